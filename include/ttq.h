@@ -1,0 +1,189 @@
+/*
+ * ttq.h -- C ABI of the TTQ linear-layer library (libttq.so, sm_100a).
+ *
+ * TTQ (activation-aware test-time quantization, arXiv:2603.19296) quantises
+ * a linear layer's weight on the fly from the activations of the current
+ * call.  For X with d input channels and T tokens and W of shape d' x d:
+ *
+ *   D_ii  = (||X_i,:||_p + lambda)^alpha                         (1)
+ *   W_hat = Q[W D^{1/2}] D^{-1/2}                                (2)
+ *   Y     = W_hat X  (+ B (A X) when a static low-rank pair is given)  (3)
+ *
+ * (1) and (2): gist.science/zh/paper/2603.19296, section 2.1 (online AWQ);
+ * also gist.science/nl/paper/2603.19296, section 2 "Kerncomponenten" 1 and
+ * gist.science/it/paper/2603.19296, section 2 "Concetti Chiave".
+ * (3): gist.science/zh/paper/2603.19296, sections 2.2 (low-rank W ~ W_q + BA)
+ * and 2.3 (projection cost O[d'dT]).  Q is the affine scale + zero-point
+ * quantiser of blog.lo0.es "Test-time quantization without calibration
+ * dataset", section "The maths that matter", applied group-wise along the
+ * input dimension.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layouts are row-major.  X is [T][d] (token-major: the pages' d x T
+ *    matrix stored column by column), W is [d'][d], A is [r][d], B is [d'][r],
+ *    Y is [T][d'].  D, D_rsqrt are float32 [d].
+ *  - Quantised weights: codes are uint32 [d'][d*bits/32]; each row is a
+ *    little-endian bit stream in which code i occupies bits [bits*i,
+ *    bits*i + bits).  scales and zeros are IEEE binary16 (as uint16 bit
+ *    patterns) [d'][d/group]; group k of row j covers input channels
+ *    [k*group, (k+1)*group).  The weight of row j, channel i is
+ *    recovered as  scales[j][k] * (code - zeros[j][k]) * D_rsqrt[i].
+ *  - The quantiser runs in binary32 in this order (bit-exact contract):
+ *      h = sqrtf(D_i);  x = W_ji * h;  m = min(0, min_group x);
+ *      M = max(0, max_group x);  s32 = (M - m) / (2^bits - 1), floored at
+ *      2^-14;  s = binary16(s32) rounded toward +inf;  inv = 1 / s;
+ *      z = clamp(rint(-m * inv), 0, 2^bits - 1);
+ *      q = clamp(rint(x * inv) + z, 0, 2^bits - 1);  rint rounds half to
+ *      even.  D == NULL means D = I (plain round-to-nearest).
+ *  - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *    caller, and must be 16-byte aligned.  The library never allocates
+ *    device memory and keeps no per-call state.  Temporary storage is the
+ *    caller's workspace `ws` of `ws_bytes` >= ttq_workspace_size(...) bytes
+ *    (256-byte aligned); its first bytes hold a device status word.
+ *    Initialise a fresh workspace once with ttq_workspace_init.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    only enqueues work on that stream and returns; the library never
+ *    synchronises.  Calls sharing one workspace must be ordered on the GPU
+ *    (same stream, or synchronised by the caller).
+ *  - Errors: invalid arguments are reported synchronously by the return
+ *    value and nothing is enqueued.  Conditions found on the device
+ *    (non-finite input or statistic, a scale beyond binary16, an internal
+ *    wait that gave up) set bits of the workspace status word and never trap
+ *    or abort the context; read them with ttq_get_status after synchronising
+ *    the stream.  Flags accumulate until ttq_workspace_init clears them.
+ *  - No function throws; every function is safe to call from C.
+ */
+#ifndef TTQ_H_
+#define TTQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ttq_status {
+  TTQ_OK = 0,
+  TTQ_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or parameter is out of range */
+  TTQ_ERR_UNSUPPORTED = 2, /* valid for the method but not built here (e.g. bits = 5) */
+  TTQ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+  TTQ_ERR_NONFINITE = 4,   /* device flag: NaN/Inf input, D_ii not in (0, inf), or scale overflow */
+  TTQ_ERR_TIMEOUT = 5,     /* device flag: an internal pipeline wait gave up (kernel returned early) */
+  TTQ_ERR_WORKSPACE = 6    /* workspace smaller than ttq_workspace_size(...) */
+} ttq_status;
+
+typedef enum ttq_dtype {
+  TTQ_F32 = 0, /* X, W, A, B and Y are float32 */
+  TTQ_BF16 = 1 /* X, W, A, B and Y are bfloat16 */
+} ttq_dtype;
+
+/* Device status word bits (ttq_get_status). */
+#define TTQ_FLAG_NONFINITE 0x1u
+#define TTQ_FLAG_SCALE_OVERFLOW 0x2u
+#define TTQ_FLAG_TIMEOUT 0x4u
+
+/* Byte offsets of the workspace regions for one problem shape (all 256-byte
+ * aligned); `total` equals ttq_workspace_size(...).  After
+ * ttq_linear_forward the regions hold that call's intermediates: D, D_rsqrt
+ * and sqrt(D) as float32 [d], the codes/scales/zeros of W_hat, and A X as
+ * bf16 [T][ax_ld].  Offsets of regions the shape does not use are 0 with
+ * size 0.  Returns TTQ_ERR_INVALID_ARG for an unsupported shape. */
+typedef struct ttq_workspace_layout {
+  size_t status;  /* uint32 status word, then internal counters */
+  size_t D;       /* float32 [d]   D_ii                          */
+  size_t D_rsqrt; /* float32 [d]   D_ii^(-1/2)                   */
+  size_t h;       /* float32 [d]   sqrtf(D_ii)                   */
+  size_t partial; /* float32 [splits][d] partial sums of |x|^p   */
+  size_t codes;   /* uint32 [d'][d*bits/32]                      */
+  size_t scales;  /* uint16 [d'][d/group]                        */
+  size_t zeros;   /* uint16 [d'][d/group]                        */
+  size_t ax;      /* bf16 [T][ax_ld]  A X                        */
+  size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32 only) */
+  size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32 only) */
+  size_t total;
+  int64_t splits; /* number of token splits of the statistic pass */
+  int64_t ax_ld;  /* row stride (elements) of A X                 */
+} ttq_workspace_layout;
+
+/* Workspace bytes needed by every entry point below for this shape
+ * (d' = dp, rank r; r = 0 means no low-rank term).  0 if the shape is
+ * unsupported. */
+size_t ttq_workspace_size(int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
+                          int group, ttq_dtype dtype);
+
+ttq_status ttq_workspace_get_layout(int64_t d, int64_t dp, int64_t T, int64_t r,
+                                    int bits, int group, ttq_dtype dtype,
+                                    ttq_workspace_layout* out);
+
+/* Clears the status word and internal counters of a workspace (enqueued on
+ * `stream`).  Call once after allocating a workspace, and to reset flags. */
+ttq_status ttq_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Step (1), the per-channel activation statistic
+ * (gist.science/zh/paper/2603.19296, section 2.1):
+ *   D[i] = (||X[:, i]||_p + lambda)^alpha,  D_rsqrt[i] = D[i]^(-1/2).
+ * X [T][d] (dtype), d % 8 == 0, T >= 0, p >= 1, lambda >= 0, alpha >= 0.
+ * The L_p norm is taken over the T tokens of this call (no 1/T factor).
+ * The sum is split over tokens and merged in a fixed order, so the result
+ * is deterministic.  D or D_rsqrt may be NULL (then they are still written
+ * to the workspace).  Flags NONFINITE if any D[i] is not finite and > 0. */
+ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
+                        float p, float lambda, float alpha, float* D,
+                        float* D_rsqrt, void* ws, size_t ws_bytes, void* stream);
+
+/* Step (2) without the rescale: codes, scales and zeros of Q[W D^{1/2}]
+ * (gist.science/zh/paper/2603.19296, section 2.1; quantiser of blog.lo0.es
+ * "The maths that matter"), in the binary32 order stated above.
+ * W [dp][d] (dtype); D float32 [d] or NULL (identity).  bits in {2, 3, 4};
+ * group in {32, 64, 128, 256} with d % group == 0.  Outputs as described
+ * above.  Flags NONFINITE for a non-finite W*sqrt(D) and SCALE_OVERFLOW
+ * (with NONFINITE) for a group whose scale exceeds binary16. */
+ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                               const float* D, int bits, int group, uint32_t* codes,
+                               uint16_t* scales, uint16_t* zeros, void* ws,
+                               size_t ws_bytes, void* stream);
+
+/* Steps (2)-(3) from already quantised weights: Y = W_hat X (+ B (A X)),
+ * with W_hat[j][i] = scales[j][k] (codes[j][i] - zeros[j][k]) D_rsqrt[i]
+ * formed in shared memory and multiplied on the tensor cores (bf16 operands,
+ * fp32 accumulation; float32 X is rounded to bf16 for the product).
+ * D_rsqrt == NULL means D = I.  A [r][d] and B [dp][r] may be NULL when
+ * r == 0; r % 8 == 0.  Y [T][dp] (dtype). */
+ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
+                            const uint16_t* zeros, const float* D_rsqrt,
+                            const void* X, const void* A, const void* B,
+                            ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,
+                            int64_t r, int bits, int group, void* Y, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/* The whole TTQ linear layer, (1) -> (2) -> (3), on `stream`:
+ *   Y = Q[W D^{1/2}] D^{-1/2} X + B (A X).
+ * X [T][d], W [dp][d], A [r][d], B [dp][r], Y [T][dp], all in `dtype`.
+ * A and B may be NULL when r == 0.  W is taken to be the residual that the
+ * static low-rank pair complements (gist.science/zh, section 2.2).
+ * The workspace keeps D, D_rsqrt, codes, scales and zeros of this call. */
+ttq_status ttq_linear_forward(const void* X, const void* W, const void* A,
+                              const void* B, ttq_dtype dtype, int64_t d, int64_t dp,
+                              int64_t T, int64_t r, float p, float lambda, float alpha,
+                              int bits, int group, void* Y, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Reads the workspace status word (a blocking device-to-host copy; the caller
+ * synchronises its stream first).  *flags receives the raw TTQ_FLAG_* bits
+ * (may be NULL).  Returns TTQ_OK if no flag is set, TTQ_ERR_TIMEOUT if the
+ * timeout flag is set, else TTQ_ERR_NONFINITE. */
+ttq_status ttq_get_status(const void* ws, uint32_t* flags);
+
+/* Static description of a status code. */
+const char* ttq_status_string(ttq_status s);
+
+/* Library version, e.g. "0.1.0". */
+const char* ttq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTQ_H_ */
