@@ -1,0 +1,390 @@
+#!/usr/bin/env python
+"""Benchmark of the TTQ linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one TTQ linear forward through the C ABI -- activation statistic,
+quantise-and-pack, dequantising tensor-core GEMM -- on one batch of seeded
+synthetic input: the Llama-7B-like q_proj prefill, d = d' = 4096, T = 2048
+tokens, INT4 with groups of 128, p = 2, lambda = 1e-3, alpha = 0.5.
+
+Metric: tokens/s of the layer (whole job over all ranks; each rank runs its
+own independent problem, so scaling is weak and there is no collective on the
+data path).  Timing: CUDA events on the launching stream around exactly K
+steps after W warm-up steps, barrier + synchronize on both sides, max over
+ranks.  The inputs rotate over enough (X, W) sets that each step's operands
+exceed the 126 MB L2, so no step reads its inputs from a warm L2.
+
+Extra keys: roofline of the dominant kernel (live CUDA-event timing of each
+kernel over the same K steps), the CPU oracle as a baseline (rank 0, N = 1),
+an end-to-end figure with host buffers and host<->device copies inside the
+timed region, clocks sampled during the run, and the number of our kernel
+launches in the timed region.
+
+--impl reference times the CPU oracle (the method written as plain loops) on
+a bounded sample of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = dict(name="q_proj_prefill_4096", d=4096, dp=4096, T=2048, bits=4, group=128, r=0,
+                p=2.0, lam=1e-3, alpha=0.5)
+METRIC = "TTQ linear tokens/s @4096^2, T=2048 (INT4 g128)"
+L2_BYTES = 126 * 2 ** 20
+
+# DRAM bytes per launch of the dominant kernel from one ncu capture, keyed by
+# the hash of the kernel source it was taken on (stale entries read as null).
+NCU_TRAFFIC = {}
+
+
+def _rank_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def _measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def _kernel_hash():
+    h = hashlib.sha256()
+    for name in ("gemm_tc.cu", "ttq_device.cuh"):
+        with open(os.path.join(ROOT, "test_weight_quantization_ttq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling in the background."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = []
+        for line in self.file.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "util": float(parts[4]),
+                             "hw": parts[6], "hwt": parts[7], "swt": parts[8], "pc": parts[9]})
+            except ValueError:
+                continue
+        os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        busy = [r for r in rows if r["util"] >= 50] or rows
+        reasons = set()
+        for r in busy:
+            if r["hw"] == "Active":
+                reasons.add("hw_slowdown")
+            if r["hwt"] == "Active":
+                reasons.add("hw_thermal_slowdown")
+            if r["swt"] == "Active":
+                reasons.add("sw_thermal_slowdown")
+            if r["pc"] == "Active":
+                reasons.add("sw_power_cap")
+        return {"sm_mhz": statistics.median(r["sm"] for r in busy), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(busy)}
+
+
+# ----------------------------------------------------------------- oracle
+def _oracle_sample(data, rows_sample: int):
+    """Times the oracle on one bounded sample of the workload: the statistic
+    and the quantiser in full, the projection for `rows_sample` output rows.
+    Returns (seconds extrapolated to the whole layer, seconds spent)."""
+    import numpy as np
+
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import ttq_oracle
+
+    from test_weight_quantization_ttq_b200 import synth
+
+    O = ttq_oracle.get()
+    w = WORKLOAD
+    X = data["X"].astype(np.float64)
+    t0 = time.perf_counter()
+    D, Dr, _ = O.act_norm(X, w["p"], w["lam"], w["alpha"])
+    codes, sc, ze, _ = O.quantize(data["W"], D.astype(np.float32), w["bits"], w["group"])
+    t1 = time.perf_counter()
+    rows = synth.sample_rows(w["dp"], rows_sample, seed=int(t0 * 1000) % 100000)
+    What = O.dequant_rows(codes, sc, ze, Dr, w["d"], w["bits"], w["group"], rows)
+    O.project(What, X)
+    t2 = time.perf_counter()
+    est = (t1 - t0) + (t2 - t1) * (w["dp"] / len(rows))
+    return est, t2 - t0
+
+
+def run_reference(args):
+    rank, world, _ = _rank_env()
+    if rank != 0:
+        return
+    from test_weight_quantization_ttq_b200 import synth
+
+    spec = synth.C2
+    data = synth.generate(spec)
+    rows_sample = 64
+    for _ in range(args.warmup):
+        _oracle_sample(data, rows_sample)
+    ests = []
+    spent = 0.0
+    for _ in range(args.steps):
+        est, s = _oracle_sample(data, rows_sample)
+        ests.append(est)
+        spent += s
+    t_step = sum(ests) / len(ests)
+    value = WORKLOAD["T"] / t_step
+    sample = (f"per step: statistic and quantiser over the full layer, projection for {rows_sample} of "
+              f"{WORKLOAD['dp']} output rows, extrapolated linearly in d'")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "cpu_seconds": spent},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config():
+    w = WORKLOAD
+    return {"workload": f"{w['name']}: TTQ linear, d=d'={w['d']}, T={w['T']}, INT{w['bits']} g{w['group']}, "
+                        f"p={w['p']}, lambda={w['lam']}, alpha={w['alpha']}, bf16 X/W/Y",
+            "d": w["d"], "d_out": w["dp"], "tokens": w["T"], "bits": w["bits"], "group": w["group"],
+            "l2": "inputs rotate over sets whose size exceeds L2 (no warm-L2 reads of X or W)"}
+
+
+# ------------------------------------------------------------------- ours
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from test_weight_quantization_ttq_b200 import synth, ttq
+
+    rank, world, local = _rank_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    w = WORKLOAD
+    spec = synth.C2
+    d, dp, T, bits, group = w["d"], w["dp"], w["T"], w["bits"], w["group"]
+    data = synth.generate(spec.with_(seed=rank))
+    set_bytes = 2 * (d * dp + T * d + T * dp)
+    nsets = max(2, -(-2 * L2_BYTES // set_bytes))
+    Xs, Ws, Ys = [], [], []
+    X0 = torch.from_numpy(data["X"]).to(torch.bfloat16)
+    W0 = torch.from_numpy(data["W"]).to(torch.bfloat16)
+    for i in range(nsets):
+        # distinct buffers with the same values: each step reads cold memory
+        Xs.append(X0.cuda())
+        Ws.append(W0.cuda())
+        Ys.append(torch.empty((T, dp), dtype=torch.bfloat16, device="cuda"))
+    ws = ttq.new_workspace(d, dp, T, 0, bits, group)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        k = i % nsets
+        ttq.ttq_linear_forward(Xs[k], Ws[k], None, None, w["p"], w["lam"], w["alpha"], bits, group,
+                               ws=ws, Y=Ys[k])
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # keep the GPU busy for ~1.5 s so the clock samples describe a loaded GPU
+    t_end = time.time() + 1.5
+    i = 0
+    while time.time() < t_end:
+        for _ in range(50):
+            step(i)
+            i += 1
+        torch.cuda.synchronize()
+
+    # ---- value: exactly K forward steps
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    clocks = sampler.stop()
+    st, flags = ttq.ttq_get_status(ws)
+    if st != ttq.TTQ_OK:
+        raise RuntimeError(f"device status {ttq.status_string(st)} (flags {flags:#x})")
+    value = world * args.steps * T / (ms / 1e3)
+
+    # ---- per-kernel durations over K steps (same kernels, one entry point each)
+    Dbuf = torch.empty(d, dtype=torch.float32, device="cuda")
+    Drbuf = torch.empty(d, dtype=torch.float32, device="cuda")
+    codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda")
+    sc = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
+    ze = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        k = i % nsets
+        ev[i][0].record(stream)
+        ttq.ttq_act_norm(Xs[k], w["p"], w["lam"], w["alpha"], ws=ws, D=Dbuf, D_rsqrt=Drbuf)
+        ev[i][1].record(stream)
+        ttq.ttq_quantize_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc, zeros=ze)
+        ev[i][2].record(stream)
+        ttq.ttq_dequant_gemm(codes, sc, ze, Drbuf, Xs[k], None, None, bits, group, ws=ws, Y=Ys[k])
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    t_act = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_qdq = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_gemm = statistics.mean(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+
+    peaks = _measured_peaks()
+    flops = 2.0 * dp * d * T
+    act_bytes = 2.0 * d * T + 8.0 * d
+    qdq_bytes = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d
+    gemm_tflops = flops / t_gemm / 1e12
+    traffic = NCU_TRAFFIC.get(_kernel_hash())
+    roofline = {"kernel": "ttq_gemm_kernel<4> (dequantising tcgen05 GEMM)", "bound": "tensor",
+                "achieved": gemm_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": gemm_tflops / peaks["bf16_tflops"], "traffic": traffic,
+                "peak_source": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
+                "algorithmic_flops_per_launch": flops}
+    kernels = [
+        {"kernel": "act_norm_kernel", "ms": t_act * 1e3, "bound": "hbm", "bytes": act_bytes,
+         "achieved_gbs": act_bytes / t_act / 1e9, "frac": act_bytes / t_act / 1e9 / peaks["hbm_gbs"]},
+        {"kernel": "qdq_pack_kernel", "ms": t_qdq * 1e3, "bound": "hbm", "bytes": qdq_bytes,
+         "achieved_gbs": qdq_bytes / t_qdq / 1e9, "frac": qdq_bytes / t_qdq / 1e9 / peaks["hbm_gbs"]},
+        {"kernel": "ttq_gemm_kernel", "ms": t_gemm * 1e3, "bound": "tensor", "flops": flops,
+         "achieved_tflops": gemm_tflops, "frac": gemm_tflops / peaks["bf16_tflops"]},
+    ]
+    rho = {"measured": (t_act + t_qdq) / t_gemm, "closed_form": 1.0 / dp + 3.0 / T}
+
+    # ---- end to end: pinned host X in, host Y out, inside the timed region
+    Xh = X0.pin_memory()
+    Yh = torch.empty((T, dp), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty_like(Xs[0])
+    barrier()
+    torch.cuda.synchronize()
+    for _ in range(2):
+        Xd.copy_(Xh, non_blocking=True)
+        ttq.ttq_linear_forward(Xd, Ws[0], None, None, w["p"], w["lam"], w["alpha"], bits, group, ws=ws, Y=Ys[0])
+        Yh.copy_(Ys[0], non_blocking=True)
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for i in range(args.steps):
+        Xd.copy_(Xh, non_blocking=True)
+        ttq.ttq_linear_forward(Xd, Ws[i % nsets], None, None, w["p"], w["lam"], w["alpha"], bits, group,
+                               ws=ws, Y=Ys[0])
+        Yh.copy_(Ys[0], non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e = {"value": world * args.steps * T / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows_sample = 512
+        est, spent = _oracle_sample(data, rows_sample)
+        cpu = {"value": T / est, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"statistic and quantiser over the full layer, projection for {rows_sample} of {dp} "
+                         f"output rows, extrapolated linearly in d' ({spent:.1f} s of CPU work)"}
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(),
+        "roofline": roofline, "kernels": kernels, "rho": rho, "cpu_baseline": cpu, "e2e": e2e,
+        "clocks": clocks, "gpu_launches": 3 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

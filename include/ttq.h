@@ -86,15 +86,14 @@ typedef enum ttq_dtype {
 
 /* Byte offsets of the workspace regions for one problem shape (all 256-byte
  * aligned); `total` equals ttq_workspace_size(...).  After
- * ttq_linear_forward the regions hold that call's intermediates: D, D_rsqrt
- * and sqrt(D) as float32 [d], the codes/scales/zeros of W_hat, and A X as
- * bf16 [T][ax_ld].  Offsets of regions the shape does not use are 0 with
+ * ttq_linear_forward the regions hold that call's intermediates: D and
+ * D_rsqrt as float32 [d], the codes/scales/zeros of W_hat, and A X as bf16
+ * [T][ax_ld].  Offsets of regions the shape does not use are 0 with
  * size 0.  Returns TTQ_ERR_INVALID_ARG for an unsupported shape. */
 typedef struct ttq_workspace_layout {
   size_t status;  /* uint32 status word, then internal counters */
   size_t D;       /* float32 [d]   D_ii                          */
   size_t D_rsqrt; /* float32 [d]   D_ii^(-1/2)                   */
-  size_t h;       /* float32 [d]   sqrtf(D_ii)                   */
   size_t partial; /* float32 [splits][d] partial sums of |x|^p   */
   size_t codes;   /* uint32 [d'][d*bits/32]                      */
   size_t scales;  /* uint16 [d'][d/group]                        */

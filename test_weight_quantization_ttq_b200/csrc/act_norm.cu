@@ -1,0 +1,205 @@
+// Step (1) of the TTQ layer: the per-channel activation statistic
+//   D_ii = (||X_i,:||_p + lambda)^alpha,  and D_ii^(-1/2)
+// (gist.science/zh/paper/2603.19296, section 2.1).  X is [T][d] (token
+// major), so channel i is a column: the reduction runs down the columns.
+//
+// Layout of the work: a block owns 256 consecutive channels and one split of
+// the tokens.  Each lane loads 8 consecutive channels of a row (one 16-byte
+// load for bf16), each of the 8 warps walks every 8th row of the split, and
+// the warps' sums are merged in shared memory in a fixed order.  The split's
+// partial sums go to global memory; the last block to finish a column block
+// (an atomic ticket) merges all splits in fp64, in split order, so the
+// result does not depend on scheduling.  The pass is HBM-bound: it reads X
+// once (2dT bytes for bf16) and writes 8d bytes.
+#include "ttq_device.cuh"
+#include "ttq_kernels.h"
+
+namespace ttq {
+namespace {
+
+constexpr int kChannelsPerBlock = 256;
+constexpr int kThreads = 256;
+
+template <int PK>  // 1: p = 1, 2: p = 2, 0: any p >= 1
+__device__ __forceinline__ float abs_pow(float x, float p) {
+  const float a = fabsf(x);
+  if (PK == 1) return a;
+  if (PK == 2) return a * a;
+  return powf(a, p);
+}
+
+__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float (&v)[8]) {
+  uint4 raw;
+  __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
+  __nv_bfloat162 h1 = __floats2bfloat162_rn(v[2], v[3]);
+  __nv_bfloat162 h2 = __floats2bfloat162_rn(v[4], v[5]);
+  __nv_bfloat162 h3 = __floats2bfloat162_rn(v[6], v[7]);
+  raw.x = *reinterpret_cast<uint32_t*>(&h0);
+  raw.y = *reinterpret_cast<uint32_t*>(&h1);
+  raw.z = *reinterpret_cast<uint32_t*>(&h2);
+  raw.w = *reinterpret_cast<uint32_t*>(&h3);
+  *reinterpret_cast<uint4*>(dst) = raw;
+}
+
+template <typename XT, int PK>
+__global__ void __launch_bounds__(kThreads) act_norm_kernel(
+    const XT* __restrict__ X, int64_t d, int64_t T, float p, double lambda, double alpha,
+    int64_t splits, int64_t rows_per_split, float* __restrict__ partial,
+    uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
+    __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
+  __shared__ float red[8][kChannelsPerBlock + 8];
+  __shared__ int is_last;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t cb = blockIdx.x;
+  const int64_t sp = blockIdx.y;
+  const int64_t c0 = cb * kChannelsPerBlock + lane * 8;
+
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+
+  const int64_t t_begin = sp * rows_per_split;
+  const int64_t t_end = min(T, t_begin + rows_per_split);
+  if (c0 < d) {
+    int64_t t = t_begin + warp;
+    // two rows in flight per warp
+    for (; t + 8 < t_end; t += 16) {
+      float v0[8], v1[8];
+      load8(X + t * d + c0, v0);
+      load8(X + (t + 8) * d + c0, v1);
+      if (xb != nullptr) {
+        store8_bf16(xb + t * d + c0, v0);
+        store8_bf16(xb + (t + 8) * d + c0, v1);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v0[e], p) + abs_pow<PK>(v1[e], p);
+    }
+    for (; t < t_end; t += 8) {
+      float v0[8];
+      load8(X + t * d + c0, v0);
+      if (xb != nullptr) store8_bf16(xb + t * d + c0, v0);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v0[e], p);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
+  __syncthreads();
+
+  const int ci = threadIdx.x;
+  const int64_t c = cb * kChannelsPerBlock + ci;
+  float sum = 0.f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) sum += red[w][ci];
+  if (c < d) partial[sp * d + c] = sum;
+
+  // Ticket: the last split block of this column block merges all splits.
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atomicAdd(&counters[cb], 1u);
+    is_last = (prev == static_cast<uint32_t>(splits - 1)) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  if (c < d) {
+    double tot = 0.0;
+    for (int64_t s = 0; s < splits; ++s) tot += static_cast<double>(__ldcg(partial + s * d + c));
+    double n;
+    if (PK == 1) {
+      n = tot;
+    } else if (PK == 2) {
+      n = sqrt(tot);
+    } else {
+      n = pow(tot, 1.0 / static_cast<double>(p));
+    }
+    const double dv = pow(n + lambda, alpha);
+    const double drv = 1.0 / sqrt(dv);
+    const float df = static_cast<float>(dv);
+    const float drf = static_cast<float>(drv);
+    D[c] = df;
+    Dr[c] = drf;
+    const bool ok = (df > 0.f) && (df <= 3.402823466e38f) && (drf > 0.f) && (drf <= 3.402823466e38f);
+    if (!ok) set_flag(status, TTQ_FLAG_NONFINITE);
+  }
+  if (threadIdx.x == 0) counters[cb] = 0u;  // ready for the next call
+}
+
+template <typename XT, int PK>
+cudaError_t launch_typed(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
+                         int64_t splits, int64_t rows_per_split, float* partial,
+                         uint32_t* counters, float* D, float* Dr, void* xb, uint32_t* status,
+                         cudaStream_t stream) {
+  const dim3 grid(static_cast<unsigned>((d + kChannelsPerBlock - 1) / kChannelsPerBlock),
+                  static_cast<unsigned>(splits));
+  act_norm_kernel<XT, PK><<<grid, kThreads, 0, stream>>>(
+      X, d, T, p, static_cast<double>(lambda), static_cast<double>(alpha), splits,
+      rows_per_split, partial, counters, D, Dr, static_cast<__nv_bfloat16*>(xb), status);
+  return cudaGetLastError();
+}
+
+template <typename XT>
+cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
+                     int64_t splits, int64_t rows_per_split, float* partial, uint32_t* counters,
+                     float* D, float* Dr, void* xb, uint32_t* status, cudaStream_t stream) {
+  if (p == 1.0f)
+    return launch_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
+                               counters, D, Dr, xb, status, stream);
+  if (p == 2.0f)
+    return launch_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
+                               counters, D, Dr, xb, status, stream);
+  return launch_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
+                             counters, D, Dr, xb, status, stream);
+}
+
+}  // namespace
+
+void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split) {
+  const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
+  const int64_t target = static_cast<int64_t>(num_sms) * 4;
+  int64_t s = (target + ncb - 1) / ncb;
+  const int64_t max_by_rows = (T + 31) / 32;  // at least 32 rows per split
+  if (s > max_by_rows) s = max_by_rows;
+  if (s > 256) s = 256;
+  if (s < 1) s = 1;
+  int64_t rps = (T + s - 1) / s;
+  if (rps < 1) rps = 1;
+  s = (T + rps - 1) / rps;
+  if (s < 1) s = 1;
+  *splits = s;
+  *rows_per_split = rps;
+}
+
+cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
+                            float lambda, float alpha, int64_t splits, int64_t rows_per_split,
+                            float* partial, uint32_t* counters, float* D, float* Dr, void* xb,
+                            uint32_t* status, cudaStream_t stream) {
+  if (x_f32)
+    return launch_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits, rows_per_split,
+                    partial, counters, D, Dr, xb, status, stream);
+  return launch_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
+                  rows_per_split, partial, counters, D, Dr, nullptr, status, stream);
+}
+
+}  // namespace ttq

@@ -1,0 +1,390 @@
+// The C ABI of libttq.so (declared in include/ttq.h): argument checks,
+// workspace layout, TMA descriptor set-up and the order of the kernels of
+// one TTQ linear call.  Nothing here allocates device memory or
+// synchronises; every call only enqueues work on the caller's stream.
+#include <cmath>
+#include <mutex>
+
+#include "ttq.h"
+#include "ttq_device.cuh"
+#include "ttq_kernels.h"
+
+namespace ttq {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 4096;           // status word + act_norm tickets
+constexpr int64_t kMaxColumnBlocks = 960;       // tickets after the first 256 bytes
+constexpr int kPlanSMs = 148;                   // fixed so the layout is device-independent
+
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return kPlanSMs;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = kPlanSMs;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
+bool valid_qparams(int bits, int group) {
+  return (bits >= 2 && bits <= 4) && (group == 32 || group == 64 || group == 128 || group == 256);
+}
+
+// Computes the workspace layout; false for an unsupported shape.
+bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
+                 ttq_dtype dtype, ttq_workspace_layout* L) {
+  if (d < 8 || d % 8 != 0 || dp < 0 || T < 0 || r < 0 || r % 8 != 0) return false;
+  if ((d + 255) / 256 > kMaxColumnBlocks) return false;
+  const bool has_q = dp > 0;
+  if (has_q && (!valid_qparams(bits, group) || d % group != 0)) return false;
+  if (dtype != TTQ_F32 && dtype != TTQ_BF16) return false;
+  ttq_workspace_layout l = {};
+  int64_t splits = 1, rps = 1;
+  act_norm_plan(d, T, kPlanSMs, &splits, &rps);
+  size_t off = 0;
+  l.status = off;
+  off += kStatusBytes;
+  l.D = off;
+  off = align_up(off + 4 * static_cast<size_t>(d));
+  l.D_rsqrt = off;
+  off = align_up(off + 4 * static_cast<size_t>(d));
+  l.partial = off;
+  off = align_up(off + 4 * static_cast<size_t>(splits) * static_cast<size_t>(d));
+  if (has_q) {
+    l.codes = off;
+    off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d * bits / 32) * 4);
+    l.scales = off;
+    off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d / group) * 2);
+    l.zeros = off;
+    off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d / group) * 2);
+  }
+  l.ax_ld = 0;
+  if (r > 0) {
+    l.ax_ld = r;
+    l.ax = off;
+    off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(r) * 2);
+  }
+  if (dtype == TTQ_F32) {
+    l.xb = off;
+    off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(d) * 2);
+    if (r > 0) {
+      l.ab = off;
+      off = align_up(off + (static_cast<size_t>(r) * d + static_cast<size_t>(dp) * r) * 2);
+    }
+  }
+  l.total = off;
+  l.splits = splits;
+  *L = l;
+  return true;
+}
+
+// ----------------------------------------------------- tensor map encoding
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                              const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                              const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [outer][inner] with row stride ld (elements), loaded as
+// box_outer rows x 64 columns into the 128-byte-swizzled layout; reads
+// outside the matrix return zeros.
+bool encode_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                 int box_outer) {
+  EncodeFn enc = get_encode();
+  if (enc == nullptr || inner < 1 || outer < 1) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
+  const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_outer)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_ERR_CUDA; }
+
+uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
+
+// Y = W_hat X (+ B (A X)) from quantised weights; X, A, B already bf16.
+ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                    const float* Dr, const void* Xb, const void* Ab, const void* Bb, int64_t d,
+                    int64_t dp, int64_t T, int64_t r, int bits, int group, void* Y, bool y_f32,
+                    void* ws, const ttq_workspace_layout& L, cudaStream_t stream) {
+  if (T == 0 || dp == 0) return TTQ_OK;
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  void* ax = r > 0 ? ws_at(ws, L.ax) : nullptr;
+  if (r > 0) {
+    // A X: the plain-operand mode of the same kernel, M = r rows of A.
+    const int bn = gemm_block_n(T);
+    GemmMaps m;
+    if (!encode_bf16(&m.a0, Ab, d, r, d, 128) || !encode_bf16(&m.b0, Xb, d, T, d, bn))
+      return TTQ_ERR_CUDA;
+    m.a1 = m.a0;
+    m.b1 = m.b0;
+    GemmArgs a;
+    a.bits = 0;
+    a.K = d;
+    a.M = r;
+    a.T = T;
+    a.K_tail = 0;
+    a.Y = ax;
+    a.ldy = L.ax_ld;
+    a.y_f32 = false;
+    a.status = status;
+    const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, stream));
+    if (st != TTQ_OK) return st;
+  }
+  const int bn = gemm_block_n(T);
+  GemmMaps m;
+  if (!encode_bf16(&m.b0, Xb, d, T, d, bn)) return TTQ_ERR_CUDA;
+  m.a0 = m.b0;
+  if (r > 0) {
+    if (!encode_bf16(&m.a1, Bb, r, dp, r, 128) || !encode_bf16(&m.b1, ax, r, T, L.ax_ld, bn))
+      return TTQ_ERR_CUDA;
+  } else {
+    m.a1 = m.b0;
+    m.b1 = m.b0;
+  }
+  GemmArgs a;
+  a.codes = codes;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.Dr = Dr;
+  a.bits = bits;
+  a.group = group;
+  a.K = d;
+  a.M = dp;
+  a.T = T;
+  a.K_tail = r;
+  a.Y = Y;
+  a.ldy = dp;
+  a.y_f32 = y_f32;
+  a.status = status;
+  return cuda_status(launch_dequant_gemm(a, m, bn, stream));
+}
+
+}  // namespace
+}  // namespace ttq
+
+using namespace ttq;
+
+extern "C" {
+
+size_t ttq_workspace_size(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
+                          ttq_dtype dtype) {
+  ttq_workspace_layout L;
+  if (!make_layout(d, dp, T, r, bits, group, dtype, &L)) return 0;
+  return L.total;
+}
+
+ttq_status ttq_workspace_get_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
+                                    int group, ttq_dtype dtype, ttq_workspace_layout* out) {
+  if (out == nullptr) return TTQ_ERR_INVALID_ARG;
+  if (!make_layout(d, dp, T, r, bits, group, dtype, out)) return TTQ_ERR_INVALID_ARG;
+  return TTQ_OK;
+}
+
+ttq_status ttq_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || ws_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return TTQ_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+}
+
+ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T, float p,
+                        float lambda, float alpha, float* D, float* D_rsqrt, void* ws,
+                        size_t ws_bytes, void* stream) {
+  ttq_workspace_layout L;
+  if (!make_layout(d, 0, T, 0, 4, 32, dtype, &L)) return TTQ_ERR_INVALID_ARG;
+  if ((T > 0 && X == nullptr) || ws == nullptr || !(p >= 1.0f) || !(lambda >= 0.0f) ||
+      !(alpha >= 0.0f) || !std::isfinite(p) || !std::isfinite(lambda) || !std::isfinite(alpha))
+    return TTQ_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (D && !aligned16(D)) || (D_rsqrt && !aligned16(D_rsqrt)) ||
+      (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return TTQ_ERR_INVALID_ARG;
+  const size_t need = L.partial + align_up(4 * static_cast<size_t>(L.splits) * d);
+  if (ws_bytes < need) return TTQ_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  float* Dw = reinterpret_cast<float*>(ws_at(ws, L.D));
+  float* Drw = reinterpret_cast<float*>(ws_at(ws, L.D_rsqrt));
+  int64_t splits, rps;
+  act_norm_plan(d, T, kPlanSMs, &splits, &rps);
+  ttq_status st = cuda_status(launch_act_norm(
+      X, dtype == TTQ_F32, d, T, p, lambda, alpha, splits, rps,
+      reinterpret_cast<float*>(ws_at(ws, L.partial)), status + 64, Dw, Drw, nullptr, status, s));
+  if (st != TTQ_OK) return st;
+  if (D) st = cuda_status(cudaMemcpyAsync(D, Dw, 4 * d, cudaMemcpyDeviceToDevice, s));
+  if (st == TTQ_OK && D_rsqrt)
+    st = cuda_status(cudaMemcpyAsync(D_rsqrt, Drw, 4 * d, cudaMemcpyDeviceToDevice, s));
+  return st;
+}
+
+ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                               const float* D, int bits, int group, uint32_t* codes,
+                               uint16_t* scales, uint16_t* zeros, void* ws, size_t ws_bytes,
+                               void* stream) {
+  if (dtype != TTQ_F32 && dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
+  if (bits < 1 || bits > 8 || group < 1) return TTQ_ERR_INVALID_ARG;
+  if (!valid_qparams(bits, group)) return TTQ_ERR_UNSUPPORTED;
+  if (d < group || d % group != 0 || dp < 0) return TTQ_ERR_INVALID_ARG;
+  if (dp > 0 && (W == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr))
+    return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if ((W && !aligned16(W)) || (D && !aligned16(D)) || (codes && !aligned16(codes)))
+    return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  return cuda_status(launch_qdq_pack(W, dtype == TTQ_F32, dp, d, D, bits, group, codes, scales,
+                                     zeros, status, device_sms(),
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
+                            const float* D_rsqrt, const void* X, const void* A, const void* B,
+                            ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
+                            int bits, int group, void* Y, void* ws, size_t ws_bytes,
+                            void* stream) {
+  if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
+    return TTQ_ERR_UNSUPPORTED;
+  ttq_workspace_layout L;
+  if (!make_layout(d, dp, T, r, bits, group, dtype, &L)) return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
+  const bool work = dp > 0 && T > 0;
+  if (work && (codes == nullptr || scales == nullptr || zeros == nullptr || X == nullptr ||
+               Y == nullptr))
+    return TTQ_ERR_INVALID_ARG;
+  if (r > 0 && (A == nullptr || B == nullptr)) return TTQ_ERR_INVALID_ARG;
+  const void* ptrs[] = {codes, scales, zeros, D_rsqrt, X, A, B, Y};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTQ_ERR_INVALID_ARG;
+  if (!work) return TTQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void* Xb = X;
+  const void* Ab = A;
+  const void* Bb = B;
+  if (dtype == TTQ_F32) {
+    void* xb = ws_at(ws, L.xb);
+    ttq_status st = cuda_status(launch_to_bf16(static_cast<const float*>(X), xb, T * d, s));
+    if (st != TTQ_OK) return st;
+    Xb = xb;
+    if (r > 0) {
+      void* ab = ws_at(ws, L.ab);
+      void* bb = static_cast<uint8_t*>(ab) + static_cast<size_t>(r) * d * 2;
+      st = cuda_status(launch_to_bf16(static_cast<const float*>(A), ab, r * d, s));
+      if (st == TTQ_OK) st = cuda_status(launch_to_bf16(static_cast<const float*>(B), bb, dp * r, s));
+      if (st != TTQ_OK) return st;
+      Ab = ab;
+      Bb = bb;
+    }
+  }
+  return run_gemm(codes, scales, zeros, D_rsqrt, Xb, Ab, Bb, d, dp, T, r, bits, group, Y,
+                  dtype == TTQ_F32, ws, L, s);
+}
+
+ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const void* B,
+                              ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
+                              float p, float lambda, float alpha, int bits, int group, void* Y,
+                              void* ws, size_t ws_bytes, void* stream) {
+  if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
+    return TTQ_ERR_UNSUPPORTED;
+  ttq_workspace_layout L;
+  if (!make_layout(d, dp, T, r, bits, group, dtype, &L)) return TTQ_ERR_INVALID_ARG;
+  if (dp == 0 && !valid_qparams(bits, group)) return TTQ_ERR_INVALID_ARG;
+  if (!(p >= 1.0f) || !(lambda >= 0.0f) || !(alpha >= 0.0f) || !std::isfinite(p) ||
+      !std::isfinite(lambda) || !std::isfinite(alpha))
+    return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
+  if ((T > 0 && X == nullptr) || (dp > 0 && W == nullptr) || (T > 0 && dp > 0 && Y == nullptr))
+    return TTQ_ERR_INVALID_ARG;
+  if (r > 0 && (A == nullptr || B == nullptr)) return TTQ_ERR_INVALID_ARG;
+  const void* ptrs[] = {X, W, A, B, Y};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return TTQ_ERR_INVALID_ARG;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  float* D = reinterpret_cast<float*>(ws_at(ws, L.D));
+  float* Dr = reinterpret_cast<float*>(ws_at(ws, L.D_rsqrt));
+  const bool f32 = dtype == TTQ_F32;
+  void* xb = f32 ? ws_at(ws, L.xb) : nullptr;
+
+  // (1) D and D^{-1/2} (float32 X is also narrowed to bf16 on the way)
+  int64_t splits, rps;
+  act_norm_plan(d, T, kPlanSMs, &splits, &rps);
+  ttq_status st = cuda_status(launch_act_norm(
+      X, f32, d, T, p, lambda, alpha, splits, rps,
+      reinterpret_cast<float*>(ws_at(ws, L.partial)), status + 64, D, Dr, xb, status, s));
+  if (st != TTQ_OK || dp == 0) return st;
+
+  // (2) codes, scales, zeros of Q[W D^{1/2}]
+  uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));
+  uint16_t* scales = reinterpret_cast<uint16_t*>(ws_at(ws, L.scales));
+  uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
+  st = cuda_status(launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros, status,
+                                   device_sms(), s));
+  if (st != TTQ_OK || T == 0) return st;
+
+  // (3) Y = W_hat X (+ B (A X))
+  const void* Ab = A;
+  const void* Bb = B;
+  if (f32 && r > 0) {
+    void* ab = ws_at(ws, L.ab);
+    void* bb = static_cast<uint8_t*>(ab) + static_cast<size_t>(r) * d * 2;
+    st = cuda_status(launch_to_bf16(static_cast<const float*>(A), ab, r * d, s));
+    if (st == TTQ_OK) st = cuda_status(launch_to_bf16(static_cast<const float*>(B), bb, dp * r, s));
+    if (st != TTQ_OK) return st;
+    Ab = ab;
+    Bb = bb;
+  }
+  return run_gemm(codes, scales, zeros, Dr, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
+                  f32, ws, L, s);
+}
+
+ttq_status ttq_get_status(const void* ws, uint32_t* flags) {
+  if (ws == nullptr) return TTQ_ERR_INVALID_ARG;
+  uint32_t f = 0;
+  if (cudaMemcpy(&f, ws, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess) return TTQ_ERR_CUDA;
+  if (flags) *flags = f;
+  if (f & TTQ_FLAG_TIMEOUT) return TTQ_ERR_TIMEOUT;
+  if (f) return TTQ_ERR_NONFINITE;
+  return TTQ_OK;
+}
+
+const char* ttq_status_string(ttq_status s) {
+  switch (s) {
+    case TTQ_OK: return "ok";
+    case TTQ_ERR_INVALID_ARG: return "invalid argument";
+    case TTQ_ERR_UNSUPPORTED: return "unsupported parameter combination";
+    case TTQ_ERR_CUDA: return "CUDA error";
+    case TTQ_ERR_NONFINITE: return "non-finite value or binary16 scale overflow";
+    case TTQ_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case TTQ_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* ttq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

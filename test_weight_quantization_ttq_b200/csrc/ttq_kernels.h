@@ -1,0 +1,66 @@
+// Host-side launchers of the TTQ kernels (internal to libttq.so).  Each
+// returns cudaSuccess or the launch error; argument checking is done by the
+// C ABI layer (ttq_api.cu) before these are called.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ttq {
+
+// Number of token splits of the statistic pass and the rows each covers.
+void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split);
+
+// Step (1): D, D^{-1/2} from X [T][d].  `partial` holds splits x d floats,
+// `counters` ceil(d/256) uint32 that start (and are left) at zero.  When
+// xb is non-null the float32 X is also written out as bf16 [T][d].
+cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
+                            float lambda, float alpha, int64_t splits, int64_t rows_per_split,
+                            float* partial, uint32_t* counters, float* D, float* Dr,
+                            void* xb, uint32_t* status, cudaStream_t stream);
+
+// Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null).
+cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
+                            int bits, int group, uint32_t* codes, uint16_t* scales,
+                            uint16_t* zeros, uint32_t* status, int num_sms,
+                            cudaStream_t stream);
+
+// float32 -> bf16 copy of n elements (n % 8 == 0).
+cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
+
+// Steps (2)-(3) on the tensor cores.
+struct GemmArgs {
+  // dequantised A operand (bits != 0) ...
+  const uint32_t* codes = nullptr;
+  const uint16_t* scales = nullptr;
+  const uint16_t* zeros = nullptr;
+  const float* Dr = nullptr;  // null: identity
+  int bits = 0;               // 0: A operand loaded by TMA from tmA0 (plain bf16)
+  int group = 0;
+  // sizes
+  int64_t K = 0;        // reduction length of the main part (d)
+  int64_t M = 0;        // output rows (d', or r for the A X product)
+  int64_t T = 0;        // tokens
+  int64_t K_tail = 0;   // low-rank reduction length r (0: none)
+  // output Y[t][j] at Y + t * ldy + j
+  void* Y = nullptr;
+  int64_t ldy = 0;
+  bool y_f32 = false;
+  uint32_t* status = nullptr;
+};
+
+struct GemmMaps {
+  CUtensorMap a0;  // plain A operand [M][K] bf16 (bits == 0)
+  CUtensorMap b0;  // X [T][K] bf16
+  CUtensorMap a1;  // low-rank B [M][r] bf16
+  CUtensorMap b1;  // A X [T][r] bf16
+};
+
+// Tile width along the tokens for T tokens.
+int gemm_block_n(int64_t T);
+
+cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,
+                                cudaStream_t stream);
+
+}  // namespace ttq

@@ -26,9 +26,10 @@ def bf16_round(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest bfloat16 (ties to even); the
     result is returned as float32 holding bf16-representable values."""
     a = np.ascontiguousarray(a, dtype=np.float32)
-    u = a.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return (u.astype(np.uint32) << 16).view(np.float32).reshape(a.shape)
+    u = a.view(np.uint32)
+    # finite inputs cannot carry past bit 31: the largest is 0xFF7FFFFF + 0x8000
+    u = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return u.view(np.float32).reshape(a.shape)
 
 
 def bf16_bits(a: np.ndarray) -> np.ndarray:

@@ -1,0 +1,235 @@
+"""Python binding of libttq.so: the C ABI of include/ttq.h, one function per
+entry point with the same name.  Argument marshalling only -- every step of
+the TTQ layer runs in the library's CUDA kernels; torch supplies device
+memory and the current stream.  There is no fallback: if the library is
+missing or the tensors are not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_HERE, "libttq.so")
+
+TTQ_OK = 0
+TTQ_ERR_INVALID_ARG = 1
+TTQ_ERR_UNSUPPORTED = 2
+TTQ_ERR_CUDA = 3
+TTQ_ERR_NONFINITE = 4
+TTQ_ERR_TIMEOUT = 5
+TTQ_ERR_WORKSPACE = 6
+
+TTQ_F32 = 0
+TTQ_BF16 = 1
+
+TTQ_FLAG_NONFINITE = 0x1
+TTQ_FLAG_SCALE_OVERFLOW = 0x2
+TTQ_FLAG_TIMEOUT = 0x4
+
+# C signatures, in the order of include/ttq.h
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_F = ctypes.c_float
+_SZ = ctypes.c_size_t
+
+
+class WorkspaceLayout(ctypes.Structure):
+    _fields_ = [("status", _SZ), ("D", _SZ), ("D_rsqrt", _SZ), ("partial", _SZ), ("codes", _SZ),
+                ("scales", _SZ), ("zeros", _SZ), ("ax", _SZ), ("xb", _SZ), ("ab", _SZ),
+                ("total", _SZ), ("splits", _I64), ("ax_ld", _I64)]
+
+
+SIGNATURES = {
+    "ttq_workspace_size": (_SZ, [_I64, _I64, _I64, _I64, _INT, _INT, _INT]),
+    "ttq_workspace_get_layout": (_INT, [_I64, _I64, _I64, _I64, _INT, _INT, _INT,
+                                        ctypes.POINTER(WorkspaceLayout)]),
+    "ttq_workspace_init": (_INT, [_P, _SZ, _P]),
+    "ttq_act_norm": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _SZ, _P]),
+    "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
+    "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
+                                _P, _P, _SZ, _P]),
+    "ttq_linear_forward": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT, _INT,
+                                  _P, _P, _SZ, _P]),
+    "ttq_get_status": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "ttq_status_string": (ctypes.c_char_p, [_INT]),
+    "ttq_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class TTQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status) if _lib else status} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIBRARY):
+            raise RuntimeError(f"libttq.so not found at {LIBRARY}; build it with "
+                               "`python -m test_weight_quantization_ttq_b200.build`")
+        L = ctypes.CDLL(LIBRARY)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(st: int) -> str:
+    return lib().ttq_status_string(int(st)).decode()
+
+
+def _check(st: int, where: str) -> None:
+    if st != TTQ_OK:
+        raise TTQError(st, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TTQ_F32
+    if t.dtype == torch.bfloat16:
+        return TTQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _dev(t: torch.Tensor | None, name: str) -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream or None
+
+
+# ------------------------------------------------------------- workspace
+def ttq_workspace_size(d, dp, T, r, bits, group, dtype=TTQ_BF16) -> int:
+    return int(lib().ttq_workspace_size(d, dp, T, r, bits, group, dtype))
+
+
+def ttq_workspace_get_layout(d, dp, T, r, bits, group, dtype=TTQ_BF16) -> WorkspaceLayout:
+    out = WorkspaceLayout()
+    _check(lib().ttq_workspace_get_layout(d, dp, T, r, bits, group, dtype, ctypes.byref(out)),
+           "ttq_workspace_get_layout")
+    return out
+
+
+def ttq_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(lib().ttq_workspace_init(_dev(ws, "ws"), ws.numel(), _stream(stream)), "ttq_workspace_init")
+
+
+def new_workspace(d, dp, T, r, bits, group, dtype=TTQ_BF16, device="cuda", stream=None) -> torch.Tensor:
+    """A zero-initialised workspace (uint8 tensor) for this shape."""
+    n = ttq_workspace_size(d, dp, T, r, bits, group, dtype)
+    if n == 0:
+        raise TTQError(TTQ_ERR_INVALID_ARG, "ttq_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    ttq_workspace_init(ws, stream)
+    return ws
+
+
+def ttq_get_status(ws: torch.Tensor) -> tuple[int, int]:
+    """(status, raw flag bits) of the workspace; synchronise the stream first."""
+    flags = ctypes.c_uint32(0)
+    st = lib().ttq_get_status(_dev(ws, "ws"), ctypes.byref(flags))
+    return int(st), int(flags.value)
+
+
+# ---------------------------------------------------------- entry points
+def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None):
+    """D[i] = (||X[:, i]||_p + lambda)^alpha and D^{-1/2}; X is [T][d]."""
+    T, d = X.shape
+    if ws is None:
+        ws = new_workspace(d, 0, T, 0, 4, 32, _dtype_code(X), X.device, stream)
+    if D is None:
+        D = torch.empty(d, dtype=torch.float32, device=X.device)
+    if D_rsqrt is None:
+        D_rsqrt = torch.empty(d, dtype=torch.float32, device=X.device)
+    _check(lib().ttq_act_norm(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, _dev(D, "D"),
+                              _dev(D_rsqrt, "D_rsqrt"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "ttq_act_norm")
+    return D, D_rsqrt
+
+
+def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zeros=None, stream=None):
+    """codes [d'][d*bits/32] uint32, scales/zeros [d'][d/group] binary16 bits (int16 storage)."""
+    dp, d = W.shape
+    dev = W.device
+    if ws is None:
+        ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
+    if codes is None:
+        codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
+    if zeros is None:
+        zeros = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
+    _check(lib().ttq_quantize_weight(_dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group,
+                                     _dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
+                                     _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "ttq_quantize_weight")
+    return codes, scales, zeros
+
+
+def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=None, Y=None, stream=None):
+    """Y [T][d'] = W_hat X (+ B (A X)) from quantised weights."""
+    T, d = X.shape
+    dp = codes.shape[0]
+    r = 0 if A is None else A.shape[0]
+    dt = _dtype_code(X)
+    if ws is None:
+        ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
+    if Y is None:
+        Y = torch.empty((T, dp), dtype=X.dtype, device=X.device)
+    _check(lib().ttq_dequant_gemm(_dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
+                                  _dev(D_rsqrt, "D_rsqrt"), _dev(X, "X"), _dev(A, "A"), _dev(B, "B"), dt,
+                                  d, dp, T, r, bits, group, _dev(Y, "Y"), _dev(ws, "ws"), ws.numel(),
+                                  _stream(stream)),
+           "ttq_dequant_gemm")
+    return Y
+
+
+def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, stream=None):
+    """The TTQ linear layer: Y [T][d'] = Q[W D^{1/2}] D^{-1/2} X + B (A X)."""
+    T, d = X.shape
+    dp = W.shape[0]
+    r = 0 if A is None else A.shape[0]
+    dt = _dtype_code(X)
+    if ws is None:
+        ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
+    if Y is None:
+        Y = torch.empty((T, dp), dtype=X.dtype, device=X.device)
+    _check(lib().ttq_linear_forward(_dev(X, "X"), _dev(W, "W"), _dev(A, "A"), _dev(B, "B"), dt, d, dp, T,
+                                    r, p, lam, alpha, bits, group, _dev(Y, "Y"), _dev(ws, "ws"), ws.numel(),
+                                    _stream(stream)),
+           "ttq_linear_forward")
+    return Y
+
+
+def workspace_views(ws: torch.Tensor, d, dp, T, r, bits, group, dtype=TTQ_BF16) -> dict:
+    """Views of the intermediates a forward call leaves in its workspace."""
+    L = ttq_workspace_get_layout(d, dp, T, r, bits, group, dtype)
+
+    def view(off, n, dt):
+        itemsize = torch.empty((), dtype=dt).element_size()
+        return ws[off: off + n * itemsize].view(dt)
+
+    out = {"D": view(L.D, d, torch.float32), "D_rsqrt": view(L.D_rsqrt, d, torch.float32)}
+    if dp > 0:
+        out["codes"] = view(L.codes, dp * (d * bits // 32), torch.int32).view(dp, -1)
+        out["scales"] = view(L.scales, dp * (d // group), torch.int16).view(dp, -1)
+        out["zeros"] = view(L.zeros, dp * (d // group), torch.int16).view(dp, -1)
+    return out

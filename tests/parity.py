@@ -1,0 +1,39 @@
+"""Helpers shared by the GPU parity tests: move seeded inputs to the device
+and compare the CUDA path with the oracle."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from test_weight_quantization_ttq_b200 import synth
+
+# Y tolerance of the layer: max |dY| <= 1e-2 * rms(Y_oracle) (bf16 operands,
+# fp32 accumulation).  D tolerance: 1e-5 relative.
+Y_TOL = 1e-2
+D_RTOL = 1e-5
+
+
+def to_dev(a: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+    t = t.to(torch.bfloat16) if dtype == "bf16" else t
+    return t.cuda()
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def u32(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint32)
+
+
+def y_error(y_gpu: np.ndarray, y_ref: np.ndarray) -> float:
+    """max |dY| / rms(Y_ref)."""
+    rms = float(np.sqrt(np.mean(y_ref.astype(np.float64) ** 2)))
+    if rms == 0.0:
+        return float(np.abs(y_gpu).max()) if y_gpu.size else 0.0
+    return float(np.abs(y_gpu.astype(np.float64) - y_ref).max()) / rms
+
+
+def inputs(spec: synth.LinearSpec, need_w: bool = True) -> dict:
+    return synth.generate(spec, need_w=need_w)

@@ -1,0 +1,90 @@
+"""The C ABI library on the CPU: it loads, exports every entry point that
+include/ttq.h declares, and its host-side logic (workspace layout, argument
+checks that reject before any device work) behaves as documented.  No
+compute call is made here."""
+import os
+import re
+
+import pytest
+
+from test_weight_quantization_ttq_b200 import build as ttq_build
+from test_weight_quantization_ttq_b200 import ttq
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ttq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    ttq_build.build()
+    return ttq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 9, names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(ttq.SIGNATURES), "binding and header disagree"
+
+
+def test_version_and_status_strings(L):
+    assert ttq.lib().ttq_version().decode().count(".") == 2
+    for st in range(7):
+        assert ttq.status_string(st)
+    assert ttq.status_string(99) == "unknown status"
+
+
+def test_workspace_layout_is_consistent(L):
+    for (d, dp, T, r, bits, g, dt) in [(4096, 4096, 2048, 0, 4, 128, ttq.TTQ_BF16),
+                                       (8192, 28672, 4096, 64, 2, 64, ttq.TTQ_BF16),
+                                       (256, 256, 64, 0, 4, 64, ttq.TTQ_F32),
+                                       (96, 200, 0, 8, 3, 32, ttq.TTQ_F32)]:
+        n = ttq.ttq_workspace_size(d, dp, T, r, bits, g, dt)
+        lay = ttq.ttq_workspace_get_layout(d, dp, T, r, bits, g, dt)
+        assert n == lay.total > 0
+        offs = [lay.status, lay.D, lay.D_rsqrt, lay.partial, lay.codes, lay.scales, lay.zeros]
+        assert all(o % 256 == 0 for o in offs)
+        assert offs == sorted(offs) and len(set(offs)) == len(offs)
+        assert lay.codes + dp * d * bits // 8 <= lay.scales
+        assert lay.scales + dp * (d // g) * 2 <= lay.zeros
+        assert lay.partial + 4 * lay.splits * d <= lay.codes
+        if r:
+            assert lay.ax_ld == r and lay.ax >= lay.zeros + dp * (d // g) * 2
+        if dt == ttq.TTQ_F32:
+            assert lay.xb > 0
+
+
+@pytest.mark.parametrize("args", [
+    (4096, 4096, 2048, 0, 5, 128),   # bits not built
+    (4096, 4096, 2048, 0, 4, 96),    # group not built
+    (4100, 4096, 2048, 0, 4, 128),   # d % group
+    (4096, 4096, 2048, 4, 4, 128),   # rank not a multiple of 8
+    (4096, -1, 2048, 0, 4, 128),
+])
+def test_workspace_size_rejects_bad_shapes(L, args):
+    assert ttq.ttq_workspace_size(*args, ttq.TTQ_BF16) == 0
+
+
+def test_rejections_before_device_work(L):
+    # unsupported bit width / group: refused before any CUDA call
+    assert L.ttq_quantize_weight(None, 1, 4, 64, None, 5, 64, None, None, None, None, 0, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert L.ttq_quantize_weight(None, 1, 4, 64, None, 4, 48, None, None, None, None, 0, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert L.ttq_quantize_weight(None, 1, 4, 64, None, 0, 64, None, None, None, None, 0, None) == ttq.TTQ_ERR_INVALID_ARG
+    # p < 1, lambda < 0, NaN alpha
+    for p, lam, a in [(0.5, 0.0, 0.5), (2.0, -1.0, 0.5), (2.0, 0.0, float("nan"))]:
+        st = L.ttq_act_norm(16, 1, 64, 4, p, lam, a, None, None, 256, 1 << 20, None)
+        assert st == ttq.TTQ_ERR_INVALID_ARG
+    # workspace too small / misaligned
+    assert L.ttq_act_norm(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
+    assert L.ttq_act_norm(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 128, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
+    # forward with a null weight
+    st = L.ttq_linear_forward(16, None, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 16, 256, 1 << 30, None)
+    assert st == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_workspace_init(None, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_get_status(None, None) == ttq.TTQ_ERR_INVALID_ARG

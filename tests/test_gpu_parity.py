@@ -1,0 +1,249 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Sizes: small and ragged shapes that span several tiles with a tail, and the
+five workloads at full size (sampled output rows for Y; D and the codes,
+scales and zeros always in full).
+"""
+import numpy as np
+import pytest
+import torch
+
+import parity as P
+import ttq_oracle
+from test_weight_quantization_ttq_b200 import synth
+from test_weight_quantization_ttq_b200 import ttq
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def O():
+    return ttq_oracle.get()
+
+
+def _small(name, d, dp, T, bits, group, dtype="bf16", r=0, p=2.0, lam=1e-3, alpha=0.5, n_out=3, seed=0):
+    return synth.LinearSpec(name, d=d, dp=dp, T=T, bits=bits, group=group, dtype=dtype, r=r, p=p,
+                            lam=lam, alpha=alpha, n_outliers=n_out, outlier_lo=20.0, outlier_hi=80.0,
+                            seed=seed)
+
+
+ACT_CASES = [
+    synth.C1,
+    synth.C2,
+    synth.C3_DOWN,
+    synth.C4.with_(T=1),
+    synth.C4.with_(T=16),
+    synth.C5.with_(T=4096, p=1.0, alpha=0.25),
+    synth.C5.with_(T=128, p=2.0, alpha=0.5),
+    _small("p3_ragged", d=264, dp=0, T=45, bits=4, group=8 * 1, p=3.0),
+    _small("one_token", d=64, dp=0, T=1, bits=4, group=32),
+    _small("f32_many_tokens", d=512, dp=0, T=3000, bits=4, group=32, dtype="f32"),
+]
+
+
+@pytest.mark.parametrize("spec", ACT_CASES, ids=lambda s: f"{s.name}-T{s.T}")
+def test_act_norm_matches_oracle(O, spec):
+    x = P.inputs(spec, need_w=False)["X"]
+    D_ref, Dr_ref, st = O.act_norm(x.astype(np.float64), spec.p, spec.lam, spec.alpha)
+    assert st == 0
+    X = P.to_dev(x, spec.dtype)
+    D, Dr = ttq.ttq_act_norm(X, spec.p, spec.lam, spec.alpha)
+    torch.cuda.synchronize()
+    D, Dr = D.cpu().numpy().astype(np.float64), Dr.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(D - D_ref) / D_ref) <= P.D_RTOL
+    assert np.max(np.abs(Dr - Dr_ref) / Dr_ref) <= P.D_RTOL
+
+
+def test_act_norm_empty_tokens(O):
+    d = 96
+    X = torch.empty((0, d), dtype=torch.bfloat16, device="cuda")
+    D, Dr = ttq.ttq_act_norm(X, 2.0, 0.25, 0.5)
+    torch.cuda.synchronize()
+    assert np.allclose(D.cpu().numpy(), 0.25 ** 0.5, rtol=1e-7)
+    assert np.allclose(Dr.cpu().numpy(), 0.25 ** -0.25, rtol=1e-7)
+
+
+QUANT_CASES = [
+    (synth.C1, None),
+    (synth.C2, None),
+    (synth.C3_GATE, None),
+    (synth.C3_DOWN, None),
+    (synth.C4, None),
+    (synth.C5, None),
+]
+for _bits in (2, 3, 4):
+    for _g in (32, 64, 128, 256):
+        QUANT_CASES.append((_small(f"b{_bits}g{_g}", d=512, dp=37, T=9, bits=_bits, group=_g), None))
+QUANT_CASES.append((_small("f32_b3g32_d96", d=96, dp=5, T=4, bits=3, group=32, dtype="f32"), None))
+QUANT_CASES.append((_small("identity_D", d=256, dp=64, T=4, bits=4, group=64), "identity"))
+
+
+@pytest.mark.parametrize("spec,mode", QUANT_CASES, ids=lambda v: getattr(v, "name", str(v)))
+def test_quantize_bit_exact(O, spec, mode):
+    data = P.inputs(spec)
+    W = data["W"]
+    if mode == "identity":
+        D32 = None
+    else:
+        D_ref, _, _ = O.act_norm(data["X"].astype(np.float64), spec.p, spec.lam, spec.alpha)
+        D32 = D_ref.astype(np.float32)  # both sides get this same D
+    codes_ref, sc_ref, ze_ref, st = O.quantize(W, D32, spec.bits, spec.group)
+    assert st == 0
+    Dd = None if D32 is None else torch.from_numpy(D32).cuda()
+    codes, sc, ze = ttq.ttq_quantize_weight(P.to_dev(W, spec.dtype), Dd, spec.bits, spec.group)
+    torch.cuda.synchronize()
+    assert np.array_equal(P.u32(codes), codes_ref)
+    assert np.array_equal(P.u16(sc), sc_ref)
+    assert np.array_equal(P.u16(ze), ze_ref)
+
+
+GEMM_CASES = [
+    # d, dp, T, bits, group, r, dtype
+    (64, 128, 1, 4, 32, 0, "bf16"),
+    (96, 200, 7, 3, 32, 0, "bf16"),
+    (320, 256, 16, 2, 64, 0, "bf16"),
+    (256, 130, 17, 4, 64, 0, "bf16"),
+    (512, 384, 100, 4, 128, 0, "bf16"),
+    (512, 256, 256, 3, 128, 0, "bf16"),
+    (768, 300, 300, 2, 64, 0, "bf16"),
+    (1024, 256, 600, 4, 256, 0, "bf16"),
+    (256, 256, 64, 4, 64, 0, "f32"),
+    (512, 200, 40, 3, 128, 32, "bf16"),
+    (512, 256, 300, 2, 64, 8, "bf16"),
+    (640, 128, 33, 4, 128, 72, "bf16"),
+    (256, 128, 20, 4, 64, 16, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", GEMM_CASES, ids=lambda c: "d{}_dp{}_T{}_b{}_g{}_r{}_{}".format(*c))
+def test_dequant_gemm_matches_oracle(O, case):
+    d, dp, T, bits, group, r, dtype = case
+    spec = _small("gemm", d=d, dp=dp, T=T, bits=bits, group=group, dtype=dtype, r=r)
+    data = P.inputs(spec)
+    X = data["X"].astype(np.float64)
+    D_ref, Dr_ref, _ = O.act_norm(X, spec.p, spec.lam, spec.alpha)
+    codes, sc, ze, _ = O.quantize(data["W"], D_ref.astype(np.float32), bits, group)
+    Dr32 = Dr_ref.astype(np.float32)
+    What = O.dequant_rows(codes, sc, ze, Dr32.astype(np.float64), d, bits, group)
+    Y_ref = O.project(What, X)
+    if r > 0:
+        Y_ref = O.lowrank_add(data["A"], data["B"], X, Y_ref)
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    A = P.to_dev(data["A"], dtype) if r > 0 else None
+    B = P.to_dev(data["B"], dtype) if r > 0 else None
+    Y = ttq.ttq_dequant_gemm(dev(codes.view(np.int32)), dev(sc.view(np.int16)), dev(ze.view(np.int16)),
+                             dev(Dr32), P.to_dev(data["X"], dtype), A, B, bits, group)
+    torch.cuda.synchronize()
+    err = P.y_error(Y.float().cpu().numpy(), Y_ref)
+    assert err <= P.Y_TOL, err
+
+
+FORWARD_CASES = [
+    synth.C1,
+    synth.C2,
+    synth.C3_GATE,
+    synth.C3_DOWN,
+    synth.C4.with_(T=1),
+    synth.C4.with_(T=4),
+    synth.C4.with_(T=16),
+    synth.C5.with_(T=1, p=2.0, alpha=0.5),
+    synth.C5.with_(T=128, p=1.0, alpha=0.25),
+    synth.C5.with_(T=4096, p=2.0, alpha=0.25),
+    _small("ragged_all", d=96, dp=200, T=19, bits=3, group=32),
+    _small("ragged_lowrank", d=448, dp=333, T=77, bits=2, group=64, r=24),
+]
+
+
+@pytest.mark.parametrize("spec", FORWARD_CASES, ids=lambda s: f"{s.name}-T{s.T}-p{s.p}-a{s.alpha}")
+def test_forward_matches_oracle(O, spec):
+    data = P.inputs(spec)
+    rows = synth.sample_rows(spec.dp, 96)
+    ref = O.forward(data["X"].astype(np.float64), data["W"], spec.p, spec.lam, spec.alpha, spec.bits,
+                    spec.group, A=data.get("A"), B=data.get("B"), rows=rows)
+    assert ref["status"] == 0
+    X = P.to_dev(data["X"], spec.dtype)
+    W = P.to_dev(data["W"], spec.dtype)
+    A = P.to_dev(data["A"], spec.dtype) if spec.r else None
+    B = P.to_dev(data["B"], spec.dtype) if spec.r else None
+    dt = ttq.TTQ_F32 if spec.dtype == "f32" else ttq.TTQ_BF16
+    ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
+    Y = ttq.ttq_linear_forward(X, W, A, B, spec.p, spec.lam, spec.alpha, spec.bits, spec.group, ws=ws)
+    torch.cuda.synchronize()
+    st, flags = ttq.ttq_get_status(ws)
+    assert st == ttq.TTQ_OK, flags
+    views = ttq.workspace_views(ws, spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
+    D = views["D"].cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(D - ref["D"]) / ref["D"]) <= P.D_RTOL
+    # codes: identical wherever both sides rounded D to the same binary32
+    codes = P.u32(views["codes"])
+    mism = np.count_nonzero(codes != ref["codes"])
+    assert mism <= max(2, codes.size // 100000), mism
+    assert np.count_nonzero(P.u16(views["scales"]) != ref["scales"]) <= max(2, ref["scales"].size // 100000)
+    err = P.y_error(Y.float().cpu().numpy()[:, rows], ref["Y"])
+    assert err <= P.Y_TOL, err
+
+
+def test_forward_is_deterministic():
+    spec = synth.C2.with_(T=300)
+    data = P.inputs(spec)
+    X, W = P.to_dev(data["X"], "bf16"), P.to_dev(data["W"], "bf16")
+    y1 = ttq.ttq_linear_forward(X, W, None, None, spec.p, spec.lam, spec.alpha, spec.bits, spec.group)
+    y2 = ttq.ttq_linear_forward(X, W, None, None, spec.p, spec.lam, spec.alpha, spec.bits, spec.group)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+
+
+def test_forward_empty_tokens():
+    d, dp = 128, 64
+    X = torch.empty((0, d), dtype=torch.bfloat16, device="cuda")
+    W = torch.randn((dp, d), device="cuda").to(torch.bfloat16)
+    Y = ttq.ttq_linear_forward(X, W, None, None, 2.0, 1e-3, 0.5, 4, 64)
+    torch.cuda.synchronize()
+    assert Y.shape == (0, dp)
+
+
+def test_status_flags_nonfinite():
+    d, dp, T = 128, 64, 8
+    X = torch.randn((T, d), device="cuda").to(torch.bfloat16)
+    W = torch.randn((dp, d), device="cuda").to(torch.bfloat16)
+    X[3, 5] = float("nan")
+    ws = ttq.new_workspace(d, dp, T, 0, 4, 64)
+    ttq.ttq_linear_forward(X, W, None, None, 2.0, 1e-3, 0.5, 4, 64, ws=ws)
+    torch.cuda.synchronize()
+    st, flags = ttq.ttq_get_status(ws)
+    assert st == ttq.TTQ_ERR_NONFINITE and flags & ttq.TTQ_FLAG_NONFINITE
+    # lambda = 0 and an all-zero channel: D_ii = 0
+    X2 = torch.randn((T, d), device="cuda").to(torch.bfloat16)
+    X2[:, 7] = 0
+    ttq.ttq_workspace_init(ws)
+    ttq.ttq_linear_forward(X2, W, None, None, 2.0, 0.0, 0.5, 4, 64, ws=ws)
+    torch.cuda.synchronize()
+    assert ttq.ttq_get_status(ws)[0] == ttq.TTQ_ERR_NONFINITE
+    # a group whose binary16 scale overflows
+    W2 = W.clone()
+    W2[0, 0] = 3.0e6
+    ttq.ttq_workspace_init(ws)
+    ttq.ttq_quantize_weight(W2, None, 4, 64, ws=ws)
+    torch.cuda.synchronize()
+    st, flags = ttq.ttq_get_status(ws)
+    assert st == ttq.TTQ_ERR_NONFINITE and flags & ttq.TTQ_FLAG_SCALE_OVERFLOW
+    # and a clean call after a reset reads OK
+    ttq.ttq_workspace_init(ws)
+    ttq.ttq_linear_forward(X2 + 1, W, None, None, 2.0, 1e-3, 0.5, 4, 64, ws=ws)
+    torch.cuda.synchronize()
+    assert ttq.ttq_get_status(ws)[0] == ttq.TTQ_OK
+
+
+def test_invalid_arguments_are_rejected():
+    X = torch.randn((4, 128), device="cuda").to(torch.bfloat16)
+    W = torch.randn((64, 128), device="cuda").to(torch.bfloat16)
+    with pytest.raises(ttq.TTQError) as e:
+        ttq.ttq_linear_forward(X, W, None, None, 0.5, 1e-3, 0.5, 4, 64)  # p < 1
+    assert e.value.status == ttq.TTQ_ERR_INVALID_ARG
+    with pytest.raises(ttq.TTQError) as e:
+        ttq.ttq_quantize_weight(W, None, 5, 64)
+    assert e.value.status == ttq.TTQ_ERR_UNSUPPORTED
+    ws = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ttq.TTQError) as e:
+        ttq.ttq_linear_forward(X, W, None, None, 2.0, 1e-3, 0.5, 4, 64, ws=ws)
+    assert e.value.status == ttq.TTQ_ERR_WORKSPACE
