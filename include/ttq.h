@@ -69,7 +69,8 @@ typedef enum ttq_status {
   TTQ_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or parameter is out of range */
   TTQ_ERR_UNSUPPORTED = 2, /* valid for the method but not built here (e.g. bits = 5) */
   TTQ_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
-  TTQ_ERR_NONFINITE = 4,   /* device flag: NaN/Inf input, D_ii not in (0, inf), or scale overflow */
+  TTQ_ERR_NONFINITE = 4,   /* device flag: NaN/Inf input, D_ii not in (0, inf), scale overflow,
+                              or an activation beyond the binary16 range */
   TTQ_ERR_TIMEOUT = 5,     /* device flag: an internal pipeline wait gave up (kernel returned early) */
   TTQ_ERR_WORKSPACE = 6    /* workspace smaller than ttq_workspace_size(...) */
 } ttq_status;
@@ -83,6 +84,7 @@ typedef enum ttq_dtype {
 #define TTQ_FLAG_NONFINITE 0x1u
 #define TTQ_FLAG_SCALE_OVERFLOW 0x2u
 #define TTQ_FLAG_TIMEOUT 0x4u
+#define TTQ_FLAG_X_RANGE 0x8u /* an activation beyond the binary16 range (|x| > 65504) */
 
 /* Byte offsets of the workspace regions for one problem shape (all 256-byte
  * aligned); `total` equals ttq_workspace_size(...).  After
@@ -94,13 +96,14 @@ typedef struct ttq_workspace_layout {
   size_t status;  /* uint32 status word, then internal counters */
   size_t D;       /* float32 [d]   D_ii                          */
   size_t D_rsqrt; /* float32 [d]   D_ii^(-1/2)                   */
-  size_t partial; /* float32 [splits][d] partial sums of |x|^p   */
+  size_t partial; /* float64 [splits][d] partial sums of |x|^p   */
   size_t codes;   /* uint32 [d'][d*bits/32]                      */
   size_t scales;  /* uint16 [d'][d/group]                        */
   size_t zeros;   /* uint16 [d'][d/group]                        */
   size_t ax;      /* bf16 [T][ax_ld]  A X                        */
-  size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32 only) */
-  size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32 only) */
+  size_t xh;      /* binary16 [T][d] copy of X for the product    */
+  size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32, r > 0) */
+  size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32, r > 0) */
   size_t total;
   int64_t splits; /* number of token splits of the statistic pass */
   int64_t ax_ld;  /* row stride (elements) of A X                 */
@@ -125,8 +128,9 @@ ttq_status ttq_workspace_init(void* ws, size_t ws_bytes, void* stream);
  *   D[i] = (||X[:, i]||_p + lambda)^alpha,  D_rsqrt[i] = D[i]^(-1/2).
  * X [T][d] (dtype), d % 8 == 0, T >= 0, p >= 1, lambda >= 0, alpha >= 0.
  * The L_p norm is taken over the T tokens of this call (no 1/T factor).
- * The sum is split over tokens and merged in a fixed order, so the result
- * is deterministic.  D or D_rsqrt may be NULL (then they are still written
+ * |x|^p is summed in fp64, split over tokens and merged in a fixed order,
+ * so the result is deterministic; n, D and D^{-1/2} are formed in fp64 and
+ * rounded once to binary32.  D or D_rsqrt may be NULL (then they are still written
  * to the workspace).  Flags NONFINITE if any D[i] is not finite and > 0. */
 ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
                         float p, float lambda, float alpha, float* D,
@@ -146,28 +150,34 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
 
 /* Steps (2)-(3) from already quantised weights: Y = W_hat X (+ B (A X)),
  * with W_hat[j][i] = scales[j][k] (codes[j][i] - zeros[j][k]) D_rsqrt[i]
- * formed in shared memory and multiplied on the tensor cores (bf16 operands,
- * fp32 accumulation; float32 X is rounded to bf16 for the product).
- * D_rsqrt == NULL means D = I.  A [r][d] and B [dp][r] may be NULL when
- * r == 0; r % 8 == 0.  Y [T][dp] (dtype). */
+ * formed in shared memory and multiplied on the tensor cores: binary16
+ * W_hat and X (X converted exactly from bf16; |x| must not exceed 65504,
+ * else flag X_RANGE), fp32 accumulation; the low-rank term B (A X) uses bf16
+ * operands with fp32 accumulation, A X held in bf16.
+ * D_rsqrt == NULL means D = I.  A [r][d] and B [dp][r] (dtype) may be NULL
+ * when r == 0; r % 8 == 0.  Y [T][dp] is written in y_dtype: TTQ_F32 keeps
+ * the fp32 accumulator as is, TTQ_BF16 rounds it to nearest-even once. */
 ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
                             const uint16_t* zeros, const float* D_rsqrt,
                             const void* X, const void* A, const void* B,
                             ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,
-                            int64_t r, int bits, int group, void* Y, void* ws,
-                            size_t ws_bytes, void* stream);
+                            int64_t r, int bits, int group, void* Y,
+                            ttq_dtype y_dtype, void* ws, size_t ws_bytes,
+                            void* stream);
 
 /* The whole TTQ linear layer, (1) -> (2) -> (3), on `stream`:
  *   Y = Q[W D^{1/2}] D^{-1/2} X + B (A X).
- * X [T][d], W [dp][d], A [r][d], B [dp][r], Y [T][dp], all in `dtype`.
- * A and B may be NULL when r == 0.  W is taken to be the residual that the
- * static low-rank pair complements (gist.science/zh, section 2.2).
- * The workspace keeps D, D_rsqrt, codes, scales and zeros of this call. */
+ * X [T][d], W [dp][d], A [r][d], B [dp][r] in `dtype`; Y [T][dp] in
+ * `y_dtype` (TTQ_F32: the fp32 accumulator; TTQ_BF16: rounded once to
+ * nearest-even).  A and B may be NULL when r == 0.  W is taken to be the
+ * residual that the static low-rank pair complements (gist.science/zh,
+ * section 2.2).  The workspace keeps D, D_rsqrt, codes, scales and zeros of
+ * this call. */
 ttq_status ttq_linear_forward(const void* X, const void* W, const void* A,
                               const void* B, ttq_dtype dtype, int64_t d, int64_t dp,
                               int64_t T, int64_t r, float p, float lambda, float alpha,
-                              int bits, int group, void* Y, void* ws, size_t ws_bytes,
-                              void* stream);
+                              int bits, int group, void* Y, ttq_dtype y_dtype, void* ws,
+                              size_t ws_bytes, void* stream);
 
 /* Reads the workspace status word (a blocking device-to-host copy; the caller
  * synchronises its stream first).  *flags receives the raw TTQ_FLAG_* bits

@@ -6,11 +6,14 @@
 // Layout of the work: a block owns 256 consecutive channels and one split of
 // the tokens.  Each lane loads 8 consecutive channels of a row (one 16-byte
 // load for bf16), each of the 8 warps walks every 8th row of the split, and
-// the warps' sums are merged in shared memory in a fixed order.  The split's
+// the warps' sums are merged in shared memory in a fixed order; sums are kept
+// in fp64 (the pass is bound by memory, not by the fp64 pipe).  The split's
 // partial sums go to global memory; the last block to finish a column block
 // (an atomic ticket) merges all splits in fp64, in split order, so the
-// result does not depend on scheduling.  The pass is HBM-bound: it reads X
-// once (2dT bytes for bf16) and writes 8d bytes.
+// result does not depend on scheduling.  On the way it writes the binary16
+// copy of X that the tensor-core product consumes (and, for float32 X with a
+// low-rank term, a bf16 copy).  The pass is HBM-bound: it reads X once (2dT
+// bytes for bf16) and writes 2dT bytes of binary16 X plus 8d bytes.
 #include "ttq_device.cuh"
 #include "ttq_kernels.h"
 
@@ -20,12 +23,14 @@ namespace {
 constexpr int kChannelsPerBlock = 256;
 constexpr int kThreads = 256;
 
+// |x|^p in fp64: exact for p = 1 and for p = 2 with 16-bit inputs, so the
+// merged sums (and hence D rounded to binary32) match an fp64 reference.
 template <int PK>  // 1: p = 1, 2: p = 2, 0: any p >= 1
-__device__ __forceinline__ float abs_pow(float x, float p) {
-  const float a = fabsf(x);
+__device__ __forceinline__ double abs_pow(float x, double p) {
+  const double a = fabs(static_cast<double>(x));
   if (PK == 1) return a;
   if (PK == 2) return a * a;
-  return powf(a, p);
+  return pow(a, p);
 }
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
@@ -45,6 +50,19 @@ __device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
+__device__ __forceinline__ void store8_f16(__half* dst, const float (&v)[8]) {
+  uint4 raw;
+  __half2 h0 = __floats2half2_rn(v[0], v[1]);
+  __half2 h1 = __floats2half2_rn(v[2], v[3]);
+  __half2 h2 = __floats2half2_rn(v[4], v[5]);
+  __half2 h3 = __floats2half2_rn(v[6], v[7]);
+  raw.x = *reinterpret_cast<uint32_t*>(&h0);
+  raw.y = *reinterpret_cast<uint32_t*>(&h1);
+  raw.z = *reinterpret_cast<uint32_t*>(&h2);
+  raw.w = *reinterpret_cast<uint32_t*>(&h3);
+  *reinterpret_cast<uint4*>(dst) = raw;
+}
+
 __device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float (&v)[8]) {
   uint4 raw;
   __nv_bfloat162 h0 = __floats2bfloat162_rn(v[0], v[1]);
@@ -60,11 +78,11 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float (&v)
 
 template <typename XT, int PK>
 __global__ void __launch_bounds__(kThreads) act_norm_kernel(
-    const XT* __restrict__ X, int64_t d, int64_t T, float p, double lambda, double alpha,
-    int64_t splits, int64_t rows_per_split, float* __restrict__ partial,
+    const XT* __restrict__ X, int64_t d, int64_t T, double p, double lambda, double alpha,
+    int64_t splits, int64_t rows_per_split, double* __restrict__ partial,
     uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
-    __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
-  __shared__ float red[8][kChannelsPerBlock + 8];
+    __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
+  __shared__ double red[8][kChannelsPerBlock + 2];
   __shared__ int is_last;
 
   const int warp = threadIdx.x >> 5;
@@ -73,12 +91,13 @@ __global__ void __launch_bounds__(kThreads) act_norm_kernel(
   const int64_t sp = blockIdx.y;
   const int64_t c0 = cb * kChannelsPerBlock + lane * 8;
 
-  float acc[8];
+  double acc[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 
   const int64_t t_begin = sp * rows_per_split;
   const int64_t t_end = min(T, t_begin + rows_per_split);
+  float amax = 0.f;
   if (c0 < d) {
     int64_t t = t_begin + warp;
     // two rows in flight per warp
@@ -86,28 +105,42 @@ __global__ void __launch_bounds__(kThreads) act_norm_kernel(
       float v0[8], v1[8];
       load8(X + t * d + c0, v0);
       load8(X + (t + 8) * d + c0, v1);
+      if (xh != nullptr) {
+        store8_f16(xh + t * d + c0, v0);
+        store8_f16(xh + (t + 8) * d + c0, v1);
+      }
       if (xb != nullptr) {
         store8_bf16(xb + t * d + c0, v0);
         store8_bf16(xb + (t + 8) * d + c0, v1);
       }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v0[e], p) + abs_pow<PK>(v1[e], p);
+      for (int e = 0; e < 8; ++e) {
+        acc[e] += abs_pow<PK>(v0[e], p) + abs_pow<PK>(v1[e], p);
+        amax = fmaxf(amax, fmaxf(fabsf(v0[e]), fabsf(v1[e])));
+      }
     }
     for (; t < t_end; t += 8) {
       float v0[8];
       load8(X + t * d + c0, v0);
+      if (xh != nullptr) store8_f16(xh + t * d + c0, v0);
       if (xb != nullptr) store8_bf16(xb + t * d + c0, v0);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v0[e], p);
+      for (int e = 0; e < 8; ++e) {
+        acc[e] += abs_pow<PK>(v0[e], p);
+        amax = fmaxf(amax, fabsf(v0[e]));
+      }
     }
   }
+  // the binary16 copy of X holds |x| <= 65504 only (NaN is caught by D)
+  if (xh != nullptr && __any_sync(0xffffffffu, amax > 65504.f) && lane == 0)
+    set_flag(status, TTQ_FLAG_X_RANGE);
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
   __syncthreads();
 
   const int ci = threadIdx.x;
   const int64_t c = cb * kChannelsPerBlock + ci;
-  float sum = 0.f;
+  double sum = 0.0;
 #pragma unroll
   for (int w = 0; w < 8; ++w) sum += red[w][ci];
   if (c < d) partial[sp * d + c] = sum;
@@ -125,14 +158,14 @@ __global__ void __launch_bounds__(kThreads) act_norm_kernel(
 
   if (c < d) {
     double tot = 0.0;
-    for (int64_t s = 0; s < splits; ++s) tot += static_cast<double>(__ldcg(partial + s * d + c));
+    for (int64_t s = 0; s < splits; ++s) tot += __ldcg(partial + s * d + c);
     double n;
     if (PK == 1) {
       n = tot;
     } else if (PK == 2) {
       n = sqrt(tot);
     } else {
-      n = pow(tot, 1.0 / static_cast<double>(p));
+      n = pow(tot, 1.0 / p);
     }
     const double dv = pow(n + lambda, alpha);
     const double drv = 1.0 / sqrt(dv);
@@ -148,29 +181,31 @@ __global__ void __launch_bounds__(kThreads) act_norm_kernel(
 
 template <typename XT, int PK>
 cudaError_t launch_typed(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
-                         int64_t splits, int64_t rows_per_split, float* partial,
-                         uint32_t* counters, float* D, float* Dr, void* xb, uint32_t* status,
-                         cudaStream_t stream) {
+                         int64_t splits, int64_t rows_per_split, double* partial,
+                         uint32_t* counters, float* D, float* Dr, void* xh, void* xb,
+                         uint32_t* status, cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>((d + kChannelsPerBlock - 1) / kChannelsPerBlock),
                   static_cast<unsigned>(splits));
   act_norm_kernel<XT, PK><<<grid, kThreads, 0, stream>>>(
-      X, d, T, p, static_cast<double>(lambda), static_cast<double>(alpha), splits,
-      rows_per_split, partial, counters, D, Dr, static_cast<__nv_bfloat16*>(xb), status);
+      X, d, T, static_cast<double>(p), static_cast<double>(lambda), static_cast<double>(alpha), splits,
+      rows_per_split, partial, counters, D, Dr, static_cast<__half*>(xh),
+      static_cast<__nv_bfloat16*>(xb), status);
   return cudaGetLastError();
 }
 
 template <typename XT>
 cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
-                     int64_t splits, int64_t rows_per_split, float* partial, uint32_t* counters,
-                     float* D, float* Dr, void* xb, uint32_t* status, cudaStream_t stream) {
+                     int64_t splits, int64_t rows_per_split, double* partial, uint32_t* counters,
+                     float* D, float* Dr, void* xh, void* xb, uint32_t* status,
+                     cudaStream_t stream) {
   if (p == 1.0f)
     return launch_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                               counters, D, Dr, xb, status, stream);
+                               counters, D, Dr, xh, xb, status, stream);
   if (p == 2.0f)
     return launch_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                               counters, D, Dr, xb, status, stream);
+                               counters, D, Dr, xh, xb, status, stream);
   return launch_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                             counters, D, Dr, xb, status, stream);
+                             counters, D, Dr, xh, xb, status, stream);
 }
 
 }  // namespace
@@ -193,13 +228,13 @@ void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* 
 
 cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                             float lambda, float alpha, int64_t splits, int64_t rows_per_split,
-                            float* partial, uint32_t* counters, float* D, float* Dr, void* xb,
-                            uint32_t* status, cudaStream_t stream) {
+                            double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
+                            void* xb, uint32_t* status, cudaStream_t stream) {
   if (x_f32)
     return launch_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits, rows_per_split,
-                    partial, counters, D, Dr, xb, status, stream);
+                    partial, counters, D, Dr, xh, xb, status, stream);
   return launch_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
-                  rows_per_split, partial, counters, D, Dr, nullptr, status, stream);
+                  rows_per_split, partial, counters, D, Dr, xh, nullptr, status, stream);
 }
 
 }  // namespace ttq

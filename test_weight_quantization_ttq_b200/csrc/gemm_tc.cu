@@ -5,7 +5,8 @@
 // static low-rank pair, 2.3 for the projection).
 //
 // One CTA computes a 128 (rows of W) x BN (tokens) tile of Y^T in tensor
-// memory with tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), cta_group::1:
+// memory with tcgen05.mma kind::f16 (binary16 x binary16 -> fp32 for the
+// quantised weight; bf16 x bf16 for the low-rank tail), cta_group::1:
 //   warp 0      TMA producer: X tiles (BN x 64, 128-byte swizzle) into the
 //               B slot of each pipeline stage; in the plain mode (no codes)
 //               and for the low-rank tail also the A slot.
@@ -16,9 +17,11 @@
 //               then (after the last stage) read the accumulator out of
 //               tensor memory and store Y.
 // W_hat is formed in fp32 -- (q - z) * s is exact, one rounding for the
-// D^(-1/2) factor -- and rounded once to bf16, so the only operand rounding
-// on the weight side is that final one.  The low-rank term rides along as
-// extra K blocks: A slot = B[j][k] (TMA), B slot = AX[t][k] (TMA).
+// D^(-1/2) factor -- and rounded once to binary16 (11 significant bits; a
+// bf16 W_hat would carry 8x the rounding error on the few large
+// outlier-channel terms).  X arrives as binary16, exact for bf16 inputs of
+// magnitude <= 65504.  The low-rank term rides along as extra K blocks: A
+// slot = B[j][k] (TMA), B slot = AX[t][k] (TMA), both bf16.
 //
 // Every barrier wait is bounded (1 s); a wait that gives up sets
 // TTQ_FLAG_TIMEOUT, tells the other roles to stop, and the CTA still frees
@@ -52,8 +55,8 @@ struct GemmDev {
   uint32_t* status;
 };
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
@@ -64,7 +67,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 }
 
 // Writes rows rb, rb+32, rb+64, rb+96 of the 128 x 64 A tile, channels
-// [8c, 8c+8) of K block kb, as bf16 W_hat in the 128-byte-swizzled layout:
+// [8c, 8c+8) of K block kb, as binary16 W_hat in the 128-byte-swizzled layout:
 // row r, 16-byte chunk c lives at (r/8)*1024 + (r%8)*128 + ((c ^ r%8) * 16).
 template <int BITS>
 __device__ __forceinline__ void dequant_rows(uint32_t a_slot, const GemmDev& g, int64_t m0,
@@ -105,10 +108,10 @@ __device__ __forceinline__ void dequant_rows(uint32_t a_slot, const GemmDev& g, 
         const int q = static_cast<int>((v >> (BITS * e)) & QMAX);
         w[e] = __fmul_rn(static_cast<float>(q - z) * s, dr[e]);
       }
-      out.x = pack_bf16x2(w[0], w[1]);
-      out.y = pack_bf16x2(w[2], w[3]);
-      out.z = pack_bf16x2(w[4], w[5]);
-      out.w = pack_bf16x2(w[6], w[7]);
+      out.x = pack_f16x2(w[0], w[1]);
+      out.y = pack_f16x2(w[2], w[3]);
+      out.z = pack_f16x2(w[4], w[5]);
+      out.w = pack_f16x2(w[6], w[7]);
     }
     const uint32_t addr = a_slot + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
     st_shared_v4(addr, out);
@@ -197,7 +200,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(kBM, static_cast<uint32_t>(BN));
+      // main K blocks: binary16 W_hat x binary16 X (bf16 x bf16 in the plain
+      // mode); low-rank tail: bf16 B x bf16 A X
+      const uint32_t idesc_main =
+          idesc_f16kind(BITS == 0 ? kFmtBF16 : kFmtF16, kBM, static_cast<uint32_t>(BN));
+      const uint32_t idesc_tail = idesc_f16kind(kFmtBF16, kBM, static_cast<uint32_t>(BN));
       for (int kb = 0; kb < kb_total; ++kb) {
         const int s = kb % stages;
         const uint32_t ph = static_cast<uint32_t>(kb / stages) & 1u;
@@ -210,9 +217,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t a_addr = smem_addr(smem + s * stage_bytes);
         const uint64_t adesc = smem_desc_sw128(a_addr);
         const uint64_t bdesc = smem_desc_sw128(a_addr + kATileBytes);
+        const uint32_t idesc = kb < kb_main ? idesc_main : idesc_tail;
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k)
-          mma_bf16_ss(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+          mma_f16kind_ss(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
         mma_commit(&empty[s]);
       }
       mma_commit(accum);

@@ -187,7 +187,54 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __r
   }
 }
 
+template <typename T>
+__global__ void to_f16_kernel(const T* __restrict__ src, __half* __restrict__ dst, int64_t n8,
+                              uint32_t* __restrict__ status) {
+  bool out_of_range = false;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n8;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float v[8];
+    if constexpr (sizeof(T) == 4) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(src) + 2 * i);
+      const float4 b = __ldg(reinterpret_cast<const float4*>(src) + 2 * i + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src) + i);
+      const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] = __uint_as_float(w[k] << 16);
+        v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      }
+    }
+    __half2 h[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      h[k] = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+      out_of_range |= !(fabsf(v[2 * k]) <= 65504.f) || !(fabsf(v[2 * k + 1]) <= 65504.f);
+    }
+    reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<uint4*>(h);
+  }
+  if (__any_sync(0xffffffffu, out_of_range) && (threadIdx.x & 31) == 0)
+    set_flag(status, TTQ_FLAG_X_RANGE);
+}
+
 }  // namespace
+
+cudaError_t launch_to_f16(const void* src, bool src_f32, void* dst, int64_t n, uint32_t* status,
+                          cudaStream_t stream) {
+  const int64_t n8 = n / 8;
+  if (n8 == 0) return cudaSuccess;
+  int64_t blocks = (n8 + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  if (src_f32)
+    to_f16_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const float*>(src), static_cast<__half*>(dst), n8, status);
+  else
+    to_f16_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(src), static_cast<__half*>(dst), n8, status);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,

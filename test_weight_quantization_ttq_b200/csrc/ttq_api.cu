@@ -56,7 +56,7 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
   l.D_rsqrt = off;
   off = align_up(off + 4 * static_cast<size_t>(d));
   l.partial = off;
-  off = align_up(off + 4 * static_cast<size_t>(splits) * static_cast<size_t>(d));
+  off = align_up(off + 8 * static_cast<size_t>(splits) * static_cast<size_t>(d));
   if (has_q) {
     l.codes = off;
     off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d * bits / 32) * 4);
@@ -71,13 +71,15 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
     l.ax = off;
     off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(r) * 2);
   }
-  if (dtype == TTQ_F32) {
+  if (has_q) {
+    l.xh = off;
+    off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(d) * 2);
+  }
+  if (dtype == TTQ_F32 && r > 0) {
     l.xb = off;
     off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(d) * 2);
-    if (r > 0) {
-      l.ab = off;
-      off = align_up(off + (static_cast<size_t>(r) * d + static_cast<size_t>(dp) * r) * 2);
-    }
+    l.ab = off;
+    off = align_up(off + (static_cast<size_t>(r) * d + static_cast<size_t>(dp) * r) * 2);
   }
   l.total = off;
   l.splits = splits;
@@ -105,18 +107,19 @@ EncodeFn get_encode() {
   return fn;
 }
 
-// bf16 matrix [outer][inner] with row stride ld (elements), loaded as
-// box_outer rows x 64 columns into the 128-byte-swizzled layout; reads
-// outside the matrix return zeros.
-bool encode_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
-                 int box_outer) {
+// 16-bit matrix [outer][inner] (bf16 or binary16) with row stride ld
+// (elements), loaded as box_outer rows x 64 columns into the
+// 128-byte-swizzled layout; reads outside the matrix return zeros.
+bool encode_16bit(CUtensorMap* m, const void* base, bool f16, int64_t inner, int64_t outer,
+                  int64_t ld, int box_outer) {
   EncodeFn enc = get_encode();
   if (enc == nullptr || inner < 1 || outer < 1) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2};
   const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_outer)};
   const cuuint32_t estr[2] = {1u, 1u};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+  return enc(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -125,19 +128,21 @@ ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_E
 
 uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
 
-// Y = W_hat X (+ B (A X)) from quantised weights; X, A, B already bf16.
+// Y = W_hat X (+ B (A X)) from quantised weights.  Xh is binary16 X; Xb, Ab,
+// Bb are bf16 X, A, B (used only when r > 0).
 ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
-                    const float* Dr, const void* Xb, const void* Ab, const void* Bb, int64_t d,
-                    int64_t dp, int64_t T, int64_t r, int bits, int group, void* Y, bool y_f32,
-                    void* ws, const ttq_workspace_layout& L, cudaStream_t stream) {
+                    const float* Dr, const void* Xh, const void* Xb, const void* Ab,
+                    const void* Bb, int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
+                    int group, void* Y, bool y_f32, void* ws, const ttq_workspace_layout& L,
+                    cudaStream_t stream) {
   if (T == 0 || dp == 0) return TTQ_OK;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   void* ax = r > 0 ? ws_at(ws, L.ax) : nullptr;
+  const int bn = gemm_block_n(T);
   if (r > 0) {
     // A X: the plain-operand mode of the same kernel, M = r rows of A.
-    const int bn = gemm_block_n(T);
     GemmMaps m;
-    if (!encode_bf16(&m.a0, Ab, d, r, d, 128) || !encode_bf16(&m.b0, Xb, d, T, d, bn))
+    if (!encode_16bit(&m.a0, Ab, false, d, r, d, 128) || !encode_16bit(&m.b0, Xb, false, d, T, d, bn))
       return TTQ_ERR_CUDA;
     m.a1 = m.a0;
     m.b1 = m.b0;
@@ -154,12 +159,12 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, stream));
     if (st != TTQ_OK) return st;
   }
-  const int bn = gemm_block_n(T);
   GemmMaps m;
-  if (!encode_bf16(&m.b0, Xb, d, T, d, bn)) return TTQ_ERR_CUDA;
+  if (!encode_16bit(&m.b0, Xh, true, d, T, d, bn)) return TTQ_ERR_CUDA;
   m.a0 = m.b0;
   if (r > 0) {
-    if (!encode_bf16(&m.a1, Bb, r, dp, r, 128) || !encode_bf16(&m.b1, ax, r, T, L.ax_ld, bn))
+    if (!encode_16bit(&m.a1, Bb, false, r, dp, r, 128) ||
+        !encode_16bit(&m.b1, ax, false, r, T, L.ax_ld, bn))
       return TTQ_ERR_CUDA;
   } else {
     m.a1 = m.b0;
@@ -221,7 +226,7 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T, fl
   if ((X && !aligned16(X)) || (D && !aligned16(D)) || (D_rsqrt && !aligned16(D_rsqrt)) ||
       (reinterpret_cast<uintptr_t>(ws) & 255u))
     return TTQ_ERR_INVALID_ARG;
-  const size_t need = L.partial + align_up(4 * static_cast<size_t>(L.splits) * d);
+  const size_t need = L.partial + align_up(8 * static_cast<size_t>(L.splits) * d);
   if (ws_bytes < need) return TTQ_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
@@ -231,7 +236,8 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T, fl
   act_norm_plan(d, T, kPlanSMs, &splits, &rps);
   ttq_status st = cuda_status(launch_act_norm(
       X, dtype == TTQ_F32, d, T, p, lambda, alpha, splits, rps,
-      reinterpret_cast<float*>(ws_at(ws, L.partial)), status + 64, Dw, Drw, nullptr, status, s));
+      reinterpret_cast<double*>(ws_at(ws, L.partial)), status + 64, Dw, Drw, nullptr, nullptr,
+      status, s));
   if (st != TTQ_OK) return st;
   if (D) st = cuda_status(cudaMemcpyAsync(D, Dw, 4 * d, cudaMemcpyDeviceToDevice, s));
   if (st == TTQ_OK && D_rsqrt)
@@ -262,8 +268,9 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
 ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
                             const float* D_rsqrt, const void* X, const void* A, const void* B,
                             ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
-                            int bits, int group, void* Y, void* ws, size_t ws_bytes,
-                            void* stream) {
+                            int bits, int group, void* Y, ttq_dtype y_dtype, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
   if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
     return TTQ_ERR_UNSUPPORTED;
   ttq_workspace_layout L;
@@ -280,32 +287,35 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
     if (p && !aligned16(p)) return TTQ_ERR_INVALID_ARG;
   if (!work) return TTQ_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  const bool f32 = dtype == TTQ_F32;
+  void* xh = ws_at(ws, L.xh);
+  ttq_status st = cuda_status(launch_to_f16(X, f32, xh, T * d, status, s));
+  if (st != TTQ_OK) return st;
   const void* Xb = X;
   const void* Ab = A;
   const void* Bb = B;
-  if (dtype == TTQ_F32) {
+  if (f32 && r > 0) {
     void* xb = ws_at(ws, L.xb);
-    ttq_status st = cuda_status(launch_to_bf16(static_cast<const float*>(X), xb, T * d, s));
+    void* ab = ws_at(ws, L.ab);
+    void* bb = static_cast<uint8_t*>(ab) + static_cast<size_t>(r) * d * 2;
+    st = cuda_status(launch_to_bf16(static_cast<const float*>(X), xb, T * d, s));
+    if (st == TTQ_OK) st = cuda_status(launch_to_bf16(static_cast<const float*>(A), ab, r * d, s));
+    if (st == TTQ_OK) st = cuda_status(launch_to_bf16(static_cast<const float*>(B), bb, dp * r, s));
     if (st != TTQ_OK) return st;
     Xb = xb;
-    if (r > 0) {
-      void* ab = ws_at(ws, L.ab);
-      void* bb = static_cast<uint8_t*>(ab) + static_cast<size_t>(r) * d * 2;
-      st = cuda_status(launch_to_bf16(static_cast<const float*>(A), ab, r * d, s));
-      if (st == TTQ_OK) st = cuda_status(launch_to_bf16(static_cast<const float*>(B), bb, dp * r, s));
-      if (st != TTQ_OK) return st;
-      Ab = ab;
-      Bb = bb;
-    }
+    Ab = ab;
+    Bb = bb;
   }
-  return run_gemm(codes, scales, zeros, D_rsqrt, Xb, Ab, Bb, d, dp, T, r, bits, group, Y,
-                  dtype == TTQ_F32, ws, L, s);
+  return run_gemm(codes, scales, zeros, D_rsqrt, xh, Xb, Ab, Bb, d, dp, T, r, bits, group, Y,
+                  y_dtype == TTQ_F32, ws, L, s);
 }
 
 ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const void* B,
                               ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
                               float p, float lambda, float alpha, int bits, int group, void* Y,
-                              void* ws, size_t ws_bytes, void* stream) {
+                              ttq_dtype y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
   if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
     return TTQ_ERR_UNSUPPORTED;
   ttq_workspace_layout L;
@@ -328,14 +338,16 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   float* D = reinterpret_cast<float*>(ws_at(ws, L.D));
   float* Dr = reinterpret_cast<float*>(ws_at(ws, L.D_rsqrt));
   const bool f32 = dtype == TTQ_F32;
-  void* xb = f32 ? ws_at(ws, L.xb) : nullptr;
+  void* xh = dp > 0 ? ws_at(ws, L.xh) : nullptr;
+  void* xb = (f32 && r > 0) ? ws_at(ws, L.xb) : nullptr;
 
-  // (1) D and D^{-1/2} (float32 X is also narrowed to bf16 on the way)
+  // (1) D and D^{-1/2}; X is also written as binary16 for the product (and
+  // as bf16 for the low-rank product when it arrives as float32)
   int64_t splits, rps;
   act_norm_plan(d, T, kPlanSMs, &splits, &rps);
   ttq_status st = cuda_status(launch_act_norm(
       X, f32, d, T, p, lambda, alpha, splits, rps,
-      reinterpret_cast<float*>(ws_at(ws, L.partial)), status + 64, D, Dr, xb, status, s));
+      reinterpret_cast<double*>(ws_at(ws, L.partial)), status + 64, D, Dr, xh, xb, status, s));
   if (st != TTQ_OK || dp == 0) return st;
 
   // (2) codes, scales, zeros of Q[W D^{1/2}]
@@ -358,8 +370,8 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
     Ab = ab;
     Bb = bb;
   }
-  return run_gemm(codes, scales, zeros, Dr, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
-                  f32, ws, L, s);
+  return run_gemm(codes, scales, zeros, Dr, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
+                  y_dtype == TTQ_F32, ws, L, s);
 }
 
 ttq_status ttq_get_status(const void* ws, uint32_t* flags) {

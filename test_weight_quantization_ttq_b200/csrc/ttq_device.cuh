@@ -126,8 +126,9 @@ __device__ __forceinline__ void tc_fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 x bf16 -> fp32, one thread issues.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit operands (types in idesc) -> fp32;
+// one thread issues.
+__device__ __forceinline__ void mma_f16kind_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -178,11 +179,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
   return desc;
 }
 
-// Instruction descriptor of kind::f16 with bf16 A and B (both K-major) and an
-// fp32 accumulator: D format (bits 4-5) = 1 (f32), A format (7-9) = 1 (bf16),
-// B format (10-12) = 1 (bf16), N >> 3 (17-22), M >> 4 (24-28).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+// Instruction descriptor of kind::f16 with A and B of one 16-bit type (both
+// K-major) and an fp32 accumulator: D format (bits 4-5) = 1 (f32), A format
+// (7-9) and B format (10-12) = 0 for binary16 or 1 for bf16, N >> 3 (17-22),
+// M >> 4 (24-28).
+constexpr uint32_t kFmtF16 = 0;
+constexpr uint32_t kFmtBF16 = 1;
+__host__ __device__ constexpr uint32_t idesc_f16kind(uint32_t fmt, uint32_t M, uint32_t N) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 }  // namespace ttq

@@ -12,12 +12,14 @@ namespace ttq {
 // Number of token splits of the statistic pass and the rows each covers.
 void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split);
 
-// Step (1): D, D^{-1/2} from X [T][d].  `partial` holds splits x d floats,
+// Step (1): D, D^{-1/2} from X [T][d].  `partial` holds splits x d doubles,
 // `counters` ceil(d/256) uint32 that start (and are left) at zero.  When
-// xb is non-null the float32 X is also written out as bf16 [T][d].
+// xh is non-null X is also written out as binary16 [T][d] (flag X_RANGE if
+// some |x| > 65504); when xb is non-null a float32 X is also written out as
+// bf16 [T][d].
 cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                             float lambda, float alpha, int64_t splits, int64_t rows_per_split,
-                            float* partial, uint32_t* counters, float* D, float* Dr,
+                            double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
                             void* xb, uint32_t* status, cudaStream_t stream);
 
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null).
@@ -29,6 +31,11 @@ cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, co
 // float32 -> bf16 copy of n elements (n % 8 == 0).
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
 
+// float32 or bf16 -> binary16 copy of n elements (n % 8 == 0); flags
+// X_RANGE if some |x| > 65504.
+cudaError_t launch_to_f16(const void* src, bool src_f32, void* dst, int64_t n, uint32_t* status,
+                          cudaStream_t stream);
+
 // Steps (2)-(3) on the tensor cores.
 struct GemmArgs {
   // dequantised A operand (bits != 0) ...
@@ -36,7 +43,7 @@ struct GemmArgs {
   const uint16_t* scales = nullptr;
   const uint16_t* zeros = nullptr;
   const float* Dr = nullptr;  // null: identity
-  int bits = 0;               // 0: A operand loaded by TMA from tmA0 (plain bf16)
+  int bits = 0;               // 0: A operand loaded by TMA from tmA0 (plain bf16 x bf16)
   int group = 0;
   // sizes
   int64_t K = 0;        // reduction length of the main part (d)
@@ -52,7 +59,7 @@ struct GemmArgs {
 
 struct GemmMaps {
   CUtensorMap a0;  // plain A operand [M][K] bf16 (bits == 0)
-  CUtensorMap b0;  // X [T][K] bf16
+  CUtensorMap b0;  // X [T][K]: binary16 with codes (bits != 0), bf16 in the plain mode
   CUtensorMap a1;  // low-rank B [M][r] bf16
   CUtensorMap b1;  // A X [T][r] bf16
 };

@@ -28,6 +28,7 @@ TTQ_BF16 = 1
 TTQ_FLAG_NONFINITE = 0x1
 TTQ_FLAG_SCALE_OVERFLOW = 0x2
 TTQ_FLAG_TIMEOUT = 0x4
+TTQ_FLAG_X_RANGE = 0x8
 
 # C signatures, in the order of include/ttq.h
 _P = ctypes.c_void_p
@@ -39,7 +40,7 @@ _SZ = ctypes.c_size_t
 
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("status", _SZ), ("D", _SZ), ("D_rsqrt", _SZ), ("partial", _SZ), ("codes", _SZ),
-                ("scales", _SZ), ("zeros", _SZ), ("ax", _SZ), ("xb", _SZ), ("ab", _SZ),
+                ("scales", _SZ), ("zeros", _SZ), ("ax", _SZ), ("xh", _SZ), ("xb", _SZ), ("ab", _SZ),
                 ("total", _SZ), ("splits", _I64), ("ax_ld", _I64)]
 
 
@@ -51,9 +52,9 @@ SIGNATURES = {
     "ttq_act_norm": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _SZ, _P]),
     "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
-                                _P, _P, _SZ, _P]),
+                                _P, _INT, _P, _SZ, _P]),
     "ttq_linear_forward": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT, _INT,
-                                  _P, _P, _SZ, _P]),
+                                  _P, _INT, _P, _SZ, _P]),
     "ttq_get_status": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "ttq_status_string": (ctypes.c_char_p, [_INT]),
     "ttq_version": (ctypes.c_char_p, []),
@@ -184,8 +185,10 @@ def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zer
     return codes, scales, zeros
 
 
-def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=None, Y=None, stream=None):
-    """Y [T][d'] = W_hat X (+ B (A X)) from quantised weights."""
+def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=None, Y=None,
+                     y_dtype=None, stream=None):
+    """Y [T][d'] = W_hat X (+ B (A X)) from quantised weights; Y in y_dtype
+    (default: the dtype of X, or of a given Y)."""
     T, d = X.shape
     dp = codes.shape[0]
     r = 0 if A is None else A.shape[0]
@@ -193,17 +196,19 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
     if ws is None:
         ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
     if Y is None:
-        Y = torch.empty((T, dp), dtype=X.dtype, device=X.device)
+        Y = torch.empty((T, dp), dtype=y_dtype or X.dtype, device=X.device)
     _check(lib().ttq_dequant_gemm(_dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
                                   _dev(D_rsqrt, "D_rsqrt"), _dev(X, "X"), _dev(A, "A"), _dev(B, "B"), dt,
-                                  d, dp, T, r, bits, group, _dev(Y, "Y"), _dev(ws, "ws"), ws.numel(),
-                                  _stream(stream)),
+                                  d, dp, T, r, bits, group, _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"),
+                                  ws.numel(), _stream(stream)),
            "ttq_dequant_gemm")
     return Y
 
 
-def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, stream=None):
-    """The TTQ linear layer: Y [T][d'] = Q[W D^{1/2}] D^{-1/2} X + B (A X)."""
+def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, y_dtype=None,
+                       stream=None):
+    """The TTQ linear layer: Y [T][d'] = Q[W D^{1/2}] D^{-1/2} X + B (A X);
+    Y in y_dtype (default: the dtype of X, or of a given Y)."""
     T, d = X.shape
     dp = W.shape[0]
     r = 0 if A is None else A.shape[0]
@@ -211,10 +216,10 @@ def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, 
     if ws is None:
         ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
     if Y is None:
-        Y = torch.empty((T, dp), dtype=X.dtype, device=X.device)
+        Y = torch.empty((T, dp), dtype=y_dtype or X.dtype, device=X.device)
     _check(lib().ttq_linear_forward(_dev(X, "X"), _dev(W, "W"), _dev(A, "A"), _dev(B, "B"), dt, d, dp, T,
-                                    r, p, lam, alpha, bits, group, _dev(Y, "Y"), _dev(ws, "ws"), ws.numel(),
-                                    _stream(stream)),
+                                    r, p, lam, alpha, bits, group, _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"),
+                                    ws.numel(), _stream(stream)),
            "ttq_linear_forward")
     return Y
 

@@ -53,11 +53,13 @@ def test_workspace_layout_is_consistent(L):
         assert offs == sorted(offs) and len(set(offs)) == len(offs)
         assert lay.codes + dp * d * bits // 8 <= lay.scales
         assert lay.scales + dp * (d // g) * 2 <= lay.zeros
-        assert lay.partial + 4 * lay.splits * d <= lay.codes
+        assert lay.partial + 8 * lay.splits * d <= lay.codes
         if r:
             assert lay.ax_ld == r and lay.ax >= lay.zeros + dp * (d // g) * 2
-        if dt == ttq.TTQ_F32:
-            assert lay.xb > 0
+        if T and dp:
+            assert lay.xh > 0
+        if dt == ttq.TTQ_F32 and r:
+            assert lay.xb > 0 and lay.ab > 0
 
 
 @pytest.mark.parametrize("args", [
@@ -84,7 +86,7 @@ def test_rejections_before_device_work(L):
     assert L.ttq_act_norm(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
     assert L.ttq_act_norm(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 128, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
     # forward with a null weight
-    st = L.ttq_linear_forward(16, None, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 16, 256, 1 << 30, None)
+    st = L.ttq_linear_forward(16, None, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 16, 1, 256, 1 << 30, None)
     assert st == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_workspace_init(None, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_get_status(None, None) == ttq.TTQ_ERR_INVALID_ARG

@@ -131,11 +131,15 @@ def test_dequant_gemm_matches_oracle(O, case):
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     A = P.to_dev(data["A"], dtype) if r > 0 else None
     B = P.to_dev(data["B"], dtype) if r > 0 else None
-    Y = ttq.ttq_dequant_gemm(dev(codes.view(np.int32)), dev(sc.view(np.int16)), dev(ze.view(np.int16)),
-                             dev(Dr32), P.to_dev(data["X"], dtype), A, B, bits, group)
+    args = (dev(codes.view(np.int32)), dev(sc.view(np.int16)), dev(ze.view(np.int16)), dev(Dr32),
+            P.to_dev(data["X"], dtype), A, B, bits, group)
+    Y = ttq.ttq_dequant_gemm(*args, y_dtype=torch.float32)
+    Yb = ttq.ttq_dequant_gemm(*args, y_dtype=torch.bfloat16)
     torch.cuda.synchronize()
-    err = P.y_error(Y.float().cpu().numpy(), Y_ref)
+    err = P.y_error(Y.cpu().numpy(), Y_ref)
     assert err <= P.Y_TOL, err
+    # the bf16 output is the fp32 accumulator rounded once to nearest-even
+    assert torch.equal(Yb, Y.to(torch.bfloat16))
 
 
 FORWARD_CASES = [
@@ -167,19 +171,30 @@ def test_forward_matches_oracle(O, spec):
     B = P.to_dev(data["B"], spec.dtype) if spec.r else None
     dt = ttq.TTQ_F32 if spec.dtype == "f32" else ttq.TTQ_BF16
     ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
-    Y = ttq.ttq_linear_forward(X, W, A, B, spec.p, spec.lam, spec.alpha, spec.bits, spec.group, ws=ws)
+    Y = ttq.ttq_linear_forward(X, W, A, B, spec.p, spec.lam, spec.alpha, spec.bits, spec.group, ws=ws,
+                               y_dtype=torch.float32)
+    Yo = ttq.ttq_linear_forward(X, W, A, B, spec.p, spec.lam, spec.alpha, spec.bits, spec.group, ws=ws,
+                                y_dtype=X.dtype)
     torch.cuda.synchronize()
+    assert torch.equal(Yo, Y.to(X.dtype))
     st, flags = ttq.ttq_get_status(ws)
     assert st == ttq.TTQ_OK, flags
     views = ttq.workspace_views(ws, spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
     D = views["D"].cpu().numpy().astype(np.float64)
     assert np.max(np.abs(D - ref["D"]) / ref["D"]) <= P.D_RTOL
-    # codes: identical wherever both sides rounded D to the same binary32
-    codes = P.u32(views["codes"])
-    mism = np.count_nonzero(codes != ref["codes"])
-    assert mism <= max(2, codes.size // 100000), mism
-    assert np.count_nonzero(P.u16(views["scales"]) != ref["scales"]) <= max(2, ref["scales"].size // 100000)
-    err = P.y_error(Y.float().cpu().numpy()[:, rows], ref["Y"])
+    # The quantiser is bit-exact for a shared D (test_quantize_bit_exact); here
+    # each side uses its own D, so codes, scales and zeros must agree in every
+    # group whose channels got the same binary32 D on both sides.
+    same_d = views["D"].cpu().numpy() == ref["D"].astype(np.float32)
+    group_ok = same_d.reshape(-1, spec.group).all(axis=1)          # [d/group]
+    wpg = spec.group * spec.bits // 32                               # words per group
+    codes = P.u32(views["codes"]).reshape(spec.dp, -1, wpg)
+    ref_codes = ref["codes"].reshape(spec.dp, -1, wpg)
+    assert np.array_equal(codes[:, group_ok], ref_codes[:, group_ok])
+    assert np.array_equal(P.u16(views["scales"])[:, group_ok], ref["scales"][:, group_ok])
+    assert np.array_equal(P.u16(views["zeros"])[:, group_ok], ref["zeros"][:, group_ok])
+    assert group_ok.mean() >= 0.99, f"D differs in {np.count_nonzero(~same_d)} channels"
+    err = P.y_error(Y.cpu().numpy()[:, rows], ref["Y"])
     assert err <= P.Y_TOL, err
 
 
@@ -227,6 +242,14 @@ def test_status_flags_nonfinite():
     torch.cuda.synchronize()
     st, flags = ttq.ttq_get_status(ws)
     assert st == ttq.TTQ_ERR_NONFINITE and flags & ttq.TTQ_FLAG_SCALE_OVERFLOW
+    # an activation beyond the binary16 range of the product's X copy
+    X3 = X2 + 1
+    X3[2, 9] = 1.0e5
+    ttq.ttq_workspace_init(ws)
+    ttq.ttq_linear_forward(X3, W, None, None, 2.0, 1e-3, 0.5, 4, 64, ws=ws)
+    torch.cuda.synchronize()
+    st, flags = ttq.ttq_get_status(ws)
+    assert st == ttq.TTQ_ERR_NONFINITE and flags & ttq.TTQ_FLAG_X_RANGE
     # and a clean call after a reset reads OK
     ttq.ttq_workspace_init(ws)
     ttq.ttq_linear_forward(X2 + 1, W, None, None, 2.0, 1e-3, 0.5, 4, 64, ws=ws)
