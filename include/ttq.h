@@ -76,8 +76,9 @@ typedef enum ttq_status {
 } ttq_status;
 
 typedef enum ttq_dtype {
-  TTQ_F32 = 0, /* X, W, A, B and Y are float32 */
-  TTQ_BF16 = 1 /* X, W, A, B and Y are bfloat16 */
+  TTQ_F32 = 0,  /* X, W, A, B and Y are float32 */
+  TTQ_BF16 = 1, /* X, W, A, B and Y are bfloat16 */
+  TTQ_F16 = 2   /* binary16: only for X of ttq_scale_activations and ttq_dequant_gemm */
 } ttq_dtype;
 
 /* Device status word bits (ttq_get_status). */
@@ -101,7 +102,7 @@ typedef struct ttq_workspace_layout {
   size_t scales;  /* uint16 [d'][d/group]                        */
   size_t zeros;   /* uint16 [d'][d/group]                        */
   size_t ax;      /* bf16 [T][ax_ld]  A X                        */
-  size_t xh;      /* binary16 [T][d] copy of X for the product    */
+  size_t xh;      /* binary16 [T][d] X D^{-1/2} for the product   */
   size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32, r > 0) */
   size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32, r > 0) */
   size_t total;
@@ -142,21 +143,37 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
  * W [dp][d] (dtype); D float32 [d] or NULL (identity).  bits in {2, 3, 4};
  * group in {32, 64, 128, 256} with d % group == 0.  Outputs as described
  * above.  Flags NONFINITE for a non-finite W*sqrt(D) and SCALE_OVERFLOW
- * (with NONFINITE) for a group whose scale exceeds binary16. */
+ * (with NONFINITE) for a group whose scale, or scale * (2^bits - 1), exceeds
+ * binary16. */
 ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
                                const float* D, int bits, int group, uint32_t* codes,
                                uint16_t* scales, uint16_t* zeros, void* ws,
                                size_t ws_bytes, void* stream);
 
+/* The B operand of the product: Xs[t][i] = binary16(X[t][i] * D_rsqrt[i])
+ * (the D^{-1/2} factor of W_hat = Q[W D^{1/2}] D^{-1/2}, carried by X;
+ * gist.science/zh/paper/2603.19296, section 2.1).  X [T][d] in dtype (F32,
+ * BF16 or F16), D_rsqrt float32 [d] or NULL (identity), Xs binary16 [T][d]
+ * (uint16 bit patterns); d % 8 == 0.  Each product is rounded once to
+ * binary16; flags X_RANGE if some |Xs| > 65504.  Needs a workspace of at
+ * least 4096 bytes (status word). */
+ttq_status ttq_scale_activations(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
+                                 const float* D_rsqrt, uint16_t* Xs, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 /* Steps (2)-(3) from already quantised weights: Y = W_hat X (+ B (A X)),
- * with W_hat[j][i] = scales[j][k] (codes[j][i] - zeros[j][k]) D_rsqrt[i]
- * formed in shared memory and multiplied on the tensor cores: binary16
- * W_hat and X (X converted exactly from bf16; |x| must not exceed 65504,
- * else flag X_RANGE), fp32 accumulation; the low-rank term B (A X) uses bf16
- * operands with fp32 accumulation, A X held in bf16.
+ * with W_hat[j][i] = scales[j][k] (codes[j][i] - zeros[j][k]) D_rsqrt[i],
+ * on the tensor cores as (s (q - z)) x (X D^{-1/2}): binary16 operands (the
+ * first formed in shared memory, the second written to the workspace;
+ * |x D^{-1/2}| and s (2^bits - 1) must not exceed 65504, else flag
+ * X_RANGE / SCALE_OVERFLOW), fp32 accumulation; the low-rank term B (A X)
+ * uses bf16 operands with fp32 accumulation, A X held in bf16.
  * D_rsqrt == NULL means D = I.  A [r][d] and B [dp][r] (dtype) may be NULL
- * when r == 0; r % 8 == 0.  Y [T][dp] is written in y_dtype: TTQ_F32 keeps
- * the fp32 accumulator as is, TTQ_BF16 rounds it to nearest-even once. */
+ * when r == 0; r % 8 == 0.  dtype TTQ_F16 means X is binary16 and already
+ * holds X D^{-1/2} when D_rsqrt is NULL (as written by
+ * ttq_scale_activations): then only the product runs; it needs r == 0.
+ * Y [T][dp] is written in y_dtype (TTQ_F32 or TTQ_BF16): TTQ_F32 keeps the
+ * fp32 accumulator as is, TTQ_BF16 rounds it to nearest-even once. */
 ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
                             const uint16_t* zeros, const float* D_rsqrt,
                             const void* X, const void* A, const void* B,

@@ -16,12 +16,13 @@
 //               the same 128-byte-swizzled K-major layout the TMA produces,
 //               then (after the last stage) read the accumulator out of
 //               tensor memory and store Y.
-// W_hat is formed in fp32 -- (q - z) * s is exact, one rounding for the
-// D^(-1/2) factor -- and rounded once to binary16 (11 significant bits; a
-// bf16 W_hat would carry 8x the rounding error on the few large
-// outlier-channel terms).  X arrives as binary16, exact for bf16 inputs of
-// magnitude <= 65504.  The low-rank term rides along as extra K blocks: A
-// slot = B[j][k] (TMA), B slot = AX[t][k] (TMA), both bf16.
+// The factor D^(-1/2) of W_hat is carried by the B operand, which arrives
+// as binary16 X D^(-1/2); the A operand is s (q - z), built in binary16 with
+// integer-free bit tricks ((1024 + q) from the code bits, minus (1024 + z),
+// times s: exact until the one rounding of the product).  Binary16 keeps 11
+// significant bits, where bf16 operands would carry 8x the rounding error on
+// the few large outlier-channel terms.  The low-rank term rides along as
+// extra K blocks: A slot = B[j][k] (TMA), B slot = AX[t][k] (TMA), both bf16.
 //
 // Every barrier wait is bounded (1 s); a wait that gives up sets
 // TTQ_FLAG_TIMEOUT, tells the other roles to stop, and the CTA still frees
@@ -42,10 +43,10 @@ constexpr int kSmemLimit = 232448;             // 227 KiB opt-in per block
 
 struct GemmDev {
   const uint32_t* codes;
-  const __half* scales;
-  const __half* zeros;
-  const float* Dr;
-  int group;
+  const uint16_t* scales;
+  const uint16_t* zeros;
+  int group_shift;      // log2(group): groups are powers of two
+  int64_t ngroups;      // K / group
   int64_t K, M, T, K_tail;
   void* Y;
   int64_t ldy;
@@ -55,66 +56,110 @@ struct GemmDev {
   uint32_t* status;
 };
 
-__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
+__device__ __forceinline__ __half2 u2h(uint32_t u) {
+  __half2 h;
+  memcpy(&h, &u, 4);
+  return h;
+}
+__device__ __forceinline__ uint32_t h2u(__half2 h) {
+  uint32_t u;
+  memcpy(&u, &h, 4);
+  return u;
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
                : "memory");
 }
 
-// Writes rows rb, rb+32, rb+64, rb+96 of the 128 x 64 A tile, channels
-// [8c, 8c+8) of K block kb, as binary16 W_hat in the 128-byte-swizzled layout:
-// row r, 16-byte chunk c lives at (r/8)*1024 + (r%8)*128 + ((c ^ r%8) * 16).
+// The operands one producer thread needs for one K block: the packed codes
+// of its 32 channels of one row, and that row's scale and zero point.
+struct CodeChunk {
+  uint32_t w[4];
+  uint16_t s, z;
+};
+
+// Loads the chunk of row `row`, channels [col0, col0 + 32) (zeros outside W).
 template <int BITS>
-__device__ __forceinline__ void dequant_rows(uint32_t a_slot, const GemmDev& g, int64_t m0,
-                                             int kb, int c, int rb) {
-  constexpr int QMAX = (1 << BITS) - 1;
-  const int64_t col = static_cast<int64_t>(kb) * kBK + c * 8;
-  const bool col_ok = col < g.K;  // K % 8 == 0: the 8 channels are all in or all out
-  float dr[8];
-  if (col_ok && g.Dr != nullptr) {
-    const float4 a = __ldg(reinterpret_cast<const float4*>(g.Dr + col));
-    const float4 b = __ldg(reinterpret_cast<const float4*>(g.Dr + col) + 1);
-    dr[0] = a.x; dr[1] = a.y; dr[2] = a.z; dr[3] = a.w;
-    dr[4] = b.x; dr[5] = b.y; dr[6] = b.z; dr[7] = b.w;
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) dr[e] = 1.0f;
-  }
-  const int64_t ng = g.K / g.group;
+__device__ __forceinline__ void load_chunk(const GemmDev& g, int64_t row, int64_t col0,
+                                           CodeChunk& ck) {
+  ck.w[0] = ck.w[1] = ck.w[2] = ck.w[3] = 0u;
+  ck.s = 0;
+  ck.z = 0;
+  if (row >= g.M || col0 >= g.K) return;
   const int64_t wpr = g.K * BITS / 32;
-  const int64_t k = col / g.group;
-  const int64_t bitoff = col * BITS;
-  const int64_t widx = bitoff >> 5;
-  const int sh = static_cast<int>(bitoff & 31);
+  const uint32_t* crow = g.codes + row * wpr + (col0 >> 5) * BITS;
+  if (BITS == 4) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(crow));
+    ck.w[0] = v.x; ck.w[1] = v.y; ck.w[2] = v.z; ck.w[3] = v.w;
+  } else if (BITS == 2) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(crow));
+    ck.w[0] = v.x; ck.w[1] = v.y;
+  } else {
+    ck.w[0] = __ldg(crow);
+    ck.w[1] = __ldg(crow + 1);
+    ck.w[2] = __ldg(crow + 2);
+  }
+  const int64_t gi = row * g.ngroups + (col0 >> g.group_shift);
+  ck.s = __ldg(g.scales + gi);
+  ck.z = __ldg(g.zeros + gi);
+}
+
+// (1024 + q) in both halves of a half2 from two codes placed at bits [0, b)
+// and [16, 16 + b) of `bits`.  0x6400 is binary16 1024.0, whose unit in the
+// last place is 1, so OR-ing a code into the fraction adds it exactly.
+__device__ __forceinline__ uint32_t magic_pair(uint32_t bits) { return bits | 0x64006400u; }
+
+// Writes the 32 channels of row r, 32-channel half `hf` of the K block, as
+// binary16 s (q - z) into the 128-byte-swizzled A tile: row r, 16-byte chunk
+// c lives at (r/8)*1024 + (r%8)*128 + ((c ^ r%8) * 16).  (q - z) is exact in
+// binary16, the product is rounded once; D^(-1/2) is carried by X.
+template <int BITS>
+__device__ __forceinline__ void dequant_chunk(uint32_t a_slot, int r, int hf, const CodeChunk& ck) {
+  const __half2 c2 = __half2half2(__hadd(__ushort_as_half(ck.z), __float2half_rn(1024.f)));
+  const __half2 s2 = __half2half2(__ushort_as_half(ck.s));
+  const uint32_t row_base = a_slot + (r >> 3) * 1024 + (r & 7) * 128;
+  auto put = [&](int chunk, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    st_shared_v4(row_base + (((4 * hf + chunk) ^ (r & 7)) << 4), a, b, c, d);
+  };
+  auto val = [&](uint32_t pairbits) { return h2u(__hmul2(__hsub2(u2h(magic_pair(pairbits)), c2), s2)); };
+  if (BITS == 4 || BITS == 3) {
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int r = rb + 32 * u;
-    const int64_t row = m0 + r;
-    uint4 out = make_uint4(0u, 0u, 0u, 0u);
-    if (col_ok && row < g.M) {
-      const uint32_t* crow = g.codes + row * wpr;
-      uint32_t v = __ldg(crow + widx) >> sh;
-      if (BITS == 3 && sh > 8) v |= __ldg(crow + widx + 1) << (32 - sh);
-      const float s = __half2float(g.scales[row * ng + k]);
-      const int z = static_cast<int>(__half2float(g.zeros[row * ng + k]));
-      float w[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int q = static_cast<int>((v >> (BITS * e)) & QMAX);
-        w[e] = __fmul_rn(static_cast<float>(q - z) * s, dr[e]);
+    for (int i = 0; i < 4; ++i) {
+      // y holds codes 0-3 of this 8-code group in bits 0-15 and codes 4-7 in
+      // bits 16-31, each at 4-bit (INT4) or 3-bit (INT3) spacing
+      uint32_t y;
+      if (BITS == 4) {
+        y = ck.w[i];
+      } else {
+        // the 24 bits of codes 8i..8i+7 start at bit 24i of the 96-bit row piece
+        const int wi = (24 * i) >> 5;
+        const uint32_t v =
+            __funnelshift_r(ck.w[wi], ck.w[wi + 1 < 3 ? wi + 1 : 2], (24 * i) & 31) & 0xFFFFFFu;
+        y = (v & 0xFFFu) | ((v << 4) & 0x0FFF0000u);
       }
-      out.x = pack_f16x2(w[0], w[1]);
-      out.y = pack_f16x2(w[2], w[3]);
-      out.z = pack_f16x2(w[4], w[5]);
-      out.w = pack_f16x2(w[6], w[7]);
+      constexpr uint32_t M = BITS == 4 ? 0x000F000Fu : 0x00070007u;
+      const uint32_t h0 = val(y & M);                       // (q0, q4)
+      const uint32_t h1 = val((y >> BITS) & M);             // (q1, q5)
+      const uint32_t h2 = val((y >> (2 * BITS)) & M);       // (q2, q6)
+      const uint32_t h3 = val((y >> (3 * BITS)) & M);       // (q3, q7)
+      put(i, __byte_perm(h0, h1, 0x5410), __byte_perm(h2, h3, 0x5410), __byte_perm(h0, h1, 0x7632),
+          __byte_perm(h2, h3, 0x7632));
     }
-    const uint32_t addr = a_slot + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
-    st_shared_v4(addr, out);
+  } else {  // BITS == 2: two words of 16 codes, each filling two chunks
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t w = ck.w[k];
+      uint32_t h[8];  // h[e] = (q_e, q_{e+8})
+#pragma unroll
+      for (int e = 0; e < 8; ++e) h[e] = val((w >> (2 * e)) & 0x00030003u);
+      put(2 * k, __byte_perm(h[0], h[1], 0x5410), __byte_perm(h[2], h[3], 0x5410),
+          __byte_perm(h[4], h[5], 0x5410), __byte_perm(h[6], h[7], 0x5410));
+      put(2 * k + 1, __byte_perm(h[0], h[1], 0x7632), __byte_perm(h[2], h[3], 0x7632),
+          __byte_perm(h[4], h[5], 0x7632), __byte_perm(h[6], h[7], 0x7632));
+    }
   }
 }
 
@@ -173,9 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
-      for (int kb = 0; kb < kb_total; ++kb) {
-        const int s = kb % stages;
-        const uint32_t ph = static_cast<uint32_t>(kb / stages) & 1u;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
           *abort_flag = 1;
           set_flag(g.status, TTQ_FLAG_TIMEOUT);
@@ -205,9 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_main =
           idesc_f16kind(BITS == 0 ? kFmtBF16 : kFmtF16, kBM, static_cast<uint32_t>(BN));
       const uint32_t idesc_tail = idesc_f16kind(kFmtBF16, kBM, static_cast<uint32_t>(BN));
-      for (int kb = 0; kb < kb_total; ++kb) {
-        const int s = kb % stages;
-        const uint32_t ph = static_cast<uint32_t>(kb / stages) & 1u;
+      int s = 0;
+      uint32_t ph = 0;
+      for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
         if (!mbar_wait(&full[s], ph, abort_flag)) {
           *abort_flag = 1;
           set_flag(g.status, TTQ_FLAG_TIMEOUT);
@@ -228,12 +273,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------- dequant producers + epilogue
+    // thread pt owns row pt/2 of the A tile and its 32-channel half pt%2;
+    // the next K block's operands are loaded before waiting on this one
     const int pt = threadIdx.x - 64;  // 0..255
-    const int c = pt & 7;
-    const int rb = pt >> 3;
-    for (int kb = 0; kb < kb_total; ++kb) {
-      const int s = kb % stages;
-      const uint32_t ph = static_cast<uint32_t>(kb / stages) & 1u;
+    const int r = pt >> 1;
+    const int hf = pt & 1;
+    constexpr int LB = BITS == 0 ? 4 : BITS;
+    CodeChunk cur, nxt;
+    if (BITS != 0) load_chunk<LB>(g, m0 + r, 32 * hf, cur);
+    int s = 0;
+    uint32_t ph = 0;
+    for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
+      if (BITS != 0 && kb + 1 < kb_main)
+        load_chunk<LB>(g, m0 + r, static_cast<int64_t>(kb + 1) * kBK + 32 * hf, nxt);
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -245,8 +297,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       if (BITS != 0 && kb < kb_main) {
-        dequant_rows<(BITS == 0 ? 4 : BITS)>(smem_addr(smem + s * stage_bytes), g, m0, kb, c, rb);
+        dequant_chunk<LB>(smem_addr(smem + s * stage_bytes), r, hf, cur);
         fence_proxy_async_smem();
+        cur = nxt;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
@@ -306,10 +359,11 @@ cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   if (err != cudaSuccess) return err;
   GemmDev g;
   g.codes = a.codes;
-  g.scales = reinterpret_cast<const __half*>(a.scales);
-  g.zeros = reinterpret_cast<const __half*>(a.zeros);
-  g.Dr = a.Dr;
-  g.group = a.group;
+  g.scales = a.scales;
+  g.zeros = a.zeros;
+  g.group_shift = 0;
+  while (a.group > 0 && (1 << (g.group_shift + 1)) <= a.group) ++g.group_shift;
+  g.ngroups = a.group > 0 ? a.K / a.group : 0;
   g.K = a.K;
   g.M = a.M;
   g.T = a.T;

@@ -44,7 +44,7 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
   if ((d + 255) / 256 > kMaxColumnBlocks) return false;
   const bool has_q = dp > 0;
   if (has_q && (!valid_qparams(bits, group) || d % group != 0)) return false;
-  if (dtype != TTQ_F32 && dtype != TTQ_BF16) return false;
+  if (dtype != TTQ_F32 && dtype != TTQ_BF16 && dtype != TTQ_F16) return false;
   ttq_workspace_layout l = {};
   int64_t splits = 1, rps = 1;
   act_norm_plan(d, T, kPlanSMs, &splits, &rps);
@@ -128,10 +128,10 @@ ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_E
 
 uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
 
-// Y = W_hat X (+ B (A X)) from quantised weights.  Xh is binary16 X; Xb, Ab,
-// Bb are bf16 X, A, B (used only when r > 0).
+// Y = W_hat X (+ B (A X)) from quantised weights.  Xh is binary16
+// X D^(-1/2); Xb, Ab, Bb are bf16 X, A, B (used only when r > 0).
 ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
-                    const float* Dr, const void* Xh, const void* Xb, const void* Ab,
+                    const void* Xh, const void* Xb, const void* Ab,
                     const void* Bb, int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
                     int group, void* Y, bool y_f32, void* ws, const ttq_workspace_layout& L,
                     cudaStream_t stream) {
@@ -174,7 +174,6 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;
-  a.Dr = Dr;
   a.bits = bits;
   a.group = group;
   a.K = d;
@@ -218,6 +217,7 @@ ttq_status ttq_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T, float p,
                         float lambda, float alpha, float* D, float* D_rsqrt, void* ws,
                         size_t ws_bytes, void* stream) {
+  if (dtype == TTQ_F16) return TTQ_ERR_INVALID_ARG;
   ttq_workspace_layout L;
   if (!make_layout(d, 0, T, 0, 4, 32, dtype, &L)) return TTQ_ERR_INVALID_ARG;
   if ((T > 0 && X == nullptr) || ws == nullptr || !(p >= 1.0f) || !(lambda >= 0.0f) ||
@@ -265,6 +265,20 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
                                      static_cast<cudaStream_t>(stream)));
 }
 
+ttq_status ttq_scale_activations(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
+                                 const float* D_rsqrt, uint16_t* Xs, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (dtype != TTQ_F32 && dtype != TTQ_BF16 && dtype != TTQ_F16) return TTQ_ERR_INVALID_ARG;
+  if (d < 8 || d % 8 != 0 || T < 0) return TTQ_ERR_INVALID_ARG;
+  if (T > 0 && (X == nullptr || Xs == nullptr)) return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (Xs && !aligned16(Xs)) || (D_rsqrt && !aligned16(D_rsqrt)))
+    return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
+  return cuda_status(launch_scale_to_f16(X, dtype, D_rsqrt, Xs, T, d, static_cast<uint32_t*>(ws),
+                                         device_sms(), static_cast<cudaStream_t>(stream)));
+}
+
 ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
                             const float* D_rsqrt, const void* X, const void* A, const void* B,
                             ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
@@ -282,6 +296,7 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
                Y == nullptr))
     return TTQ_ERR_INVALID_ARG;
   if (r > 0 && (A == nullptr || B == nullptr)) return TTQ_ERR_INVALID_ARG;
+  if (dtype == TTQ_F16 && r > 0) return TTQ_ERR_UNSUPPORTED;
   const void* ptrs[] = {codes, scales, zeros, D_rsqrt, X, A, B, Y};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return TTQ_ERR_INVALID_ARG;
@@ -289,9 +304,14 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   const bool f32 = dtype == TTQ_F32;
-  void* xh = ws_at(ws, L.xh);
-  ttq_status st = cuda_status(launch_to_f16(X, f32, xh, T * d, status, s));
-  if (st != TTQ_OK) return st;
+  const void* xh = X;  // binary16 X D^{-1/2} given as is
+  ttq_status st = TTQ_OK;
+  if (!(dtype == TTQ_F16 && D_rsqrt == nullptr)) {
+    void* xs = ws_at(ws, L.xh);
+    st = cuda_status(launch_scale_to_f16(X, dtype, D_rsqrt, xs, T, d, status, device_sms(), s));
+    if (st != TTQ_OK) return st;
+    xh = xs;
+  }
   const void* Xb = X;
   const void* Ab = A;
   const void* Bb = B;
@@ -307,7 +327,7 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
     Ab = ab;
     Bb = bb;
   }
-  return run_gemm(codes, scales, zeros, D_rsqrt, xh, Xb, Ab, Bb, d, dp, T, r, bits, group, Y,
+  return run_gemm(codes, scales, zeros, xh, Xb, Ab, Bb, d, dp, T, r, bits, group, Y,
                   y_dtype == TTQ_F32, ws, L, s);
 }
 
@@ -318,6 +338,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
   if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
     return TTQ_ERR_UNSUPPORTED;
+  if (dtype == TTQ_F16) return TTQ_ERR_INVALID_ARG;
   ttq_workspace_layout L;
   if (!make_layout(d, dp, T, r, bits, group, dtype, &L)) return TTQ_ERR_INVALID_ARG;
   if (dp == 0 && !valid_qparams(bits, group)) return TTQ_ERR_INVALID_ARG;
@@ -341,14 +362,16 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   void* xh = dp > 0 ? ws_at(ws, L.xh) : nullptr;
   void* xb = (f32 && r > 0) ? ws_at(ws, L.xb) : nullptr;
 
-  // (1) D and D^{-1/2}; X is also written as binary16 for the product (and
-  // as bf16 for the low-rank product when it arrives as float32)
+  // (1) D and D^{-1/2} (a float32 X is also written as bf16 for the
+  // low-rank product), then the product's B operand X D^{-1/2} in binary16
   int64_t splits, rps;
   act_norm_plan(d, T, kPlanSMs, &splits, &rps);
   ttq_status st = cuda_status(launch_act_norm(
       X, f32, d, T, p, lambda, alpha, splits, rps,
-      reinterpret_cast<double*>(ws_at(ws, L.partial)), status + 64, D, Dr, xh, xb, status, s));
+      reinterpret_cast<double*>(ws_at(ws, L.partial)), status + 64, D, Dr, nullptr, xb, status, s));
   if (st != TTQ_OK || dp == 0) return st;
+  st = cuda_status(launch_scale_to_f16(X, dtype, Dr, xh, T, d, status, device_sms(), s));
+  if (st != TTQ_OK) return st;
 
   // (2) codes, scales, zeros of Q[W D^{1/2}]
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));
@@ -370,7 +393,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
     Ab = ab;
     Bb = bb;
   }
-  return run_gemm(codes, scales, zeros, Dr, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
+  return run_gemm(codes, scales, zeros, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
                   y_dtype == TTQ_F32, ws, L, s);
 }
 

@@ -31,10 +31,15 @@ cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, co
 // float32 -> bf16 copy of n elements (n % 8 == 0).
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
 
-// float32 or bf16 -> binary16 copy of n elements (n % 8 == 0); flags
-// X_RANGE if some |x| > 65504.
-cudaError_t launch_to_f16(const void* src, bool src_f32, void* dst, int64_t n, uint32_t* status,
-                          cudaStream_t stream);
+// X' [T][d] = binary16(X[t][i] * Dr[i]) from float32, bf16 or binary16 X
+// (Dr null: plain conversion); d % 8 == 0; flags X_RANGE if some
+// |X'| > 65504.
+constexpr int kSrcF32 = 0;
+constexpr int kSrcBF16 = 1;
+constexpr int kSrcF16 = 2;
+cudaError_t launch_scale_to_f16(const void* src, int src_kind, const float* Dr, void* dst,
+                                int64_t T, int64_t d, uint32_t* status, int num_sms,
+                                cudaStream_t stream);
 
 // Steps (2)-(3) on the tensor cores.
 struct GemmArgs {
@@ -42,7 +47,6 @@ struct GemmArgs {
   const uint32_t* codes = nullptr;
   const uint16_t* scales = nullptr;
   const uint16_t* zeros = nullptr;
-  const float* Dr = nullptr;  // null: identity
   int bits = 0;               // 0: A operand loaded by TMA from tmA0 (plain bf16 x bf16)
   int group = 0;
   // sizes
@@ -59,7 +63,7 @@ struct GemmArgs {
 
 struct GemmMaps {
   CUtensorMap a0;  // plain A operand [M][K] bf16 (bits == 0)
-  CUtensorMap b0;  // X [T][K]: binary16 with codes (bits != 0), bf16 in the plain mode
+  CUtensorMap b0;  // binary16 X D^(-1/2) [T][K] with codes (bits != 0); bf16 X in the plain mode
   CUtensorMap a1;  // low-rank B [M][r] bf16
   CUtensorMap b1;  // A X [T][r] bf16
 };

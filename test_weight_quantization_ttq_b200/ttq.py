@@ -24,6 +24,7 @@ TTQ_ERR_WORKSPACE = 6
 
 TTQ_F32 = 0
 TTQ_BF16 = 1
+TTQ_F16 = 2
 
 TTQ_FLAG_NONFINITE = 0x1
 TTQ_FLAG_SCALE_OVERFLOW = 0x2
@@ -51,6 +52,7 @@ SIGNATURES = {
     "ttq_workspace_init": (_INT, [_P, _SZ, _P]),
     "ttq_act_norm": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _SZ, _P]),
     "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
+    "ttq_scale_activations": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
                                 _P, _INT, _P, _SZ, _P]),
     "ttq_linear_forward": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT, _INT,
@@ -99,7 +101,9 @@ def _dtype_code(t: torch.Tensor) -> int:
         return TTQ_F32
     if t.dtype == torch.bfloat16:
         return TTQ_BF16
-    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+    if t.dtype == torch.float16:
+        return TTQ_F16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32, bfloat16 or float16)")
 
 
 def _dev(t: torch.Tensor | None, name: str) -> int | None:
@@ -185,6 +189,19 @@ def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zer
     return codes, scales, zeros
 
 
+def ttq_scale_activations(X, D_rsqrt, ws=None, Xs=None, stream=None):
+    """Xs [T][d] binary16 (torch.float16) = X * D^{-1/2}, the product's B operand."""
+    T, d = X.shape
+    if ws is None:
+        ws = new_workspace(d, 0, 0, 0, 4, 32, TTQ_BF16, X.device, stream)
+    if Xs is None:
+        Xs = torch.empty((T, d), dtype=torch.float16, device=X.device)
+    _check(lib().ttq_scale_activations(_dev(X, "X"), _dtype_code(X), d, T, _dev(D_rsqrt, "D_rsqrt"),
+                                       _dev(Xs, "Xs"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "ttq_scale_activations")
+    return Xs
+
+
 def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=None, Y=None,
                      y_dtype=None, stream=None):
     """Y [T][d'] = W_hat X (+ B (A X)) from quantised weights; Y in y_dtype
@@ -196,7 +213,8 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
     if ws is None:
         ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
     if Y is None:
-        Y = torch.empty((T, dp), dtype=y_dtype or X.dtype, device=X.device)
+        Y = torch.empty((T, dp), dtype=y_dtype or (torch.bfloat16 if dt == TTQ_F16 else X.dtype),
+                        device=X.device)
     _check(lib().ttq_dequant_gemm(_dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
                                   _dev(D_rsqrt, "D_rsqrt"), _dev(X, "X"), _dev(A, "A"), _dev(B, "B"), dt,
                                   d, dp, T, r, bits, group, _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"),

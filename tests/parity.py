@@ -35,5 +35,15 @@ def y_error(y_gpu: np.ndarray, y_ref: np.ndarray) -> float:
     return float(np.abs(y_gpu.astype(np.float64) - y_ref).max()) / rms
 
 
+def f32(v: float) -> float:
+    """The binary32 value the C ABI receives for a float parameter (p,
+    lambda, alpha); the oracle is given the same value."""
+    return float(np.float32(v))
+
+
+def params(spec: synth.LinearSpec) -> tuple[float, float, float]:
+    return f32(spec.p), f32(spec.lam), f32(spec.alpha)
+
+
 def inputs(spec: synth.LinearSpec, need_w: bool = True) -> dict:
     return synth.generate(spec, need_w=need_w)

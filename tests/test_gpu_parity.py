@@ -44,7 +44,7 @@ ACT_CASES = [
 @pytest.mark.parametrize("spec", ACT_CASES, ids=lambda s: f"{s.name}-T{s.T}")
 def test_act_norm_matches_oracle(O, spec):
     x = P.inputs(spec, need_w=False)["X"]
-    D_ref, Dr_ref, st = O.act_norm(x.astype(np.float64), spec.p, spec.lam, spec.alpha)
+    D_ref, Dr_ref, st = O.act_norm(x.astype(np.float64), *P.params(spec))
     assert st == 0
     X = P.to_dev(x, spec.dtype)
     D, Dr = ttq.ttq_act_norm(X, spec.p, spec.lam, spec.alpha)
@@ -85,7 +85,7 @@ def test_quantize_bit_exact(O, spec, mode):
     if mode == "identity":
         D32 = None
     else:
-        D_ref, _, _ = O.act_norm(data["X"].astype(np.float64), spec.p, spec.lam, spec.alpha)
+        D_ref, _, _ = O.act_norm(data["X"].astype(np.float64), *P.params(spec))
         D32 = D_ref.astype(np.float32)  # both sides get this same D
     codes_ref, sc_ref, ze_ref, st = O.quantize(W, D32, spec.bits, spec.group)
     assert st == 0
@@ -121,7 +121,7 @@ def test_dequant_gemm_matches_oracle(O, case):
     spec = _small("gemm", d=d, dp=dp, T=T, bits=bits, group=group, dtype=dtype, r=r)
     data = P.inputs(spec)
     X = data["X"].astype(np.float64)
-    D_ref, Dr_ref, _ = O.act_norm(X, spec.p, spec.lam, spec.alpha)
+    D_ref, Dr_ref, _ = O.act_norm(X, *P.params(spec))
     codes, sc, ze, _ = O.quantize(data["W"], D_ref.astype(np.float32), bits, group)
     Dr32 = Dr_ref.astype(np.float32)
     What = O.dequant_rows(codes, sc, ze, Dr32.astype(np.float64), d, bits, group)
@@ -162,7 +162,7 @@ FORWARD_CASES = [
 def test_forward_matches_oracle(O, spec):
     data = P.inputs(spec)
     rows = synth.sample_rows(spec.dp, 96)
-    ref = O.forward(data["X"].astype(np.float64), data["W"], spec.p, spec.lam, spec.alpha, spec.bits,
+    ref = O.forward(data["X"].astype(np.float64), data["W"], *P.params(spec), spec.bits,
                     spec.group, A=data.get("A"), B=data.get("B"), rows=rows)
     assert ref["status"] == 0
     X = P.to_dev(data["X"], spec.dtype)
@@ -196,6 +196,39 @@ def test_forward_matches_oracle(O, spec):
     assert group_ok.mean() >= 0.99, f"D differs in {np.count_nonzero(~same_d)} channels"
     err = P.y_error(Y.cpu().numpy()[:, rows], ref["Y"])
     assert err <= P.Y_TOL, err
+
+
+def test_scale_activations_rounds_once():
+    """X D^{-1/2} in binary16 is the float32 product rounded once."""
+    rng = np.random.default_rng(3)
+    T, d = 37, 264
+    x = P.inputs(_small("scale", d=d, dp=0, T=T, bits=4, group=8), need_w=False)["X"]
+    dr = np.exp(rng.uniform(-3, 1, d)).astype(np.float32)
+    for dtype in ("bf16", "f32"):
+        Xs = ttq.ttq_scale_activations(P.to_dev(x, dtype), torch.from_numpy(dr).cuda())
+        torch.cuda.synchronize()
+        ref = (x.astype(np.float32) * dr[None, :]).astype(np.float16)
+        assert np.array_equal(Xs.cpu().numpy().view(np.uint16), ref.view(np.uint16)), dtype
+
+
+def test_composed_steps_equal_forward(O):
+    """act_norm -> scale_activations -> quantize_weight -> dequant_gemm (binary16
+    X D^{-1/2}) is the forward, bit for bit, and matches the oracle."""
+    spec = synth.C2.with_(T=300, dp=640)
+    data = P.inputs(spec)
+    X, W = P.to_dev(data["X"], "bf16"), P.to_dev(data["W"], "bf16")
+    p, lam, alpha = spec.p, spec.lam, spec.alpha
+    Y = ttq.ttq_linear_forward(X, W, None, None, p, lam, alpha, spec.bits, spec.group, y_dtype=torch.float32)
+    D, Dr = ttq.ttq_act_norm(X, p, lam, alpha)
+    Xs = ttq.ttq_scale_activations(X, Dr)
+    codes, sc, ze = ttq.ttq_quantize_weight(W, D, spec.bits, spec.group)
+    Y2 = ttq.ttq_dequant_gemm(codes, sc, ze, None, Xs, None, None, spec.bits, spec.group,
+                              y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+    rows = synth.sample_rows(spec.dp, 64)
+    ref = O.forward(data["X"].astype(np.float64), data["W"], *P.params(spec), spec.bits, spec.group, rows=rows)
+    assert P.y_error(Y2.cpu().numpy()[:, rows], ref["Y"]) <= P.Y_TOL
 
 
 def test_forward_is_deterministic():
@@ -242,11 +275,12 @@ def test_status_flags_nonfinite():
     torch.cuda.synchronize()
     st, flags = ttq.ttq_get_status(ws)
     assert st == ttq.TTQ_ERR_NONFINITE and flags & ttq.TTQ_FLAG_SCALE_OVERFLOW
-    # an activation beyond the binary16 range of the product's X copy
+    # X D^{-1/2} beyond the binary16 range of the product's operand (alpha = 0
+    # gives D = I; with alpha > 0 the outlier's own norm would shrink it)
     X3 = X2 + 1
     X3[2, 9] = 1.0e5
     ttq.ttq_workspace_init(ws)
-    ttq.ttq_linear_forward(X3, W, None, None, 2.0, 1e-3, 0.5, 4, 64, ws=ws)
+    ttq.ttq_linear_forward(X3, W, None, None, 2.0, 1e-3, 0.0, 4, 64, ws=ws)
     torch.cuda.synchronize()
     st, flags = ttq.ttq_get_status(ws)
     assert st == ttq.TTQ_ERR_NONFINITE and flags & ttq.TTQ_FLAG_X_RANGE
