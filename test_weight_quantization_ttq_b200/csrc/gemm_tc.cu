@@ -4,9 +4,11 @@
 // (gist.science/zh/paper/2603.19296, section 2.1 for W_hat, 2.2 for the
 // static low-rank pair, 2.3 for the projection).
 //
-// One CTA computes a 128 (rows of W) x BN (tokens) tile of Y^T in tensor
-// memory with tcgen05.mma kind::f16 (binary16 x binary16 -> fp32 for the
-// quantised weight; bf16 x bf16 for the low-rank tail), cta_group::1:
+// One CTA computes a BM (rows of W: 128 or 256) x BN (tokens) tile of Y^T in
+// tensor memory with tcgen05.mma kind::f16 (binary16 x binary16 -> fp32 for
+// the quantised weight; bf16 x bf16 for the low-rank tail), cta_group::1; a
+// 256-row tile is two 128-row MMAs that share each X tile, which halves the
+// X traffic per FLOP:
 //   warp 0      TMA producer: X tiles (BN x 64, 128-byte swizzle) into the
 //               B slot of each pipeline stage; in the plain mode (no codes)
 //               and for the low-rank tail also the A slot.
@@ -33,12 +35,11 @@
 namespace ttq {
 namespace {
 
-constexpr int kBM = 128;
-constexpr int kBK = 64;                        // bf16 elements per 128-byte row
-constexpr int kATileBytes = kBM * kBK * 2;     // 16 KiB
+constexpr int kBK = 64;                        // 16-bit elements per 128-byte row
+constexpr int kSubTileBytes = 128 * kBK * 2;   // one 128-row operand tile: 16 KiB
 constexpr int kThreads = 320;
 constexpr int kProducerWarps = 8;
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 232448;             // 227 KiB opt-in per block
 
 struct GemmDev {
@@ -112,17 +113,19 @@ __device__ __forceinline__ void load_chunk(const GemmDev& g, int64_t row, int64_
 // last place is 1, so OR-ing a code into the fraction adds it exactly.
 __device__ __forceinline__ uint32_t magic_pair(uint32_t bits) { return bits | 0x64006400u; }
 
-// Writes the 32 channels of row r, 32-channel half `hf` of the K block, as
-// binary16 s (q - z) into the 128-byte-swizzled A tile: row r, 16-byte chunk
-// c lives at (r/8)*1024 + (r%8)*128 + ((c ^ r%8) * 16).  (q - z) is exact in
-// binary16, the product is rounded once; D^(-1/2) is carried by X.
+// Writes the 32 channels of one row, 32-channel half `hf` of the K block, as
+// binary16 s (q - z) into the 128-byte-swizzled A tile: in a 128-row
+// sub-tile, row r's 16-byte chunk c lives at (r/8)*1024 + (r%8)*128 +
+// ((c ^ r%8) * 16); row_base is the row's address and rsw = r % 8.  (q - z)
+// is exact in binary16, the product is rounded once; D^(-1/2) is carried by
+// X.
 template <int BITS>
-__device__ __forceinline__ void dequant_chunk(uint32_t a_slot, int r, int hf, const CodeChunk& ck) {
-  const __half2 c2 = __half2half2(__hadd(__ushort_as_half(ck.z), __float2half_rn(1024.f)));
+__device__ __forceinline__ void dequant_chunk(uint32_t row_base, int rsw, int hf,
+                                              const CodeChunk& ck) {
+  const __half2 c2 = __half2half2(__hadd(__ushort_as_half(ck.z), __ushort_as_half(0x6400)));
   const __half2 s2 = __half2half2(__ushort_as_half(ck.s));
-  const uint32_t row_base = a_slot + (r >> 3) * 1024 + (r & 7) * 128;
   auto put = [&](int chunk, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    st_shared_v4(row_base + (((4 * hf + chunk) ^ (r & 7)) << 4), a, b, c, d);
+    st_shared_v4(row_base + (((4 * hf + chunk) ^ rsw) << 4), a, b, c, d);
   };
   auto val = [&](uint32_t pairbits) { return h2u(__hmul2(__hsub2(u2h(magic_pair(pairbits)), c2), s2)); };
   if (BITS == 4 || BITS == 3) {
@@ -163,17 +166,19 @@ __device__ __forceinline__ void dequant_chunk(uint32_t a_slot, int r, int hf, co
   }
 }
 
-template <int BITS>
+template <int BITS, int BM>
 __global__ void __launch_bounds__(kThreads, 1)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                     const GemmDev g) {
+  constexpr int kSub = BM / 128;                 // 128-row MMAs per K step
+  constexpr int kATile = BM * kBK * 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int BN = g.BN;
   const int stages = g.stages;
-  const int stage_bytes = kATileBytes + BN * 128;
+  const int stage_bytes = kATile + BN * 128;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
   uint64_t* empty = full + kMaxStages;
   uint64_t* accum = empty + kMaxStages;
@@ -182,12 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * kBM;
+  const int64_t m0 = static_cast<int64_t>(blockIdx.x) * BM;
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * BN;
   const int kb_main = static_cast<int>((g.K + kBK - 1) / kBK);
   const int kb_tail = static_cast<int>((g.K_tail + kBK - 1) / kBK);
   const int kb_total = kb_main + kb_tail;
-  const uint32_t tmem_cols = BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u;
+  // accumulator h of a 256-row tile starts at column 256 * h
+  const uint32_t tmem_cols =
+      kSub == 2 ? 512u : (BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
@@ -227,15 +234,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* a_slot = smem + s * stage_bytes;
-        uint8_t* b_slot = a_slot + kATileBytes;
+        uint8_t* b_slot = a_slot + kATile;
         if (kb < kb_main) {
-          const uint32_t bytes = BN * 128 + (BITS == 0 ? kATileBytes : 0);
+          const uint32_t bytes = BN * 128 + (BITS == 0 ? kATile : 0);
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(&tmB0, &full[s], b_slot, kb * kBK, static_cast<int32_t>(n0));
           if (BITS == 0) tma_load_2d(&tmA0, &full[s], a_slot, kb * kBK, static_cast<int32_t>(m0));
         } else {
           const int kt = (kb - kb_main) * kBK;
-          mbar_arrive_expect_tx(&full[s], BN * 128 + kATileBytes);
+          mbar_arrive_expect_tx(&full[s], BN * 128 + kATile);
           tma_load_2d(&tmB1, &full[s], b_slot, kt, static_cast<int32_t>(n0));
           tma_load_2d(&tmA1, &full[s], a_slot, kt, static_cast<int32_t>(m0));
         }
@@ -245,11 +252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      // main K blocks: binary16 W_hat x binary16 X (bf16 x bf16 in the plain
-      // mode); low-rank tail: bf16 B x bf16 A X
+      // main K blocks: binary16 W_hat x binary16 X D^(-1/2) (bf16 x bf16 in
+      // the plain mode); low-rank tail: bf16 B x bf16 A X
       const uint32_t idesc_main =
-          idesc_f16kind(BITS == 0 ? kFmtBF16 : kFmtF16, kBM, static_cast<uint32_t>(BN));
-      const uint32_t idesc_tail = idesc_f16kind(kFmtBF16, kBM, static_cast<uint32_t>(BN));
+          idesc_f16kind(BITS == 0 ? kFmtBF16 : kFmtF16, 128, static_cast<uint32_t>(BN));
+      const uint32_t idesc_tail = idesc_f16kind(kFmtBF16, 128, static_cast<uint32_t>(BN));
       int s = 0;
       uint32_t ph = 0;
       for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
@@ -260,12 +267,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after_sync();
         const uint32_t a_addr = smem_addr(smem + s * stage_bytes);
-        const uint64_t adesc = smem_desc_sw128(a_addr);
-        const uint64_t bdesc = smem_desc_sw128(a_addr + kATileBytes);
+        const uint64_t bdesc = smem_desc_sw128(a_addr + kATile);
         const uint32_t idesc = kb < kb_main ? idesc_main : idesc_tail;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)
-          mma_f16kind_ss(tmem_base, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+        for (int k = 0; k < kBK / 16; ++k) {
+#pragma unroll
+          for (int h = 0; h < kSub; ++h) {
+            const uint64_t adesc = smem_desc_sw128(a_addr + h * kSubTileBytes);
+            mma_f16kind_ss(tmem_base + 256u * h, adesc + 2u * k, bdesc + 2u * k, idesc,
+                           (kb | k) != 0 ? 1u : 0u);
+          }
+        }
         mma_commit(&empty[s]);
       }
       mma_commit(accum);
@@ -273,19 +285,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------- dequant producers + epilogue
-    // thread pt owns row pt/2 of the A tile and its 32-channel half pt%2;
-    // the next K block's operands are loaded before waiting on this one
+    // BM = 128: thread pt owns row pt % 128 and the 32-channel half pt / 128
+    // of each K block; BM = 256: row pt and both halves.  A warp thus writes
+    // 32 consecutive rows of one 16-byte chunk column: conflict-free.  The
+    // next K block's operands are loaded before waiting on this one.
     const int pt = threadIdx.x - 64;  // 0..255
-    const int r = pt >> 1;
-    const int hf = pt & 1;
+    const int r = BM == 128 ? (pt & 127) : pt;
+    constexpr int kChunks = BM == 128 ? 1 : 2;
+    const int hf0 = BM == 128 ? (pt >> 7) : 0;
+    const int rl = r & 127;
+    const int rsw = r & 7;
+    const uint32_t row_off = (r >> 7) * kSubTileBytes + (rl >> 3) * 1024 + (rl & 7) * 128;
     constexpr int LB = BITS == 0 ? 4 : BITS;
-    CodeChunk cur, nxt;
-    if (BITS != 0) load_chunk<LB>(g, m0 + r, 32 * hf, cur);
+    CodeChunk cur[kChunks], nxt[kChunks];
+    if (BITS != 0) {
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) load_chunk<LB>(g, m0 + r, 32 * (hf0 + c), cur[c]);
+    }
     int s = 0;
     uint32_t ph = 0;
     for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
-      if (BITS != 0 && kb + 1 < kb_main)
-        load_chunk<LB>(g, m0 + r, static_cast<int64_t>(kb + 1) * kBK + 32 * hf, nxt);
+      if (BITS != 0 && kb + 1 < kb_main) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          load_chunk<LB>(g, m0 + r, static_cast<int64_t>(kb + 1) * kBK + 32 * (hf0 + c), nxt[c]);
+      }
       int ok = 1;
       if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -297,9 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       if (BITS != 0 && kb < kb_main) {
-        dequant_chunk<LB>(smem_addr(smem + s * stage_bytes), r, hf, cur);
+        const uint32_t row_base = smem_addr(smem + s * stage_bytes) + row_off;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          dequant_chunk<LB>(row_base, rsw, hf0 + c, cur[c]);
+          cur[c] = nxt[c];
+        }
         fence_proxy_async_smem();
-        cur = nxt;
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
@@ -313,14 +341,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       set_flag(g.status, TTQ_FLAG_TIMEOUT);
     }
     tc_fence_after_sync();
-    const int q = warp & 3;             // tensor-memory lane quadrant of this warp
-    const int half = (warp - 2) >> 2;   // two warps per quadrant split the columns
-    const int64_t j = m0 + q * 32 + lane;
+    // warp w may read tensor-memory lanes 32 (w % 4) .. +31.  BM = 128: the
+    // two warps of a lane quadrant split the columns; BM = 256: warps 2-5
+    // read accumulator 0 (rows 0-127), warps 6-9 accumulator 1.
+    const int q = warp & 3;
+    const int wg = (warp - 2) >> 2;
+    const int acc = BM == 128 ? 0 : wg;
+    const int ch0 = BM == 128 ? wg : 0;
+    const int chs = BM == 128 ? 2 : 1;
+    const int64_t j = m0 + acc * 128 + q * 32 + lane;
     const int nchunks = BN / 16;
     const bool store = ok && (*abort_flag == 0) && j < g.M;
-    for (int ch = half; ch < nchunks; ch += 2) {
-      uint32_t r[16];
-      tmem_load_16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, r);
+    for (int ch = ch0; ch < nchunks; ch += chs) {
+      uint32_t rr[16];
+      tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
       tmem_load_wait();
       if (store) {
         const int64_t t0 = n0 + ch * 16;
@@ -328,12 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           float* Y = static_cast<float*>(g.Y);
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __uint_as_float(r[i]);
+            if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __uint_as_float(rr[i]);
         } else {
           __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(g.Y);
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __float2bfloat16_rn(__uint_as_float(r[i]));
+            if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __float2bfloat16_rn(__uint_as_float(rr[i]));
         }
       }
     }
@@ -347,14 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BITS>
-cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStream_t stream) {
-  const int stage_bytes = kATileBytes + BN * 128;
+template <int BITS, int BM>
+cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStream_t stream) {
+  const int stage_bytes = BM * kBK * 2 + BN * 128;
   int stages = (kSmemLimit - 2048) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
   const int smem = stages * stage_bytes + 2048;
-  cudaError_t err = cudaFuncSetAttribute(ttq_gemm_kernel<BITS>,
+  cudaError_t err = cudaFuncSetAttribute(ttq_gemm_kernel<BITS, BM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   GemmDev g;
@@ -374,10 +408,17 @@ cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.BN = BN;
   g.stages = stages;
   g.status = a.status;
-  const dim3 grid(static_cast<unsigned>((a.M + kBM - 1) / kBM),
+  const dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM),
                   static_cast<unsigned>((a.T + BN - 1) / BN));
-  ttq_gemm_kernel<BITS><<<grid, kThreads, smem, stream>>>(maps.a0, maps.b0, maps.a1, maps.b1, g);
+  ttq_gemm_kernel<BITS, BM><<<grid, kThreads, smem, stream>>>(maps.a0, maps.b0, maps.a1, maps.b1, g);
   return cudaGetLastError();
+}
+
+template <int BITS>
+cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, int BM,
+                        cudaStream_t stream) {
+  if (BM == 256) return launch_tile<BITS, 256>(a, maps, BN, stream);
+  return launch_tile<BITS, 128>(a, maps, BN, stream);
 }
 
 }  // namespace
@@ -389,19 +430,32 @@ int gemm_block_n(int64_t T) {
   return static_cast<int>(bn);
 }
 
+int gemm_block_m(int bits, int64_t M, int64_t T, int block_n, int num_sms) {
+  if (bits == 0 || M <= 128) return 128;
+  // waves of CTAs times the work of one CTA; 128-row tiles move twice the
+  // X bytes per FLOP, which costs about 40% at full tensor rate
+  const int64_t nt = (T + block_n - 1) / block_n;
+  const int64_t c256 = (M + 255) / 256 * nt;
+  const int64_t c128 = (M + 127) / 128 * nt;
+  const double t256 = static_cast<double>((c256 + num_sms - 1) / num_sms) * 2.0;
+  const double t128 = static_cast<double>((c128 + num_sms - 1) / num_sms) * 1.4;
+  return t256 <= t128 ? 256 : 128;
+}
+
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,
-                                cudaStream_t stream) {
+                                int block_m, cudaStream_t stream) {
   if (args.M == 0 || args.T == 0) return cudaSuccess;
   if (block_n % 16 != 0 || block_n < 16 || block_n > 256) return cudaErrorInvalidValue;
+  if (block_m != 128 && !(block_m == 256 && args.bits != 0)) return cudaErrorInvalidValue;
   switch (args.bits) {
     case 0:
-      return launch_bits<0>(args, maps, block_n, stream);
+      return launch_bits<0>(args, maps, block_n, 128, stream);
     case 2:
-      return launch_bits<2>(args, maps, block_n, stream);
+      return launch_bits<2>(args, maps, block_n, block_m, stream);
     case 3:
-      return launch_bits<3>(args, maps, block_n, stream);
+      return launch_bits<3>(args, maps, block_n, block_m, stream);
     case 4:
-      return launch_bits<4>(args, maps, block_n, stream);
+      return launch_bits<4>(args, maps, block_n, block_m, stream);
     default:
       return cudaErrorInvalidValue;
   }

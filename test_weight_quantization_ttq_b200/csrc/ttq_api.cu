@@ -156,14 +156,15 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     a.ldy = L.ax_ld;
     a.y_f32 = false;
     a.status = status;
-    const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, stream));
+    const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, 128, stream));
     if (st != TTQ_OK) return st;
   }
+  const int bm = gemm_block_m(bits, dp, T, bn, device_sms());
   GemmMaps m;
   if (!encode_16bit(&m.b0, Xh, true, d, T, d, bn)) return TTQ_ERR_CUDA;
   m.a0 = m.b0;
   if (r > 0) {
-    if (!encode_16bit(&m.a1, Bb, false, r, dp, r, 128) ||
+    if (!encode_16bit(&m.a1, Bb, false, r, dp, r, bm) ||
         !encode_16bit(&m.b1, ax, false, r, T, L.ax_ld, bn))
       return TTQ_ERR_CUDA;
   } else {
@@ -184,7 +185,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   a.ldy = dp;
   a.y_f32 = y_f32;
   a.status = status;
-  return cuda_status(launch_dequant_gemm(a, m, bn, stream));
+  return cuda_status(launch_dequant_gemm(a, m, bn, bm, stream));
 }
 
 }  // namespace

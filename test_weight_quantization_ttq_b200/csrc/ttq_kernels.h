@@ -71,7 +71,11 @@ struct GemmMaps {
 // Tile width along the tokens for T tokens.
 int gemm_block_n(int64_t T);
 
+// Tile height (128 or 256 rows of W) for this problem; 256 only with codes.
+int gemm_block_m(int bits, int64_t M, int64_t T, int block_n, int num_sms);
+
+// The operand boxes: a0/a1 are loaded as block_m x 64, b0/b1 as block_n x 64.
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,
-                                cudaStream_t stream);
+                                int block_m, cudaStream_t stream);
 
 }  // namespace ttq

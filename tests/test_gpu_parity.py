@@ -154,6 +154,9 @@ FORWARD_CASES = [
     synth.C5.with_(T=128, p=1.0, alpha=0.25),
     synth.C5.with_(T=4096, p=2.0, alpha=0.25),
     _small("ragged_all", d=96, dp=200, T=19, bits=3, group=32),
+    # 256-row tiles with ragged row and token tails
+    _small("ragged_256row_tiles", d=4096, dp=4296, T=2000, bits=4, group=128, n_out=40),
+    _small("ragged_256row_tiles_int2_lowrank", d=1024, dp=4296, T=2000, bits=2, group=64, r=40, n_out=10),
     _small("ragged_lowrank", d=448, dp=333, T=77, bits=2, group=64, r=24),
 ]
 
