@@ -52,6 +52,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale(LIBRARY):
         return LIBRARY
     nvcc = _nvcc()
+    # a failed build must not leave an older library behind to be loaded
+    if os.path.exists(LIBRARY):
+        os.remove(LIBRARY)
     os.makedirs(BUILD_DIR, exist_ok=True)
     extra = ["-Xptxas", "-v"] if verbose else []
 

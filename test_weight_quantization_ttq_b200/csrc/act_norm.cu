@@ -77,7 +77,7 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16* dst, const float (&v)
 }
 
 template <typename XT, int PK>
-__global__ void __launch_bounds__(kThreads) act_norm_kernel(
+__global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
     const XT* __restrict__ X, int64_t d, int64_t T, double p, double lambda, double alpha,
     int64_t splits, int64_t rows_per_split, double* __restrict__ partial,
     uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
@@ -99,36 +99,47 @@ __global__ void __launch_bounds__(kThreads) act_norm_kernel(
   const int64_t t_end = min(T, t_begin + rows_per_split);
   float amax = 0.f;
   if (c0 < d) {
-    int64_t t = t_begin + warp;
-    // two rows in flight per warp
-    for (; t + 8 < t_end; t += 16) {
-      float v0[8], v1[8];
-      load8(X + t * d + c0, v0);
-      load8(X + (t + 8) * d + c0, v1);
-      if (xh != nullptr) {
-        store8_f16(xh + t * d + c0, v0);
-        store8_f16(xh + (t + 8) * d + c0, v1);
-      }
-      if (xb != nullptr) {
-        store8_bf16(xb + t * d + c0, v0);
-        store8_bf16(xb + (t + 8) * d + c0, v1);
-      }
+    // each warp takes rows t_begin + warp + 8k, kBatch at a time; the next
+    // batch is loaded while the current one is summed
+    constexpr int kBatch = 4;
+    float v[kBatch][8], vn[kBatch][8];
+    auto load_batch = [&](int64_t t0, float (&dst)[kBatch][8]) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        acc[e] += abs_pow<PK>(v0[e], p) + abs_pow<PK>(v1[e], p);
-        amax = fmaxf(amax, fmaxf(fabsf(v0[e]), fabsf(v1[e])));
-      }
-    }
-    for (; t < t_end; t += 8) {
-      float v0[8];
-      load8(X + t * d + c0, v0);
-      if (xh != nullptr) store8_f16(xh + t * d + c0, v0);
-      if (xb != nullptr) store8_bf16(xb + t * d + c0, v0);
+      for (int k = 0; k < kBatch; ++k) {
+        const int64_t t = t0 + 8 * k;
+        if (t < t_end) {
+          load8(X + t * d + c0, dst[k]);
+        } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        acc[e] += abs_pow<PK>(v0[e], p);
-        amax = fmaxf(amax, fabsf(v0[e]));
+          for (int e = 0; e < 8; ++e) dst[k][e] = 0.f;
+        }
       }
+    };
+    auto consume = [&](int64_t t0, const float(&buf)[kBatch][8]) {
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) {
+        const int64_t t = t0 + 8 * k;
+        if (t < t_end) {
+          if (xh != nullptr) store8_f16(xh + t * d + c0, buf[k]);
+          if (xb != nullptr) store8_bf16(xb + t * d + c0, buf[k]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc[e] += abs_pow<PK>(buf[k][e], p);
+          amax = fmaxf(amax, fabsf(buf[k][e]));
+        }
+      }
+    };
+    // ping-pong between two buffers (loop unrolled twice)
+    constexpr int kStep = 8 * kBatch;
+    int64_t t0 = t_begin + warp;
+    if (t0 < t_end) load_batch(t0, v);
+    for (; t0 < t_end; t0 += 2 * kStep) {
+      if (t0 + kStep < t_end) load_batch(t0 + kStep, vn);
+      consume(t0, v);
+      if (t0 + kStep >= t_end) break;
+      if (t0 + 2 * kStep < t_end) load_batch(t0 + 2 * kStep, v);
+      consume(t0 + kStep, vn);
     }
   }
   // the binary16 copy of X holds |x| <= 65504 only (NaN is caught by D)
@@ -157,8 +168,13 @@ __global__ void __launch_bounds__(kThreads) act_norm_kernel(
   __threadfence();
 
   if (c < d) {
+    // fixed order; up to 16 partials loaded at once (one L2 round trip)
+    double v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
     double tot = 0.0;
-    for (int64_t s = 0; s < splits; ++s) tot += __ldcg(partial + s * d + c);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) tot += v[k];
     double n;
     if (PK == 1) {
       n = tot;
@@ -211,12 +227,14 @@ cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, f
 }  // namespace
 
 void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split) {
+  // about two resident blocks per SM, and at most 16 splits so that the
+  // final merge is one batch of loads
   const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
-  const int64_t target = static_cast<int64_t>(num_sms) * 4;
+  const int64_t target = static_cast<int64_t>(num_sms) * 2;
   int64_t s = (target + ncb - 1) / ncb;
   const int64_t max_by_rows = (T + 31) / 32;  // at least 32 rows per split
   if (s > max_by_rows) s = max_by_rows;
-  if (s > 256) s = 256;
+  if (s > 16) s = 16;
   if (s < 1) s = 1;
   int64_t rps = (T + s - 1) / s;
   if (rps < 1) rps = 1;

@@ -48,6 +48,7 @@ struct GemmDev {
   const uint16_t* zeros;
   int group_shift;      // log2(group): groups are powers of two
   int64_t ngroups;      // K / group
+  int sz_shift;         // scales/zeros are loaded 2^sz_shift groups at a time (<= 8)
   int64_t K, M, T, K_tail;
   void* Y;
   int64_t ldy;
@@ -108,6 +109,78 @@ __device__ __forceinline__ void load_chunk(const GemmDev& g, int64_t row, int64_
   ck.z = __ldg(g.zeros + gi);
 }
 
+// Reads the packed codes of one 32-channel chunk from the K block's code
+// tile in shared memory (rows of cw words, first needed word at `off`).
+template <int BITS>
+__device__ __forceinline__ void read_codes_smem(uint32_t row_addr, int hf, CodeChunk& ck) {
+  if (BITS == 4) {
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(ck.w[0]), "=r"(ck.w[1]), "=r"(ck.w[2]), "=r"(ck.w[3])
+                 : "r"(row_addr + 16 * hf));
+  } else if (BITS == 2) {
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];"
+                 : "=r"(ck.w[0]), "=r"(ck.w[1])
+                 : "r"(row_addr + 8 * hf));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      asm volatile("ld.shared.b32 %0, [%1];" : "=r"(ck.w[i]) : "r"(row_addr + 12 * hf + 4 * i));
+  }
+}
+
+// Per-thread cache of one row's scales and zero points, 2^sz_shift groups
+// per load (the largest of 8, 4, 2, 1 that divides K/group, so every load is
+// aligned): `cur` holds group block gb, `nxt` the block after it, loaded
+// one block ahead so its latency is hidden.
+struct SZCache {
+  int64_t gb;
+  uint4 s_cur, z_cur, s_nxt, z_nxt;
+};
+
+__device__ __forceinline__ void sz_load(const GemmDev& g, int64_t row, int64_t gb, uint4& sv,
+                                        uint4& zv) {
+  sv = make_uint4(0u, 0u, 0u, 0u);
+  zv = sv;
+  const int64_t k0 = gb << g.sz_shift;
+  if (row >= g.M || k0 >= g.ngroups) return;
+  const int64_t i = row * g.ngroups + k0;
+  switch (g.sz_shift) {
+    case 3:
+      sv = __ldg(reinterpret_cast<const uint4*>(g.scales + i));
+      zv = __ldg(reinterpret_cast<const uint4*>(g.zeros + i));
+      break;
+    case 2: {
+      const uint2 a = __ldg(reinterpret_cast<const uint2*>(g.scales + i));
+      const uint2 b = __ldg(reinterpret_cast<const uint2*>(g.zeros + i));
+      sv.x = a.x; sv.y = a.y; zv.x = b.x; zv.y = b.y;
+      break;
+    }
+    case 1:
+      sv.x = __ldg(reinterpret_cast<const uint32_t*>(g.scales + i));
+      zv.x = __ldg(reinterpret_cast<const uint32_t*>(g.zeros + i));
+      break;
+    default:
+      sv.x = __ldg(g.scales + i);
+      zv.x = __ldg(g.zeros + i);
+  }
+}
+
+__device__ __forceinline__ uint16_t u16_at(const uint4& v, int idx) {
+  const int w = idx >> 1;
+  const uint32_t word = w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+  return static_cast<uint16_t>(word >> (16 * (idx & 1)));
+}
+
+// Scale and zero of group k (k lies in block gb or gb + 1 of the cache).
+__device__ __forceinline__ void sz_get(const GemmDev& g, const SZCache& c, int64_t k, uint16_t& sc,
+                                       uint16_t& ze) {
+  const int64_t blk = k >> g.sz_shift;
+  const int idx = static_cast<int>(k - (blk << g.sz_shift));
+  const bool in_cur = blk == c.gb;
+  sc = u16_at(in_cur ? c.s_cur : c.s_nxt, idx);
+  ze = u16_at(in_cur ? c.z_cur : c.z_nxt, idx);
+}
+
 // (1024 + q) in both halves of a half2 from two codes placed at bits [0, b)
 // and [16, 16 + b) of `bits`.  0x6400 is binary16 1024.0, whose unit in the
 // last place is 1, so OR-ing a code into the fraction adds it exactly.
@@ -166,22 +239,30 @@ __device__ __forceinline__ void dequant_chunk(uint32_t row_base, int rsw, int hf
   }
 }
 
-template <int BITS, int BM>
+// Words of packed codes per row that the TMA brings in for one K block
+// (INT3 reads a 16-byte-aligned window of 8 words that holds the 6 needed).
+template <int BITS>
+constexpr int code_tile_words() { return BITS == 2 ? 4 : 8; }
+
+template <int BITS, int BM, bool TC>
 __global__ void __launch_bounds__(kThreads, 1)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                    const GemmDev g) {
+                    const __grid_constant__ CUtensorMap tmC, const GemmDev g) {
   constexpr int kSub = BM / 128;                 // 128-row MMAs per K step
   constexpr int kATile = BM * kBK * 2;
+  constexpr int kCW = code_tile_words<BITS == 0 ? 4 : BITS>();
+  constexpr int kCTile = TC ? BM * kCW * 4 : 0;  // code tile of one K block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int BN = g.BN;
   const int stages = g.stages;
-  const int stage_bytes = kATile + BN * 128;
+  const int stage_bytes = kATile + BN * 128 + kCTile;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
   uint64_t* empty = full + kMaxStages;
-  uint64_t* accum = empty + kMaxStages;
+  uint64_t* cfull = empty + kMaxStages;
+  uint64_t* accum = cfull + kMaxStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accum + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -200,6 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < stages; ++s) {
       mbar_init(&full[s], 1 + kProducerWarps);
       mbar_init(&empty[s], 1);
+      mbar_init(&cfull[s], 1);
     }
     mbar_init(accum, 1);
     *abort_flag = 0;
@@ -208,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tmB0);
     if (BITS == 0) prefetch_tensormap(&tmA0);
+    if (TC) prefetch_tensormap(&tmC);
     if (kb_tail > 0) {
       prefetch_tensormap(&tmA1);
       prefetch_tensormap(&tmB1);
@@ -236,6 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* a_slot = smem + s * stage_bytes;
         uint8_t* b_slot = a_slot + kATile;
         if (kb < kb_main) {
+          if (TC) {
+            // code tile first: the producers wait for it, the MMA does not
+            const int32_t xw = BITS == 3 ? ((6 * kb) & ~3) : kb * kCW;
+            mbar_arrive_expect_tx(&cfull[s], kCTile);
+            tma_load_2d(&tmC, &cfull[s], b_slot + BN * 128, xw, static_cast<int32_t>(m0));
+          }
           const uint32_t bytes = BN * 128 + (BITS == 0 ? kATile : 0);
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(&tmB0, &full[s], b_slot, kb * kBK, static_cast<int32_t>(n0));
@@ -297,40 +386,98 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int rsw = r & 7;
     const uint32_t row_off = (r >> 7) * kSubTileBytes + (rl >> 3) * 1024 + (rl & 7) * 128;
     constexpr int LB = BITS == 0 ? 4 : BITS;
-    CodeChunk cur[kChunks], nxt[kChunks];
-    if (BITS != 0) {
-#pragma unroll
-      for (int c = 0; c < kChunks; ++c) load_chunk<LB>(g, m0 + r, 32 * (hf0 + c), cur[c]);
-    }
     int s = 0;
     uint32_t ph = 0;
-    for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
-      if (BITS != 0 && kb + 1 < kb_main) {
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c)
-          load_chunk<LB>(g, m0 + r, static_cast<int64_t>(kb + 1) * kBK + 32 * (hf0 + c), nxt[c]);
-      }
+    bool alive = true;
+    auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(&empty[s], ph ^ 1u, abort_flag) ? 1 : 0;
+      if (lane == 0) ok = mbar_wait(bar, parity, abort_flag) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) {
           *abort_flag = 1;
           set_flag(g.status, TTQ_FLAG_TIMEOUT);
         }
-        break;
+        alive = false;
       }
-      if (BITS != 0 && kb < kb_main) {
-        const uint32_t row_base = smem_addr(smem + s * stage_bytes) + row_off;
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c) {
-          dequant_chunk<LB>(row_base, rsw, hf0 + c, cur[c]);
-          cur[c] = nxt[c];
-        }
-        fence_proxy_async_smem();
-      }
+      return ok != 0;
+    };
+    auto next_stage = [&]() {
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
+      s = (s + 1 == stages) ? 0 : s + 1;
+      ph ^= (s == 0);
+    };
+    if (TC) {
+      // Codes arrive by TMA with the stage (cfull); scales and zeros come
+      // from the per-thread cache, two blocks of groups in registers.
+      SZCache cache;
+      cache.gb = 0;
+      if (BITS != 0) {
+        sz_load(g, m0 + r, 0, cache.s_cur, cache.z_cur);
+        sz_load(g, m0 + r, 1, cache.s_nxt, cache.z_nxt);
+      }
+      for (int kb = 0; kb < kb_total; ++kb) {
+        if (!wait_bar(&empty[s], ph ^ 1u)) break;
+        if (BITS != 0 && kb < kb_main) {
+          const int64_t col_first = static_cast<int64_t>(kb) * kBK + 32 * hf0;
+          while (((col_first >> g.group_shift) >> g.sz_shift) > cache.gb) {
+            // moved into the next block of groups: shift the cache by one
+            cache.gb += 1;
+            cache.s_cur = cache.s_nxt;
+            cache.z_cur = cache.z_nxt;
+            sz_load(g, m0 + r, cache.gb + 1, cache.s_nxt, cache.z_nxt);
+          }
+          if (!wait_bar(&cfull[s], ph)) break;
+          const uint8_t* stage_base = smem + s * stage_bytes;
+          const uint32_t crow = smem_addr(stage_base + kATile + BN * 128) + r * kCW * 4 +
+                                (BITS == 3 ? 4 * ((6 * kb) & 3) : 0);
+          const uint32_t row_base = smem_addr(stage_base) + row_off;
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) {
+            CodeChunk ck;
+            ck.w[3] = 0u;
+            read_codes_smem<LB>(crow, hf0 + c, ck);
+            sz_get(g, cache, (col_first + 32 * c) >> g.group_shift, ck.s, ck.z);
+            dequant_chunk<LB>(row_base, rsw, hf0 + c, ck);
+          }
+          fence_proxy_async_smem();
+        }
+        next_stage();
+      }
+    } else {
+      // Codes, scales and zeros loaded by each thread from global memory,
+      // three K blocks ahead; the ring is walked by a loop unrolled four
+      // times, so no register copy forces an early wait on a load in flight.
+      CodeChunk c0[kChunks], c1[kChunks], c2[kChunks], c3[kChunks];
+      auto load_kb = [&](int kbl, CodeChunk(&dst)[kChunks]) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          load_chunk<LB>(g, m0 + r, static_cast<int64_t>(kbl) * kBK + 32 * (hf0 + c), dst[c]);
+      };
+      if (BITS != 0) {
+        if (0 < kb_main) load_kb(0, c0);
+        if (1 < kb_main) load_kb(1, c1);
+        if (2 < kb_main) load_kb(2, c2);
+      }
+      // one K block: prefetch block kb + 3 into `pre`, dequantise `use`
+      auto step = [&](int kb, CodeChunk(&use)[kChunks], CodeChunk(&pre)[kChunks]) {
+        if (BITS != 0 && kb + 3 < kb_main) load_kb(kb + 3, pre);
+        if (!wait_bar(&empty[s], ph ^ 1u)) return;
+        if (BITS != 0 && kb < kb_main) {
+          const uint32_t row_base = smem_addr(smem + s * stage_bytes) + row_off;
+#pragma unroll
+          for (int c = 0; c < kChunks; ++c) dequant_chunk<LB>(row_base, rsw, hf0 + c, use[c]);
+          fence_proxy_async_smem();
+        }
+        next_stage();
+      };
+      for (int kb = 0; kb < kb_total && alive; kb += 4) {
+        step(kb, c0, c3);
+        if (kb + 1 < kb_total && alive) step(kb + 1, c1, c0);
+        if (kb + 2 < kb_total && alive) step(kb + 2, c2, c1);
+        if (kb + 3 < kb_total && alive) step(kb + 3, c3, c2);
+      }
     }
 
     int ok = 1;
@@ -381,14 +528,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BITS, int BM>
+template <int BITS, int BM, bool TC>
 cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStream_t stream) {
-  const int stage_bytes = BM * kBK * 2 + BN * 128;
+  const int stage_bytes =
+      BM * kBK * 2 + BN * 128 + (TC ? BM * code_tile_words<BITS == 0 ? 4 : BITS>() * 4 : 0);
   int stages = (kSmemLimit - 2048) / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages < 2) return cudaErrorInvalidValue;
   const int smem = stages * stage_bytes + 2048;
-  cudaError_t err = cudaFuncSetAttribute(ttq_gemm_kernel<BITS, BM>,
+  cudaError_t err = cudaFuncSetAttribute(ttq_gemm_kernel<BITS, BM, TC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   GemmDev g;
@@ -398,6 +546,8 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.group_shift = 0;
   while (a.group > 0 && (1 << (g.group_shift + 1)) <= a.group) ++g.group_shift;
   g.ngroups = a.group > 0 ? a.K / a.group : 0;
+  g.sz_shift = 0;
+  while (g.sz_shift < 3 && g.ngroups % (int64_t{2} << g.sz_shift) == 0) ++g.sz_shift;
   g.K = a.K;
   g.M = a.M;
   g.T = a.T;
@@ -410,18 +560,26 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.status = a.status;
   const dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM),
                   static_cast<unsigned>((a.T + BN - 1) / BN));
-  ttq_gemm_kernel<BITS, BM><<<grid, kThreads, smem, stream>>>(maps.a0, maps.b0, maps.a1, maps.b1, g);
+  ttq_gemm_kernel<BITS, BM, TC><<<grid, kThreads, smem, stream>>>(maps.a0, maps.b0, maps.a1,
+                                                                  maps.b1, maps.c0, g);
   return cudaGetLastError();
 }
 
 template <int BITS>
 cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, int BM,
                         cudaStream_t stream) {
-  if (BM == 256) return launch_tile<BITS, 256>(a, maps, BN, stream);
-  return launch_tile<BITS, 128>(a, maps, BN, stream);
+  if (BITS == 0) return launch_tile<BITS, 128, false>(a, maps, BN, stream);
+  if (a.codes_tma) {
+    if (BM == 256) return launch_tile<BITS, 256, true>(a, maps, BN, stream);
+    return launch_tile<BITS, 128, true>(a, maps, BN, stream);
+  }
+  if (BM == 256) return launch_tile<BITS, 256, false>(a, maps, BN, stream);
+  return launch_tile<BITS, 128, false>(a, maps, BN, stream);
 }
 
 }  // namespace
+
+int gemm_code_tile_words(int bits) { return bits == 2 ? 4 : 8; }
 
 int gemm_block_n(int64_t T) {
   if (T >= 256) return 256;

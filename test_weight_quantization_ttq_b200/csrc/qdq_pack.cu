@@ -12,11 +12,13 @@
 // can change a result.
 //
 // Layout of the work: a block owns a tile of `cw` consecutive input channels
-// and walks rows of W with a grid stride.  A thread owns 8 consecutive
-// channels (one 16-byte load of bf16 W), keeps their sqrt(D) in registers
-// for every row it visits, and the group's g/8 threads reduce min/max with
-// shuffles.  Codes are assembled into 32-bit words across the 4 lanes that
-// hold 32 consecutive codes (b words per 32 codes) and stored directly.
+// and walks rows of W with a grid stride.  A thread owns 16 consecutive
+// channels (two 16-byte loads of bf16 W), keeps their sqrt(D) in registers
+// for every row it visits, and the group's g/16 threads reduce min/max with
+// shuffles.  A lane's 16 codes fill two words (INT4), one word (INT2) or 48
+// bits (INT3: an even/odd lane pair makes 3 words).  Pairs of weights go
+// through the packed f32x2 multiply/add, which round each lane exactly like
+// the scalar operations.
 // The kernel is HBM-bound: it reads W once and writes d*b/8 + 4d/g bytes per
 // row.
 #include <type_traits>
@@ -29,128 +31,181 @@ namespace {
 
 constexpr int kThreads = 256;
 
-__device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
-  const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(src));
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+// 16 consecutive weights of one row, kept packed until they are used.
+template <typename WT>
+struct Raw16;
+template <>
+struct Raw16<__nv_bfloat16> {
+  uint4 v[2];
+};
+template <>
+struct Raw16<float> {
+  float4 v[4];
+};
+
+__device__ __forceinline__ void load16(const __nv_bfloat16* src, Raw16<__nv_bfloat16>& r) {
+  r.v[0] = __ldcs(reinterpret_cast<const uint4*>(src));
+  r.v[1] = __ldcs(reinterpret_cast<const uint4*>(src) + 1);
+}
+__device__ __forceinline__ void load16(const float* src, Raw16<float>& r) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.v[i] = __ldcs(reinterpret_cast<const float4*>(src) + i);
+}
+__device__ __forceinline__ void zero16(Raw16<__nv_bfloat16>& r) {
+  r.v[0] = r.v[1] = make_uint4(0u, 0u, 0u, 0u);
+}
+__device__ __forceinline__ void zero16(Raw16<float>& r) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) r.v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+__device__ __forceinline__ void unpack16(const Raw16<__nv_bfloat16>& r, float2 (&x)[8]) {
+  const uint32_t w[8] = {r.v[0].x, r.v[0].y, r.v[0].z, r.v[0].w, r.v[1].x, r.v[1].y, r.v[1].z, r.v[1].w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+__device__ __forceinline__ void unpack16(const Raw16<float>& r, float2 (&x)[8]) {
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    v[2 * i] = __uint_as_float(w[i] << 16);
-    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    x[2 * i] = make_float2(r.v[i].x, r.v[i].y);
+    x[2 * i + 1] = make_float2(r.v[i].z, r.v[i].w);
   }
 }
 
-__device__ __forceinline__ void load8(const float* src, float (&v)[8]) {
-  const float4 a = __ldcs(reinterpret_cast<const float4*>(src));
-  const float4 b = __ldcs(reinterpret_cast<const float4*>(src) + 1);
-  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-}
-
 template <typename WT, int BITS>
-__global__ void __launch_bounds__(kThreads) qdq_pack_kernel(
+__global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
     const WT* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D, int group,
     int cw, uint32_t* __restrict__ codes, __half* __restrict__ scales,
     __half* __restrict__ zeros, uint32_t* __restrict__ status) {
   constexpr int QMAX = (1 << BITS) - 1;
-  const int tpr = cw >> 3;            // threads per row of the tile
+  const int tpr = cw >> 4;            // threads per row of the tile (16 weights each)
   const int rpi = kThreads / tpr;     // rows per iteration of the block
   const int tx = threadIdx.x % tpr;
   const int ty = threadIdx.x / tpr;
   const int lane = threadIdx.x & 31;
-  const int gthreads = group >> 3;    // threads sharing one group (4..32)
-  const int64_t col = static_cast<int64_t>(blockIdx.x) * cw + tx * 8;
+  const int gthreads = group >> 4;    // threads sharing one group (2..16)
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * cw + tx * 16;
   const int64_t ngroups = d / group;
   const int64_t kgroup = col / group;  // this thread's group within the row
-  const int64_t wpr = d * BITS / 32;  // words per row
+  const int64_t wpr = d * BITS / 32;   // words per row
 
-  float h[8];
+  float2 h[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) h[e] = (D != nullptr) ? __fsqrt_rn(__ldg(D + col + e)) : 1.0f;
-  bool bad = false;
+  for (int i = 0; i < 8; ++i)
+    h[i] = D != nullptr ? make_float2(__fsqrt_rn(__ldg(D + col + 2 * i)), __fsqrt_rn(__ldg(D + col + 2 * i + 1)))
+                        : make_float2(1.f, 1.f);
+  float hchk = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) bad |= !(h[e] <= 3.402823466e38f);
-
+  for (int i = 0; i < 8; ++i) hchk += h[i].x + h[i].y;
+  bool bad = !(hchk <= 3.402823466e38f);
   bool ovf = false;
+
   // The loop bound is block-uniform so every lane takes part in the
-  // shuffles; rows past the end are computed on zeros and not stored.  Each
-  // iteration issues the loads of kRows rows before using any of them.
+  // shuffles; rows past the end are computed on zeros and not stored.  The
+  // next kRows rows are loaded while the current ones are quantised.
   constexpr int kRows = 4;
   const int64_t step = static_cast<int64_t>(gridDim.y) * rpi;
-  for (int64_t base = static_cast<int64_t>(blockIdx.y) * rpi; base < dp; base += kRows * step) {
-    float x[kRows][8];
+  const int64_t stride = kRows * step;
+  Raw16<WT> cur[kRows], nxt[kRows];
+  auto load_rows = [&](int64_t b, Raw16<WT>(&dst)[kRows]) {
 #pragma unroll
     for (int u = 0; u < kRows; ++u) {
-      const int64_t row = base + u * step + ty;
-      if (row < dp) {
-        load8(W + row * d + col, x[u]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
-      }
+      const int64_t row = b + u * step + ty;
+      if (row < dp) load16(W + row * d + col, dst[u]);
+      else zero16(dst[u]);
     }
+  };
+  // quantise the kRows rows held in `buf`, starting at row b
+  auto process = [&](int64_t b, const Raw16<WT>(&buf)[kRows]) {
+    const int64_t base = b;
 #pragma unroll
-    for (int u = 0; u < kRows; ++u) {
-      const int64_t row = base + u * step + ty;
-      const bool active = row < dp;
-      float mn = 0.f, mx = 0.f;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        x[u][e] = __fmul_rn(x[u][e], h[e]);
-        bad |= !(fabsf(x[u][e]) <= 3.402823466e38f);
-        mn = fminf(mn, x[u][e]);
-        mx = fmaxf(mx, x[u][e]);
+      for (int u = 0; u < kRows; ++u) {
+        const int64_t row = base + u * step + ty;
+        const bool active = row < dp;
+        float2 x[8];
+        unpack16(buf[u], x);
+        float2 sum2 = make_float2(0.f, 0.f);
+        float mn = 0.f, mx = 0.f;
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x[i].x = __fmul_rn(x[i].x, h[i].x);
+          x[i].y = __fmul_rn(x[i].y, h[i].y);
+          sum2 = __fadd2_rn(sum2, x[i]);  // NaN and Inf survive the sum
+          mn = fminf(mn, fminf(x[i].x, x[i].y));
+          mx = fmaxf(mx, fmaxf(x[i].x, x[i].y));
+        }
+        bad |= !(fabsf(sum2.x + sum2.y) <= 3.402823466e38f);
+        for (int o = gthreads >> 1; o > 0; o >>= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        float s32 = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
+        if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
+        const __half s16 = __float2half_ru(s32);
+        const float s = __half2float(s16);
+        const float inv = __fdiv_rn(1.0f, s);
+        const float zr = rintf(__fmul_rn(-mn, inv));
+        const int z = static_cast<int>(fminf(fmaxf(zr, 0.f), static_cast<float>(QMAX)));
+        // rint(x * inv): adding 1.5 * 2^23 rounds to an integer, ties to even,
+        // for |x * inv| < 2^22 (here |x * inv| <= 2^b); the integer is then read
+        // from the low fraction bits
+        const int zoff = z - 0x4B400000;
+        uint32_t lo = 0, hi = 0;  // codes 0-7 and 8-15 (INT3: 24 bits each)
+  #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float r0 = __fadd_rn(__fmul_rn(x[i].x, inv), 12582912.0f);
+          const float r1 = __fadd_rn(__fmul_rn(x[i].y, inv), 12582912.0f);
+          const int q0 = min(max(__float_as_int(r0) + zoff, 0), QMAX);
+          const int q1 = min(max(__float_as_int(r1) + zoff, 0), QMAX);
+          const uint32_t pair = static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << BITS);
+          if (i < 4) lo |= pair << (2 * BITS * i);
+          else hi |= pair << (2 * BITS * (i - 4));
+        }
+        if (active && (tx & (gthreads - 1)) == 0) {
+          scales[row * ngroups + kgroup] = s16;
+          zeros[row * ngroups + kgroup] = __int2half_rn(z);
+          // s (q - z) is formed in binary16 by the product: |q - z| <= 2^b - 1
+          ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QMAX) > 65504.f;
+        }
+        // the lane's 16 codes are 16*BITS bits at bit 16*BITS*(col/16)
+        if (BITS == 4) {
+          if (active) *reinterpret_cast<uint2*>(codes + row * wpr + (col >> 3)) = make_uint2(lo, hi);
+        } else if (BITS == 2) {
+          if (active) codes[row * wpr + (col >> 4)] = lo | (hi << 16);
+        } else {
+          // 48 bits per lane; an even/odd lane pair makes 3 words
+          const uint32_t a = lo | (hi << 24);  // bits 0-31
+          const uint32_t b = hi >> 8;          // bits 32-47
+          const uint32_t oa = __shfl_down_sync(0xffffffffu, a, 1);
+          const uint32_t ob = __shfl_down_sync(0xffffffffu, b, 1);
+          if (active && (tx & 1) == 0) {
+            uint32_t* dst = codes + row * wpr + (col >> 5) * 3;
+            dst[0] = a;
+            dst[1] = b | (oa << 16);
+            dst[2] = (oa >> 16) | (ob << 16);
+          }
+        }
       }
-      for (int o = gthreads >> 1; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      float s32 = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
-      if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
-      const __half s16 = __float2half_ru(s32);
-      const float s = __half2float(s16);
-      const float inv = __fdiv_rn(1.0f, s);
-      const float zr = rintf(__fmul_rn(-mn, inv));
-      const int z = static_cast<int>(fminf(fmaxf(zr, 0.f), static_cast<float>(QMAX)));
-      uint32_t packed = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        int q = __float2int_rn(__fmul_rn(x[u][e], inv)) + z;
-        q = min(max(q, 0), QMAX);
-        packed |= static_cast<uint32_t>(q) << (BITS * e);
-      }
-      if (active && (tx & (gthreads - 1)) == 0) {
-        scales[row * ngroups + kgroup] = s16;
-        zeros[row * ngroups + kgroup] = __int2half_rn(z);
-        // s (q - z) is formed in binary16 by the product: |q - z| <= 2^b - 1
-        ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QMAX) > 65504.f;
-      }
-      // 4 lanes hold 32 codes = BITS words; lane i of the quad writes word i.
-      const int qbase = lane & ~3;
-      const uint32_t v0 = __shfl_sync(0xffffffffu, packed, qbase + 0);
-      const uint32_t v1 = __shfl_sync(0xffffffffu, packed, qbase + 1);
-      const uint32_t v2 = __shfl_sync(0xffffffffu, packed, qbase + 2);
-      const uint32_t v3 = __shfl_sync(0xffffffffu, packed, qbase + 3);
-      const int qi = lane & 3;
-      if (active && qi < BITS) {
-        const unsigned __int128 stream =
-            static_cast<unsigned __int128>(v0) | (static_cast<unsigned __int128>(v1) << (8 * BITS)) |
-            (static_cast<unsigned __int128>(v2) << (16 * BITS)) |
-            (static_cast<unsigned __int128>(v3) << (24 * BITS));
-        const uint32_t word = static_cast<uint32_t>(stream >> (32 * qi));
-        const int64_t quad_col = col - (tx & 3) * 8;  // first channel of the quad
-        codes[row * wpr + (quad_col >> 5) * BITS + qi] = word;
-      }
-    }
+  };
+  // ping-pong between two buffers (loop unrolled twice): the loads for the
+  // next rows are in flight while the current ones are quantised
+  int64_t base = static_cast<int64_t>(blockIdx.y) * rpi;
+  if (base < dp) load_rows(base, cur);
+  for (; base < dp; base += 2 * stride) {
+    if (base + stride < dp) load_rows(base + stride, nxt);
+    process(base, cur);
+    if (base + stride >= dp) break;
+    if (base + 2 * stride < dp) load_rows(base + 2 * stride, cur);
+    process(base + stride, nxt);
   }
   if (__any_sync(0xffffffffu, ovf) && lane == 0)
     set_flag(status, TTQ_FLAG_NONFINITE | TTQ_FLAG_SCALE_OVERFLOW);
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_flag(status, TTQ_FLAG_NONFINITE);
 }
 
-// Largest tile width (a power of two in [32, 2048]) that divides d and is a
+// Largest tile width (a power of two in [32, 4096]) that divides d and is a
 // multiple of the group.
 int tile_width(int64_t d, int group) {
-  for (int c = 2048; c >= 32; c >>= 1)
+  for (int c = 4096; c >= 32; c >>= 1)
     if (c >= group && d % c == 0) return c;
   return group;
 }
@@ -160,9 +215,9 @@ cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bit
                      uint32_t* codes, uint16_t* scales, uint16_t* zeros, uint32_t* status,
                      int num_sms, cudaStream_t stream) {
   const int cw = tile_width(d, group);
-  const int rpi = kThreads / (cw >> 3);
+  const int rpi = kThreads / (cw >> 4);
   const int64_t gx = d / cw;
-  const int64_t want = static_cast<int64_t>(num_sms) * 8;
+  const int64_t want = static_cast<int64_t>(num_sms) * 2;  // two resident blocks per SM
   int64_t gy = (want + gx - 1) / gx;
   const int64_t max_gy = (dp + rpi - 1) / rpi;  // each block still takes >= 1 row
   if (gy > max_gy) gy = max_gy;
@@ -220,39 +275,54 @@ __global__ void __launch_bounds__(256) scale_to_f16_kernel(const T* __restrict__
 #pragma unroll
       for (int k = 0; k < 8; ++k) f[k] = 1.0f;
     }
-    for (int64_t t = blockIdx.y; t < T_; t += gridDim.y) {
-      float v[8];
-      if constexpr (sizeof(T) == 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(src + t * d + col));
-        const float4 b = __ldg(reinterpret_cast<const float4*>(src + t * d + col) + 1);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-      } else if constexpr (std::is_same<T, __half>::value) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + t * d + col));
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+    constexpr int kRows = 4;  // rows loaded before any is converted
+    for (int64_t t0 = blockIdx.y; t0 < T_; t0 += static_cast<int64_t>(gridDim.y) * kRows) {
+      uint4 raw[kRows][2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
-          v[2 * k] = f2.x;
-          v[2 * k + 1] = f2.y;
-        }
-      } else {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + t * d + col));
-        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          v[2 * k] = __uint_as_float(w[k] << 16);
-          v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+      for (int u = 0; u < kRows; ++u) {
+        const int64_t t = t0 + static_cast<int64_t>(u) * gridDim.y;
+        if (t < T_) {
+          const uint4* p = reinterpret_cast<const uint4*>(src + t * d + col);
+          raw[u][0] = __ldcs(p);
+          if constexpr (sizeof(T) == 4) raw[u][1] = __ldcs(p + 1);
         }
       }
-      __half2 h[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float a = v[2 * k] * f[2 * k];
-        const float b = v[2 * k + 1] * f[2 * k + 1];
-        h[k] = __floats2half2_rn(a, b);
-        out_of_range |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
+      for (int u = 0; u < kRows; ++u) {
+        const int64_t t = t0 + static_cast<int64_t>(u) * gridDim.y;
+        if (t >= T_) continue;
+        float v[8];
+        if constexpr (sizeof(T) == 4) {
+          v[0] = __uint_as_float(raw[u][0].x); v[1] = __uint_as_float(raw[u][0].y);
+          v[2] = __uint_as_float(raw[u][0].z); v[3] = __uint_as_float(raw[u][0].w);
+          v[4] = __uint_as_float(raw[u][1].x); v[5] = __uint_as_float(raw[u][1].y);
+          v[6] = __uint_as_float(raw[u][1].z); v[7] = __uint_as_float(raw[u][1].w);
+        } else if constexpr (std::is_same<T, __half>::value) {
+          const uint32_t w[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+            v[2 * k] = f2.x;
+            v[2 * k + 1] = f2.y;
+          }
+        } else {
+          const uint32_t w[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            v[2 * k] = __uint_as_float(w[k] << 16);
+            v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+          }
+        }
+        __half2 h[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float a = v[2 * k] * f[2 * k];
+          const float b = v[2 * k + 1] * f[2 * k + 1];
+          h[k] = __floats2half2_rn(a, b);
+          out_of_range |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
+        }
+        *reinterpret_cast<uint4*>(dst + t * d + col) = *reinterpret_cast<uint4*>(h);
       }
-      *reinterpret_cast<uint4*>(dst + t * d + col) = *reinterpret_cast<uint4*>(h);
     }
   }
   if (__any_sync(0xffffffffu, out_of_range) && (threadIdx.x & 31) == 0)

@@ -124,6 +124,21 @@ bool encode_16bit(CUtensorMap* m, const void* base, bool f16, int64_t inner, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Packed codes [rows][wpr] as uint32, loaded as box_rows x box_words tiles
+// without swizzle.  The row stride must be a multiple of 16 bytes.
+bool encode_codes(CUtensorMap* m, const uint32_t* base, int64_t wpr, int64_t rows, int box_words,
+                  int box_rows) {
+  EncodeFn enc = get_encode();
+  if (enc == nullptr || wpr < 1 || rows < 1 || (wpr * 4) % 16 != 0) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(wpr) * 4};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_words), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_ERR_CUDA; }
 
 uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
@@ -146,6 +161,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
       return TTQ_ERR_CUDA;
     m.a1 = m.a0;
     m.b1 = m.b0;
+    m.c0 = m.b0;
     GemmArgs a;
     a.bits = 0;
     a.K = d;
@@ -171,7 +187,12 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     m.a1 = m.b0;
     m.b1 = m.b0;
   }
+  // the code tile comes in by TMA when the code rows are 16-byte strided
+  const int64_t wpr = d * bits / 32;
+  const bool codes_tma = encode_codes(&m.c0, codes, wpr, dp, gemm_code_tile_words(bits), bm);
+  if (!codes_tma) m.c0 = m.b0;
   GemmArgs a;
+  a.codes_tma = codes_tma;
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;

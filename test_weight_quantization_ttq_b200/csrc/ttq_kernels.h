@@ -59,6 +59,7 @@ struct GemmArgs {
   int64_t ldy = 0;
   bool y_f32 = false;
   uint32_t* status = nullptr;
+  bool codes_tma = false;  // codes tile loaded by TMA (maps.c0); else per-thread loads
 };
 
 struct GemmMaps {
@@ -66,7 +67,11 @@ struct GemmMaps {
   CUtensorMap b0;  // binary16 X D^(-1/2) [T][K] with codes (bits != 0); bf16 X in the plain mode
   CUtensorMap a1;  // low-rank B [M][r] bf16
   CUtensorMap b1;  // A X [T][r] bf16
+  CUtensorMap c0;  // packed codes [M][K*bits/32] uint32, box gemm_code_tile_words x block_m
 };
+
+// Words per row of the code tile one K block of 64 channels needs.
+int gemm_code_tile_words(int bits);
 
 // Tile width along the tokens for T tokens.
 int gemm_block_n(int64_t T);
