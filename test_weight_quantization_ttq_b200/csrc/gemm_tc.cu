@@ -53,6 +53,7 @@ struct GemmDev {
   void* Y;
   int64_t ldy;
   int y_f32;
+  int y_tma;            // bf16 Y written by one TMA store per CTA (tmY)
   int BN;
   int stages;
   uint32_t* status;
@@ -248,7 +249,8 @@ template <int BITS, int BM, bool TC>
 __global__ void __launch_bounds__(kThreads, 1)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                    const __grid_constant__ CUtensorMap tmC, const GemmDev g) {
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
+                    const GemmDev g) {
   constexpr int kSub = BM / 128;                 // 128-row MMAs per K step
   constexpr int kATile = BM * kBK * 2;
   constexpr int kCW = code_tile_words<BITS == 0 ? 4 : BITS>();
@@ -288,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
+    if (g.y_tma) prefetch_tensormap(&tmY);
     prefetch_tensormap(&tmB0);
     if (BITS == 0) prefetch_tensormap(&tmA0);
     if (TC) prefetch_tensormap(&tmC);
@@ -496,25 +499,60 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int acc = BM == 128 ? 0 : wg;
     const int ch0 = BM == 128 ? wg : 0;
     const int chs = BM == 128 ? 2 : 1;
-    const int64_t j = m0 + acc * 128 + q * 32 + lane;
+    const int jl = acc * 128 + q * 32 + lane;  // row of W within the tile
+    const int64_t j = m0 + jl;
     const int nchunks = BN / 16;
-    const bool store = ok && (*abort_flag == 0) && j < g.M;
-    for (int ch = ch0; ch < nchunks; ch += chs) {
-      uint32_t rr[16];
-      tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
-      tmem_load_wait();
-      if (store) {
-        const int64_t t0 = n0 + ch * 16;
-        if (g.y_f32) {
-          float* Y = static_cast<float*>(g.Y);
+    const bool good = ok && (*abort_flag == 0);
+    if (g.y_tma) {
+      // bf16 Y: stage the BN x BM tile [t][j] in the (now idle) pipeline
+      // memory, then one TMA store.  Lanes 2k and 2k+1 swap one value per
+      // token pair so each writes a bf16 pair (j, j+1) of one token.
+      const uint32_t tile = smem_addr(smem);
+      const bool odd = lane & 1;
+      for (int ch = ch0; ch < nchunks; ch += chs) {
+        uint32_t rr[16];
+        tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
+        tmem_load_wait();
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __uint_as_float(rr[i]);
-        } else {
-          __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(g.Y);
+        for (int i = 0; i < 16; i += 2) {
+          // even lane keeps token i and receives its partner's token i;
+          // odd lane keeps token i+1 and receives its partner's token i+1
+          const uint32_t give = odd ? rr[i] : rr[i + 1];
+          const uint32_t got = __shfl_xor_sync(0xffffffffu, give, 1);
+          const float lo = __uint_as_float(odd ? got : rr[i]);
+          const float hi = __uint_as_float(odd ? rr[i + 1] : got);
+          __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
+          const int tl = ch * 16 + i + (odd ? 1 : 0);
+          const uint32_t addr = tile + (tl * BM + (jl & ~1)) * 2;
+          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(*reinterpret_cast<uint32_t*>(&pr))
+                       : "memory");
+        }
+      }
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+      if (threadIdx.x == 64 && good) {
+        tma_store_2d(&tmY, tile, static_cast<int32_t>(m0), static_cast<int32_t>(n0));
+        tma_store_commit_and_wait();
+      }
+    } else {
+      const bool store = good && j < g.M;
+      for (int ch = ch0; ch < nchunks; ch += chs) {
+        uint32_t rr[16];
+        tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
+        tmem_load_wait();
+        if (store) {
+          const int64_t t0 = n0 + ch * 16;
+          if (g.y_f32) {
+            float* Y = static_cast<float*>(g.Y);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __float2bfloat16_rn(__uint_as_float(rr[i]));
+            for (int i = 0; i < 16; ++i)
+              if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __uint_as_float(rr[i]);
+          } else {
+            __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(g.Y);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __float2bfloat16_rn(__uint_as_float(rr[i]));
+          }
         }
       }
     }
@@ -555,13 +593,15 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.Y = a.Y;
   g.ldy = a.ldy;
   g.y_f32 = a.y_f32 ? 1 : 0;
+  // the staged Y tile (BN x BM bf16) must fit in the pipeline memory
+  g.y_tma = (a.y_tma && !a.y_f32 && BN * BM * 2 <= stages * stage_bytes) ? 1 : 0;
   g.BN = BN;
   g.stages = stages;
   g.status = a.status;
   const dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM),
                   static_cast<unsigned>((a.T + BN - 1) / BN));
   ttq_gemm_kernel<BITS, BM, TC><<<grid, kThreads, smem, stream>>>(maps.a0, maps.b0, maps.a1,
-                                                                  maps.b1, maps.c0, g);
+                                                                  maps.b1, maps.c0, maps.y, g);
   return cudaGetLastError();
 }
 

@@ -139,6 +139,21 @@ bool encode_codes(CUtensorMap* m, const uint32_t* base, int64_t wpr, int64_t row
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// bf16 Y [rows][cols] (row stride cols), stored as box_rows x box_cols tiles
+// without swizzle.
+bool encode_y_bf16(CUtensorMap* m, void* base, int64_t cols, int64_t rows, int box_cols,
+                   int box_rows) {
+  EncodeFn enc = get_encode();
+  if (enc == nullptr || cols < 1 || rows < 1 || (cols * 2) % 16 != 0) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_ERR_CUDA; }
 
 uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
@@ -162,6 +177,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     m.a1 = m.a0;
     m.b1 = m.b0;
     m.c0 = m.b0;
+    m.y = m.b0;
     GemmArgs a;
     a.bits = 0;
     a.K = d;
@@ -191,8 +207,12 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   const int64_t wpr = d * bits / 32;
   const bool codes_tma = encode_codes(&m.c0, codes, wpr, dp, gemm_code_tile_words(bits), bm);
   if (!codes_tma) m.c0 = m.b0;
+  // bf16 Y goes out through one TMA store per tile when its rows are 16-byte strided
+  const bool y_tma = !y_f32 && dp % 8 == 0 && encode_y_bf16(&m.y, Y, dp, T, bm, bn);
+  if (!y_tma) m.y = m.b0;
   GemmArgs a;
   a.codes_tma = codes_tma;
+  a.y_tma = y_tma;
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;

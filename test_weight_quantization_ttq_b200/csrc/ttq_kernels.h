@@ -60,6 +60,7 @@ struct GemmArgs {
   bool y_f32 = false;
   uint32_t* status = nullptr;
   bool codes_tma = false;  // codes tile loaded by TMA (maps.c0); else per-thread loads
+  bool y_tma = false;      // bf16 Y stored by TMA (maps.y, box block_m x block_n)
 };
 
 struct GemmMaps {
@@ -68,6 +69,7 @@ struct GemmMaps {
   CUtensorMap a1;  // low-rank B [M][r] bf16
   CUtensorMap b1;  // A X [T][r] bf16
   CUtensorMap c0;  // packed codes [M][K*bits/32] uint32, box gemm_code_tile_words x block_m
+  CUtensorMap y;   // bf16 Y [T][ldy], box block_m x block_n, no swizzle
 };
 
 // Words per row of the code tile one K block of 64 channels needs.
