@@ -14,10 +14,11 @@
 //               and for the low-rank tail also the A slot.
 //   warp 1      allocates tensor memory; one lane issues the MMAs and
 //               commits each stage back to its "empty" barrier.
-//   warps 2-9   dequantise packed codes straight into the A slot, written in
-//               the same 128-byte-swizzled K-major layout the TMA produces,
-//               then (after the last stage) read the accumulator out of
-//               tensor memory and store Y.
+//   warps 2..   two threads per tile row (8 or 16 warps) dequantise packed
+//               codes straight into the A slot, written in the same
+//               128-byte-swizzled K-major layout the TMA produces, then
+//               (after the last stage) read the accumulator out of tensor
+//               memory and store Y.
 // The factor D^(-1/2) of W_hat is carried by the B operand, which arrives
 // as binary16 X D^(-1/2); the A operand is s (q - z), built in binary16 with
 // integer-free bit tricks ((1024 + q) from the code bits, minus (1024 + z),
@@ -37,8 +38,10 @@ namespace {
 
 constexpr int kBK = 64;                        // 16-bit elements per 128-byte row
 constexpr int kSubTileBytes = 128 * kBK * 2;   // one 128-row operand tile: 16 KiB
-constexpr int kThreads = 320;
-constexpr int kProducerWarps = 8;
+// Threads of a CTA: warp 0 (TMA), warp 1 (MMA), then two producer /
+// epilogue threads per row of the tile.
+template <int BM>
+constexpr int cta_threads() { return 64 + 2 * BM; }
 constexpr int kMaxStages = 8;
 constexpr int kSmemLimit = 232448;             // 227 KiB opt-in per block
 
@@ -246,12 +249,13 @@ template <int BITS>
 constexpr int code_tile_words() { return BITS == 2 ? 4 : 8; }
 
 template <int BITS, int BM, bool TC>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(cta_threads<BM>(), 1)
     ttq_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmY,
                     const GemmDev g) {
   constexpr int kSub = BM / 128;                 // 128-row MMAs per K step
+  constexpr int kProducerWarps = BM / 16;        // 2 threads per tile row
   constexpr int kATile = BM * kBK * 2;
   constexpr int kCW = code_tile_words<BITS == 0 ? 4 : BITS>();
   constexpr int kCTile = TC ? BM * kCW * 4 : 0;  // code tile of one K block
@@ -377,14 +381,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------- dequant producers + epilogue
-    // BM = 128: thread pt owns row pt % 128 and the 32-channel half pt / 128
-    // of each K block; BM = 256: row pt and both halves.  A warp thus writes
-    // 32 consecutive rows of one 16-byte chunk column: conflict-free.  The
-    // next K block's operands are loaded before waiting on this one.
-    const int pt = threadIdx.x - 64;  // 0..255
-    const int r = BM == 128 ? (pt & 127) : pt;
-    constexpr int kChunks = BM == 128 ? 1 : 2;
-    const int hf0 = BM == 128 ? (pt >> 7) : 0;
+    // Thread pt owns row pt % BM and the 32-channel half pt / BM of each K
+    // block.  A warp thus writes 32 consecutive rows of one 16-byte chunk
+    // column: conflict-free.
+    const int pt = threadIdx.x - 64;  // 0 .. 2*BM-1
+    const int r = pt % BM;
+    constexpr int kChunks = 1;
+    const int hf0 = pt / BM;
     const int rl = r & 127;
     const int rsw = r & 7;
     const uint32_t row_off = (r >> 7) * kSubTileBytes + (rl >> 3) * 1024 + (rl & 7) * 128;
@@ -495,10 +498,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // two warps of a lane quadrant split the columns; BM = 256: warps 2-5
     // read accumulator 0 (rows 0-127), warps 6-9 accumulator 1.
     const int q = warp & 3;
+    // lane quadrant q = warp % 4 holds BM/64 warps: one per accumulator and
+    // per half of the token chunks
     const int wg = (warp - 2) >> 2;
-    const int acc = BM == 128 ? 0 : wg;
-    const int ch0 = BM == 128 ? wg : 0;
-    const int chs = BM == 128 ? 2 : 1;
+    const int acc = wg % kSub;
+    const int ch0 = wg / kSub;
+    const int chs = 2;
     const int jl = acc * 128 + q * 32 + lane;  // row of W within the tile
     const int64_t j = m0 + jl;
     const int nchunks = BN / 16;
@@ -529,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+      asm volatile("bar.sync 1, %0;" ::"n"(2 * BM) : "memory");  // the epilogue warps
       if (threadIdx.x == 64 && good) {
         tma_store_2d(&tmY, tile, static_cast<int32_t>(m0), static_cast<int32_t>(n0));
         tma_store_commit_and_wait();
@@ -600,7 +605,7 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.status = a.status;
   const dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM),
                   static_cast<unsigned>((a.T + BN - 1) / BN));
-  ttq_gemm_kernel<BITS, BM, TC><<<grid, kThreads, smem, stream>>>(maps.a0, maps.b0, maps.a1,
+  ttq_gemm_kernel<BITS, BM, TC><<<grid, cta_threads<BM>(), smem, stream>>>(maps.a0, maps.b0, maps.a1,
                                                                   maps.b1, maps.c0, maps.y, g);
   return cudaGetLastError();
 }
