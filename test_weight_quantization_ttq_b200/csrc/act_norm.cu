@@ -84,6 +84,8 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
     __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
   __shared__ double red[8][kChannelsPerBlock + 2];
   __shared__ int is_last;
+  allow_dependents_launch();
+  grid_dependency_wait();
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -199,29 +201,28 @@ template <typename XT, int PK>
 cudaError_t launch_typed(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
                          int64_t splits, int64_t rows_per_split, double* partial,
                          uint32_t* counters, float* D, float* Dr, void* xh, void* xb,
-                         uint32_t* status, cudaStream_t stream) {
+                         uint32_t* status, cudaStream_t stream, bool pdl) {
   const dim3 grid(static_cast<unsigned>((d + kChannelsPerBlock - 1) / kChannelsPerBlock),
                   static_cast<unsigned>(splits));
-  act_norm_kernel<XT, PK><<<grid, kThreads, 0, stream>>>(
-      X, d, T, static_cast<double>(p), static_cast<double>(lambda), static_cast<double>(alpha), splits,
-      rows_per_split, partial, counters, D, Dr, static_cast<__half*>(xh),
-      static_cast<__nv_bfloat16*>(xb), status);
-  return cudaGetLastError();
+  return launch_kernel(act_norm_kernel<XT, PK>, grid, dim3(kThreads), 0, stream, pdl, X, d, T,
+                       static_cast<double>(p), static_cast<double>(lambda),
+                       static_cast<double>(alpha), splits, rows_per_split, partial, counters, D,
+                       Dr, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
 }
 
 template <typename XT>
 cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
                      int64_t splits, int64_t rows_per_split, double* partial, uint32_t* counters,
                      float* D, float* Dr, void* xh, void* xb, uint32_t* status,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool pdl) {
   if (p == 1.0f)
     return launch_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                               counters, D, Dr, xh, xb, status, stream);
+                               counters, D, Dr, xh, xb, status, stream, pdl);
   if (p == 2.0f)
     return launch_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                               counters, D, Dr, xh, xb, status, stream);
+                               counters, D, Dr, xh, xb, status, stream, pdl);
   return launch_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                             counters, D, Dr, xh, xb, status, stream);
+                             counters, D, Dr, xh, xb, status, stream, pdl);
 }
 
 }  // namespace
@@ -247,12 +248,12 @@ void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* 
 cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                             float lambda, float alpha, int64_t splits, int64_t rows_per_split,
                             double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
-                            void* xb, uint32_t* status, cudaStream_t stream) {
+                            void* xb, uint32_t* status, cudaStream_t stream, bool pdl) {
   if (x_f32)
     return launch_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits, rows_per_split,
-                    partial, counters, D, Dr, xh, xb, status, stream);
+                    partial, counters, D, Dr, xh, xb, status, stream, pdl);
   return launch_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
-                  rows_per_split, partial, counters, D, Dr, xh, nullptr, status, stream);
+                  rows_per_split, partial, counters, D, Dr, xh, nullptr, status, stream, pdl);
 }
 
 }  // namespace ttq

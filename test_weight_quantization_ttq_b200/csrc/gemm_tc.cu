@@ -311,6 +311,10 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_holder;
+  // everything above overlaps the previous kernel; its outputs (codes, X)
+  // are read only after this
+  allow_dependents_launch();
+  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -572,7 +576,8 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
 }
 
 template <int BITS, int BM, bool TC>
-cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStream_t stream) {
+cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStream_t stream,
+                        bool pdl) {
   const int stage_bytes =
       BM * kBK * 2 + BN * 128 + (TC ? BM * code_tile_words<BITS == 0 ? 4 : BITS>() * 4 : 0);
   int stages = (kSmemLimit - 2048) / stage_bytes;
@@ -605,21 +610,20 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.status = a.status;
   const dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM),
                   static_cast<unsigned>((a.T + BN - 1) / BN));
-  ttq_gemm_kernel<BITS, BM, TC><<<grid, cta_threads<BM>(), smem, stream>>>(maps.a0, maps.b0, maps.a1,
-                                                                  maps.b1, maps.c0, maps.y, g);
-  return cudaGetLastError();
+  return launch_kernel(ttq_gemm_kernel<BITS, BM, TC>, grid, dim3(cta_threads<BM>()), smem, stream,
+                       pdl, maps.a0, maps.b0, maps.a1, maps.b1, maps.c0, maps.y, g);
 }
 
 template <int BITS>
 cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, int BM,
-                        cudaStream_t stream) {
-  if (BITS == 0) return launch_tile<BITS, 128, false>(a, maps, BN, stream);
+                        cudaStream_t stream, bool pdl) {
+  if (BITS == 0) return launch_tile<BITS, 128, false>(a, maps, BN, stream, pdl);
   if (a.codes_tma) {
-    if (BM == 256) return launch_tile<BITS, 256, true>(a, maps, BN, stream);
-    return launch_tile<BITS, 128, true>(a, maps, BN, stream);
+    if (BM == 256) return launch_tile<BITS, 256, true>(a, maps, BN, stream, pdl);
+    return launch_tile<BITS, 128, true>(a, maps, BN, stream, pdl);
   }
-  if (BM == 256) return launch_tile<BITS, 256, false>(a, maps, BN, stream);
-  return launch_tile<BITS, 128, false>(a, maps, BN, stream);
+  if (BM == 256) return launch_tile<BITS, 256, false>(a, maps, BN, stream, pdl);
+  return launch_tile<BITS, 128, false>(a, maps, BN, stream, pdl);
 }
 
 }  // namespace
@@ -646,19 +650,19 @@ int gemm_block_m(int bits, int64_t M, int64_t T, int block_n, int num_sms) {
 }
 
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,
-                                int block_m, cudaStream_t stream) {
+                                int block_m, cudaStream_t stream, bool pdl) {
   if (args.M == 0 || args.T == 0) return cudaSuccess;
   if (block_n % 16 != 0 || block_n < 16 || block_n > 256) return cudaErrorInvalidValue;
   if (block_m != 128 && !(block_m == 256 && args.bits != 0)) return cudaErrorInvalidValue;
   switch (args.bits) {
     case 0:
-      return launch_bits<0>(args, maps, block_n, 128, stream);
+      return launch_bits<0>(args, maps, block_n, 128, stream, pdl);
     case 2:
-      return launch_bits<2>(args, maps, block_n, block_m, stream);
+      return launch_bits<2>(args, maps, block_n, block_m, stream, pdl);
     case 3:
-      return launch_bits<3>(args, maps, block_n, block_m, stream);
+      return launch_bits<3>(args, maps, block_n, block_m, stream, pdl);
     case 4:
-      return launch_bits<4>(args, maps, block_n, block_m, stream);
+      return launch_bits<4>(args, maps, block_n, block_m, stream, pdl);
     default:
       return cudaErrorInvalidValue;
   }

@@ -87,6 +87,24 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
   const int64_t ngroups = d / group;
   const int64_t kgroup = col / group;  // this thread's group within the row
   const int64_t wpr = d * BITS / 32;   // words per row
+  allow_dependents_launch();
+
+  // the first rows of W do not depend on the previous kernel: load them
+  // before waiting for it (D does)
+  constexpr int kRows = 4;
+  const int64_t step = static_cast<int64_t>(gridDim.y) * rpi;
+  const int64_t stride = kRows * step;
+  Raw16<WT> cur[kRows], nxt[kRows];
+  auto load_rows = [&](int64_t b, Raw16<WT>(&dst)[kRows]) {
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      const int64_t row = b + u * step + ty;
+      if (row < dp) load16(W + row * d + col, dst[u]);
+      else zero16(dst[u]);
+    }
+  };
+  if (static_cast<int64_t>(blockIdx.y) * rpi < dp) load_rows(static_cast<int64_t>(blockIdx.y) * rpi, cur);
+  grid_dependency_wait();
 
   float2 h[8];
 #pragma unroll
@@ -102,18 +120,6 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
   // The loop bound is block-uniform so every lane takes part in the
   // shuffles; rows past the end are computed on zeros and not stored.  The
   // next kRows rows are loaded while the current ones are quantised.
-  constexpr int kRows = 4;
-  const int64_t step = static_cast<int64_t>(gridDim.y) * rpi;
-  const int64_t stride = kRows * step;
-  Raw16<WT> cur[kRows], nxt[kRows];
-  auto load_rows = [&](int64_t b, Raw16<WT>(&dst)[kRows]) {
-#pragma unroll
-    for (int u = 0; u < kRows; ++u) {
-      const int64_t row = b + u * step + ty;
-      if (row < dp) load16(W + row * d + col, dst[u]);
-      else zero16(dst[u]);
-    }
-  };
   // quantise the kRows rows held in `buf`, starting at row b
   auto process = [&](int64_t b, const Raw16<WT>(&buf)[kRows]) {
     const int64_t base = b;
@@ -189,7 +195,6 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
   // ping-pong between two buffers (loop unrolled twice): the loads for the
   // next rows are in flight while the current ones are quantised
   int64_t base = static_cast<int64_t>(blockIdx.y) * rpi;
-  if (base < dp) load_rows(base, cur);
   for (; base < dp; base += 2 * stride) {
     if (base + stride < dp) load_rows(base + stride, nxt);
     process(base, cur);
@@ -213,7 +218,7 @@ int tile_width(int64_t d, int group) {
 template <typename WT>
 cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bits, int group,
                      uint32_t* codes, uint16_t* scales, uint16_t* zeros, uint32_t* status,
-                     int num_sms, cudaStream_t stream) {
+                     int num_sms, cudaStream_t stream, bool pdl) {
   const int cw = tile_width(d, group);
   const int rpi = kThreads / (cw >> 4);
   const int64_t gx = d / cw;
@@ -228,18 +233,17 @@ cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bit
   __half* z = reinterpret_cast<__half*>(zeros);
   switch (bits) {
     case 2:
-      qdq_pack_kernel<WT, 2><<<grid, kThreads, 0, stream>>>(W, dp, d, D, group, cw, codes, s, z, status);
-      break;
+      return launch_kernel(qdq_pack_kernel<WT, 2>, grid, dim3(kThreads), 0, stream, pdl, W, dp, d, D,
+                           group, cw, codes, s, z, status);
     case 3:
-      qdq_pack_kernel<WT, 3><<<grid, kThreads, 0, stream>>>(W, dp, d, D, group, cw, codes, s, z, status);
-      break;
+      return launch_kernel(qdq_pack_kernel<WT, 3>, grid, dim3(kThreads), 0, stream, pdl, W, dp, d, D,
+                           group, cw, codes, s, z, status);
     case 4:
-      qdq_pack_kernel<WT, 4><<<grid, kThreads, 0, stream>>>(W, dp, d, D, group, cw, codes, s, z, status);
-      break;
+      return launch_kernel(qdq_pack_kernel<WT, 4>, grid, dim3(kThreads), 0, stream, pdl, W, dp, d, D,
+                           group, cw, codes, s, z, status);
     default:
       return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 __global__ void to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* __restrict__ dst,
@@ -265,6 +269,8 @@ __global__ void __launch_bounds__(256) scale_to_f16_kernel(const T* __restrict__
                                                            int64_t d, uint32_t* __restrict__ status) {
   const int64_t col = (static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x) * 8;
   bool out_of_range = false;
+  allow_dependents_launch();
+  grid_dependency_wait();  // Dr comes from the previous kernel
   if (col < d) {
     float f[8];
     if (Dr != nullptr) {
@@ -333,35 +339,34 @@ __global__ void __launch_bounds__(256) scale_to_f16_kernel(const T* __restrict__
 
 cudaError_t launch_scale_to_f16(const void* src, int src_kind, const float* Dr, void* dst,
                                 int64_t T, int64_t d, uint32_t* status, int num_sms,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, bool pdl) {
   if (T == 0 || d == 0) return cudaSuccess;
   const int64_t gx = (d / 8 + 255) / 256;
   int64_t gy = (static_cast<int64_t>(num_sms) * 8 + gx - 1) / gx;
   if (gy > T) gy = T;
   if (gy > 65535) gy = 65535;
   const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  __half* out = static_cast<__half*>(dst);
   if (src_kind == kSrcF32)
-    scale_to_f16_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(src), Dr,
-                                                         static_cast<__half*>(dst), T, d, status);
-  else if (src_kind == kSrcF16)
-    scale_to_f16_kernel<__half><<<grid, 256, 0, stream>>>(static_cast<const __half*>(src), Dr,
-                                                          static_cast<__half*>(dst), T, d, status);
-  else
-    scale_to_f16_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(src), Dr, static_cast<__half*>(dst), T, d, status);
-  return cudaGetLastError();
+    return launch_kernel(scale_to_f16_kernel<float>, grid, dim3(256), 0, stream, pdl,
+                         static_cast<const float*>(src), Dr, out, T, d, status);
+  if (src_kind == kSrcF16)
+    return launch_kernel(scale_to_f16_kernel<__half>, grid, dim3(256), 0, stream, pdl,
+                         static_cast<const __half*>(src), Dr, out, T, d, status);
+  return launch_kernel(scale_to_f16_kernel<__nv_bfloat16>, grid, dim3(256), 0, stream, pdl,
+                       static_cast<const __nv_bfloat16*>(src), Dr, out, T, d, status);
 }
 
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,
                             uint16_t* zeros, uint32_t* status, int num_sms,
-                            cudaStream_t stream) {
+                            cudaStream_t stream, bool pdl) {
   if (dp == 0) return cudaSuccess;
   if (w_f32)
     return launch_w(static_cast<const float*>(W), dp, d, D, bits, group, codes, scales, zeros,
-                    status, num_sms, stream);
+                    status, num_sms, stream, pdl);
   return launch_w(static_cast<const __nv_bfloat16*>(W), dp, d, D, bits, group, codes, scales,
-                  zeros, status, num_sms, stream);
+                  zeros, status, num_sms, stream, pdl);
 }
 
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {

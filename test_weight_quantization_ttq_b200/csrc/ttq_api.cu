@@ -164,7 +164,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
                     const void* Xh, const void* Xb, const void* Ab,
                     const void* Bb, int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
                     int group, void* Y, bool y_f32, void* ws, const ttq_workspace_layout& L,
-                    cudaStream_t stream) {
+                    cudaStream_t stream, bool pdl) {
   if (T == 0 || dp == 0) return TTQ_OK;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   void* ax = r > 0 ? ws_at(ws, L.ax) : nullptr;
@@ -188,8 +188,9 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     a.ldy = L.ax_ld;
     a.y_f32 = false;
     a.status = status;
-    const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, 128, stream));
+    const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, 128, stream, pdl));
     if (st != TTQ_OK) return st;
+    pdl = true;
   }
   const int bm = gemm_block_m(bits, dp, T, bn, device_sms());
   GemmMaps m;
@@ -226,7 +227,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   a.ldy = dp;
   a.y_f32 = y_f32;
   a.status = status;
-  return cuda_status(launch_dequant_gemm(a, m, bn, bm, stream));
+  return cuda_status(launch_dequant_gemm(a, m, bn, bm, stream, pdl));
 }
 
 }  // namespace
@@ -348,7 +349,9 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
   const bool f32 = dtype == TTQ_F32;
   const void* xh = X;  // binary16 X D^{-1/2} given as is
   ttq_status st = TTQ_OK;
+  bool pdl = false;    // the first kernel of the call waits for earlier work normally
   if (!(dtype == TTQ_F16 && D_rsqrt == nullptr)) {
+    pdl = true;
     void* xs = ws_at(ws, L.xh);
     st = cuda_status(launch_scale_to_f16(X, dtype, D_rsqrt, xs, T, d, status, device_sms(), s));
     if (st != TTQ_OK) return st;
@@ -370,7 +373,7 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
     Bb = bb;
   }
   return run_gemm(codes, scales, zeros, xh, Xb, Ab, Bb, d, dp, T, r, bits, group, Y,
-                  y_dtype == TTQ_F32, ws, L, s);
+                  y_dtype == TTQ_F32, ws, L, s, pdl);
 }
 
 ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const void* B,
@@ -412,7 +415,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
       X, f32, d, T, p, lambda, alpha, splits, rps,
       reinterpret_cast<double*>(ws_at(ws, L.partial)), status + 64, D, Dr, nullptr, xb, status, s));
   if (st != TTQ_OK || dp == 0) return st;
-  st = cuda_status(launch_scale_to_f16(X, dtype, Dr, xh, T, d, status, device_sms(), s));
+  st = cuda_status(launch_scale_to_f16(X, dtype, Dr, xh, T, d, status, device_sms(), s, true));
   if (st != TTQ_OK) return st;
 
   // (2) codes, scales, zeros of Q[W D^{1/2}]
@@ -420,7 +423,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   uint16_t* scales = reinterpret_cast<uint16_t*>(ws_at(ws, L.scales));
   uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
   st = cuda_status(launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros, status,
-                                   device_sms(), s));
+                                   device_sms(), s, true));
   if (st != TTQ_OK || T == 0) return st;
 
   // (3) Y = W_hat X (+ B (A X))
@@ -436,7 +439,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
     Bb = bb;
   }
   return run_gemm(codes, scales, zeros, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
-                  y_dtype == TTQ_F32, ws, L, s);
+                  y_dtype == TTQ_F32, ws, L, s, true);
 }
 
 ttq_status ttq_get_status(const void* ws, uint32_t* flags) {

@@ -7,7 +7,28 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace ttq {
+
+// Launches `kernel`; with pdl the launch may overlap the previous kernel on
+// the stream (programmatic dependent launch: the kernel waits on the device
+// before it reads that kernel's outputs).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t stream, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? attr : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Number of token splits of the statistic pass and the rows each covers.
 void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split);
@@ -20,13 +41,13 @@ void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* 
 cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                             float lambda, float alpha, int64_t splits, int64_t rows_per_split,
                             double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
-                            void* xb, uint32_t* status, cudaStream_t stream);
+                            void* xb, uint32_t* status, cudaStream_t stream, bool pdl = false);
 
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null).
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,
                             uint16_t* zeros, uint32_t* status, int num_sms,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool pdl = false);
 
 // float32 -> bf16 copy of n elements (n % 8 == 0).
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
@@ -39,7 +60,7 @@ constexpr int kSrcBF16 = 1;
 constexpr int kSrcF16 = 2;
 cudaError_t launch_scale_to_f16(const void* src, int src_kind, const float* Dr, void* dst,
                                 int64_t T, int64_t d, uint32_t* status, int num_sms,
-                                cudaStream_t stream);
+                                cudaStream_t stream, bool pdl = false);
 
 // Steps (2)-(3) on the tensor cores.
 struct GemmArgs {
@@ -83,6 +104,6 @@ int gemm_block_m(int bits, int64_t M, int64_t T, int block_n, int num_sms);
 
 // The operand boxes: a0/a1 are loaded as block_m x 64, b0/b1 as block_n x 64.
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,
-                                int block_m, cudaStream_t stream);
+                                int block_m, cudaStream_t stream, bool pdl = false);
 
 }  // namespace ttq
