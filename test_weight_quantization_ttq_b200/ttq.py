@@ -155,11 +155,18 @@ def ttq_get_status(ws: torch.Tensor) -> tuple[int, int]:
 
 
 # ---------------------------------------------------------- entry points
-def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None):
-    """D[i] = (||X[:, i]||_p + lambda)^alpha and D^{-1/2}; X is [T][d]."""
+def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None, copy_out=True):
+    """D[i] = (||X[:, i]||_p + lambda)^alpha and D^{-1/2}; X is [T][d].
+    With copy_out=False nothing is copied out: D and D^{-1/2} are returned
+    as views of the workspace, where the entry point writes them."""
     T, d = X.shape
     if ws is None:
         ws = new_workspace(d, 0, T, 0, 4, 32, _dtype_code(X), X.device, stream)
+    if not copy_out:
+        _check(lib().ttq_act_norm(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, None, None,
+                                  _dev(ws, "ws"), ws.numel(), _stream(stream)), "ttq_act_norm")
+        L = ttq_workspace_get_layout(d, 0, T, 0, 4, 32, _dtype_code(X))
+        return (ws[L.D: L.D + 4 * d].view(torch.float32), ws[L.D_rsqrt: L.D_rsqrt + 4 * d].view(torch.float32))
     if D is None:
         D = torch.empty(d, dtype=torch.float32, device=X.device)
     if D_rsqrt is None:
