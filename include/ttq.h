@@ -137,6 +137,28 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
                         float p, float lambda, float alpha, float* D,
                         float* D_rsqrt, void* ws, size_t ws_bytes, void* stream);
 
+/* ttq_act_norm without a workspace, for callers that cannot allocate device
+ * memory: for example a plug-in that runs inside another framework's memory
+ * manager and may neither call cudaMalloc nor reserve a buffer of its own,
+ * or a real-time loop that must not allocate once it has started.  The
+ * method has no counterpart to this entry point (an interface choice of this
+ * library, not a step of the paper).
+ *   Same inputs, outputs and results as ttq_act_norm, except that D and
+ * D_rsqrt are required.  The scratch memory (fp64 partial sums, merge
+ * tickets, a status word) is one array compiled into the library: every GPU
+ * that loads the library holds 2 MiB + 4 KiB for it until the process exits,
+ * and d may be at most 16384 (larger d returns TTQ_ERR_UNSUPPORTED).
+ *   The first call on a device looks up the array's device address on the
+ * current device; make that first call before any stream capture.  All calls
+ * share the one array, so calls whose work overlaps on the GPU (other
+ * streams, other threads) race: order them on one stream.  Each call clears
+ * the array's status word and tickets first; device flags are not reported
+ * (a non-finite input shows up as a non-finite D).  The array keeps the last
+ * call's partial sums. */
+ttq_status ttq_act_norm_noalloc(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
+                                float p, float lambda, float alpha, float* D,
+                                float* D_rsqrt, void* stream);
+
 /* Step (2) without the rescale: codes, scales and zeros of Q[W D^{1/2}]
  * (gist.science/zh/paper/2603.19296, section 2.1; quantiser of blog.lo0.es
  * "The maths that matter"), in the binary32 order stated above.

@@ -51,6 +51,7 @@ SIGNATURES = {
                                         ctypes.POINTER(WorkspaceLayout)]),
     "ttq_workspace_init": (_INT, [_P, _SZ, _P]),
     "ttq_act_norm": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _SZ, _P]),
+    "ttq_act_norm_noalloc": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P]),
     "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
     "ttq_scale_activations": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
@@ -174,6 +175,20 @@ def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None, c
     _check(lib().ttq_act_norm(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, _dev(D, "D"),
                               _dev(D_rsqrt, "D_rsqrt"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
            "ttq_act_norm")
+    return D, D_rsqrt
+
+
+def ttq_act_norm_noalloc(X, p, lam, alpha, D=None, D_rsqrt=None, stream=None):
+    """ttq_act_norm without a workspace: the library's own fixed scratch array
+    is used (d <= 16384; calls overlapping on the GPU race)."""
+    T, d = X.shape
+    if D is None:
+        D = torch.empty(d, dtype=torch.float32, device=X.device)
+    if D_rsqrt is None:
+        D_rsqrt = torch.empty(d, dtype=torch.float32, device=X.device)
+    _check(lib().ttq_act_norm_noalloc(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, _dev(D, "D"),
+                                      _dev(D_rsqrt, "D_rsqrt"), _stream(stream)),
+           "ttq_act_norm_noalloc")
     return D, D_rsqrt
 
 
