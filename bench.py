@@ -282,38 +282,36 @@ def run_ours(args):
         raise RuntimeError(f"device status {ttq.status_string(st)} (flags {flags:#x})")
     value = world * args.steps * T / (ms / 1e3)
 
-    # ---- per-kernel durations over K steps: the same four kernels, one entry
-    # point each (statistic, X D^{-1/2} in binary16, quantiser, product)
+    # ---- per-kernel durations over K steps: the forward's kernels, one entry
+    # point each (statistic fused with X D^{-1/2} in binary16, quantiser,
+    # product)
+    n_kernels = ttq.ttq_linear_forward_kernels(d, dp, T, 0, w["p"])
     views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
-    Dbuf, Drbuf = views["D"], views["D_rsqrt"]  # written in place by ttq_act_norm
+    Dbuf = views["D"]  # written in place by ttq_act_norm_scale (copy_out=False)
     Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
     codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda")
     sc = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
     ze = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     for i in range(args.steps):
         k = i % nsets
         ev[i][0].record(stream)
-        ttq.ttq_act_norm(Xs[k], w["p"], w["lam"], w["alpha"], ws=ws, copy_out=False)
+        ttq.ttq_act_norm_scale(Xs[k], w["p"], w["lam"], w["alpha"], ws=ws, Xs=Xsbuf, copy_out=False)
         ev[i][1].record(stream)
-        ttq.ttq_scale_activations(Xs[k], Drbuf, ws=ws, Xs=Xsbuf)
-        ev[i][2].record(stream)
         ttq.ttq_quantize_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc, zeros=ze)
-        ev[i][3].record(stream)
+        ev[i][2].record(stream)
         ttq.ttq_dequant_gemm(codes, sc, ze, None, Xsbuf, None, None, bits, group, ws=ws, Y=Ys[k])
-        ev[i][4].record(stream)
+        ev[i][3].record(stream)
     torch.cuda.synchronize()
-    t_act = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_scale = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t_qdq = statistics.mean(e[2].elapsed_time(e[3]) for e in ev) / 1e3
-    t_gemm = statistics.mean(e[3].elapsed_time(e[4]) for e in ev) / 1e3
+    t_stat = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_qdq = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_gemm = statistics.mean(e[2].elapsed_time(e[3]) for e in ev) / 1e3
 
     peaks = _measured_peaks()
     flops = 2.0 * dp * d * T
-    act_bytes = 2.0 * d * T + 8.0 * d
-    scale_bytes = 4.0 * d * T + 4.0 * d
+    stat_bytes = 4.0 * d * T + 8.0 * d  # X read once, X D^{-1/2} written, D and D^{-1/2}
     qdq_bytes = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d
     gemm_tflops = flops / t_gemm / 1e12
     traffic = NCU_TRAFFIC.get(_kernel_hash())
@@ -323,16 +321,14 @@ def run_ours(args):
                 "peak_source": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
                 "algorithmic_flops_per_launch": flops}
     kernels = [
-        {"kernel": "act_norm_kernel", "ms": t_act * 1e3, "bound": "hbm", "bytes": act_bytes,
-         "achieved_gbs": act_bytes / t_act / 1e9, "frac": act_bytes / t_act / 1e9 / peaks["hbm_gbs"]},
-        {"kernel": "scale_to_f16_kernel", "ms": t_scale * 1e3, "bound": "hbm", "bytes": scale_bytes,
-         "achieved_gbs": scale_bytes / t_scale / 1e9, "frac": scale_bytes / t_scale / 1e9 / peaks["hbm_gbs"]},
+        {"kernel": "act_norm_scale_kernel", "ms": t_stat * 1e3, "bound": "hbm", "bytes": stat_bytes,
+         "achieved_gbs": stat_bytes / t_stat / 1e9, "frac": stat_bytes / t_stat / 1e9 / peaks["hbm_gbs"]},
         {"kernel": "qdq_pack_kernel", "ms": t_qdq * 1e3, "bound": "hbm", "bytes": qdq_bytes,
          "achieved_gbs": qdq_bytes / t_qdq / 1e9, "frac": qdq_bytes / t_qdq / 1e9 / peaks["hbm_gbs"]},
         {"kernel": "ttq_gemm_kernel", "ms": t_gemm * 1e3, "bound": "tensor", "flops": flops,
          "achieved_tflops": gemm_tflops, "frac": gemm_tflops / peaks["bf16_tflops"]},
     ]
-    rho = {"measured": (t_act + t_scale + t_qdq) / t_gemm, "closed_form": 1.0 / dp + 3.0 / T}
+    rho = {"measured": (t_stat + t_qdq) / t_gemm, "closed_form": 1.0 / dp + 3.0 / T}
 
     if args.profile:
         if world > 1:
@@ -384,7 +380,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(),
         "roofline": roofline, "kernels": kernels, "rho": rho, "cpu_baseline": cpu, "e2e": e2e,
-        "clocks": clocks, "gpu_launches": 4 * args.steps,
+        "clocks": clocks, "gpu_launches": n_kernels * args.steps,
     }
     print(json.dumps(line), flush=True)
 

@@ -137,6 +137,30 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
                         float p, float lambda, float alpha, float* D,
                         float* D_rsqrt, void* ws, size_t ws_bytes, void* stream);
 
+/* Step (1) together with the B operand of the product, in one pass over X:
+ * D and D_rsqrt exactly as ttq_act_norm computes them
+ * (gist.science/zh/paper/2603.19296, section 2.1), and
+ *   Xs[t][i] = binary16(X[t][i] * D_rsqrt[i])
+ * exactly as ttq_scale_activations computes it (the D^{-1/2} factor of
+ * W_hat = Q[W D^{1/2}] D^{-1/2}, carried by X).  X [T][d] in TTQ_F32 or
+ * TTQ_BF16, d % 8 == 0; Xs binary16 [T][d] (uint16 bit patterns), required
+ * when T > 0; D and D_rsqrt float32 [d] or NULL (then written to the
+ * workspace only).  When each token split of the statistic pass has at
+ * most 128 rows (64 for float32 X; the splits are those of ttq_act_norm:
+ * about 296 blocks of 256 channels, at most 16 splits) and the whole grid
+ * can be resident at once, this is one cooperative kernel that reads X
+ * from HBM once and keeps it in registers; otherwise it is the two kernels
+ * of ttq_act_norm and ttq_scale_activations.  The results are the same bits
+ * either way.  The
+ * workspace is the one ttq_act_norm needs (it must have been cleared by
+ * ttq_workspace_init once; the call leaves its counters at zero).  Flags as
+ * ttq_act_norm and ttq_scale_activations (NONFINITE, X_RANGE; TIMEOUT if
+ * the fused kernel's wait for the other splits gave up). */
+ttq_status ttq_act_norm_scale(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
+                              float p, float lambda, float alpha, float* D,
+                              float* D_rsqrt, uint16_t* Xs, void* ws, size_t ws_bytes,
+                              void* stream);
+
 /* ttq_act_norm without a workspace, for callers that cannot allocate device
  * memory: for example a plug-in that runs inside another framework's memory
  * manager and may neither call cudaMalloc nor reserve a buffer of its own,
@@ -217,6 +241,15 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A,
                               int64_t T, int64_t r, float p, float lambda, float alpha,
                               int bits, int group, void* Y, ttq_dtype y_dtype, void* ws,
                               size_t ws_bytes, void* stream);
+
+/* Number of kernels one ttq_linear_forward call with these sizes enqueues
+ * on the current device (host query; no device work), in *kernels:
+ * the statistic pass (fused with the scaling of X when it fits, see
+ * ttq_act_norm_scale), the quantiser, the product, and for r > 0 the A X
+ * product (plus two bf16 conversions of a float32 A and B).  An interface
+ * query of this library; the method has no counterpart. */
+ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,
+                                      int64_t r, float p, int* kernels);
 
 /* Reads the workspace status word (a blocking device-to-host copy; the caller
  * synchronises its stream first).  *flags receives the raw TTQ_FLAG_* bits

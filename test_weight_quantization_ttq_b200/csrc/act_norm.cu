@@ -14,6 +14,10 @@
 // copy of X that the tensor-core product consumes (and, for float32 X with a
 // low-rank term, a bf16 copy).  The pass is HBM-bound: it reads X once (2dT
 // bytes for bf16) and writes 2dT bytes of binary16 X plus 8d bytes.
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "ttq_device.cuh"
 #include "ttq_kernels.h"
 
@@ -31,6 +35,26 @@ __device__ __forceinline__ double abs_pow(float x, double p) {
   if (PK == 1) return a;
   if (PK == 2) return a * a;
   return pow(a, p);
+}
+
+// D_ii and D_ii^(-1/2) (binary32) from the merged sum of |x|^p of channel
+// i; false when either is zero, infinite or NaN.
+template <int PK>
+__device__ __forceinline__ bool finish_channel(double tot, double p, double lambda, double alpha,
+                                               float* df, float* drf) {
+  double n;
+  if (PK == 1) {
+    n = tot;
+  } else if (PK == 2) {
+    n = sqrt(tot);
+  } else {
+    n = pow(tot, 1.0 / p);
+  }
+  const double dv = pow(n + lambda, alpha);
+  const double drv = 1.0 / sqrt(dv);
+  *df = static_cast<float>(dv);
+  *drf = static_cast<float>(drv);
+  return (*df > 0.f) && (*df <= 3.402823466e38f) && (*drf > 0.f) && (*drf <= 3.402823466e38f);
 }
 
 __device__ __forceinline__ void load8(const __nv_bfloat16* src, float (&v)[8]) {
@@ -177,24 +201,168 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
     double tot = 0.0;
 #pragma unroll
     for (int k = 0; k < 16; ++k) tot += v[k];
-    double n;
-    if (PK == 1) {
-      n = tot;
-    } else if (PK == 2) {
-      n = sqrt(tot);
-    } else {
-      n = pow(tot, 1.0 / p);
-    }
-    const double dv = pow(n + lambda, alpha);
-    const double drv = 1.0 / sqrt(dv);
-    const float df = static_cast<float>(dv);
-    const float drf = static_cast<float>(drv);
+    float df, drf;
+    const bool ok = finish_channel<PK>(tot, p, lambda, alpha, &df, &drf);
     D[c] = df;
     Dr[c] = drf;
-    const bool ok = (df > 0.f) && (df <= 3.402823466e38f) && (drf > 0.f) && (drf <= 3.402823466e38f);
     if (!ok) set_flag(status, TTQ_FLAG_NONFINITE);
   }
   if (threadIdx.x == 0) counters[cb] = 0u;  // ready for the next call
+}
+
+// ---------------------------------------------------------------------------
+// Fused form of the statistic pass and of the binary16 operand X D^(-1/2).
+// Block (cb, sp) is the block of act_norm_kernel with the same index: warp w
+// takes rows w, w + 8, ... of the split, lane l channels 8l..8l+7 of the
+// column block.  Each thread loads all of its rows (at most kRegRows<XT>)
+// into registers at once, sums |x|^p over them in the same order as
+// act_norm_kernel, publishes the split's partial sums, and waits until every
+// split of its column block has done so (a barrier among the blocks of the
+// column block; the grid is launched cooperatively so that all of them are
+// resident).  Each block then merges its column block's splits in split
+// order (the same merge as act_norm_kernel, so D is identical), and writes
+// binary16(x * D^(-1/2)) from the registers.  X is read from HBM once.
+
+// Rows per warp held in registers: 16 uint4 of X per thread.
+template <typename XT>
+__host__ __device__ constexpr int reg_rows() { return sizeof(XT) == 2 ? 16 : 8; }
+
+template <typename XT>
+struct Raw8;  // eight consecutive elements of X as loaded
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 w;
+  __device__ __forceinline__ void load(const __nv_bfloat16* src) {
+    w = __ldcs(reinterpret_cast<const uint4*>(src));
+  }
+  __device__ __forceinline__ void unpack(float (&v)[8]) const {
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(u[i] << 16);
+      v[2 * i + 1] = __uint_as_float(u[i] & 0xFFFF0000u);
+    }
+  }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* src) {
+    a = __ldcs(reinterpret_cast<const float4*>(src));
+    b = __ldcs(reinterpret_cast<const float4*>(src) + 1);
+  }
+  __device__ __forceinline__ void unpack(float (&v)[8]) const {
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+template <typename XT, int PK>
+__global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
+    const XT* __restrict__ X, int64_t d, int64_t T, double p, double lambda, double alpha,
+    int64_t splits, int64_t rows_per_split, double* __restrict__ partial,
+    uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
+    __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
+  constexpr int R = reg_rows<XT>();
+  __shared__ double red[8][kChannelsPerBlock + 2];
+  __shared__ float dr_s[kChannelsPerBlock];
+  __shared__ int barrier_ok;
+  allow_dependents_launch();
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t cb = blockIdx.x;
+  const int64_t sp = blockIdx.y;
+  const int cl = lane * 8;
+  const int64_t c0 = cb * kChannelsPerBlock + cl;
+  const bool active = c0 < d;
+  const int64_t t_begin = sp * rows_per_split;
+  const int64_t t_end = min(T, t_begin + rows_per_split);
+
+  // all rows of this thread in flight at once
+  Raw8<XT> raw[R];
+  if (active) {
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int64_t t = t_begin + warp + 8 * k;
+      if (t < t_end) raw[k].load(X + t * d + c0);
+    }
+  }
+
+  // (1) this split's sums of |x|^p, rows in increasing order
+  double acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  if (active) {
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      if (t_begin + warp + 8 * k < t_end) {
+        float v[8];
+        raw[k].unpack(v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v[e], p);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[warp][cl + e] = acc[e];
+  __syncthreads();
+  const int ci = threadIdx.x;
+  const int64_t c = cb * kChannelsPerBlock + ci;
+  {
+    double sum = 0.0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) sum += red[w][ci];
+    if (c < d) partial[sp * d + c] = sum;
+  }
+
+  // (2) every split of this column block has published; merge in split order
+  group_barrier(counters + cb, static_cast<uint32_t>(splits), status, &barrier_ok);
+  float drf = 0.f;
+  if (c < d) {
+    double v[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
+    double tot = 0.0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) tot += v[k];
+    float df;
+    const bool ok = finish_channel<PK>(tot, p, lambda, alpha, &df, &drf);
+    if (sp == 0) {
+      D[c] = df;
+      Dr[c] = drf;
+      if (!ok) set_flag(status, TTQ_FLAG_NONFINITE);
+    }
+  }
+  dr_s[ci] = drf;
+  __syncthreads();
+
+  // (3) binary16(x * D^(-1/2)) (and the bf16 copy of a float32 X)
+  bool out_of_range = false;
+  if (active) {
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) f[e] = dr_s[cl + e];
+#pragma unroll
+    for (int k = 0; k < R; ++k) {
+      const int64_t t = t_begin + warp + 8 * k;
+      if (t < t_end) {
+        float v[8];
+        raw[k].unpack(v);
+        __half2 h[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float a = __fmul_rn(v[2 * q], f[2 * q]);
+          const float b = __fmul_rn(v[2 * q + 1], f[2 * q + 1]);
+          h[q] = __floats2half2_rn(a, b);
+          out_of_range |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
+        }
+        *reinterpret_cast<uint4*>(xh + t * d + c0) = *reinterpret_cast<const uint4*>(h);
+        if (xb != nullptr) store8_bf16(xb + t * d + c0, v);
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, out_of_range) && lane == 0) set_flag(status, TTQ_FLAG_X_RANGE);
 }
 
 template <typename XT, int PK>
@@ -223,6 +391,86 @@ cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, f
                                counters, D, Dr, xh, xb, status, stream, pdl);
   return launch_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
                              counters, D, Dr, xh, xb, status, stream, pdl);
+}
+
+// How many blocks of the fused kernel fit on one SM (0 when the query
+// fails), cached per device.
+template <typename XT, int PK>
+int fused_blocks_per_sm() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, act_norm_scale_kernel<XT, PK>, kThreads,
+                                                      0) != cudaSuccess)
+      return 0;
+    cache[dev] = n > 0 ? n : -1;
+  }
+  return cache[dev] > 0 ? cache[dev] : 0;
+}
+
+// Whether the fused kernel applies: every thread's rows fit in its
+// registers and the grid (ceil(d/256) x splits blocks) is resident at once.
+template <typename XT, int PK>
+bool fused_fits(int64_t d, int64_t splits, int64_t rows_per_split, int num_sms) {
+  if (rows_per_split > 8 * reg_rows<XT>()) return false;
+  const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
+  const int per_sm = fused_blocks_per_sm<XT, PK>();
+  return per_sm > 0 && ncb * splits <= static_cast<int64_t>(per_sm) * num_sms;
+}
+
+template <typename XT>
+bool fused_fits_p(float p, int64_t d, int64_t splits, int64_t rows_per_split, int num_sms) {
+  if (p == 1.0f) return fused_fits<XT, 1>(d, splits, rows_per_split, num_sms);
+  if (p == 2.0f) return fused_fits<XT, 2>(d, splits, rows_per_split, num_sms);
+  return fused_fits<XT, 0>(d, splits, rows_per_split, num_sms);
+}
+
+template <typename XT, int PK>
+cudaError_t launch_fused_typed(const XT* X, int64_t d, int64_t T, float p, float lambda,
+                               float alpha, int64_t splits, int64_t rows_per_split,
+                               double* partial, uint32_t* counters, float* D, float* Dr,
+                               void* xh, void* xb, uint32_t* status, int num_sms,
+                               cudaStream_t stream, bool* launched) {
+  *launched = false;
+  if (!fused_fits<XT, PK>(d, splits, rows_per_split, num_sms)) return cudaSuccess;
+  const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ncb), static_cast<unsigned>(splits));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, act_norm_scale_kernel<XT, PK>, X, d, T, static_cast<double>(p),
+      static_cast<double>(lambda), static_cast<double>(alpha), splits, rows_per_split, partial,
+      counters, D, Dr, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
+  *launched = e == cudaSuccess;
+  return e;
+}
+
+template <typename XT>
+cudaError_t launch_fused_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
+                           int64_t splits, int64_t rows_per_split, double* partial,
+                           uint32_t* counters, float* D, float* Dr, void* xh, void* xb,
+                           uint32_t* status, int num_sms, cudaStream_t stream, bool* launched) {
+  if (p == 1.0f)
+    return launch_fused_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
+                                     counters, D, Dr, xh, xb, status, num_sms, stream,
+                                     launched);
+  if (p == 2.0f)
+    return launch_fused_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
+                                     counters, D, Dr, xh, xb, status, num_sms, stream,
+                                     launched);
+  return launch_fused_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
+                                   counters, D, Dr, xh, xb, status, num_sms, stream, launched);
 }
 
 }  // namespace
@@ -254,6 +502,27 @@ cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, flo
                     partial, counters, D, Dr, xh, xb, status, stream, pdl);
   return launch_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
                   rows_per_split, partial, counters, D, Dr, xh, nullptr, status, stream, pdl);
+}
+
+bool act_norm_scale_fused(bool x_f32, int64_t d, int64_t splits, int64_t rows_per_split, float p,
+                          int num_sms) {
+  return x_f32 ? fused_fits_p<float>(p, d, splits, rows_per_split, num_sms)
+               : fused_fits_p<__nv_bfloat16>(p, d, splits, rows_per_split, num_sms);
+}
+
+cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t T, float p,
+                                  float lambda, float alpha, int64_t splits,
+                                  int64_t rows_per_split, double* partial,
+                                  uint32_t* counters, float* D, float* Dr, void* xh,
+                                  void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
+                                  bool* launched) {
+  if (x_f32)
+    return launch_fused_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits,
+                          rows_per_split, partial, counters, D, Dr, xh, xb, status, num_sms,
+                          stream, launched);
+  return launch_fused_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
+                        rows_per_split, partial, counters, D, Dr, xh, nullptr, status,
+                        num_sms, stream, launched);
 }
 
 }  // namespace ttq

@@ -13,7 +13,9 @@ namespace ttq {
 namespace {
 
 constexpr size_t kAlign = 256;
-constexpr size_t kStatusBytes = 4096;           // status word + act_norm tickets
+// status header: word 0 the flags, words 64.. one counter per column block
+// of the statistic pass (merge tickets / barrier counts, left at zero)
+constexpr size_t kStatusBytes = 4096;
 constexpr int64_t kMaxColumnBlocks = 960;       // tickets after the first 256 bytes
 constexpr int kPlanSMs = 148;                   // fixed so the layout is device-independent
 
@@ -230,6 +232,35 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   return cuda_status(launch_dequant_gemm(a, m, bn, bm, stream, pdl));
 }
 
+// Step (1) and, when xh is non-null, the product's binary16 operand
+// X D^(-1/2) in xh: one fused cooperative kernel when every block's tile of
+// X fits in shared memory and the grid is resident at once, else the
+// statistic kernel followed by the scaling kernel.  Either way D and D_rsqrt
+// are the same bits (same splits, same merge order).  xb: bf16 copy of a
+// float32 X (or null).
+ttq_status run_statistic(const void* X, ttq_dtype dtype, int64_t d, int64_t T, float p,
+                         float lambda, float alpha, const ttq_workspace_layout& L, void* ws,
+                         float* D, float* Dr, void* xh, void* xb, cudaStream_t s) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  double* partial = reinterpret_cast<double*>(ws_at(ws, L.partial));
+  const bool f32 = dtype == TTQ_F32;
+  int64_t splits, rps;
+  act_norm_plan(d, T, kPlanSMs, &splits, &rps);
+  if (xh != nullptr) {
+    bool fused = false;
+    const ttq_status st = cuda_status(launch_act_norm_scale(X, f32, d, T, p, lambda, alpha,
+                                                            splits, rps, partial, status + 64, D,
+                                                            Dr, xh, xb, status, device_sms(), s,
+                                                            &fused));
+    if (st != TTQ_OK || fused) return st;
+  }
+  ttq_status st = cuda_status(launch_act_norm(X, f32, d, T, p, lambda, alpha, splits, rps,
+                                              partial, status + 64, D, Dr, nullptr, xb, status,
+                                              s));
+  if (st != TTQ_OK || xh == nullptr) return st;
+  return cuda_status(launch_scale_to_f16(X, dtype, Dr, xh, T, d, status, device_sms(), s, true));
+}
+
 }  // namespace
 }  // namespace ttq
 
@@ -286,6 +317,46 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T, fl
   if (st == TTQ_OK && D_rsqrt)
     st = cuda_status(cudaMemcpyAsync(D_rsqrt, Drw, 4 * d, cudaMemcpyDeviceToDevice, s));
   return st;
+}
+
+ttq_status ttq_act_norm_scale(const void* X, ttq_dtype dtype, int64_t d, int64_t T, float p,
+                              float lambda, float alpha, float* D, float* D_rsqrt, uint16_t* Xs,
+                              void* ws, size_t ws_bytes, void* stream) {
+  if (dtype == TTQ_F16) return TTQ_ERR_INVALID_ARG;
+  ttq_workspace_layout L;
+  if (!make_layout(d, 0, T, 0, 4, 32, dtype, &L)) return TTQ_ERR_INVALID_ARG;
+  if ((T > 0 && (X == nullptr || Xs == nullptr)) || ws == nullptr || !(p >= 1.0f) ||
+      !(lambda >= 0.0f) || !(alpha >= 0.0f) || !std::isfinite(p) || !std::isfinite(lambda) ||
+      !std::isfinite(alpha))
+    return TTQ_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (Xs && !aligned16(Xs)) || (D && !aligned16(D)) ||
+      (D_rsqrt && !aligned16(D_rsqrt)) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return TTQ_ERR_INVALID_ARG;
+  const size_t need = L.partial + align_up(8 * static_cast<size_t>(L.splits) * d);
+  if (ws_bytes < need) return TTQ_ERR_WORKSPACE;
+  float* Dw = D ? D : reinterpret_cast<float*>(ws_at(ws, L.D));
+  float* Drw = D_rsqrt ? D_rsqrt : reinterpret_cast<float*>(ws_at(ws, L.D_rsqrt));
+  if (T == 0) Xs = nullptr;  // nothing to scale
+  return run_statistic(X, dtype, d, T, p, lambda, alpha, L, ws, Dw, Drw, Xs, nullptr,
+                       static_cast<cudaStream_t>(stream));
+}
+
+ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,
+                                      int64_t r, float p, int* kernels) {
+  if (kernels == nullptr || (dtype != TTQ_F32 && dtype != TTQ_BF16)) return TTQ_ERR_INVALID_ARG;
+  if (d < 8 || d % 8 != 0 || dp < 0 || T < 0 || r < 0 || !(p >= 1.0f) || !std::isfinite(p))
+    return TTQ_ERR_INVALID_ARG;
+  int64_t splits, rps;
+  act_norm_plan(d, T, kPlanSMs, &splits, &rps);
+  const bool f32 = dtype == TTQ_F32;
+  int n = 1;  // statistic
+  if (dp > 0) {
+    if (!act_norm_scale_fused(f32, d, splits, rps, p, device_sms())) ++n;  // separate scaling
+    ++n;                                                                   // quantiser
+    if (T > 0) n += 1 + (r > 0 ? 1 + (f32 ? 2 : 0) : 0);  // product (+ A X, + bf16 A, B)
+  }
+  *kernels = n;
+  return TTQ_OK;
 }
 
 ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
@@ -409,14 +480,8 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
 
   // (1) D and D^{-1/2} (a float32 X is also written as bf16 for the
   // low-rank product), then the product's B operand X D^{-1/2} in binary16
-  int64_t splits, rps;
-  act_norm_plan(d, T, kPlanSMs, &splits, &rps);
-  ttq_status st = cuda_status(launch_act_norm(
-      X, f32, d, T, p, lambda, alpha, splits, rps,
-      reinterpret_cast<double*>(ws_at(ws, L.partial)), status + 64, D, Dr, nullptr, xb, status, s));
+  ttq_status st = run_statistic(X, dtype, d, T, p, lambda, alpha, L, ws, D, Dr, xh, xb, s);
   if (st != TTQ_OK || dp == 0) return st;
-  st = cuda_status(launch_scale_to_f16(X, dtype, Dr, xh, T, d, status, device_sms(), s, true));
-  if (st != TTQ_OK) return st;
 
   // (2) codes, scales, zeros of Q[W D^{1/2}]
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));

@@ -99,6 +99,43 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// ------------------------------------------------------ inter-block barrier
+// Barrier among the n blocks of a grid that share the global word `count`
+// (all of them resident at once: a cooperative launch).  `count` is zero
+// before and after every use: each block adds 1 when it arrives (a release
+// that publishes the block's earlier global writes), waits with acquire
+// loads until all n have arrived, and adds 1 when it leaves; the block that
+// brings it to 2n sets it back to zero.  A wait
+// longer than kWaitLimitNs sets TTQ_FLAG_TIMEOUT and lets the block go on
+// (its later results are then not valid); the result is false in that case.
+// `ok_smem` is a shared int used to broadcast the outcome to the block.
+__device__ __forceinline__ bool group_barrier(uint32_t* count, uint32_t n, uint32_t* status,
+                                              int* ok_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    // release at gpu scope: the block's writes (ordered before this thread
+    // by the block barrier) are visible to whoever observes the increment
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+      uint32_t cur;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(count) : "memory");
+      if (cur >= n) break;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        set_flag(status, TTQ_FLAG_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(32);
+    }
+    if (atomicAdd(count, 1u) == 2u * n - 1u) atomicExch(count, 0u);
+    *ok_smem = ok;
+  }
+  __syncthreads();
+  return *ok_smem != 0;
+}
+
 // -------------------------------------------------------------------- TMA
 // 2-D tiled bulk copy global -> shared (no cluster multicast), completing
 // `bytes` of transaction count on `bar`.  x is the innermost coordinate.

@@ -43,6 +43,25 @@ cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, flo
                             double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
                             void* xb, uint32_t* status, cudaStream_t stream, bool pdl = false);
 
+// Whether launch_act_norm_scale would run (on the current device).
+bool act_norm_scale_fused(bool x_f32, int64_t d, int64_t splits, int64_t rows_per_split, float p,
+                          int num_sms);
+
+// Step (1) fused with the binary16 operand X D^(-1/2) (written to xh, which
+// must be non-null; xb as for launch_act_norm).  One cooperative launch over
+// the same splits as launch_act_norm, with D bit-identical to it; X is read
+// once and held in registers.  `counters` as for launch_act_norm.  Launches
+// only when each thread's rows of X fit in its registers (rows_per_split <=
+// 128 for bf16, 64 for float32) and the whole grid is resident at once;
+// *launched tells whether it ran (when it did not, nothing was queued and
+// the result is cudaSuccess).
+cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t T, float p,
+                                  float lambda, float alpha, int64_t splits,
+                                  int64_t rows_per_split, double* partial,
+                                  uint32_t* counters, float* D, float* Dr, void* xh,
+                                  void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
+                                  bool* launched);
+
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null).
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,

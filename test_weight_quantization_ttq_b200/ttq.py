@@ -52,12 +52,14 @@ SIGNATURES = {
     "ttq_workspace_init": (_INT, [_P, _SZ, _P]),
     "ttq_act_norm": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _SZ, _P]),
     "ttq_act_norm_noalloc": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P]),
+    "ttq_act_norm_scale": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _P, _SZ, _P]),
     "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
     "ttq_scale_activations": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
                                 _P, _INT, _P, _SZ, _P]),
     "ttq_linear_forward": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT, _INT,
                                   _P, _INT, _P, _SZ, _P]),
+    "ttq_linear_forward_kernels": (_INT, [_INT, _I64, _I64, _I64, _I64, _F, ctypes.POINTER(ctypes.c_int)]),
     "ttq_get_status": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "ttq_status_string": (ctypes.c_char_p, [_INT]),
     "ttq_version": (ctypes.c_char_p, []),
@@ -178,6 +180,43 @@ def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None, c
     return D, D_rsqrt
 
 
+def ttq_act_norm_scale(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, Xs=None, stream=None,
+                       copy_out=True):
+    """D, D^{-1/2} and Xs [T][d] binary16 = X * D^{-1/2} in one pass over X.
+    With copy_out=False, D and D^{-1/2} are not given to the entry point and
+    are returned as views of the workspace, where it writes them."""
+    T, d = X.shape
+    if ws is None:
+        ws = new_workspace(d, 0, T, 0, 4, 32, _dtype_code(X), X.device, stream)
+    if Xs is None:
+        Xs = torch.empty((T, d), dtype=torch.float16, device=X.device)
+    if copy_out:
+        if D is None:
+            D = torch.empty(d, dtype=torch.float32, device=X.device)
+        if D_rsqrt is None:
+            D_rsqrt = torch.empty(d, dtype=torch.float32, device=X.device)
+        dptr, drptr = _dev(D, "D"), _dev(D_rsqrt, "D_rsqrt")
+    else:
+        dptr = drptr = None
+    _check(lib().ttq_act_norm_scale(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, dptr, drptr,
+                                    _dev(Xs, "Xs"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "ttq_act_norm_scale")
+    if not copy_out:
+        L = ttq_workspace_get_layout(d, 0, T, 0, 4, 32, _dtype_code(X))
+        D = ws[L.D: L.D + 4 * d].view(torch.float32)
+        D_rsqrt = ws[L.D_rsqrt: L.D_rsqrt + 4 * d].view(torch.float32)
+    return D, D_rsqrt, Xs
+
+
+def ttq_linear_forward_kernels(d, dp, T, r=0, p=2.0, dtype=TTQ_BF16) -> int:
+    """Kernels one ttq_linear_forward call of these sizes enqueues on the
+    current device."""
+    n = ctypes.c_int(0)
+    _check(lib().ttq_linear_forward_kernels(dtype, d, dp, T, r, p, ctypes.byref(n)),
+           "ttq_linear_forward_kernels")
+    return n.value
+
+
 def ttq_act_norm_noalloc(X, p, lam, alpha, D=None, D_rsqrt=None, stream=None):
     """ttq_act_norm without a workspace: the library's own fixed scratch array
     is used (d <= 16384; calls overlapping on the GPU race)."""
@@ -277,4 +316,5 @@ def workspace_views(ws: torch.Tensor, d, dp, T, r, bits, group, dtype=TTQ_BF16) 
         out["codes"] = view(L.codes, dp * (d * bits // 32), torch.int32).view(dp, -1)
         out["scales"] = view(L.scales, dp * (d // group), torch.int16).view(dp, -1)
         out["zeros"] = view(L.zeros, dp * (d // group), torch.int16).view(dp, -1)
+        out["xh"] = view(L.xh, T * d, torch.float16).view(T, d)
     return out

@@ -85,6 +85,12 @@ def test_rejections_before_device_work(L):
     # workspace too small / misaligned
     assert L.ttq_act_norm(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
     assert L.ttq_act_norm(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 128, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
+    # fused statistic + operand: Xs required, binary16 X refused, workspace checked
+    assert L.ttq_act_norm_scale(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, None, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_act_norm_scale(16, 2, 64, 4, 2.0, 0.0, 0.5, None, None, 32, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_act_norm_scale(16, 1, 64, 4, 0.5, 0.0, 0.5, None, None, 32, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_act_norm_scale(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 32, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
+    assert L.ttq_act_norm_scale(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 40, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
     # forward with a null weight
     st = L.ttq_linear_forward(16, None, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 16, 1, 256, 1 << 30, None)
     assert st == ttq.TTQ_ERR_INVALID_ARG
