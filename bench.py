@@ -3,8 +3,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step is one TTQ linear forward through the C ABI -- activation statistic,
-quantise-and-pack, dequantising tensor-core GEMM -- on one batch of seeded
+One step is one TTQ linear forward through the C ABI -- activation statistic
+with the scaled binary16 X, quantise-and-pack with the dequantised binary16
+weight, tensor-core GEMM -- on one batch of seeded
 synthetic input: the Llama-7B-like q_proj prefill, d = d' = 4096, T = 2048
 tokens, INT4 with groups of 128, p = 2, lambda = 1e-3, alpha = 0.5.
 
@@ -283,8 +284,8 @@ def run_ours(args):
     value = world * args.steps * T / (ms / 1e3)
 
     # ---- per-kernel durations over K steps: the forward's kernels, one entry
-    # point each (statistic fused with X D^{-1/2} in binary16, quantiser,
-    # product)
+    # point each (statistic fused with X D^{-1/2} in binary16, quantiser with
+    # the dequantised binary16 weight, product on it)
     n_kernels = ttq.ttq_linear_forward_kernels(d, dp, T, 0, w["p"])
     views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
     Dbuf = views["D"]  # written in place by ttq_act_norm_scale (copy_out=False)
@@ -292,6 +293,7 @@ def run_ours(args):
     codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda")
     sc = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
     ze = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
+    W_hat = torch.empty((dp, d), dtype=torch.float16, device="cuda")
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
@@ -300,9 +302,10 @@ def run_ours(args):
         ev[i][0].record(stream)
         ttq.ttq_act_norm_scale(Xs[k], w["p"], w["lam"], w["alpha"], ws=ws, Xs=Xsbuf, copy_out=False)
         ev[i][1].record(stream)
-        ttq.ttq_quantize_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc, zeros=ze)
+        ttq.ttq_quantize_dequant_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc,
+                                        zeros=ze, W_hat=W_hat)
         ev[i][2].record(stream)
-        ttq.ttq_dequant_gemm(codes, sc, ze, None, Xsbuf, None, None, bits, group, ws=ws, Y=Ys[k])
+        ttq.ttq_dequantized_gemm(W_hat, Xsbuf, ws=ws, Y=Ys[k])
         ev[i][3].record(stream)
     torch.cuda.synchronize()
     t_stat = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
@@ -312,10 +315,11 @@ def run_ours(args):
     peaks = _measured_peaks()
     flops = 2.0 * dp * d * T
     stat_bytes = 4.0 * d * T + 8.0 * d  # X read once, X D^{-1/2} written, D and D^{-1/2}
-    qdq_bytes = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d
+    # W read, codes, scales and zeros and the binary16 W_hat written, D read
+    qdq_bytes = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d + 2.0 * dp * d
     gemm_tflops = flops / t_gemm / 1e12
     traffic = NCU_TRAFFIC.get(_kernel_hash())
-    roofline = {"kernel": "ttq_gemm_kernel<4> (dequantising tcgen05 GEMM)", "bound": "tensor",
+    roofline = {"kernel": "ttq_gemm_kernel<0, 256> (tcgen05 GEMM on the binary16 dequantised weight)", "bound": "tensor",
                 "achieved": gemm_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": gemm_tflops / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_source": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",

@@ -105,6 +105,8 @@ typedef struct ttq_workspace_layout {
   size_t xh;      /* binary16 [T][d] X D^{-1/2} for the product   */
   size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32, r > 0) */
   size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32, r > 0) */
+  size_t wq;      /* binary16 [d'][d] s (q - z) that ttq_linear_forward's
+                     product reads when T > 256 (0: not in this layout) */
   size_t total;
   int64_t splits; /* number of token splits of the statistic pass */
   int64_t ax_ld;  /* row stride (elements) of A X                 */
@@ -196,6 +198,19 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
                                uint16_t* scales, uint16_t* zeros, void* ws,
                                size_t ws_bytes, void* stream);
 
+/* ttq_quantize_weight that also writes the dequantised weight
+ *   W_hat[j][i] = binary16(s[j][k] * (q[j][i] - z[j][k]))
+ * (binary16 bit patterns, [dp][d] row-major, 16-byte aligned; required
+ * when dp > 0): W_hat of the paper (gist.science/zh/paper/2603.19296,
+ * section 2.1) without its D^{-1/2} factor, which the product's other
+ * operand X D^{-1/2} carries.  q - z is exact and the product is rounded
+ * once, so these are the operand values ttq_dequant_gemm forms from the
+ * codes.  Everything else as ttq_quantize_weight. */
+ttq_status ttq_quantize_dequant_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                                       const float* D, int bits, int group, uint32_t* codes,
+                                       uint16_t* scales, uint16_t* zeros, uint16_t* W_hat,
+                                       void* ws, size_t ws_bytes, void* stream);
+
 /* The B operand of the product: Xs[t][i] = binary16(X[t][i] * D_rsqrt[i])
  * (the D^{-1/2} factor of W_hat = Q[W D^{1/2}] D^{-1/2}, carried by X;
  * gist.science/zh/paper/2603.19296, section 2.1).  X [T][d] in dtype (F32,
@@ -228,6 +243,18 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
                             ttq_dtype y_dtype, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* Step (3) on a dequantised weight: Y[t][j] = sum_i W_hat[j][i] Xs[t][i]
+ * (gist.science/zh/paper/2603.19296, section 2.3), on the tensor cores
+ * with binary16 operands and fp32 accumulation.  W_hat binary16 [dp][d]
+ * (as written by ttq_quantize_dequant_weight), Xs binary16 [T][d] (X
+ * D^{-1/2}, as written by ttq_scale_activations); d % 8 == 0; all pointers
+ * 16-byte aligned.  Y [T][dp] in y_dtype (TTQ_F32 or TTQ_BF16, rounded
+ * once).  No low-rank term.  Needs a workspace of at least 4096 bytes
+ * (status word). */
+ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64_t d,
+                                int64_t dp, int64_t T, void* Y, ttq_dtype y_dtype, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* The whole TTQ linear layer, (1) -> (2) -> (3), on `stream`:
  *   Y = Q[W D^{1/2}] D^{-1/2} X + B (A X).
  * X [T][d], W [dp][d], A [r][d], B [dp][r] in `dtype`; Y [T][dp] in
@@ -235,7 +262,12 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
  * nearest-even).  A and B may be NULL when r == 0.  W is taken to be the
  * residual that the static low-rank pair complements (gist.science/zh,
  * section 2.2).  The workspace keeps D, D_rsqrt, codes, scales and zeros of
- * this call. */
+ * this call.  For T > 256 the quantiser also writes the dequantised weight
+ * s (q - z) in binary16 to the workspace (layout field wq) and the product
+ * reads it as a plain tensor-core operand, so that no 256-token tile
+ * dequantises the codes again; for T <= 256 the product dequantises the
+ * codes itself (as ttq_dequant_gemm does).  Both give the same operand
+ * values. */
 ttq_status ttq_linear_forward(const void* X, const void* W, const void* A,
                               const void* B, ttq_dtype dtype, int64_t d, int64_t dp,
                               int64_t T, int64_t r, float p, float lambda, float alpha,

@@ -56,7 +56,8 @@ struct GemmDev {
   void* Y;
   int64_t ldy;
   int y_f32;
-  int y_tma;            // bf16 Y written by one TMA store per CTA (tmY)
+  int y_tma;            // bf16 Y written by TMA stores of 32 x 16 slabs (tmY)
+  int a_f16;            // plain mode: binary16 A operand (else bf16)
   int BN;
   int stages;
   uint32_t* status;
@@ -285,7 +286,8 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1 + kProducerWarps);
+      // the producer warps take part only when they build the A operand
+      mbar_init(&full[s], 1 + (BITS != 0 ? kProducerWarps : 0));
       mbar_init(&empty[s], 1);
       mbar_init(&cfull[s], 1);
     }
@@ -354,8 +356,8 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
     if (lane == 0) {
       // main K blocks: binary16 W_hat x binary16 X D^(-1/2) (bf16 x bf16 in
       // the plain mode); low-rank tail: bf16 B x bf16 A X
-      const uint32_t idesc_main =
-          idesc_f16kind(BITS == 0 ? kFmtBF16 : kFmtF16, 128, static_cast<uint32_t>(BN));
+      const uint32_t idesc_main = idesc_f16kind(
+          (BITS != 0 || g.a_f16) ? kFmtF16 : kFmtBF16, 128, static_cast<uint32_t>(BN));
       const uint32_t idesc_tail = idesc_f16kind(kFmtBF16, 128, static_cast<uint32_t>(BN));
       int s = 0;
       uint32_t ph = 0;
@@ -418,7 +420,9 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
       s = (s + 1 == stages) ? 0 : s + 1;
       ph ^= (s == 0);
     };
-    if (TC) {
+    if (BITS == 0) {
+      // plain mode: the A operand comes by TMA; nothing to build
+    } else if (TC) {
       // Codes arrive by TMA with the stage (cfull); scales and zeros come
       // from the per-thread cache, two blocks of groups in registers.
       SZCache cache;
@@ -513,42 +517,50 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
     const int nchunks = BN / 16;
     const bool good = ok && (*abort_flag == 0);
     if (g.y_tma) {
-      // bf16 Y: stage the BN x BM tile [t][j] in the (now idle) pipeline
-      // memory, then one TMA store.  Lanes 2k and 2k+1 swap one value per
-      // token pair so each writes a bf16 pair (j, j+1) of one token.
-      const uint32_t tile = smem_addr(smem);
-      const bool odd = lane & 1;
-      for (int ch = ch0; ch < nchunks; ch += chs) {
-        uint32_t rr[16];
-        tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
-        tmem_load_wait();
+      // bf16 Y: each warp converts its 32 rows x 16 tokens of a chunk into a
+      // 1 KiB slab [t][j] of the (now idle) pipeline memory and one lane
+      // sends it out with a TMA store, while the next chunk's tensor-memory
+      // load is in flight.
+      const int iters = (nchunks + chs - 1) / chs;
+      const uint32_t slabs = smem_addr(smem) + static_cast<uint32_t>((warp - 2) * iters) * 1024u;
+      const int32_t jx = static_cast<int32_t>(m0 + acc * 128 + q * 32);
+      const uint32_t tcol = tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16);
+      uint32_t ra[16], rb[16];
+      if (ch0 < nchunks) {
+        tmem_load_16(tcol + ch0 * 16, ra);
+        tmem_load_wait(ra);
+      }
+      int it = 0;
+      for (int ch = ch0; ch < nchunks; ch += chs, ++it) {
+        const bool more = ch + chs < nchunks;
+        if (more) tmem_load_16(tcol + (ch + chs) * 16, rb);
+        const uint32_t slab = slabs + static_cast<uint32_t>(it) * 1024u;
 #pragma unroll
-        for (int i = 0; i < 16; i += 2) {
-          // even lane keeps token i and receives its partner's token i;
-          // odd lane keeps token i+1 and receives its partner's token i+1
-          const uint32_t give = odd ? rr[i] : rr[i + 1];
-          const uint32_t got = __shfl_xor_sync(0xffffffffu, give, 1);
-          const float lo = __uint_as_float(odd ? got : rr[i]);
-          const float hi = __uint_as_float(odd ? rr[i + 1] : got);
-          __nv_bfloat162 pr = __floats2bfloat162_rn(lo, hi);
-          const int tl = ch * 16 + i + (odd ? 1 : 0);
-          const uint32_t addr = tile + (tl * BM + (jl & ~1)) * 2;
-          asm volatile("st.shared.b32 [%0], %1;" ::"r"(addr), "r"(*reinterpret_cast<uint32_t*>(&pr))
+        for (int i = 0; i < 16; ++i) {
+          const __nv_bfloat16 v = __float2bfloat16_rn(__uint_as_float(ra[i]));
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(slab + (i * 32 + lane) * 2),
+                       "h"(*reinterpret_cast<const uint16_t*>(&v))
                        : "memory");
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && good) {
+          tma_store_2d(&tmY, slab, jx, static_cast<int32_t>(n0 + ch * 16));
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (more) {
+          tmem_load_wait(rb);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ra[i] = rb[i];
+        }
       }
-      fence_proxy_async_smem();
-      asm volatile("bar.sync 1, %0;" ::"n"(2 * BM) : "memory");  // the epilogue warps
-      if (threadIdx.x == 64 && good) {
-        tma_store_2d(&tmY, tile, static_cast<int32_t>(m0), static_cast<int32_t>(n0));
-        tma_store_commit_and_wait();
-      }
+      if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     } else {
       const bool store = good && j < g.M;
       for (int ch = ch0; ch < nchunks; ch += chs) {
         uint32_t rr[16];
         tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
-        tmem_load_wait();
+        tmem_load_wait(rr);
         if (store) {
           const int64_t t0 = n0 + ch * 16;
           if (g.y_f32) {
@@ -603,8 +615,11 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.Y = a.Y;
   g.ldy = a.ldy;
   g.y_f32 = a.y_f32 ? 1 : 0;
-  // the staged Y tile (BN x BM bf16) must fit in the pipeline memory
-  g.y_tma = (a.y_tma && !a.y_f32 && BN * BM * 2 <= stages * stage_bytes) ? 1 : 0;
+  g.a_f16 = a.a_f16 ? 1 : 0;
+  // the Y slabs (1 KiB per producer warp and chunk pair) must fit in the
+  // pipeline memory
+  const int slab_bytes = (2 * BM / 32) * ((BN / 16 + 1) / 2) * 1024;
+  g.y_tma = (a.y_tma && !a.y_f32 && slab_bytes <= stages * stage_bytes) ? 1 : 0;
   g.BN = BN;
   g.stages = stages;
   g.status = a.status;
@@ -617,7 +632,10 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
 template <int BITS>
 cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, int BM,
                         cudaStream_t stream, bool pdl) {
-  if (BITS == 0) return launch_tile<BITS, 128, false>(a, maps, BN, stream, pdl);
+  if (BITS == 0) {
+    if (BM == 256) return launch_tile<BITS, 256, false>(a, maps, BN, stream, pdl);
+    return launch_tile<BITS, 128, false>(a, maps, BN, stream, pdl);
+  }
   if (a.codes_tma) {
     if (BM == 256) return launch_tile<BITS, 256, true>(a, maps, BN, stream, pdl);
     return launch_tile<BITS, 128, true>(a, maps, BN, stream, pdl);
@@ -637,26 +655,42 @@ int gemm_block_n(int64_t T) {
   return static_cast<int>(bn);
 }
 
-int gemm_block_m(int bits, int64_t M, int64_t T, int block_n, int num_sms) {
-  if (bits == 0 || M <= 128) return 128;
-  // waves of CTAs times the work of one CTA; 128-row tiles move twice the
-  // X bytes per FLOP, which costs about 40% at full tensor rate
-  const int64_t nt = (T + block_n - 1) / block_n;
-  const int64_t c256 = (M + 255) / 256 * nt;
-  const int64_t c128 = (M + 127) / 128 * nt;
-  const double t256 = static_cast<double>((c256 + num_sms - 1) / num_sms) * 2.0;
-  const double t128 = static_cast<double>((c128 + num_sms - 1) / num_sms) * 1.4;
-  return t256 <= t128 ? 256 : 128;
+void gemm_tile_shape(int bits, int64_t M, int64_t T, int num_sms, int* block_m, int* block_n) {
+  // Cost of a shape: waves of CTAs times the time of one CTA, taken as
+  // proportional to (BN + 24) (24: the fixed prologue / epilogue share) and
+  // to 2.0 for 256-row tiles, 1.4 for 128-row tiles (which move twice the X
+  // bytes per FLOP).  With codes, the dequantisation of a K block takes
+  // about as long as 256 tokens of MMA whatever BN is, so BN counts as at
+  // least 256 there.  256-row tiles need M > 128.
+  const int64_t bn_max = T >= 256 ? 256 : (T + 15) / 16 * 16;
+  double best = 0.0;
+  int best_m = 128, best_n = 16;
+  for (int bm = 256; bm >= 128; bm -= 128) {
+    if (bm == 256 && M <= 128) continue;
+    for (int bn = static_cast<int>(bn_max); bn >= 16; bn -= 16) {
+      const int64_t tiles = (M + bm - 1) / bm * ((T + bn - 1) / bn);
+      const int64_t waves = (tiles + num_sms - 1) / num_sms;
+      const int work = bits != 0 && bn < 256 ? 256 : bn;
+      const double cost = static_cast<double>(waves) * (bm == 256 ? 2.0 : 1.4) * (work + 24);
+      if (best == 0.0 || cost < best) {
+        best = cost;
+        best_m = bm;
+        best_n = bn;
+      }
+    }
+  }
+  *block_m = best_m;
+  *block_n = best_n;
 }
 
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,
                                 int block_m, cudaStream_t stream, bool pdl) {
   if (args.M == 0 || args.T == 0) return cudaSuccess;
   if (block_n % 16 != 0 || block_n < 16 || block_n > 256) return cudaErrorInvalidValue;
-  if (block_m != 128 && !(block_m == 256 && args.bits != 0)) return cudaErrorInvalidValue;
+  if (block_m != 128 && block_m != 256) return cudaErrorInvalidValue;
   switch (args.bits) {
     case 0:
-      return launch_bits<0>(args, maps, block_n, 128, stream, pdl);
+      return launch_bits<0>(args, maps, block_n, block_m, stream, pdl);
     case 2:
       return launch_bits<2>(args, maps, block_n, block_m, stream, pdl);
     case 3:

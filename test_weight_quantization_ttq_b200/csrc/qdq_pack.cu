@@ -71,11 +71,15 @@ __device__ __forceinline__ void unpack16(const Raw16<float>& r, float2 (&x)[8]) 
   }
 }
 
-template <typename WT, int BITS>
+// With WQ the kernel also writes the dequantised weight s (q - z) as
+// binary16 [dp][d] (wq), formed exactly as the product's A operand is
+// formed from the codes: (1024 + q) - (1024 + z) is exact in binary16 and
+// the product with s is rounded once.
+template <typename WT, int BITS, bool WQ>
 __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
     const WT* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D, int group,
     int cw, uint32_t* __restrict__ codes, __half* __restrict__ scales,
-    __half* __restrict__ zeros, uint32_t* __restrict__ status) {
+    __half* __restrict__ zeros, __half* __restrict__ wq, uint32_t* __restrict__ status) {
   constexpr int QMAX = (1 << BITS) - 1;
   const int tpr = cw >> 4;            // threads per row of the tile (16 weights each)
   const int rpi = kThreads / tpr;     // rows per iteration of the block
@@ -156,6 +160,9 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         // from the low fraction bits
         const int zoff = z - 0x4B400000;
         uint32_t lo = 0, hi = 0;  // codes 0-7 and 8-15 (INT3: 24 bits each)
+        uint32_t wh[8];           // s (q - z) of weights 2i, 2i+1 (WQ)
+        const __half2 zc2 = __half2half2(__hadd(__int2half_rn(z), __ushort_as_half(0x6400)));
+        const __half2 s2 = __half2half2(s16);
   #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float r0 = __fadd_rn(__fmul_rn(x[i].x, inv), 12582912.0f);
@@ -165,6 +172,18 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
           const uint32_t pair = static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << BITS);
           if (i < 4) lo |= pair << (2 * BITS * i);
           else hi |= pair << (2 * BITS * (i - 4));
+          if (WQ) {
+            const uint32_t m = static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << 16) | 0x64006400u;
+            __half2 hm;
+            memcpy(&hm, &m, 4);
+            const __half2 v = __hmul2(__hsub2(hm, zc2), s2);
+            memcpy(&wh[i], &v, 4);
+          }
+        }
+        if (WQ && active) {
+          uint4* dst = reinterpret_cast<uint4*>(wq + row * d + col);
+          dst[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+          dst[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
         }
         if (active && (tx & (gthreads - 1)) == 0) {
           scales[row * ngroups + kgroup] = s16;
@@ -215,10 +234,10 @@ int tile_width(int64_t d, int group) {
   return group;
 }
 
-template <typename WT>
+template <typename WT, bool WQ>
 cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bits, int group,
-                     uint32_t* codes, uint16_t* scales, uint16_t* zeros, uint32_t* status,
-                     int num_sms, cudaStream_t stream, bool pdl) {
+                     uint32_t* codes, uint16_t* scales, uint16_t* zeros, void* wq,
+                     uint32_t* status, int num_sms, cudaStream_t stream, bool pdl) {
   const int cw = tile_width(d, group);
   const int rpi = kThreads / (cw >> 4);
   const int64_t gx = d / cw;
@@ -233,14 +252,14 @@ cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bit
   __half* z = reinterpret_cast<__half*>(zeros);
   switch (bits) {
     case 2:
-      return launch_kernel(qdq_pack_kernel<WT, 2>, grid, dim3(kThreads), 0, stream, pdl, W, dp, d, D,
-                           group, cw, codes, s, z, status);
+      return launch_kernel(qdq_pack_kernel<WT, 2, WQ>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
+                           d, D, group, cw, codes, s, z, static_cast<__half*>(wq), status);
     case 3:
-      return launch_kernel(qdq_pack_kernel<WT, 3>, grid, dim3(kThreads), 0, stream, pdl, W, dp, d, D,
-                           group, cw, codes, s, z, status);
+      return launch_kernel(qdq_pack_kernel<WT, 3, WQ>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
+                           d, D, group, cw, codes, s, z, static_cast<__half*>(wq), status);
     case 4:
-      return launch_kernel(qdq_pack_kernel<WT, 4>, grid, dim3(kThreads), 0, stream, pdl, W, dp, d, D,
-                           group, cw, codes, s, z, status);
+      return launch_kernel(qdq_pack_kernel<WT, 4, WQ>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
+                           d, D, group, cw, codes, s, z, static_cast<__half*>(wq), status);
     default:
       return cudaErrorInvalidValue;
   }
@@ -360,13 +379,20 @@ cudaError_t launch_scale_to_f16(const void* src, int src_kind, const float* Dr, 
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,
                             uint16_t* zeros, uint32_t* status, int num_sms,
-                            cudaStream_t stream, bool pdl) {
+                            cudaStream_t stream, bool pdl, void* wq) {
   if (dp == 0) return cudaSuccess;
-  if (w_f32)
-    return launch_w(static_cast<const float*>(W), dp, d, D, bits, group, codes, scales, zeros,
-                    status, num_sms, stream, pdl);
-  return launch_w(static_cast<const __nv_bfloat16*>(W), dp, d, D, bits, group, codes, scales,
-                  zeros, status, num_sms, stream, pdl);
+  if (w_f32) {
+    const float* w = static_cast<const float*>(W);
+    return wq ? launch_w<float, true>(w, dp, d, D, bits, group, codes, scales, zeros, wq, status,
+                                      num_sms, stream, pdl)
+              : launch_w<float, false>(w, dp, d, D, bits, group, codes, scales, zeros, wq, status,
+                                       num_sms, stream, pdl);
+  }
+  const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(W);
+  return wq ? launch_w<__nv_bfloat16, true>(w, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                            status, num_sms, stream, pdl)
+            : launch_w<__nv_bfloat16, false>(w, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                             status, num_sms, stream, pdl);
 }
 
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {

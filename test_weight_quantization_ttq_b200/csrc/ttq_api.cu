@@ -39,6 +39,12 @@ bool valid_qparams(int bits, int group) {
   return (bits >= 2 && bits <= 4) && (group == 32 || group == 64 || group == 128 || group == 256);
 }
 
+// Whether ttq_linear_forward materialises the dequantised weight s (q - z)
+// in binary16 and runs the product on it (more than one 256-token tile:
+// dequantising inside the product would repeat the work once per tile)
+// instead of dequantising the codes inside the product.
+bool materialize_w(int64_t dp, int64_t T) { return dp > 0 && T > 256; }
+
 // Computes the workspace layout; false for an unsupported shape.
 bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
                  ttq_dtype dtype, ttq_workspace_layout* L) {
@@ -82,6 +88,10 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
     off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(d) * 2);
     l.ab = off;
     off = align_up(off + (static_cast<size_t>(r) * d + static_cast<size_t>(dp) * r) * 2);
+  }
+  if (has_q && materialize_w(dp, T)) {
+    l.wq = off;
+    off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d) * 2);
   }
   l.total = off;
   l.splits = splits;
@@ -166,7 +176,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
                     const void* Xh, const void* Xb, const void* Ab,
                     const void* Bb, int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
                     int group, void* Y, bool y_f32, void* ws, const ttq_workspace_layout& L,
-                    cudaStream_t stream, bool pdl) {
+                    cudaStream_t stream, bool pdl, const void* wq = nullptr) {
   if (T == 0 || dp == 0) return TTQ_OK;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   void* ax = r > 0 ? ws_at(ws, L.ax) : nullptr;
@@ -194,13 +204,16 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     if (st != TTQ_OK) return st;
     pdl = true;
   }
-  const int bm = gemm_block_m(bits, dp, T, bn, device_sms());
+  // wq: the product reads the materialised binary16 s (q - z) by TMA
+  int bm = 128, bnm = 16;
+  gemm_tile_shape(wq ? 0 : bits, dp, T, device_sms(), &bm, &bnm);
   GemmMaps m;
-  if (!encode_16bit(&m.b0, Xh, true, d, T, d, bn)) return TTQ_ERR_CUDA;
+  if (!encode_16bit(&m.b0, Xh, true, d, T, d, bnm)) return TTQ_ERR_CUDA;
   m.a0 = m.b0;
+  if (wq && !encode_16bit(&m.a0, wq, true, d, dp, d, bm)) return TTQ_ERR_CUDA;
   if (r > 0) {
     if (!encode_16bit(&m.a1, Bb, false, r, dp, r, bm) ||
-        !encode_16bit(&m.b1, ax, false, r, T, L.ax_ld, bn))
+        !encode_16bit(&m.b1, ax, false, r, T, L.ax_ld, bnm))
       return TTQ_ERR_CUDA;
   } else {
     m.a1 = m.b0;
@@ -208,10 +221,12 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   }
   // the code tile comes in by TMA when the code rows are 16-byte strided
   const int64_t wpr = d * bits / 32;
-  const bool codes_tma = encode_codes(&m.c0, codes, wpr, dp, gemm_code_tile_words(bits), bm);
+  const bool codes_tma =
+      !wq && encode_codes(&m.c0, codes, wpr, dp, gemm_code_tile_words(bits), bm);
   if (!codes_tma) m.c0 = m.b0;
-  // bf16 Y goes out through one TMA store per tile when its rows are 16-byte strided
-  const bool y_tma = !y_f32 && dp % 8 == 0 && encode_y_bf16(&m.y, Y, dp, T, bm, bn);
+  // bf16 Y goes out through TMA stores of 32 x 16 slabs when its rows are
+  // 16-byte strided
+  const bool y_tma = !y_f32 && dp % 8 == 0 && encode_y_bf16(&m.y, Y, dp, T, 32, 16);
   if (!y_tma) m.y = m.b0;
   GemmArgs a;
   a.codes_tma = codes_tma;
@@ -219,7 +234,8 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   a.codes = codes;
   a.scales = scales;
   a.zeros = zeros;
-  a.bits = bits;
+  a.bits = wq ? 0 : bits;
+  a.a_f16 = wq != nullptr;
   a.group = group;
   a.K = d;
   a.M = dp;
@@ -229,7 +245,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   a.ldy = dp;
   a.y_f32 = y_f32;
   a.status = status;
-  return cuda_status(launch_dequant_gemm(a, m, bn, bm, stream, pdl));
+  return cuda_status(launch_dequant_gemm(a, m, bnm, bm, stream, pdl));
 }
 
 // Step (1) and, when xh is non-null, the product's binary16 operand
@@ -379,6 +395,45 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
                                      static_cast<cudaStream_t>(stream)));
 }
 
+ttq_status ttq_quantize_dequant_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                                       const float* D, int bits, int group, uint32_t* codes,
+                                       uint16_t* scales, uint16_t* zeros, uint16_t* W_hat,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  if (dp > 0 && W_hat == nullptr) return TTQ_ERR_INVALID_ARG;
+  if (W_hat && !aligned16(W_hat)) return TTQ_ERR_INVALID_ARG;
+  if (dtype != TTQ_F32 && dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
+  if (bits < 1 || bits > 8 || group < 1) return TTQ_ERR_INVALID_ARG;
+  if (!valid_qparams(bits, group)) return TTQ_ERR_UNSUPPORTED;
+  if (d < group || d % group != 0 || dp < 0) return TTQ_ERR_INVALID_ARG;
+  if (dp > 0 && (W == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr))
+    return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if ((W && !aligned16(W)) || (D && !aligned16(D)) || (codes && !aligned16(codes)))
+    return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
+  return cuda_status(launch_qdq_pack(W, dtype == TTQ_F32, dp, d, D, bits, group, codes, scales,
+                                     zeros, static_cast<uint32_t*>(ws), device_sms(),
+                                     static_cast<cudaStream_t>(stream), false, W_hat));
+}
+
+ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64_t d, int64_t dp,
+                                int64_t T, void* Y, ttq_dtype y_dtype, void* ws, size_t ws_bytes,
+                                void* stream) {
+  if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
+  if (d < 8 || d % 8 != 0 || dp < 0 || T < 0) return TTQ_ERR_INVALID_ARG;
+  const bool work = dp > 0 && T > 0;
+  if (work && (W_hat == nullptr || Xs == nullptr || Y == nullptr)) return TTQ_ERR_INVALID_ARG;
+  const void* ptrs[] = {W_hat, Xs, Y};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
+  if (!work) return TTQ_OK;
+  ttq_workspace_layout L = {};  // only the status word (offset 0) is used
+  return run_gemm(nullptr, nullptr, nullptr, Xs, nullptr, nullptr, nullptr, d, dp, T, 0, 4, 32,
+                  Y, y_dtype == TTQ_F32, ws, L, static_cast<cudaStream_t>(stream), false, W_hat);
+}
+
 ttq_status ttq_scale_activations(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
                                  const float* D_rsqrt, uint16_t* Xs, void* ws, size_t ws_bytes,
                                  void* stream) {
@@ -487,8 +542,9 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));
   uint16_t* scales = reinterpret_cast<uint16_t*>(ws_at(ws, L.scales));
   uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
+  void* wq = materialize_w(dp, T) ? ws_at(ws, L.wq) : nullptr;
   st = cuda_status(launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros, status,
-                                   device_sms(), s, true));
+                                   device_sms(), s, true, wq));
   if (st != TTQ_OK || T == 0) return st;
 
   // (3) Y = W_hat X (+ B (A X))
@@ -504,7 +560,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
     Bb = bb;
   }
   return run_gemm(codes, scales, zeros, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
-                  y_dtype == TTQ_F32, ws, L, s, true);
+                  y_dtype == TTQ_F32, ws, L, s, true, wq);
 }
 
 ttq_status ttq_get_status(const void* ws, uint32_t* flags) {
@@ -530,6 +586,6 @@ const char* ttq_status_string(ttq_status s) {
   return "unknown status";
 }
 
-const char* ttq_version(void) { return "0.1.0"; }
+const char* ttq_version(void) { return "0.2.0"; }
 
 }  // extern "C"

@@ -62,11 +62,12 @@ cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t 
                                   void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
                                   bool* launched);
 
-// Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null).
+// Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null); with wq
+// non-null also the dequantised weight s (q - z) as binary16 [dp][d].
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,
                             uint16_t* zeros, uint32_t* status, int num_sms,
-                            cudaStream_t stream, bool pdl = false);
+                            cudaStream_t stream, bool pdl = false, void* wq = nullptr);
 
 // float32 -> bf16 copy of n elements (n % 8 == 0).
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);
@@ -87,7 +88,7 @@ struct GemmArgs {
   const uint32_t* codes = nullptr;
   const uint16_t* scales = nullptr;
   const uint16_t* zeros = nullptr;
-  int bits = 0;               // 0: A operand loaded by TMA from tmA0 (plain bf16 x bf16)
+  int bits = 0;               // 0: A operand loaded by TMA from tmA0 (plain mode)
   int group = 0;
   // sizes
   int64_t K = 0;        // reduction length of the main part (d)
@@ -99,17 +100,18 @@ struct GemmArgs {
   int64_t ldy = 0;
   bool y_f32 = false;
   uint32_t* status = nullptr;
+  bool a_f16 = false;      // plain mode: the A operand (maps.a0) is binary16, not bf16
   bool codes_tma = false;  // codes tile loaded by TMA (maps.c0); else per-thread loads
   bool y_tma = false;      // bf16 Y stored by TMA (maps.y, box block_m x block_n)
 };
 
 struct GemmMaps {
-  CUtensorMap a0;  // plain A operand [M][K] bf16 (bits == 0)
+  CUtensorMap a0;  // plain A operand [M][K] bf16 or binary16 (bits == 0), box 64 x block_m
   CUtensorMap b0;  // binary16 X D^(-1/2) [T][K] with codes (bits != 0); bf16 X in the plain mode
   CUtensorMap a1;  // low-rank B [M][r] bf16
   CUtensorMap b1;  // A X [T][r] bf16
   CUtensorMap c0;  // packed codes [M][K*bits/32] uint32, box gemm_code_tile_words x block_m
-  CUtensorMap y;   // bf16 Y [T][ldy], box block_m x block_n, no swizzle
+  CUtensorMap y;   // bf16 Y [T][ldy], box 32 x 16 (rows of W x tokens), no swizzle
 };
 
 // Words per row of the code tile one K block of 64 channels needs.
@@ -118,8 +120,10 @@ int gemm_code_tile_words(int bits);
 // Tile width along the tokens for T tokens.
 int gemm_block_n(int64_t T);
 
-// Tile height (128 or 256 rows of W) for this problem; 256 only with codes.
-int gemm_block_m(int bits, int64_t M, int64_t T, int block_n, int num_sms);
+// Tile shape of the product for this problem: block_m 128 or 256 rows of W
+// (256 only with codes), block_n a multiple of 16 up to 256 tokens, chosen
+// so that the CTAs fill the SMs in as few, as full waves as possible.
+void gemm_tile_shape(int bits, int64_t M, int64_t T, int num_sms, int* block_m, int* block_n);
 
 // The operand boxes: a0/a1 are loaded as block_m x 64, b0/b1 as block_n x 64.
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,

@@ -42,7 +42,7 @@ _SZ = ctypes.c_size_t
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("status", _SZ), ("D", _SZ), ("D_rsqrt", _SZ), ("partial", _SZ), ("codes", _SZ),
                 ("scales", _SZ), ("zeros", _SZ), ("ax", _SZ), ("xh", _SZ), ("xb", _SZ), ("ab", _SZ),
-                ("total", _SZ), ("splits", _I64), ("ax_ld", _I64)]
+                ("wq", _SZ), ("total", _SZ), ("splits", _I64), ("ax_ld", _I64)]
 
 
 SIGNATURES = {
@@ -54,6 +54,9 @@ SIGNATURES = {
     "ttq_act_norm_noalloc": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P]),
     "ttq_act_norm_scale": (_INT, [_P, _INT, _I64, _I64, _F, _F, _F, _P, _P, _P, _P, _SZ, _P]),
     "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
+    "ttq_quantize_dequant_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _P,
+                                           _SZ, _P]),
+    "ttq_dequantized_gemm": (_INT, [_P, _P, _I64, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "ttq_scale_activations": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
                                 _P, _INT, _P, _SZ, _P]),
@@ -250,6 +253,42 @@ def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zer
     return codes, scales, zeros
 
 
+def ttq_quantize_dequant_weight(W, D, bits, group, ws=None, codes=None, scales=None, zeros=None,
+                                W_hat=None, stream=None):
+    """ttq_quantize_weight plus W_hat [d'][d] binary16 (torch.float16) = s (q - z)."""
+    dp, d = W.shape
+    dev = W.device
+    if ws is None:
+        ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
+    if codes is None:
+        codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
+    if zeros is None:
+        zeros = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
+    if W_hat is None:
+        W_hat = torch.empty((dp, d), dtype=torch.float16, device=dev)
+    _check(lib().ttq_quantize_dequant_weight(
+        _dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group, _dev(codes, "codes"),
+        _dev(scales, "scales"), _dev(zeros, "zeros"), _dev(W_hat, "W_hat"), _dev(ws, "ws"),
+        ws.numel(), _stream(stream)), "ttq_quantize_dequant_weight")
+    return codes, scales, zeros, W_hat
+
+
+def ttq_dequantized_gemm(W_hat, Xs, ws=None, Y=None, y_dtype=torch.bfloat16, stream=None):
+    """Y [T][d'] = W_hat Xs^T from a binary16 dequantised weight and binary16 X D^{-1/2}."""
+    dp, d = W_hat.shape
+    T = Xs.shape[0]
+    if ws is None:
+        ws = new_workspace(d, 0, 0, 0, 4, 32, TTQ_BF16, W_hat.device, stream)
+    if Y is None:
+        Y = torch.empty((T, dp), dtype=y_dtype, device=W_hat.device)
+    _check(lib().ttq_dequantized_gemm(_dev(W_hat, "W_hat"), _dev(Xs, "Xs"), d, dp, T, _dev(Y, "Y"),
+                                      _dtype_code(Y), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+           "ttq_dequantized_gemm")
+    return Y
+
+
 def ttq_scale_activations(X, D_rsqrt, ws=None, Xs=None, stream=None):
     """Xs [T][d] binary16 (torch.float16) = X * D^{-1/2}, the product's B operand."""
     T, d = X.shape
@@ -317,4 +356,6 @@ def workspace_views(ws: torch.Tensor, d, dp, T, r, bits, group, dtype=TTQ_BF16) 
         out["scales"] = view(L.scales, dp * (d // group), torch.int16).view(dp, -1)
         out["zeros"] = view(L.zeros, dp * (d // group), torch.int16).view(dp, -1)
         out["xh"] = view(L.xh, T * d, torch.float16).view(T, d)
+        if L.wq:
+            out["wq"] = view(L.wq, dp * d, torch.float16).view(dp, d)
     return out

@@ -62,6 +62,14 @@ def test_workspace_layout_is_consistent(L):
             assert lay.xb > 0 and lay.ab > 0
 
 
+def test_dequantised_weight_only_for_long_inputs(L):
+    """The forward materialises s (q - z) only for more than 256 tokens."""
+    for T in (0, 1, 16, 256):
+        assert ttq.ttq_workspace_get_layout(4096, 4096, T, 0, 4, 128, ttq.TTQ_BF16).wq == 0
+    lay = ttq.ttq_workspace_get_layout(4096, 4096, 257, 0, 4, 128, ttq.TTQ_BF16)
+    assert lay.wq % 256 == 0 and lay.wq > lay.zeros and lay.wq + 4096 * 4096 * 2 <= lay.total
+
+
 @pytest.mark.parametrize("args", [
     (4096, 4096, 2048, 0, 5, 128),   # bits not built
     (4096, 4096, 2048, 0, 4, 96),    # group not built
@@ -91,6 +99,13 @@ def test_rejections_before_device_work(L):
     assert L.ttq_act_norm_scale(16, 1, 64, 4, 0.5, 0.0, 0.5, None, None, 32, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_act_norm_scale(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 32, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
     assert L.ttq_act_norm_scale(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 40, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
+    # dequantised-weight entry points: W_hat required, shapes checked before any CUDA call
+    assert L.ttq_quantize_dequant_weight(16, 1, 4, 64, None, 4, 64, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_quantize_dequant_weight(16, 1, 4, 64, None, 5, 64, 16, 16, 16, 16, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert L.ttq_dequantized_gemm(16, 16, 60, 4, 4, 16, 1, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_dequantized_gemm(16, None, 64, 4, 4, 16, 1, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_dequantized_gemm(16, 16, 64, 4, 4, 16, 1, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
+    assert L.ttq_dequantized_gemm(16, 16, 64, 4, 4, 16, 2, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
     # forward with a null weight
     st = L.ttq_linear_forward(16, None, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 16, 1, 256, 1 << 30, None)
     assert st == ttq.TTQ_ERR_INVALID_ARG
