@@ -22,7 +22,8 @@
  *   - the range is min/max extended to include 0; the scale is rounded to
  *     binary16 toward +infinity and floored at 2^-14; the zero point is an
  *     integer in [0, 2^b-1]; codes are q = clamp(rint(x * (1/s)) + z);
- *     rint is round-half-to-even; reconstruction is s (q - z);
+ *     rint is round-half-to-even of the exact product; reconstruction is
+ *     s (q - z);
  *   - the W given to the forward is the residual W_q is formed from; B, A
  *     are static and B (A X) is added unscaled.
  *
@@ -164,6 +165,9 @@ static void put_code(uint32_t* row, int64_t i, int bits, uint32_t q) {
  *   inv  = 1 / s
  *   z    = clamp(rint(-m * inv), 0, 2^b - 1)   -> zeros[j][k] (binary16)
  *   q    = clamp(rint(x * inv) + z, 0, 2^b - 1) -> codes
+ * The two products inside rint are exact (binary32 x binary32 fits in
+ * binary64), so each code is rint of the true x * inv: one rounding, to the
+ * integer, half to even.
  * W and D are binary32 arrays (bf16 inputs widen to binary32 exactly).    */
 int ttqo_quantize(const float* W, int64_t dp, int64_t d, const float* D,
                   int bits, int group, uint32_t* codes, uint16_t* scales,
@@ -206,12 +210,12 @@ int ttqo_quantize(const float* W, int64_t dp, int64_t d, const float* D,
       if ((s16 & 0x7c00) == 0x7c00) flags |= TTQO_NONFINITE;
       float s = ttqo_f16_to_f32(s16);
       float inv = 1.0f / s;
-      float zr = rintf(-m * inv);
-      int z = (int)(zr < 0.0f ? 0.0f : (zr > (float)qmax ? (float)qmax : zr));
+      double zr = rint(-(double)m * (double)inv);
+      int z = (int)(zr < 0.0 ? 0.0 : (zr > (double)qmax ? (double)qmax : zr));
       scales[j * ngroups + k] = s16;
       zeros[j * ngroups + k] = f16_from_small_int(z);
       for (int c = 0; c < group; ++c) {
-        float r = rintf(x[c] * inv);
+        double r = rint((double)x[c] * (double)inv);
         long q = (long)r + z;
         if (q < 0) q = 0;
         if (q > qmax) q = qmax;

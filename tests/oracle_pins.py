@@ -200,6 +200,26 @@ def check_ties_even(O):
     assert q[1, 2:8].tolist() == [8, 6, 6, 8, 10, 10], q[1]
 
 
+def check_code_rounding_exact_product(O):
+    """The code rounds the exact product x * (1/s), not its binary32 rounding.
+    Group [0, 45] gives s = 3 and z = 0, inv = binary32(1/3).  For x =
+    28.499998092651367 the binary32 product is exactly 9.5 (rint: 10) while
+    the true product is 9.49999964... (rint: 9); x = 28.5 is a control."""
+    bits, group = 4, 32
+    row = np.zeros(32, np.float32)
+    row[0], row[1] = 0.0, 45.0
+    x_tie = np.float32(28.499998092651367)
+    row[2], row[3] = x_tie, 28.5
+    inv = np.float32(1.0) / np.float32(3.0)
+    assert np.float32(x_tie * inv) == np.float32(9.5)            # the binary32 product is a tie
+    assert float(x_tie) * float(inv) < 9.5                       # the true one is below it
+    codes, sc, ze, st = O.quantize(row[None, :], None, bits, group)
+    assert st == 0
+    assert _f16_bits_to_f64(sc).tolist() == [[3.0]] and _f16_bits_to_f64(ze).tolist() == [[0.0]]
+    q = _unpack_np(codes, 32, bits)
+    assert q[0, 1] == 15 and q[0, 2] == 9 and q[0, 3] == 10, q[0, :4]
+
+
 def check_quantizer_properties(O):
     """Codes in range; per-element error <= s/2 (+ reciprocal slack); the
     stored scale is the smallest binary16 value covering the group range;
@@ -354,6 +374,7 @@ ALL_CHECKS = [
     check_act_norm,
     check_exact_grid,
     check_ties_even,
+    check_code_rounding_exact_product,
     check_quantizer_properties,
     check_scaling_and_rows,
     check_dequant_layout,

@@ -23,9 +23,14 @@ MUTANTS = [
     ("range_without_zero", "float m = 0.0f, M = 0.0f;", "float m = 3e38f, M = -3e38f;"),
     ("levels_off_by_one", "float s32 = range / (float)qmax;", "float s32 = range / (float)(qmax + 1);"),
     ("scale_floor_dropped", "if (!(s32 >= 0x1p-14f)) s32 = 0x1p-14f;", ""),
-    ("codes_floor_not_rint", "float r = rintf(x[c] * inv);", "float r = floorf(x[c] * inv);"),
-    ("codes_half_away", "float r = rintf(x[c] * inv);", "float r = roundf(x[c] * inv);"),
-    ("zero_sign_flipped", "float zr = rintf(-m * inv);", "float zr = rintf(m * inv);"),
+    ("codes_floor_not_rint", "double r = rint((double)x[c] * (double)inv);",
+     "double r = floor((double)x[c] * (double)inv);"),
+    ("codes_half_away", "double r = rint((double)x[c] * (double)inv);",
+     "double r = round((double)x[c] * (double)inv);"),
+    ("codes_product_rounded_first", "double r = rint((double)x[c] * (double)inv);",
+     "double r = rint((double)(x[c] * inv));"),
+    ("zero_sign_flipped", "double zr = rint(-(double)m * (double)inv);",
+     "double zr = rint((double)m * (double)inv);"),
     ("zero_point_subtracted", "long q = (long)r + z;", "long q = (long)r - z;"),
     ("min_tracks_max", "if (x[c] < m) m = x[c];", "if (x[c] > m) m = x[c];"),
     ("scale_round_nearest", "double n = sign ? floor(m) : ceil(m);", "double n = nearbyint(m);"),
