@@ -34,8 +34,9 @@
  *      M = max(0, max_group x);  s32 = (M - m) / (2^bits - 1), floored at
  *      2^-14;  s = binary16(s32) rounded toward +inf;  inv = 1 / s;
  *      z = clamp(rint(-m * inv), 0, 2^bits - 1);
- *      q = clamp(rint(x * inv) + z, 0, 2^bits - 1);  rint rounds half to
- *      even.  D == NULL means D = I (plain round-to-nearest).
+ *      q = clamp(rint(x * inv) + z, 0, 2^bits - 1);  rint rounds the
+ *      exact product (no binary32 rounding before it) half to even.
+ *      D == NULL means D = I (plain round-to-nearest).
  *  - All tensor pointers are DEVICE pointers, allocated and owned by the
  *    caller, and must be 16-byte aligned.  The library never allocates
  *    device memory and keeps no per-call state.  Temporary storage is the

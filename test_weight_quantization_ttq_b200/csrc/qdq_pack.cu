@@ -7,9 +7,10 @@
 // the CPU oracle bit for bit:
 //   h = sqrt(D_i); x = W_ji * h; m = min(0, min x); M = max(0, max x);
 //   s32 = (M - m) / (2^b - 1), floored at 2^-14; s = binary16 round-up(s32);
-//   inv = 1 / s; z = clamp(rint(-m * inv)); q = clamp(rint(x * inv) + z).
-// Every operation is an explicitly rounded intrinsic, so no FMA contraction
-// can change a result.
+//   inv = 1 / s; z = clamp(rint(-m * inv)); q = clamp(rint(x * inv) + z),
+// where the two products inside rint are exact (one fused multiply-add
+// rounds them straight to the integer).  Every other operation is an
+// explicitly rounded intrinsic, so no contraction can change a result.
 //
 // Layout of the work: a block owns a tile of `cw` consecutive input channels
 // and walks rows of W with a grid stride.  A thread owns 16 consecutive
@@ -17,8 +18,8 @@
 // for every row it visits, and the group's g/16 threads reduce min/max with
 // shuffles.  A lane's 16 codes fill two words (INT4), one word (INT2) or 48
 // bits (INT3: an even/odd lane pair makes 3 words).  Pairs of weights go
-// through the packed f32x2 multiply/add, which round each lane exactly like
-// the scalar operations.
+// through the packed f32x2 multiply, which rounds each lane exactly like the
+// scalar one (checked on B200 against __fmul_rn).
 // The kernel is HBM-bound: it reads W once and writes d*b/8 + 4d/g bytes per
 // row.
 #include <type_traits>
@@ -69,6 +70,29 @@ __device__ __forceinline__ void unpack16(const Raw16<float>& r, float2 (&x)[8]) 
     x[2 * i] = make_float2(r.v[i].x, r.v[i].y);
     x[2 * i + 1] = make_float2(r.v[i].z, r.v[i].w);
   }
+}
+
+// Three-input minimum / maximum that return NaN if any input is NaN (so a
+// NaN weight reaches the group's range and is flagged there).
+__device__ __forceinline__ float min3_nan(float a, float b, float c) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float max3_nan(float a, float b, float c) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
 }
 
 // With WQ the kernel also writes the dequantised weight s (q - z) as
@@ -133,31 +157,32 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         const bool active = row < dp;
         float2 x[8];
         unpack16(buf[u], x);
-        float2 sum2 = make_float2(0.f, 0.f);
         float mn = 0.f, mx = 0.f;
   #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          x[i].x = __fmul_rn(x[i].x, h[i].x);
-          x[i].y = __fmul_rn(x[i].y, h[i].y);
-          sum2 = __fadd2_rn(sum2, x[i]);  // NaN and Inf survive the sum
-          mn = fminf(mn, fminf(x[i].x, x[i].y));
-          mx = fmaxf(mx, fmaxf(x[i].x, x[i].y));
+          x[i] = __fmul2_rn(x[i], h[i]);
+          mn = min3_nan(mn, x[i].x, x[i].y);
+          mx = max3_nan(mx, x[i].x, x[i].y);
         }
-        bad |= !(fabsf(sum2.x + sum2.y) <= 3.402823466e38f);
         for (int o = gthreads >> 1; o > 0; o >>= 1) {
-          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          mn = min_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = max_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
         }
-        float s32 = __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(QMAX));
+        const float range = __fsub_rn(mx, mn);
+        bad |= !(range <= 3.402823466e38f);  // a NaN or infinite x, or a range beyond binary32
+        float s32 = __fdiv_rn(range, static_cast<float>(QMAX));
         if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
         const __half s16 = __float2half_ru(s32);
         const float s = __half2float(s16);
         const float inv = __fdiv_rn(1.0f, s);
-        const float zr = rintf(__fmul_rn(-mn, inv));
-        const int z = static_cast<int>(fminf(fmaxf(zr, 0.f), static_cast<float>(QMAX)));
-        // rint(x * inv): adding 1.5 * 2^23 rounds to an integer, ties to even,
-        // for |x * inv| < 2^22 (here |x * inv| <= 2^b); the integer is then read
-        // from the low fraction bits
+        // rint of the exact product x * inv: a fused multiply-add with
+        // 1.5 * 2^23 rounds the true product to an integer, ties to even, for
+        // |x * inv| < 2^22 (here |x * inv| <= 2^b + 1); the integer is read
+        // from the low fraction bits.  For a finite group rint(x * inv) + z
+        // is never below 0 (x >= m and rint is odd), so only the top is
+        // clamped.
+        const int zi = __float_as_int(__fmaf_rn(-mn, inv, 12582912.0f)) - 0x4B400000;
+        const int z = min(max(zi, 0), QMAX);
         const int zoff = z - 0x4B400000;
         uint32_t lo = 0, hi = 0;  // codes 0-7 and 8-15 (INT3: 24 bits each)
         uint32_t wh[8];           // s (q - z) of weights 2i, 2i+1 (WQ)
@@ -165,10 +190,10 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         const __half2 s2 = __half2half2(s16);
   #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float r0 = __fadd_rn(__fmul_rn(x[i].x, inv), 12582912.0f);
-          const float r1 = __fadd_rn(__fmul_rn(x[i].y, inv), 12582912.0f);
-          const int q0 = min(max(__float_as_int(r0) + zoff, 0), QMAX);
-          const int q1 = min(max(__float_as_int(r1) + zoff, 0), QMAX);
+          const float r0 = __fmaf_rn(x[i].x, inv, 12582912.0f);
+          const float r1 = __fmaf_rn(x[i].y, inv, 12582912.0f);
+          const int q0 = min(__float_as_int(r0) + zoff, QMAX);
+          const int q1 = min(__float_as_int(r1) + zoff, QMAX);
           const uint32_t pair = static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << BITS);
           if (i < 4) lo |= pair << (2 * BITS * i);
           else hi |= pair << (2 * BITS * (i - 4));
