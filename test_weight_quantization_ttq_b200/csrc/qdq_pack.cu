@@ -72,6 +72,31 @@ __device__ __forceinline__ void unpack16(const Raw16<float>& r, float2 (&x)[8]) 
   }
 }
 
+__device__ __forceinline__ __half2 u32_as_half2(uint32_t u) {
+  __half2 h;
+  memcpy(&h, &u, 4);
+  return h;
+}
+__device__ __forceinline__ uint32_t half2_as_u32(__half2 h) {
+  uint32_t u;
+  memcpy(&u, &h, 4);
+  return u;
+}
+
+// Codes 4k..4k+3 (each < 16) from two pairs of 16-bit lanes a = (q0, q1),
+// b = (q2, q3), as four 4-bit fields in the low 16 bits: a + b * 256 holds
+// q0 | q2 << 8 and q1 | q3 << 8 in its lanes, and OR-ing it with itself
+// shifted right by 12 brings q1 and q3 down to bits 4 and 12.
+__device__ __forceinline__ uint32_t nibbles4(uint32_t a, uint32_t b) {
+  const uint32_t t = a + (b << 8);
+  return t | (t >> 12);
+}
+// The same for codes < 4: four 2-bit fields in the low byte.
+__device__ __forceinline__ uint32_t crumbs4(uint32_t a, uint32_t b) {
+  const uint32_t t = a + (b << 4);
+  return t | (t >> 14);
+}
+
 // Three-input minimum / maximum that return NaN if any input is NaN (so a
 // NaN weight reaches the group's range and is flagged there).
 __device__ __forceinline__ float min3_nan(float a, float b, float c) {
@@ -144,6 +169,13 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
   for (int i = 0; i < 8; ++i) hchk += h[i].x + h[i].y;
   bool bad = !(hchk <= 3.402823466e38f);
   bool ovf = false;
+  // binary32(1 / m) for the 1024 binary16 significands m = 1 + k/1024; the
+  // reciprocal of a normal binary16 s = m 2^e is then this value times
+  // 2^-e, exactly (a power-of-two scaling in the normal range)
+  __shared__ float rcp_sig[1024];
+  for (int k = threadIdx.x; k < 1024; k += kThreads)
+    rcp_sig[k] = __fdiv_rn(1.0f, 1.0f + static_cast<float>(k) * 0.0009765625f);
+  __syncthreads();
 
   // The loop bound is block-uniform so every lane takes part in the
   // shuffles; rows past the end are computed on zeros and not stored.  The
@@ -174,7 +206,11 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
         const __half s16 = __float2half_ru(s32);
         const float s = __half2float(s16);
-        const float inv = __fdiv_rn(1.0f, s);
+        // inv = binary32(1 / s) from the significand table and the exponent
+        // (s >= 2^-14 is normal; an infinite s is flagged below)
+        const uint32_t sbits = __half_as_ushort(s16);
+        const int sexp = static_cast<int>((sbits >> 10) & 31u) - 15;
+        const float inv = __int_as_float(__float_as_int(rcp_sig[sbits & 1023u]) - sexp * (1 << 23));
         // rint of the exact product x * inv: a fused multiply-add with
         // 1.5 * 2^23 rounds the true product to an integer, ties to even, for
         // |x * inv| < 2^22 (here |x * inv| <= 2^b + 1); the integer is read
@@ -183,36 +219,52 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         // clamped.
         const int zi = __float_as_int(__fmaf_rn(-mn, inv, 12582912.0f)) - 0x4B400000;
         const int z = min(max(zi, 0), QMAX);
-        const int zoff = z - 0x4B400000;
-        uint32_t lo = 0, hi = 0;  // codes 0-7 and 8-15 (INT3: 24 bits each)
-        uint32_t wh[8];           // s (q - z) of weights 2i, 2i+1 (WQ)
-        const __half2 zc2 = __half2half2(__hadd(__int2half_rn(z), __ushort_as_half(0x6400)));
-        const __half2 s2 = __half2half2(s16);
+        // the 16 codes as eight (q_2i, q_2i+1) pairs of 16-bit lanes:
+        // rint(x * inv) from the low bits of the fused multiply-add, plus z,
+        // clamped at the top (one packed add-and-min per pair)
+        const uint32_t zz = static_cast<uint32_t>(z) * 0x00010001u;
+        constexpr uint32_t QQ = static_cast<uint32_t>(QMAX) * 0x00010001u;
+        const float2 inv2 = make_float2(inv, inv);
+        const float2 magic2 = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+        uint32_t qp[8];
   #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const float r0 = __fmaf_rn(x[i].x, inv, 12582912.0f);
-          const float r1 = __fmaf_rn(x[i].y, inv, 12582912.0f);
-          const int q0 = min(__float_as_int(r0) + zoff, QMAX);
-          const int q1 = min(__float_as_int(r1) + zoff, QMAX);
-          const uint32_t pair = static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << BITS);
-          if (i < 4) lo |= pair << (2 * BITS * i);
-          else hi |= pair << (2 * BITS * (i - 4));
-          if (WQ) {
-            const uint32_t m = static_cast<uint32_t>(q0) | (static_cast<uint32_t>(q1) << 16) | 0x64006400u;
-            __half2 hm;
-            memcpy(&hm, &m, 4);
-            const __half2 v = __hmul2(__hsub2(hm, zc2), s2);
-            memcpy(&wh[i], &v, 4);
-          }
+          const float2 r = __ffma2_rn(x[i], inv2, magic2);
+          const uint32_t n = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
+          qp[i] = __viaddmin_s16x2(n, zz, QQ);
         }
         if (WQ && active) {
+          // s (q - z): (1024 + q) - (1024 + z) is exact in binary16, the
+          // product with s rounds once
+          const __half2 zc2 = u32_as_half2((0x6400u | static_cast<uint32_t>(z)) * 0x00010001u);
+          const __half2 s2 = __half2half2(s16);
+          uint32_t wh[8];
+  #pragma unroll
+          for (int i = 0; i < 8; ++i)
+            wh[i] = half2_as_u32(__hmul2(__hsub2(u32_as_half2(qp[i] | 0x64006400u), zc2), s2));
           uint4* dst = reinterpret_cast<uint4*>(wq + row * d + col);
           dst[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
           dst[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
         }
+        uint32_t lo = 0, hi = 0;  // INT4: codes 0-7 and 8-15; INT3: 24 bits each
+        if (BITS == 4) {
+          lo = __byte_perm(nibbles4(qp[0], qp[1]), nibbles4(qp[2], qp[3]), 0x5410);
+          hi = __byte_perm(nibbles4(qp[4], qp[5]), nibbles4(qp[6], qp[7]), 0x5410);
+        } else if (BITS == 2) {
+          lo = __byte_perm(__byte_perm(crumbs4(qp[0], qp[1]), crumbs4(qp[2], qp[3]), 0x0040),
+                           __byte_perm(crumbs4(qp[4], qp[5]), crumbs4(qp[6], qp[7]), 0x0040), 0x5410);
+        } else {
+  #pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t pair = (qp[i] & 0xFFFFu) | ((qp[i] >> 16) << BITS);
+            if (i < 4) lo |= pair << (2 * BITS * i);
+            else hi |= pair << (2 * BITS * (i - 4));
+          }
+        }
         if (active && (tx & (gthreads - 1)) == 0) {
           scales[row * ngroups + kgroup] = s16;
-          zeros[row * ngroups + kgroup] = __int2half_rn(z);
+          zeros[row * ngroups + kgroup] =
+              __hsub(__ushort_as_half(static_cast<uint16_t>(0x6400u | z)), __ushort_as_half(0x6400));
           // s (q - z) is formed in binary16 by the product: |q - z| <= 2^b - 1
           ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QMAX) > 65504.f;
         }
@@ -220,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         if (BITS == 4) {
           if (active) *reinterpret_cast<uint2*>(codes + row * wpr + (col >> 3)) = make_uint2(lo, hi);
         } else if (BITS == 2) {
-          if (active) codes[row * wpr + (col >> 4)] = lo | (hi << 16);
+          if (active) codes[row * wpr + (col >> 4)] = lo;
         } else {
           // 48 bits per lane; an even/odd lane pair makes 3 words
           const uint32_t a = lo | (hi << 24);  // bits 0-31
