@@ -228,6 +228,77 @@ int ttqo_quantize(const float* W, int64_t dp, int64_t d, const float* D,
   return flags;
 }
 
+/* Step 2, symmetric variant (blog.lo0.es "Test-time quantization ...",
+ * section "The maths that matter": a symmetric b-bit range has levels
+ * +-(2^(b-1) - 1) and the scale that covers a group of largest magnitude M
+ * is M / (2^(b-1) - 1); every element is then off by at most s/2).
+ * Binary32, in this order:
+ *   h_i  = sqrt(D_i)                     (1 when D is NULL)
+ *   x    = W[j][i] * h_i
+ *   M    = max_group |x|
+ *   s32  = M / (2^(b-1) - 1);  if !(s32 >= 2^-14) s32 = 2^-14
+ *   s    = binary16(s32, toward +inf)   -> scales[j][k]
+ *   inv  = 1 / s
+ *   l    = clamp(rint(x * inv), -(2^(b-1) - 1), 2^(b-1) - 1)  (exact product)
+ *   code = l + 2^(b-1)  in [1, 2^b - 1];  zeros[j][k] = 2^(b-1)
+ * so that the stored (code, scale, zero) reconstruct s (code - zero) = s l
+ * exactly as the asymmetric format does.  Needs bits >= 2.                */
+int ttqo_quantize_sym(const float* W, int64_t dp, int64_t d, const float* D,
+                      int bits, int group, uint32_t* codes, uint16_t* scales,
+                      uint16_t* zeros) {
+  if (!W || !codes || !scales || !zeros || dp < 0 || d < 1 || bits < 2 ||
+      bits > 8 || group < 1 || d % group != 0)
+    return TTQO_BAD_ARG;
+  int flags = TTQO_OK;
+  const int lmax = (1 << (bits - 1)) - 1;
+  const int zero = 1 << (bits - 1);
+  const int64_t wpr = ttqo_words_per_row(d, bits);
+  const int64_t ngroups = d / group;
+  float* sq = (float*)malloc(sizeof(float) * (size_t)d);  /* sqrt(D_i) */
+  float* v = (float*)malloc(sizeof(float) * (size_t)group);  /* prescaled group */
+  if (!sq || !v) {
+    free(sq);
+    free(v);
+    return TTQO_BAD_ARG;
+  }
+  for (int64_t i = 0; i < d; ++i) {
+    sq[i] = D ? sqrtf(D[i]) : 1.0f;
+    if (!isfinite(sq[i])) flags |= TTQO_NONFINITE;
+  }
+  memset(codes, 0, sizeof(uint32_t) * (size_t)(dp * wpr));
+  for (int64_t j = 0; j < dp; ++j) {
+    uint32_t* crow = codes + j * wpr;
+    for (int64_t k = 0; k < ngroups; ++k) {
+      float M = 0.0f;
+      for (int c = 0; c < group; ++c) {
+        int64_t i = k * group + c;
+        float w = W[j * d + i];
+        if (!isfinite(w)) flags |= TTQO_NONFINITE;
+        v[c] = w * sq[i];
+        float a = fabsf(v[c]);
+        if (a > M) M = a;
+      }
+      float s32 = M / (float)lmax;
+      if (!(s32 >= 0x1p-14f)) s32 = 0x1p-14f; /* binary16 normal range */
+      uint16_t s16 = ttqo_f32_to_f16_ru(s32);
+      if ((s16 & 0x7c00) == 0x7c00) flags |= TTQO_NONFINITE;
+      float s = ttqo_f16_to_f32(s16);
+      float inv = 1.0f / s;
+      scales[j * ngroups + k] = s16;
+      zeros[j * ngroups + k] = f16_from_small_int(zero);
+      for (int c = 0; c < group; ++c) {
+        long l = (long)rint((double)v[c] * (double)inv);
+        if (l < -lmax) l = -lmax;
+        if (l > lmax) l = lmax;
+        put_code(crow, k * group + c, bits, (uint32_t)(l + zero));
+      }
+    }
+  }
+  free(sq);
+  free(v);
+  return flags;
+}
+
 /* Step 3: W_hat = Q[.] D^{-1/2}: w_hat[j][i] = s_jk (q_ji - z_jk) Dr_i, in
  * fp64, for the listed rows only (rows == NULL means rows 0..nrows-1).
  * Dr == NULL means D = I.                                                  */

@@ -73,6 +73,8 @@ class Oracle:
         lib.ttqo_unpack.restype = ctypes.c_int
         lib.ttqo_quantize.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P]
         lib.ttqo_quantize.restype = ctypes.c_int
+        lib.ttqo_quantize_sym.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P]
+        lib.ttqo_quantize_sym.restype = ctypes.c_int
         lib.ttqo_dequant_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _I64, _P]
         lib.ttqo_dequant_rows.restype = ctypes.c_int
         lib.ttqo_project.argtypes = [_P, _I64, _P, _I64, _I64, _P]
@@ -106,8 +108,11 @@ class Oracle:
     def words_per_row(self, d: int, bits: int) -> int:
         return int(self.lib.ttqo_words_per_row(d, bits))
 
-    def quantize(self, W: np.ndarray, D: np.ndarray | None, bits: int, group: int):
-        """Q[W D^{1/2}] in the binary32 operation order; W is [d'][d]."""
+    def quantize(self, W: np.ndarray, D: np.ndarray | None, bits: int, group: int,
+                 symmetric: bool = False):
+        """Q[W D^{1/2}] in the binary32 operation order; W is [d'][d].
+        symmetric=True: the symmetric quantiser (levels +-(2^(b-1)-1), zero
+        point 2^(b-1) stored with the codes)."""
         W = np.ascontiguousarray(W, dtype=np.float32)
         dp, d = W.shape
         wpr = self.words_per_row(d, bits)
@@ -119,8 +124,9 @@ class Oracle:
         if D is not None:
             D32 = np.ascontiguousarray(D, dtype=np.float32)
             Dp = D32.ctypes.data
-        st = self.lib.ttqo_quantize(W.ctypes.data, dp, d, Dp, bits, group,
-                                    codes.ctypes.data, scales.ctypes.data, zeros.ctypes.data)
+        fn = self.lib.ttqo_quantize_sym if symmetric else self.lib.ttqo_quantize
+        st = fn(W.ctypes.data, dp, d, Dp, bits, group,
+                codes.ctypes.data, scales.ctypes.data, zeros.ctypes.data)
         return codes, scales, zeros, st
 
     def code_at(self, codes_row: np.ndarray, i: int, bits: int) -> int:
@@ -184,7 +190,8 @@ class Oracle:
         return Y
 
     # -- the whole layer ----------------------------------------------------
-    def forward(self, X, W, p, lam, alpha, bits, group, A=None, B=None, rows=None):
+    def forward(self, X, W, p, lam, alpha, bits, group, A=None, B=None, rows=None,
+                symmetric=False):
         """The TTQ linear layer for the listed output rows.
 
         Returns a dict with D, Dr (fp64), the codes/scales/zeros of all rows
@@ -192,7 +199,7 @@ class Oracle:
         """
         X = np.ascontiguousarray(X, dtype=np.float64)
         D, Dr, st1 = self.act_norm(X, p, lam, alpha)
-        codes, scales, zeros, st2 = self.quantize(W, D.astype(np.float32), bits, group)
+        codes, scales, zeros, st2 = self.quantize(W, D.astype(np.float32), bits, group, symmetric)
         d = X.shape[1]
         What = self.dequant_rows(codes, scales, zeros, Dr, d, bits, group, rows)
         Y = self.project(What, X)

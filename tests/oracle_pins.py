@@ -220,6 +220,84 @@ def check_code_rounding_exact_product(O):
     assert q[0, 1] == 15 and q[0, 2] == 9 and q[0, 3] == 10, q[0, :4]
 
 
+def check_symmetric_worked_example(O):
+    """The symmetric INT4 quantiser on the blog's group ("The maths that
+    matter"): magnitudes 1 with one 30 give s = 30/7 (here the binary16 value
+    just above it) and errors up to s/2 ~ 2.14 on the unit values; without
+    the 30 the scale is 1/7 and the errors at most ~0.071, thirty times
+    less.  Levels are +-7 around the stored zero point 8."""
+    bits, group = 4, 32
+    row = np.ones(32, np.float32)
+    row[1::2] = -1.0
+    row[5] = 30.0
+    codes, sc, ze, st = O.quantize(row[None, :], None, bits, group, symmetric=True)
+    assert st == 0
+    s = float(_f16_bits_to_f64(sc)[0, 0])
+    assert 30.0 / 7.0 <= s <= 30.0 / 7.0 * (1 + 2.0 ** -10), s
+    assert _f16_bits_to_f64(ze).tolist() == [[8.0]]
+    q = _unpack_np(codes, 32, bits)[0]
+    assert q[5] == 15 and q.min() >= 1 and q.max() <= 15
+    rec = s * (q.astype(np.float64) - 8.0)
+    unit_err = np.abs(rec - row)[np.arange(32) != 5]
+    assert unit_err.max() <= s / 2 and abs(s / 2 - 2.1428571) < 2e-3, (unit_err.max(), s)
+    # segregated: the same unit values without the outlier
+    row2 = row.copy()
+    row2[5] = 1.0
+    codes2, sc2, _, _ = O.quantize(row2[None, :], None, bits, group, symmetric=True)
+    s2 = float(_f16_bits_to_f64(sc2)[0, 0])
+    assert 1.0 / 7.0 <= s2 <= 1.0 / 7.0 * (1 + 2.0 ** -10), s2
+    err2 = np.abs(s2 * (_unpack_np(codes2, 32, bits)[0] - 8.0) - row2)
+    assert err2.max() <= s2 / 2 and abs(s2 / 2 - 0.0714286) < 1e-4
+    assert 29.0 < s / s2 < 31.0
+    # the asymmetric quantiser on the outlier group: s = (30 - m) / 15, m = -1
+    codes3, sc3, ze3, _ = O.quantize(row[None, :], None, bits, group)
+    s3 = float(_f16_bits_to_f64(sc3)[0, 0])
+    assert 31.0 / 15.0 <= s3 <= 31.0 / 15.0 * (1 + 2.0 ** -10)
+    rec3 = s3 * (_unpack_np(codes3, 32, bits)[0] - _f16_bits_to_f64(ze3)[0, 0])
+    assert np.abs(rec3 - row).max() <= s3 / 2 * (1 + 1e-6)
+
+
+def check_symmetric_properties(O):
+    """Symmetric quantiser: codes in [1, 2^b - 1], zero point 2^(b-1), every
+    element within s/2, the nearest of the 2^b - 1 levels (ties to even),
+    s the smallest binary16 covering max|x| (or the 2^-14 floor), and odd
+    symmetry: -W gives the mirrored codes."""
+    rng = np.random.default_rng(11)
+    for bits in (2, 3, 4):
+        for group in (32, 128):
+            dp, d = 8, 256
+            W = _rand_weights(rng, dp, d)
+            W[0, :group] = 0.0
+            D = np.exp(rng.uniform(-3, 3, d)).astype(np.float32)
+            codes, sc, ze, st = O.quantize(W, D, bits, group, symmetric=True)
+            assert st == 0
+            lmax = (1 << (bits - 1)) - 1
+            zero = 1 << (bits - 1)
+            q = _unpack_np(codes, d, bits)
+            assert q.min() >= 1 and q.max() <= 2 * lmax + 1, (bits, group)
+            assert np.all(_f16_bits_to_f64(ze) == zero)
+            x = (W.astype(np.float32) * np.sqrt(D).astype(np.float32)[None, :]).astype(np.float64)
+            s = np.repeat(_f16_bits_to_f64(sc), group, axis=1)
+            lev = q.astype(np.float64) - zero
+            err = np.abs(x - s * lev)
+            assert np.all(err <= s / 2 * (1 + 1e-6)), (bits, group)
+            levels = np.arange(-lmax, lmax + 1)[None, None, :]
+            dist = np.abs(x[:, :, None] - s[:, :, None] * levels)
+            best = dist.min(axis=2)
+            near_tie = np.abs(np.abs(x / s - np.round(x / s)) - 0.5) < 1e-5
+            assert np.all((err <= best * (1 + 1e-9) + 1e-300) | near_tie), (bits, group)
+            M = np.abs(x).reshape(dp, d // group, group).max(axis=2)
+            s16 = sc.view(np.float16)
+            sv = s16.astype(np.float64)
+            floor_ok = sv == 2.0 ** -14
+            assert np.all(sv * lmax >= M * (1 - 2.0 ** -22))
+            below = np.nextafter(s16, np.float16(0)).astype(np.float64)
+            assert np.all(floor_ok | (below * lmax < M * (1 + 2.0 ** -22))), (bits, group)
+            codes_n, sc_n, _, _ = O.quantize(-W, D, bits, group, symmetric=True)
+            assert np.array_equal(sc_n, sc)
+            assert np.array_equal(_unpack_np(codes_n, d, bits), 2 * zero - q), (bits, group)
+
+
 def check_quantizer_properties(O):
     """Codes in range; per-element error <= s/2 (+ reciprocal slack); the
     stored scale is the smallest binary16 value covering the group range;
@@ -375,6 +453,8 @@ ALL_CHECKS = [
     check_exact_grid,
     check_ties_even,
     check_code_rounding_exact_product,
+    check_symmetric_worked_example,
+    check_symmetric_properties,
     check_quantizer_properties,
     check_scaling_and_rows,
     check_dequant_layout,

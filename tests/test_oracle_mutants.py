@@ -22,13 +22,22 @@ MUTANTS = [
     ("prescale_divides", "x[c] = w * h[i];", "x[c] = w / h[i];"),
     ("range_without_zero", "float m = 0.0f, M = 0.0f;", "float m = 3e38f, M = -3e38f;"),
     ("levels_off_by_one", "float s32 = range / (float)qmax;", "float s32 = range / (float)(qmax + 1);"),
-    ("scale_floor_dropped", "if (!(s32 >= 0x1p-14f)) s32 = 0x1p-14f;", ""),
+    ("scale_floor_dropped", "float s32 = range / (float)qmax;\n      if (!(s32 >= 0x1p-14f)) s32 = 0x1p-14f;",
+     "float s32 = range / (float)qmax;"),
+    ("sym_scale_floor_dropped", "if (!(s32 >= 0x1p-14f)) s32 = 0x1p-14f; /* binary16 normal range */", ""),
     ("codes_floor_not_rint", "double r = rint((double)x[c] * (double)inv);",
      "double r = floor((double)x[c] * (double)inv);"),
     ("codes_half_away", "double r = rint((double)x[c] * (double)inv);",
      "double r = round((double)x[c] * (double)inv);"),
     ("codes_product_rounded_first", "double r = rint((double)x[c] * (double)inv);",
      "double r = rint((double)(x[c] * inv));"),
+    ("sym_levels_unsigned", "const int lmax = (1 << (bits - 1)) - 1;", "const int lmax = (1 << bits) - 1;"),
+    ("sym_range_signed_max", "float a = fabsf(v[c]);", "float a = v[c];"),
+    ("sym_prescale_divides", "v[c] = w * sq[i];", "v[c] = w / sq[i];"),
+    ("sym_codes_floor", "long l = (long)rint((double)v[c] * (double)inv);",
+     "long l = (long)floor((double)v[c] * (double)inv);"),
+    ("sym_zero_dropped", "zeros[j * ngroups + k] = f16_from_small_int(zero);",
+     "zeros[j * ngroups + k] = f16_from_small_int(0);"),
     ("zero_sign_flipped", "double zr = rint(-(double)m * (double)inv);",
      "double zr = rint((double)m * (double)inv);"),
     ("zero_point_subtracted", "long q = (long)r + z;", "long q = (long)r - z;"),
