@@ -82,6 +82,18 @@ typedef enum ttq_dtype {
   TTQ_F16 = 2   /* binary16: only for X of ttq_scale_activations and ttq_dequant_gemm */
 } ttq_dtype;
 
+/* The quantiser's code scheme (blog.lo0.es "Test-time quantization ...",
+ * section "The maths that matter").  TTQ_QSCHEME_ASYMMETRIC: the range
+ * [min(0, min x), max(0, max x)] over 2^bits - 1 steps with an integer zero
+ * point (the default everywhere).  TTQ_QSCHEME_SYMMETRIC: levels
+ * +-(2^(bits-1) - 1) with scale max|x| / (2^(bits-1) - 1); the codes are
+ * stored as level + 2^(bits-1), and the zero point 2^(bits-1) is stored in
+ * `zeros`, so both schemes dequantise as scales * (code - zeros). */
+typedef enum ttq_qscheme {
+  TTQ_QSCHEME_ASYMMETRIC = 0,
+  TTQ_QSCHEME_SYMMETRIC = 1
+} ttq_qscheme;
+
 /* Device status word bits (ttq_get_status). */
 #define TTQ_FLAG_NONFINITE 0x1u
 #define TTQ_FLAG_SCALE_OVERFLOW 0x2u
@@ -199,6 +211,21 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
                                uint16_t* scales, uint16_t* zeros, void* ws,
                                size_t ws_bytes, void* stream);
 
+/* ttq_quantize_weight with a choice of code scheme and an optional
+ * dequantised binary16 weight (as ttq_quantize_dequant_weight writes it;
+ * W_hat may be NULL).  With TTQ_QSCHEME_SYMMETRIC the binary32 order is
+ *   h = sqrtf(D_i); x = W_ji * h; M = max_group |x|;
+ *   s32 = M / (2^(bits-1) - 1), floored at 2^-14; s = binary16 round-up;
+ *   inv = 1 / s; level = clamp(rint(x * inv), -(2^(bits-1)-1), 2^(bits-1)-1)
+ *   (exact product, half to even); code = level + 2^(bits-1);
+ *   zeros = 2^(bits-1)
+ * (a finite group never needs the clamp).  Flags as ttq_quantize_weight
+ * (SCALE_OVERFLOW when s * (2^(bits-1) - 1) exceeds binary16). */
+ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                                  const float* D, int bits, int group, ttq_qscheme scheme,
+                                  uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                                  uint16_t* W_hat, void* ws, size_t ws_bytes, void* stream);
+
 /* ttq_quantize_weight that also writes the dequantised weight
  *   W_hat[j][i] = binary16(s[j][k] * (q[j][i] - z[j][k]))
  * (binary16 bit patterns, [dp][d] row-major, 16-byte aligned; required
@@ -274,6 +301,14 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A,
                               int64_t T, int64_t r, float p, float lambda, float alpha,
                               int bits, int group, void* Y, ttq_dtype y_dtype, void* ws,
                               size_t ws_bytes, void* stream);
+
+/* ttq_linear_forward with a choice of code scheme (TTQ_QSCHEME_ASYMMETRIC
+ * is exactly ttq_linear_forward). */
+ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A,
+                                 const void* B, ttq_dtype dtype, int64_t d, int64_t dp,
+                                 int64_t T, int64_t r, float p, float lambda, float alpha,
+                                 int bits, int group, ttq_qscheme scheme, void* Y,
+                                 ttq_dtype y_dtype, void* ws, size_t ws_bytes, void* stream);
 
 /* Number of kernels one ttq_linear_forward call with these sizes enqueues
  * on the current device (host query; no device work), in *kernels:

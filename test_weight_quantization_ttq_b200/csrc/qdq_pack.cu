@@ -124,12 +124,16 @@ __device__ __forceinline__ float max_nan(float a, float b) {
 // binary16 [dp][d] (wq), formed exactly as the product's A operand is
 // formed from the codes: (1024 + q) - (1024 + z) is exact in binary16 and
 // the product with s is rounded once.
-template <typename WT, int BITS, bool WQ>
+// With SYM the symmetric quantiser: the scale covers max|x| with levels
+// +-(2^(b-1) - 1) and the zero point is the constant 2^(b-1), so the stored
+// (code, scale, zero) triples dequantise exactly as the asymmetric ones.
+template <typename WT, int BITS, bool WQ, bool SYM>
 __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
     const WT* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D, int group,
     int cw, uint32_t* __restrict__ codes, __half* __restrict__ scales,
     __half* __restrict__ zeros, __half* __restrict__ wq, uint32_t* __restrict__ status) {
-  constexpr int QMAX = (1 << BITS) - 1;
+  constexpr int QMAX = (1 << BITS) - 1;                     // largest code
+  constexpr int QSPAN = SYM ? (1 << (BITS - 1)) - 1 : QMAX;  // levels the scale spans
   const int tpr = cw >> 4;            // threads per row of the tile (16 weights each)
   const int rpi = kThreads / tpr;     // rows per iteration of the block
   const int tx = threadIdx.x % tpr;
@@ -202,7 +206,10 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         }
         const float range = __fsub_rn(mx, mn);
         bad |= !(range <= 3.402823466e38f);  // a NaN or infinite x, or a range beyond binary32
-        float s32 = __fdiv_rn(range, static_cast<float>(QMAX));
+        // asymmetric: the range [m, M] over 2^b - 1 steps; symmetric: max|x|
+        // over 2^(b-1) - 1 steps
+        const float span = SYM ? max_nan(mx, -mn) : range;
+        float s32 = __fdiv_rn(span, static_cast<float>(QSPAN));
         if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
         const __half s16 = __float2half_ru(s32);
         const float s = __half2float(s16);
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         // is never below 0 (x >= m and rint is odd), so only the top is
         // clamped.
         const int zi = __float_as_int(__fmaf_rn(-mn, inv, 12582912.0f)) - 0x4B400000;
-        const int z = min(max(zi, 0), QMAX);
+        const int z = SYM ? (1 << (BITS - 1)) : min(max(zi, 0), QMAX);
         // the 16 codes as eight (q_2i, q_2i+1) pairs of 16-bit lanes:
         // rint(x * inv) from the low bits of the fused multiply-add, plus z,
         // clamped at the top (one packed add-and-min per pair)
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
           zeros[row * ngroups + kgroup] =
               __hsub(__ushort_as_half(static_cast<uint16_t>(0x6400u | z)), __ushort_as_half(0x6400));
           // s (q - z) is formed in binary16 by the product: |q - z| <= 2^b - 1
-          ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QMAX) > 65504.f;
+          ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QSPAN) > 65504.f;
         }
         // the lane's 16 codes are 16*BITS bits at bit 16*BITS*(col/16)
         if (BITS == 4) {
@@ -311,7 +318,7 @@ int tile_width(int64_t d, int group) {
   return group;
 }
 
-template <typename WT, bool WQ>
+template <typename WT, bool WQ, bool SYM>
 cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bits, int group,
                      uint32_t* codes, uint16_t* scales, uint16_t* zeros, void* wq,
                      uint32_t* status, int num_sms, cudaStream_t stream, bool pdl) {
@@ -329,13 +336,13 @@ cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bit
   __half* z = reinterpret_cast<__half*>(zeros);
   switch (bits) {
     case 2:
-      return launch_kernel(qdq_pack_kernel<WT, 2, WQ>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
+      return launch_kernel(qdq_pack_kernel<WT, 2, WQ, SYM>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
                            d, D, group, cw, codes, s, z, static_cast<__half*>(wq), status);
     case 3:
-      return launch_kernel(qdq_pack_kernel<WT, 3, WQ>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
+      return launch_kernel(qdq_pack_kernel<WT, 3, WQ, SYM>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
                            d, D, group, cw, codes, s, z, static_cast<__half*>(wq), status);
     case 4:
-      return launch_kernel(qdq_pack_kernel<WT, 4, WQ>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
+      return launch_kernel(qdq_pack_kernel<WT, 4, WQ, SYM>, grid, dim3(kThreads), 0, stream, pdl, W, dp,
                            d, D, group, cw, codes, s, z, static_cast<__half*>(wq), status);
     default:
       return cudaErrorInvalidValue;
@@ -453,23 +460,37 @@ cudaError_t launch_scale_to_f16(const void* src, int src_kind, const float* Dr, 
                        static_cast<const __nv_bfloat16*>(src), Dr, out, T, d, status);
 }
 
+template <typename WT, bool SYM>
+cudaError_t launch_wq(const WT* W, int64_t dp, int64_t d, const float* D, int bits, int group,
+                      uint32_t* codes, uint16_t* scales, uint16_t* zeros, void* wq,
+                      uint32_t* status, int num_sms, cudaStream_t stream, bool pdl) {
+  return wq ? launch_w<WT, true, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq, status,
+                                      num_sms, stream, pdl)
+            : launch_w<WT, false, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq, status,
+                                       num_sms, stream, pdl);
+}
+
+template <typename WT>
+cudaError_t launch_scheme(const WT* W, int64_t dp, int64_t d, const float* D, int bits, int group,
+                          bool symmetric, uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                          void* wq, uint32_t* status, int num_sms, cudaStream_t stream,
+                          bool pdl) {
+  return symmetric ? launch_wq<WT, true>(W, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                         status, num_sms, stream, pdl)
+                   : launch_wq<WT, false>(W, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                          status, num_sms, stream, pdl);
+}
+
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,
                             uint16_t* zeros, uint32_t* status, int num_sms,
-                            cudaStream_t stream, bool pdl, void* wq) {
+                            cudaStream_t stream, bool pdl, void* wq, bool symmetric) {
   if (dp == 0) return cudaSuccess;
-  if (w_f32) {
-    const float* w = static_cast<const float*>(W);
-    return wq ? launch_w<float, true>(w, dp, d, D, bits, group, codes, scales, zeros, wq, status,
-                                      num_sms, stream, pdl)
-              : launch_w<float, false>(w, dp, d, D, bits, group, codes, scales, zeros, wq, status,
-                                       num_sms, stream, pdl);
-  }
-  const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(W);
-  return wq ? launch_w<__nv_bfloat16, true>(w, dp, d, D, bits, group, codes, scales, zeros, wq,
-                                            status, num_sms, stream, pdl)
-            : launch_w<__nv_bfloat16, false>(w, dp, d, D, bits, group, codes, scales, zeros, wq,
-                                             status, num_sms, stream, pdl);
+  if (w_f32)
+    return launch_scheme(static_cast<const float*>(W), dp, d, D, bits, group, symmetric, codes,
+                         scales, zeros, wq, status, num_sms, stream, pdl);
+  return launch_scheme(static_cast<const __nv_bfloat16*>(W), dp, d, D, bits, group, symmetric,
+                       codes, scales, zeros, wq, status, num_sms, stream, pdl);
 }
 
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {

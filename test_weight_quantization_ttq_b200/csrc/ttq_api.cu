@@ -375,31 +375,13 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
   return TTQ_OK;
 }
 
-ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
-                               const float* D, int bits, int group, uint32_t* codes,
-                               uint16_t* scales, uint16_t* zeros, void* ws, size_t ws_bytes,
-                               void* stream) {
-  if (dtype != TTQ_F32 && dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
-  if (bits < 1 || bits > 8 || group < 1) return TTQ_ERR_INVALID_ARG;
-  if (!valid_qparams(bits, group)) return TTQ_ERR_UNSUPPORTED;
-  if (d < group || d % group != 0 || dp < 0) return TTQ_ERR_INVALID_ARG;
-  if (dp > 0 && (W == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr))
-    return TTQ_ERR_INVALID_ARG;
-  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
-  if ((W && !aligned16(W)) || (D && !aligned16(D)) || (codes && !aligned16(codes)))
-    return TTQ_ERR_INVALID_ARG;
-  if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
-  uint32_t* status = static_cast<uint32_t*>(ws);
-  return cuda_status(launch_qdq_pack(W, dtype == TTQ_F32, dp, d, D, bits, group, codes, scales,
-                                     zeros, status, device_sms(),
-                                     static_cast<cudaStream_t>(stream)));
-}
 
-ttq_status ttq_quantize_dequant_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
-                                       const float* D, int bits, int group, uint32_t* codes,
-                                       uint16_t* scales, uint16_t* zeros, uint16_t* W_hat,
-                                       void* ws, size_t ws_bytes, void* stream) {
-  if (dp > 0 && W_hat == nullptr) return TTQ_ERR_INVALID_ARG;
+ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                                  const float* D, int bits, int group, ttq_qscheme scheme,
+                                  uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                                  uint16_t* W_hat, void* ws, size_t ws_bytes, void* stream) {
+  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC)
+    return TTQ_ERR_INVALID_ARG;
   if (W_hat && !aligned16(W_hat)) return TTQ_ERR_INVALID_ARG;
   if (dtype != TTQ_F32 && dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
   if (bits < 1 || bits > 8 || group < 1) return TTQ_ERR_INVALID_ARG;
@@ -413,7 +395,25 @@ ttq_status ttq_quantize_dequant_weight(const void* W, ttq_dtype dtype, int64_t d
   if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
   return cuda_status(launch_qdq_pack(W, dtype == TTQ_F32, dp, d, D, bits, group, codes, scales,
                                      zeros, static_cast<uint32_t*>(ws), device_sms(),
-                                     static_cast<cudaStream_t>(stream), false, W_hat));
+                                     static_cast<cudaStream_t>(stream), false, W_hat,
+                                     scheme == TTQ_QSCHEME_SYMMETRIC));
+}
+
+ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                               const float* D, int bits, int group, uint32_t* codes,
+                               uint16_t* scales, uint16_t* zeros, void* ws, size_t ws_bytes,
+                               void* stream) {
+  return ttq_quantize_weight_ex(W, dtype, dp, d, D, bits, group, TTQ_QSCHEME_ASYMMETRIC, codes,
+                                scales, zeros, nullptr, ws, ws_bytes, stream);
+}
+
+ttq_status ttq_quantize_dequant_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
+                                       const float* D, int bits, int group, uint32_t* codes,
+                                       uint16_t* scales, uint16_t* zeros, uint16_t* W_hat,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  if (dp > 0 && W_hat == nullptr) return TTQ_ERR_INVALID_ARG;
+  return ttq_quantize_weight_ex(W, dtype, dp, d, D, bits, group, TTQ_QSCHEME_ASYMMETRIC, codes,
+                                scales, zeros, W_hat, ws, ws_bytes, stream);
 }
 
 ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64_t d, int64_t dp,
@@ -502,11 +502,14 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
                   y_dtype == TTQ_F32, ws, L, s, pdl);
 }
 
-ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const void* B,
-                              ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
-                              float p, float lambda, float alpha, int bits, int group, void* Y,
-                              ttq_dtype y_dtype, void* ws, size_t ws_bytes, void* stream) {
+ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, const void* B,
+                                 ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
+                                 float p, float lambda, float alpha, int bits, int group,
+                                 ttq_qscheme scheme, void* Y, ttq_dtype y_dtype, void* ws,
+                                 size_t ws_bytes, void* stream) {
   if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
+  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC)
+    return TTQ_ERR_INVALID_ARG;
   if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
     return TTQ_ERR_UNSUPPORTED;
   if (dtype == TTQ_F16) return TTQ_ERR_INVALID_ARG;
@@ -544,7 +547,7 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
   void* wq = materialize_w(dp, T) ? ws_at(ws, L.wq) : nullptr;
   st = cuda_status(launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros, status,
-                                   device_sms(), s, true, wq));
+                                   device_sms(), s, true, wq, scheme == TTQ_QSCHEME_SYMMETRIC));
   if (st != TTQ_OK || T == 0) return st;
 
   // (3) Y = W_hat X (+ B (A X))
@@ -561,6 +564,14 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
   }
   return run_gemm(codes, scales, zeros, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
                   y_dtype == TTQ_F32, ws, L, s, true, wq);
+}
+
+ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const void* B,
+                              ttq_dtype dtype, int64_t d, int64_t dp, int64_t T, int64_t r,
+                              float p, float lambda, float alpha, int bits, int group, void* Y,
+                              ttq_dtype y_dtype, void* ws, size_t ws_bytes, void* stream) {
+  return ttq_linear_forward_ex(X, W, A, B, dtype, d, dp, T, r, p, lambda, alpha, bits, group,
+                               TTQ_QSCHEME_ASYMMETRIC, Y, y_dtype, ws, ws_bytes, stream);
 }
 
 ttq_status ttq_get_status(const void* ws, uint32_t* flags) {

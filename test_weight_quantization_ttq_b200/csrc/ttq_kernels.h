@@ -64,10 +64,12 @@ cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t 
 
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null); with wq
 // non-null also the dequantised weight s (q - z) as binary16 [dp][d].
+// symmetric: the symmetric quantiser (zero point 2^(b-1)).
 cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
                             int bits, int group, uint32_t* codes, uint16_t* scales,
                             uint16_t* zeros, uint32_t* status, int num_sms,
-                            cudaStream_t stream, bool pdl = false, void* wq = nullptr);
+                            cudaStream_t stream, bool pdl = false, void* wq = nullptr,
+                            bool symmetric = false);
 
 // float32 -> bf16 copy of n elements (n % 8 == 0).
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream);

@@ -26,6 +26,9 @@ TTQ_F32 = 0
 TTQ_BF16 = 1
 TTQ_F16 = 2
 
+TTQ_QSCHEME_ASYMMETRIC = 0
+TTQ_QSCHEME_SYMMETRIC = 1
+
 TTQ_FLAG_NONFINITE = 0x1
 TTQ_FLAG_SCALE_OVERFLOW = 0x2
 TTQ_FLAG_TIMEOUT = 0x4
@@ -56,6 +59,10 @@ SIGNATURES = {
     "ttq_quantize_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _SZ, _P]),
     "ttq_quantize_dequant_weight": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _P, _P, _P, _P, _P,
                                            _SZ, _P]),
+    "ttq_quantize_weight_ex": (_INT, [_P, _INT, _I64, _I64, _P, _INT, _INT, _INT, _P, _P, _P, _P, _P,
+                                      _SZ, _P]),
+    "ttq_linear_forward_ex": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT,
+                                     _INT, _INT, _P, _INT, _P, _SZ, _P]),
     "ttq_dequantized_gemm": (_INT, [_P, _P, _I64, _I64, _I64, _P, _INT, _P, _SZ, _P]),
     "ttq_scale_activations": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
@@ -253,6 +260,27 @@ def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zer
     return codes, scales, zeros
 
 
+def ttq_quantize_weight_ex(W, D, bits, group, scheme, ws=None, codes=None, scales=None, zeros=None,
+                           W_hat=None, stream=None):
+    """Codes, scales and zeros under the given TTQ_QSCHEME_*; W_hat (binary16
+    s (q - z), optional) is written when given."""
+    dp, d = W.shape
+    dev = W.device
+    if ws is None:
+        ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
+    if codes is None:
+        codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device=dev)
+    if scales is None:
+        scales = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
+    if zeros is None:
+        zeros = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
+    _check(lib().ttq_quantize_weight_ex(
+        _dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group, scheme, _dev(codes, "codes"),
+        _dev(scales, "scales"), _dev(zeros, "zeros"), _dev(W_hat, "W_hat"), _dev(ws, "ws"), ws.numel(),
+        _stream(stream)), "ttq_quantize_weight_ex")
+    return codes, scales, zeros
+
+
 def ttq_quantize_dequant_weight(W, D, bits, group, ws=None, codes=None, scales=None, zeros=None,
                                 W_hat=None, stream=None):
     """ttq_quantize_weight plus W_hat [d'][d] binary16 (torch.float16) = s (q - z)."""
@@ -324,9 +352,10 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
 
 
 def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, y_dtype=None,
-                       stream=None):
+                       stream=None, scheme=None):
     """The TTQ linear layer: Y [T][d'] = Q[W D^{1/2}] D^{-1/2} X + B (A X);
-    Y in y_dtype (default: the dtype of X, or of a given Y)."""
+    Y in y_dtype (default: the dtype of X, or of a given Y).  scheme: None
+    (ttq_linear_forward) or a TTQ_QSCHEME_* code (ttq_linear_forward_ex)."""
     T, d = X.shape
     dp = W.shape[0]
     r = 0 if A is None else A.shape[0]
@@ -335,10 +364,13 @@ def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, 
         ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
     if Y is None:
         Y = torch.empty((T, dp), dtype=y_dtype or X.dtype, device=X.device)
-    _check(lib().ttq_linear_forward(_dev(X, "X"), _dev(W, "W"), _dev(A, "A"), _dev(B, "B"), dt, d, dp, T,
-                                    r, p, lam, alpha, bits, group, _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"),
-                                    ws.numel(), _stream(stream)),
-           "ttq_linear_forward")
+    args = (_dev(X, "X"), _dev(W, "W"), _dev(A, "A"), _dev(B, "B"), dt, d, dp, T, r, p, lam, alpha, bits,
+            group)
+    tail = (_dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"), ws.numel(), _stream(stream))
+    if scheme is None:
+        _check(lib().ttq_linear_forward(*args, *tail), "ttq_linear_forward")
+    else:
+        _check(lib().ttq_linear_forward_ex(*args, scheme, *tail), "ttq_linear_forward_ex")
     return Y
 
 

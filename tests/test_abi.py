@@ -106,6 +106,10 @@ def test_rejections_before_device_work(L):
     assert L.ttq_dequantized_gemm(16, None, 64, 4, 4, 16, 1, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_dequantized_gemm(16, 16, 64, 4, 4, 16, 1, 256, 64, None) == ttq.TTQ_ERR_WORKSPACE
     assert L.ttq_dequantized_gemm(16, 16, 64, 4, 4, 16, 2, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    # an unknown code scheme is refused before any CUDA call
+    assert L.ttq_quantize_weight_ex(16, 1, 4, 64, None, 4, 64, 7, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    st = L.ttq_linear_forward_ex(16, 16, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 9, 16, 1, 256, 1 << 30, None)
+    assert st == ttq.TTQ_ERR_INVALID_ARG
     # forward with a null weight
     st = L.ttq_linear_forward(16, None, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 4, 64, 16, 1, 256, 1 << 30, None)
     assert st == ttq.TTQ_ERR_INVALID_ARG
