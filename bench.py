@@ -208,6 +208,25 @@ def _config():
             "l2": "inputs rotate over sets whose size exceeds L2 (no warm-L2 reads of X or W)"}
 
 
+# ------------------------------------------------------- multi-rank helpers
+def _max_over_ranks(v: float, world: int, device: str) -> float:
+    """The largest of the ranks' values (every rank gets it); a time taken
+    on each rank's device becomes the job's time."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _job_throughput(world: int, steps: int, tokens: int, ms: float) -> float:
+    """Tokens per second of the whole job: every rank runs `steps` forwards
+    of `tokens` tokens on its own problem within the max-over-ranks time."""
+    return world * steps * tokens / (ms / 1e3)
+
+
 # ------------------------------------------------------------------- ours
 def run_ours(args):
     import numpy as np
@@ -227,11 +246,7 @@ def run_ours(args):
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return _max_over_ranks(v, world, "cuda")
 
     w = WORKLOAD
     spec = synth.C2
@@ -284,7 +299,7 @@ def run_ours(args):
     st, flags = ttq.ttq_get_status(ws)
     if st != ttq.TTQ_OK:
         raise RuntimeError(f"device status {ttq.status_string(st)} (flags {flags:#x})")
-    value = world * args.steps * T / (ms / 1e3)
+    value = _job_throughput(world, args.steps, T, ms)
 
     # ---- per-kernel durations over K steps: the forward's kernels, one entry
     # point each (statistic fused with X D^{-1/2} in binary16, quantiser with
@@ -367,7 +382,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(f0.elapsed_time(f1))
-    e2e = {"value": world * args.steps * T / (e2e_ms / 1e3), "unit": "tokens/s",
+    e2e = {"value": _job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
            "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2)}
 
     cpu = None
