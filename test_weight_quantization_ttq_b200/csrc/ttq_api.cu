@@ -204,6 +204,33 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     if (st != TTQ_OK) return st;
     pdl = true;
   }
+  if (!wq && T <= 16) {
+    // a few tokens: the product is bound by the code bytes; they stream
+    // through shared memory and are dequantised in registers for
+    // warp-level MMAs (when the code rows are 16-byte strided)
+    CUtensorMap tmC, tmX;
+    if (encode_codes(&tmC, codes, d * bits / 32, dp, decode_code_box_words(bits),
+                     decode_code_box_rows()) &&
+        encode_16bit(&tmX, Xh, true, d, T, d, T <= 8 ? 8 : 16)) {
+      DecodeArgs a;
+      a.scales = scales;
+      a.zeros = zeros;
+      a.K = d;
+      a.M = dp;
+      a.T = T;
+      a.bits = bits;
+      a.group = group;
+      a.Blr = Bb;
+      a.AX = ax;
+      a.r = r;
+      a.ax_ld = L.ax_ld;
+      a.Y = Y;
+      a.ldy = dp;
+      a.y_f32 = y_f32;
+      a.status = status;
+      return cuda_status(launch_decode_gemm(a, tmC, tmX, stream, pdl));
+    }
+  }
   // wq: the product reads the materialised binary16 s (q - z) by TMA
   int bm = 128, bnm = 16;
   gemm_tile_shape(wq ? 0 : bits, dp, T, device_sms(), &bm, &bnm);

@@ -116,6 +116,32 @@ struct GemmMaps {
   CUtensorMap y;   // bf16 Y [T][ldy], box 32 x 16 (rows of W x tokens), no swizzle
 };
 
+// Steps (2)-(3) for T <= 16 tokens: Y[t][j] = sum_i s (q - z) Xh[t][i]
+// (+ sum_k Blr[j][k] AX[t][k] when r > 0, both bf16) with the codes
+// dequantised in registers for warp-level tensor-core MMAs.  K % 32 == 0,
+// group a power of two >= 32; Y [T][ldy] float32 or bf16.
+struct DecodeArgs {
+  const uint16_t* scales = nullptr;  // [M][K / group] binary16
+  const uint16_t* zeros = nullptr;
+  int64_t K = 0, M = 0, T = 0;
+  int bits = 4, group = 128;
+  const void* Blr = nullptr;         // bf16 [M][r]
+  const void* AX = nullptr;          // bf16 [T][ax_ld]
+  int64_t r = 0, ax_ld = 0;
+  void* Y = nullptr;
+  int64_t ldy = 0;
+  bool y_f32 = false;
+  uint32_t* status = nullptr;
+};
+// The tensor maps it reads: tmC the codes [M][K bits / 32] as uint32 in
+// boxes of decode_code_box_words(bits) x decode_code_box_rows() without
+// swizzle; tmX binary16 Xh [T][K] in boxes of 64 channels x (T <= 8 ? 8 : 16)
+// tokens, 128-byte swizzled.
+int decode_code_box_words(int bits);
+int decode_code_box_rows();
+cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
+                               const CUtensorMap& tmX, cudaStream_t stream, bool pdl = false);
+
 // Words per row of the code tile one K block of 64 channels needs.
 int gemm_code_tile_words(int bits);
 

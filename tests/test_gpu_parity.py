@@ -112,6 +112,15 @@ GEMM_CASES = [
     (512, 256, 300, 2, 64, 8, "bf16"),
     (640, 128, 33, 4, 128, 72, "bf16"),
     (256, 128, 20, 4, 64, 16, "f32"),
+    # at most 16 tokens: the register-dequantising product, with K tails of
+    # 32 channels, ragged rows and the low-rank term
+    (96, 64, 5, 4, 32, 0, "bf16"),
+    (512, 200, 9, 4, 64, 16, "bf16"),
+    (288, 100, 3, 3, 32, 8, "f32"),
+    (352, 70, 16, 2, 32, 24, "bf16"),
+    (4096, 333, 2, 4, 128, 64, "bf16"),
+    (384, 100, 5, 3, 64, 8, "bf16"),
+    (1024, 64, 13, 3, 256, 0, "f32"),
 ]
 
 
@@ -158,6 +167,9 @@ FORWARD_CASES = [
     _small("ragged_256row_tiles", d=4096, dp=4296, T=2000, bits=4, group=128, n_out=40),
     _small("ragged_256row_tiles_int2_lowrank", d=1024, dp=4296, T=2000, bits=2, group=64, r=40, n_out=10),
     _small("ragged_lowrank", d=448, dp=333, T=77, bits=2, group=64, r=24),
+    _small("decode_lowrank", d=480, dp=150, T=11, bits=4, group=32, r=16),
+    _small("decode_int3_lowrank", d=736, dp=77, T=1, bits=3, group=32, r=8, dtype="f32"),
+    _small("decode_int3_k768", d=768, dp=129, T=8, bits=3, group=128, r=16),
 ]
 
 
