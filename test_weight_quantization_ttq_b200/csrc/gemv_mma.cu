@@ -3,26 +3,36 @@
 // with X' = X D^(-1/2) in binary16 (gist.science/zh/paper/2603.19296,
 // section 2.1 for W_hat, 2.2 for the static low-rank pair).
 //
-// With so few tokens the product is a matrix-vector product bound by the
-// bytes of the packed codes, so the kernel is built to keep many of them in
-// flight: one producer warp streams, per stage of 128 input channels, the
-// code tile of the CTA's 64 rows of W and the matching 128 channels of X'
-// into shared memory by TMA (8 stages deep); four consumer warps, 16 rows
-// each, dequantise the codes in registers and feed them to warp-level
-// tensor-core MMAs (m16n8k16, binary16 x binary16 -> fp32).  The weights never
-// exist in binary16 outside registers.  The operand values are those the
-// large-tile product forms: binary16 (1024 + q) - (1024 + z) is exact and
-// the product with s rounds once.
+// With so few tokens the product is a matrix-vector product over the packed
+// codes, and turning codes into tensor-core operands costs as much as
+// reading them, so the kernel is laid out to spend few instructions per
+// code.  One producer warp streams, per stage of 512 input channels, the
+// code tile of the CTA's 64 rows of W and the matching 512 channels of X'
+// into shared memory, one 3-D TMA copy each (few, large stages: issuing a
+// stage costs the producer about as much as a consumer spends on a small
+// one).  The code tile lands unit-major -- 64-channel units, each a block of
+// 64 rows -- so the rows a warp reads at once sit 16 to 48 bytes apart, free
+// of bank conflicts.  Eight consumer warps -- two groups of 32 rows x four
+// quarters of every stage (units 2kq, 2kq + 1) -- turn the codes into
+// binary16 operands in registers and run warp-level MMAs (m16n8k16,
+// binary16 x binary16 -> fp32); each warp's two 16-row tiles share the X'
+// operand.  The quarters are added in a fixed order at the end, so the
+// result is deterministic.
 //
 // The order of the 16 products inside one MMA is free as long as the A and
-// B operands agree on it, so each lane (g = lane / 4, c = lane % 4) owns 32
-// contiguous channels of a stage -- its codes are one vector load from
-// shared memory -- and pairs codes the way the packing makes cheap: INT4
-// channels (i, i + 4) of a 16-channel unit come out of one word with one
-// mask, INT2 (i, i + 8), INT3 (2i, 2i + 1).  The matching pairs of X' are
-// put together with byte permutes.  Lanes with c >= 2 walk their two units
-// in the opposite order, which together with the 128-byte swizzle of the X'
-// tiles keeps the shared-memory reads free of bank conflicts.
+// B operands agree on it.  Each lane (g = lane / 4, c = lane % 4) owns
+// channels 16c .. 16c + 15 of each 64-channel half ("unit") of a stage and
+// pairs codes the way the packing makes cheap: a code at bit b of a 16-bit
+// half, OR-ed into the exponent of m = 2^(10 - b), reads as the binary16
+// m + q, so INT4 channels (i, i + 4) and INT2 (i, i + 8) of a unit come out
+// of a word with one mask each (INT3: (2i, 2i + 1) after a shift).  The
+// matching pairs of X' are put together with byte permutes.  The X' tiles
+// are 128-byte swizzled, which makes their reads free of bank conflicts.
+//
+// The operand is (m + q) - (m + z) = q - z, exact in binary16.  For up to 8
+// tokens with quantisation groups that span whole stages (group >= 128) s
+// multiplies the fp32 sum of a stage once per row; otherwise the operand is
+// the binary16 s (q - z) (one rounding), as in the large-tile product.
 //
 // Register layout of m16n8k16 (PTX ISA, warp-level MMA): the A registers
 // hold rows g and g + 8 at the lane's K pair 0 (registers 0, 1) and K pair 1
@@ -40,25 +50,36 @@
 namespace ttq {
 namespace {
 
-constexpr int kRowGroups = 4;                   // 16-row groups per CTA
-constexpr int kRowsPerCta = 16 * kRowGroups;
-constexpr int kConsumers = 2 * kRowGroups;      // x 2: even and odd stages
-constexpr int kStageK = 128;                    // input channels per stage
-constexpr int kStages = 8;
+constexpr int kRowGroups = 2;                   // 32-row groups per CTA
+constexpr int kRowsPerCta = 32 * kRowGroups;
+constexpr int kQuarters = 4;                    // consumer warps per row group
+constexpr int kConsumers = kRowGroups * kQuarters;
+constexpr int kUnitK = 64;                      // channels per unit
+constexpr int kUnits = 8;                       // units per stage
+constexpr int kStageK = kUnitK * kUnits;
 
+// The code tile is copied in pieces of one unit (two for INT3, whose unit
+// of 24 bytes is not a multiple of 16): [piece][row][piece bytes].
 template <int BITS>
-constexpr int stage_words() { return kStageK * BITS / 32; }   // code words per row and stage
+constexpr int piece_units() { return BITS == 3 ? 2 : 1; }
 template <int BITS>
-constexpr uint32_t code_tile_bytes() { return kRowsPerCta * stage_words<BITS>() * 4; }
+constexpr int piece_words() { return kUnitK * BITS / 32 * piece_units<BITS>(); }
+template <int BITS>
+constexpr int pieces() { return kUnits / piece_units<BITS>(); }
+template <int BITS>
+constexpr uint32_t code_tile_bytes() { return kRowsPerCta * kStageK * BITS / 8; }
+// X' of a stage: [unit][8 NTT tokens][64 channels], 128-byte swizzled
 template <int NTT>
-constexpr uint32_t xh_tile_bytes() { return 2u * 8u * NTT * 128u; }  // two 64-channel boxes
+constexpr uint32_t xh_tile_bytes() { return kUnits * 8u * NTT * 128u; }
+template <int NTT>
+constexpr int num_stages() { return NTT == 1 ? 4 : 3; }
 template <int BITS, int NTT>
 constexpr uint32_t stage_bytes() {
   return (xh_tile_bytes<NTT>() + code_tile_bytes<BITS>() + 1023u) & ~1023u;
 }
 template <int BITS, int NTT>
 constexpr size_t decode_smem_bytes() {
-  return static_cast<size_t>(kStages) * stage_bytes<BITS, NTT>() + 1024;
+  return static_cast<size_t>(num_stages<NTT>()) * stage_bytes<BITS, NTT>() + 1024;
 }
 
 __device__ __forceinline__ void mma_m16n8k16_f16(float (&c)[4], const uint32_t (&a)[4],
@@ -78,27 +99,15 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&c)[4], const uint32_t 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// (m + q) - (m + z) on a binary16 pair (exact)
-__device__ __forceinline__ uint32_t hsub2_bits(uint32_t magic_pair, uint32_t zc2) {
-  __half2 a, zc;
-  memcpy(&a, &magic_pair, 4);
-  memcpy(&zc, &zc2, 4);
-  const __half2 v = __hsub2(a, zc);
+__device__ __forceinline__ uint32_t h2_bits(__half2 v) {
   uint32_t u;
   memcpy(&u, &v, 4);
   return u;
 }
-
-// s ((m + q) - (m + z)) on a binary16 pair
-__device__ __forceinline__ uint32_t dequant_pair(uint32_t magic_pair, uint32_t zc2, uint32_t s2) {
-  __half2 a, zc, s;
-  memcpy(&a, &magic_pair, 4);
-  memcpy(&zc, &zc2, 4);
-  memcpy(&s, &s2, 4);
-  const __half2 v = __hmul2(__hsub2(a, zc), s);
-  uint32_t u;
-  memcpy(&u, &v, 4);
-  return u;
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) {
+  __half2 v;
+  memcpy(&v, &u, 4);
+  return v;
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -119,66 +128,40 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   return v;
 }
 
-// The lane's code words of one row for the current stage (its 32 channels).
+// Number of distinct magics m a unit's pairs use, and pair p's index into
+// them: INT4 {1024, 64}; INT2 {1024, 256, 64, 16, 4}; INT3 {1024}.
 template <int BITS>
-struct LaneCodes {
-  uint32_t w[BITS];
-};
-
+constexpr int num_kinds() { return BITS == 4 ? 2 : (BITS == 2 ? 5 : 1); }
 template <int BITS>
-__device__ __forceinline__ LaneCodes<BITS> load_lane_codes(uint32_t row_addr, int c) {
-  LaneCodes<BITS> v;
-  if (BITS == 4) {
-    const uint4 a = lds128(row_addr + 16 * c);
-    v.w[0] = a.x; v.w[1] = a.y; v.w[2 % BITS] = a.z; v.w[3 % BITS] = a.w;
-  } else if (BITS == 2) {
-    const uint2 a = lds64(row_addr + 8 * c);
-    v.w[0] = a.x; v.w[1] = a.y;
-  } else {
-#pragma unroll
-    for (int i = 0; i < BITS; ++i) v.w[i] = lds32(row_addr + 12 * c + 4 * i);
-  }
-  return v;
+__device__ __forceinline__ constexpr int pair_kind(int p) {
+  return BITS == 4 ? (p & 1) : (BITS == 2 ? (p < 5 ? p : p - 5) : 0);
+}
+template <int BITS>
+__device__ __forceinline__ constexpr uint32_t kind_magic(int k) {
+  return BITS == 2 ? (k == 0 ? 0x6400u : k == 1 ? 0x5C00u : k == 2 ? 0x5400u
+                                       : k == 3 ? 0x4C00u : 0x4400u)
+                   : (k == 0 ? 0x6400u : 0x5400u);
 }
 
-// Code pairs of 16-channel unit uu of the lane's 32 channels as binary16
-// pairs (m + q), m a power of two per pair, so that no shift is needed
-// where the code bits already sit inside the significand: a code at bit b
-// of a 16-bit half, OR-ed into the exponent of m = 2^(10 - b), reads m + q.
-// INT4: P[i] = channels (i, i + 4), P[4 + i] = (8 + i, 12 + i); INT2: P[i] =
-// (i, i + 8); INT3: P[i] = (2i, 2i + 1) (all with m = 1024).
-// kind[i] = log2(m) of pair i.
+// (m + q) pairs P[0..7] of the lane's 16 channels of unit u of its piece,
+// for one row (row_addr: the row's first byte in the piece).  INT4: P[i] =
+// channels (i, i + 4), P[4 + i] = (8 + i, 12 + i); INT2: P[i] = (i, i + 8);
+// INT3: P[i] = (2i, 2i + 1).
 template <int BITS>
-struct PairSpec {
-  static constexpr int kinds = BITS == 4 ? 2 : (BITS == 2 ? 5 : 1);
-};
-template <int BITS>
-__device__ __forceinline__ constexpr int pair_kind(int i) {
-  // index into the per-row table of (m + z): INT4 {1024, 64}; INT2 {1024,
-  // 256, 64, 16, 4}; INT3 {1024}
-  return BITS == 4 ? (i & 1) : (BITS == 2 ? (i < 5 ? i : i - 5) : 0);
-}
-__device__ __forceinline__ constexpr uint32_t kind_magic(int bits, int k) {
-  return bits == 2 ? (k == 0 ? 0x64006400u : k == 1 ? 0x5C005C00u : k == 2 ? 0x54005400u
-                                                 : k == 3 ? 0x4C004C00u : 0x44004400u)
-                   : (k == 0 ? 0x64006400u : 0x54005400u);
-}
-template <int BITS>
-__device__ __forceinline__ void magic_pairs(const LaneCodes<BITS>& v, int uu, uint32_t (&P)[8]) {
+__device__ __forceinline__ void code_pairs(uint32_t row_addr, int u, int c, uint32_t (&P)[8]) {
   if (BITS == 4) {
-    const uint32_t lo = uu ? v.w[2 % BITS] : v.w[0];
-    const uint32_t hi = uu ? v.w[3 % BITS] : v.w[1];
-    const uint32_t lo8 = lo >> 8, hi8 = hi >> 8;
-    P[0] = (lo & 0x000F000Fu) | 0x64006400u;    // channels 0, 4
-    P[1] = (lo & 0x00F000F0u) | 0x54005400u;    // 1, 5
+    const uint2 w = lds64(row_addr + 32 * u + 8 * c);
+    const uint32_t lo8 = w.x >> 8, hi8 = w.y >> 8;
+    P[0] = (w.x & 0x000F000Fu) | 0x64006400u;   // channels 0, 4
+    P[1] = (w.x & 0x00F000F0u) | 0x54005400u;   // 1, 5
     P[2] = (lo8 & 0x000F000Fu) | 0x64006400u;   // 2, 6
     P[3] = (lo8 & 0x00F000F0u) | 0x54005400u;   // 3, 7
-    P[4] = (hi & 0x000F000Fu) | 0x64006400u;
-    P[5] = (hi & 0x00F000F0u) | 0x54005400u;
+    P[4] = (w.y & 0x000F000Fu) | 0x64006400u;
+    P[5] = (w.y & 0x00F000F0u) | 0x54005400u;
     P[6] = (hi8 & 0x000F000Fu) | 0x64006400u;
     P[7] = (hi8 & 0x00F000F0u) | 0x54005400u;
   } else if (BITS == 2) {
-    const uint32_t w = uu ? v.w[1] : v.w[0];
+    const uint32_t w = lds32(row_addr + 16 * u + 4 * c);
     const uint32_t w10 = w >> 10;
     P[0] = (w & 0x00030003u) | 0x64006400u;     // channels 0, 8
     P[1] = (w & 0x000C000Cu) | 0x5C005C00u;     // 1, 9
@@ -189,9 +172,12 @@ __device__ __forceinline__ void magic_pairs(const LaneCodes<BITS>& v, int uu, ui
     P[6] = (w10 & 0x000C000Cu) | 0x5C005C00u;   // 6, 14
     P[7] = (w10 & 0x00300030u) | 0x54005400u;   // 7, 15
   } else {
-    // unit 0: bits 0..47 of the lane's 96; unit 1: bits 48..95
-    const uint64_t b = uu ? ((static_cast<uint64_t>(v.w[2 % BITS]) << 16) | (v.w[1] >> 16))
-                          : (static_cast<uint64_t>(v.w[1] & 0xFFFFu) << 32 | v.w[0]);
+    // the unit's channels 16c.. start at bit 48c of the unit's 192 bits:
+    // word 6u + (3c >> 1), plus 16 bits for odd c
+    const uint32_t wi = 6u * u + (static_cast<uint32_t>(3 * c) >> 1);
+    const uint64_t win = static_cast<uint64_t>(lds32(row_addr + 4 * wi)) |
+                         (static_cast<uint64_t>(lds32(row_addr + 4 * wi + 4)) << 32);
+    const uint64_t b = win >> ((c & 1) * 16);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint32_t t = static_cast<uint32_t>(b >> (6 * i));
@@ -200,7 +186,7 @@ __device__ __forceinline__ void magic_pairs(const LaneCodes<BITS>& v, int uu, ui
   }
 }
 
-// The X' pairs B[0..7] matching magic_pairs, from the unit's 16 channels
+// The X' pairs B[0..7] matching code_pairs, from the unit's 16 channels
 // X[m] = channels (2m, 2m + 1).
 template <int BITS>
 __device__ __forceinline__ void x_pairs(const uint32_t (&X)[8], uint32_t (&B)[8]) {
@@ -221,37 +207,40 @@ __device__ __forceinline__ void x_pairs(const uint32_t (&X)[8], uint32_t (&B)[8]
   }
 }
 
-// PS: the quantisation group spans whole stages (group >= 128), so s is
-// applied once per stage and row to the fp32 sum of (q - z) X' (exact
-// operands); otherwise every operand is the binary16 s (q - z).
+// PS: s applied per 128-channel block to fp32 sums of exact (q - z)
+// operands (group >= 128); otherwise binary16 s (q - z) operands.
 template <int BITS, int NTT, bool PS>
-__global__ void __launch_bounds__(32 * (1 + kConsumers)) ttq_decode_kernel(
+__global__ void __launch_bounds__(32 * (1 + kConsumers), 2) ttq_decode_kernel(
     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmX,
-    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros, int64_t K,
-    int64_t M, int64_t T, int group_shift, const __nv_bfloat16* __restrict__ Blr,
-    const __nv_bfloat16* __restrict__ AX, int64_t r, int64_t ax_ld, void* __restrict__ Y,
-    int64_t ldy, int y_f32, uint32_t* status) {
+    const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros, int K, int M,
+    int T, int group_shift, const __nv_bfloat16* __restrict__ Blr,
+    const __nv_bfloat16* __restrict__ AX, int r, int ax_ld, void* __restrict__ Y, int ldy,
+    int y_f32, uint32_t* status) {
+  constexpr int kStages = num_stages<NTT>();
   extern __shared__ uint8_t dsm[];
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ __align__(8) uint64_t empty[kStages];
   __shared__ int abort_s;
-  __shared__ float red[kRowGroups][NTT][4][32];   // odd-stage sums
+  __shared__ float red[kQuarters - 1][kRowGroups][2][NTT][4][32];   // quarters 1..3
   constexpr uint32_t kXh = xh_tile_bytes<NTT>();
   constexpr uint32_t kCode = code_tile_bytes<BITS>();
   constexpr uint32_t kStage = stage_bytes<BITS, NTT>();
-  constexpr int kKinds = PairSpec<BITS>::kinds;
+  constexpr uint32_t kPieceRow = piece_words<BITS>() * 4;        // bytes of a row in a piece
+  constexpr uint32_t kPiece = kPieceRow * kRowsPerCta;
+  constexpr int kKinds = num_kinds<BITS>();
+  constexpr int kUnitsSz = PS ? 1 : 2;           // (s, z) per row: per block or per unit
   const uint32_t smem = (smem_addr(dsm) + 1023u) & ~1023u;
   uint8_t* smem_ptr = dsm + (smem - smem_addr(dsm));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int nsteps = static_cast<int>((K + kStageK - 1) / kStageK);
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  const int nsteps = (K + kStageK - 1) / kStageK;
+  const int row0 = blockIdx.x * kRowsPerCta;
   volatile int* abort_flag = &abort_s;
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kRowGroups);
+      mbar_init(&empty[s], kConsumers);
     }
     abort_s = 0;
     fence_barrier_init();
@@ -276,10 +265,8 @@ __global__ void __launch_bounds__(32 * (1 + kConsumers)) ttq_decode_kernel(
         }
         uint8_t* base = smem_ptr + s * kStage;
         mbar_arrive_expect_tx(&full[s], kXh + kCode);
-        tma_load_2d(&tmX, &full[s], base, st * kStageK, 0);
-        tma_load_2d(&tmX, &full[s], base + kXh / 2, st * kStageK + 64, 0);
-        tma_load_2d(&tmC, &full[s], base + kXh, st * stage_words<BITS>(),
-                    static_cast<int32_t>(row0));
+        tma_load_3d(&tmX, &full[s], base, 0, 0, st * kUnits);
+        tma_load_3d(&tmC, &full[s], base + kXh, 0, row0, st * pieces<BITS>());
         issued = st + 1;
       }
       if (*abort_flag) {
@@ -293,59 +280,68 @@ __global__ void __launch_bounds__(32 * (1 + kConsumers)) ttq_decode_kernel(
   }
 
   // ------------------------------------------------------------ consumers
-  // warp 1 + rg + 4 kpar: rows 16 rg .. 16 rg + 15 of the CTA, stages
-  // kpar, kpar + 2, ...
+  // warp 1 + rg + 2 kq: rows 32 rg + {g, g + 8, g + 16, g + 24} of the CTA
+  // (two 16-row MMA tiles), units 2 kq and 2 kq + 1 of every stage
   const int cw = warp - 1;
   const int rg = cw % kRowGroups;
-  const int kpar = cw / kRowGroups;
+  const int kq = cw / kRowGroups;
   const int g = lane >> 2;
   const int c = lane & 3;
-  const int rla = 16 * rg + g, rlb = rla + 8;   // rows within the CTA
-  const int64_t ra = row0 + rla, rb = row0 + rlb;
-  const int64_t ngroups = K >> group_shift;
-  const int64_t sra = (ra < M ? ra : M - 1) * ngroups;
-  const int64_t srb = (rb < M ? rb : M - 1) * ngroups;
-  // s | z << 16 of both rows for stage st (the lane's 32 channels lie in one
-  // quantisation group); past K the group index is clamped (the matching X'
-  // is zero)
-  auto load_sz = [&](int st, uint32_t& za_s, uint32_t& zb_s) {
-    int64_t gi = (static_cast<int64_t>(st) * kStageK + 32 * c) >> group_shift;
-    if (gi >= ngroups) gi = ngroups - 1;
-    za_s = static_cast<uint32_t>(__ldg(scales + sra + gi)) |
-           (static_cast<uint32_t>(__ldg(zeros + sra + gi)) << 16);
-    zb_s = static_cast<uint32_t>(__ldg(scales + srb + gi)) |
-           (static_cast<uint32_t>(__ldg(zeros + srb + gi)) << 16);
-  };
-  const int my_n = (nsteps - kpar + 1) / 2;     // stages of this warp
-  // the loads of s, z run kSzAhead stages ahead in a ring whose slot index
-  // is static after unrolling (moving a register still being loaded would
-  // wait for the load)
-  constexpr int kSzAhead = 4;
-  uint32_t sz_a[kSzAhead], sz_b[kSzAhead];
+  const int ngroups = K >> group_shift;
+  int rloc[4];
+  const uint16_t* srow[4];
+  const uint16_t* zrow[4];
 #pragma unroll
-  for (int i = 0; i < kSzAhead; ++i) {
-    sz_a[i] = sz_b[i] = 0u;
-    if (i < my_n) load_sz(kpar + 2 * i, sz_a[i], sz_b[i]);
+  for (int i = 0; i < 4; ++i) {
+    rloc[i] = 32 * rg + g + 8 * i;
+    const int row = row0 + rloc[i] < M ? row0 + rloc[i] : M - 1;
+    srow[i] = scales + static_cast<int64_t>(row) * ngroups;
+    zrow[i] = zeros + static_cast<int64_t>(row) * ngroups;
   }
-  float acc[NTT][4];
+  // s | z << 16 of the lane's four rows for stage st and unit 2 kq + v (the
+  // lane's 16 channels lie in one quantisation group; with PS the whole
+  // 128-channel block does); past K the group index is clamped (the
+  // matching X' is zero)
+  auto load_sz = [&](int st, int v, uint32_t (&dst)[4]) {
+    int gi = (st * kStageK + (2 * kq + v) * kUnitK + (PS ? 0 : 16 * c)) >> group_shift;
+    gi = gi < ngroups ? gi : ngroups - 1;
 #pragma unroll
-  for (int tt = 0; tt < NTT; ++tt) acc[tt][0] = acc[tt][1] = acc[tt][2] = acc[tt][3] = 0.f;
+    for (int i = 0; i < 4; ++i)
+      dst[i] = static_cast<uint32_t>(__ldg(srow[i] + gi)) |
+               (static_cast<uint32_t>(__ldg(zrow[i] + gi)) << 16);
+  };
+  // (s, z) run one stage ahead, in two slots whose index is static after
+  // unrolling (moving a register still being loaded would wait for the load)
+  uint32_t sz[2][kUnitsSz][4];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+#pragma unroll
+    for (int v = 0; v < kUnitsSz; ++v) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sz[j][v][i] = 0u;
+      if (j < nsteps) load_sz(j, v, sz[j][v]);
+    }
+  // with one token tile the two units accumulate apart (four independent
+  // MMA chains per warp instead of two); added in unit order
+  constexpr int kUA = NTT == 1 ? 2 : 1;
+  float acc[kUA][2][NTT][4];
+#pragma unroll
+  for (int ua = 0; ua < kUA; ++ua)
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int tt = 0; tt < NTT; ++tt)
+        acc[ua][mt][tt][0] = acc[ua][mt][tt][1] = acc[ua][mt][tt][2] = acc[ua][mt][tt][3] = 0.f;
   bool ok = true;
-  const uint32_t xbox = static_cast<uint32_t>(c >> 1) * (kXh / 2);
-  const uint32_t flip = static_cast<uint32_t>(c >> 1);
 
-  for (int i0 = 0; i0 < my_n && ok; i0 += kSzAhead) {
+  for (int i0 = 0; i0 < nsteps && ok; i0 += 2) {
 #pragma unroll
-    for (int j = 0; j < kSzAhead; ++j) {
-      const int i = i0 + j;
-      if (i >= my_n) break;
-      const int st = kpar + 2 * i;
+    for (int j = 0; j < 2; ++j) {
+      const int st = i0 + j;
+      if (st >= nsteps) break;
       const int s = st % kStages;
       const uint32_t ph = static_cast<uint32_t>(st / kStages) & 1u;
-      int got = 1;
-      if (lane == 0) got = mbar_wait(&full[s], ph, abort_flag) ? 1 : 0;
-      got = __shfl_sync(0xffffffffu, got, 0);
-      if (!got) {
+      if (!mbar_wait(&full[s], ph, abort_flag)) {
         if (lane == 0) {
           *abort_flag = 1;
           set_flag(status, TTQ_FLAG_TIMEOUT);
@@ -354,132 +350,165 @@ __global__ void __launch_bounds__(32 * (1 + kConsumers)) ttq_decode_kernel(
         break;
       }
       const uint32_t base = smem + s * kStage;
-      const uint32_t code_base = base + kXh;
-      const LaneCodes<BITS> va =
-          load_lane_codes<BITS>(code_base + rla * (stage_words<BITS>() * 4), c);
-      const LaneCodes<BITS> vb =
-          load_lane_codes<BITS>(code_base + rlb * (stage_words<BITS>() * 4), c);
-      // (m + z) pairs of both rows for every magic m in use (exact), and s
-      const __half za = __ushort_as_half(static_cast<uint16_t>(sz_a[j] >> 16));
-      const __half zb = __ushort_as_half(static_cast<uint16_t>(sz_b[j] >> 16));
-      uint32_t zca[kKinds], zcb[kKinds];
+      float part[kUA][2][NTT][4];
+      if (PS) {
 #pragma unroll
-      for (int k = 0; k < kKinds; ++k) {
-        const __half m = __ushort_as_half(static_cast<uint16_t>(kind_magic(BITS, k) & 0xFFFFu));
-        zca[k] = static_cast<uint32_t>(__half_as_ushort(__hadd(za, m))) * 0x00010001u;
-        zcb[k] = static_cast<uint32_t>(__half_as_ushort(__hadd(zb, m))) * 0x00010001u;
+        for (int ua = 0; ua < kUA; ++ua)
+#pragma unroll
+          for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int tt = 0; tt < NTT; ++tt)
+              part[ua][mt][tt][0] = part[ua][mt][tt][1] = part[ua][mt][tt][2] = part[ua][mt][tt][3] = 0.f;
       }
-      const uint32_t s2a = (sz_a[j] & 0xFFFFu) * 0x00010001u;
-      const uint32_t s2b = (sz_b[j] & 0xFFFFu) * 0x00010001u;
-      const float sfa = __half2float(__ushort_as_half(static_cast<uint16_t>(sz_a[j] & 0xFFFFu)));
-      const float sfb = __half2float(__ushort_as_half(static_cast<uint16_t>(sz_b[j] & 0xFFFFu)));
-      if (i + kSzAhead < my_n) load_sz(st + 2 * kSzAhead, sz_a[j], sz_b[j]);
-
-      float part[NTT][4];
+      float sf[4];
 #pragma unroll
-      for (int tt = 0; tt < NTT; ++tt) part[tt][0] = part[tt][1] = part[tt][2] = part[tt][3] = 0.f;
+      for (int v = 0; v < 2; ++v) {
+        const int u = 2 * kq + v;                  // unit of the stage
+        if (st * kStageK + u * kUnitK >= K) break;  // past the end of the row
+        const int vs = PS ? 0 : v;
+        // (m + z) pairs of the four rows for every magic m in use (exact),
+        // and s (a binary16 pair, or a float for the per-block scaling)
+        uint32_t zc[4][kKinds], s2[4];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int uu = u ^ static_cast<int>(flip);
-        uint32_t Pa[8], Pb[8];
-        magic_pairs<BITS>(va, uu, Pa);
-        magic_pairs<BITS>(vb, uu, Pb);
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t zz = __byte_perm(sz[j][vs][i], 0u, 0x3232u);   // z in both halves
+          const uint32_t ss = __byte_perm(sz[j][vs][i], 0u, 0x1010u);   // s in both halves
 #pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const int k = pair_kind<BITS>(p);
-          if (PS) {
-            Pa[p] = hsub2_bits(Pa[p], zca[k]);
-            Pb[p] = hsub2_bits(Pb[p], zcb[k]);
-          } else {
-            Pa[p] = dequant_pair(Pa[p], zca[k], s2a);
-            Pb[p] = dequant_pair(Pb[p], zcb[k], s2b);
+          for (int k = 0; k < kKinds; ++k)
+            zc[i][k] = h2_bits(__hadd2(bits_h2(zz), bits_h2(kind_magic<BITS>(k) * 0x00010001u)));
+          s2[i] = ss;
+          if (PS && v == 0) sf[i] = __half2float(__ushort_as_half(static_cast<uint16_t>(ss & 0xFFFFu)));
+        }
+        const int piece = u / piece_units<BITS>();
+        const int h = u % piece_units<BITS>();
+        const uint32_t prow = base + kXh + static_cast<uint32_t>(piece) * kPiece +
+                              static_cast<uint32_t>(32 * rg + g) * kPieceRow;
+        uint32_t P[4][8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          code_pairs<BITS>(prow + 8u * i * kPieceRow, h, c, P[i]);
+#pragma unroll
+          for (int p = 0; p < 8; ++p) {
+            const __half2 x = __hsub2(bits_h2(P[i][p]), bits_h2(zc[i][pair_kind<BITS>(p)]));
+            P[i][p] = PS ? h2_bits(x) : h2_bits(__hmul2(x, bits_h2(s2[i])));
           }
         }
-        // the unit's 16 channels of X' are chunks 4 (c & 1) + 2 uu and the
-        // next one of the 128-byte rows of box c >> 1, swizzled by row & 7
-        const uint32_t ch0 = static_cast<uint32_t>(4 * (c & 1) + 2 * uu);
+        // the unit's 16 channels of X' are chunks 2c, 2c + 1 of the 128-byte
+        // token rows of unit u, swizzled by row & 7 (= g)
+        const uint32_t xrow = base + static_cast<uint32_t>(u) * (8u * NTT * 128u) +
+                              static_cast<uint32_t>(g) * 128u;
+        const uint32_t off0 = (static_cast<uint32_t>(2 * c) ^ static_cast<uint32_t>(g)) << 4;
+        const uint32_t off1 = (static_cast<uint32_t>(2 * c + 1) ^ static_cast<uint32_t>(g)) << 4;
 #pragma unroll
         for (int tt = 0; tt < NTT; ++tt) {
-          const uint32_t rowa = base + xbox + static_cast<uint32_t>(8 * tt + g) * 128u;
-          const uint4 x0 = lds128(rowa + ((ch0 ^ static_cast<uint32_t>(g)) << 4));
-          const uint4 x1 = lds128(rowa + (((ch0 + 1) ^ static_cast<uint32_t>(g)) << 4));
+          const uint4 x0 = lds128(xrow + 1024u * tt + off0);
+          const uint4 x1 = lds128(xrow + 1024u * tt + off1);
           const uint32_t X[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
           uint32_t B[8];
           x_pairs<BITS>(X, B);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint32_t a[4] = {Pa[2 * k], Pb[2 * k], Pa[2 * k + 1], Pb[2 * k + 1]};
-            mma_m16n8k16_f16(PS ? part[tt] : acc[tt], a, B[2 * k], B[2 * k + 1]);
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+              const uint32_t a[4] = {P[2 * mt][2 * k], P[2 * mt + 1][2 * k], P[2 * mt][2 * k + 1],
+                                     P[2 * mt + 1][2 * k + 1]};
+              const int ua = kUA > 1 ? v : 0;
+              mma_m16n8k16_f16(PS ? part[ua][mt][tt] : acc[ua][mt][tt], a, B[2 * k], B[2 * k + 1]);
+            }
           }
         }
       }
-      if (PS) {
+      // refill this slot with the (s, z) of the stage after next
+      if (st + 2 < nsteps) {
 #pragma unroll
-        for (int tt = 0; tt < NTT; ++tt) {
-          acc[tt][0] = fmaf(sfa, part[tt][0], acc[tt][0]);
-          acc[tt][1] = fmaf(sfa, part[tt][1], acc[tt][1]);
-          acc[tt][2] = fmaf(sfb, part[tt][2], acc[tt][2]);
-          acc[tt][3] = fmaf(sfb, part[tt][3], acc[tt][3]);
-        }
+        for (int v = 0; v < kUnitsSz; ++v) load_sz(st + 2, v, sz[j][v]);
       }
-      (void)s2a;
-      (void)s2b;
-      (void)sfa;
-      (void)sfb;
+      if (PS && st * kStageK + 2 * kq * kUnitK < K) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int tt = 0; tt < NTT; ++tt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float x = part[0][mt][tt][e];
+              if (kUA > 1) x += part[kUA - 1][mt][tt][e];
+              acc[0][mt][tt][e] = fmaf(sf[2 * mt + (e >> 1)], x, acc[0][mt][tt][e]);
+            }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[s]);
     }
   }
 
   // the low-rank term B (A X), bf16 operands in the plain register layout
-  // (K pair 0 = k 2c, 2c + 1; K pair 1 = k 2c + 8, 2c + 9), on the odd-stage
-  // warps
-  if (kpar == 1 && r > 0 && ok) {
-    const bool ra_ok = ra < M, rb_ok = rb < M;
-    const __nv_bfloat16* ba = Blr + (ra_ok ? ra : 0) * r;
-    const __nv_bfloat16* bb = Blr + (rb_ok ? rb : 0) * r;
-    for (int64_t k0 = 0; k0 < r; k0 += 16) {
-      const int64_t kc = k0 + 2 * c;
+  // (K pair 0 = k 2c, 2c + 1; K pair 1 = k 2c + 8, 2c + 9), on the last
+  // quarter's warps
+  if (kq == kQuarters - 1 && r > 0 && ok) {
+    for (int k0 = 0; k0 < r; k0 += 16) {
+      const int kc = k0 + 2 * c;
       const bool lo_ok = kc < r, hi_ok = kc + 8 < r;
-      uint32_t a[4];
-      a[0] = (ra_ok && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(ba + kc)) : 0u;
-      a[1] = (rb_ok && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bb + kc)) : 0u;
-      a[2] = (ra_ok && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(ba + kc + 8)) : 0u;
-      a[3] = (rb_ok && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bb + kc + 8)) : 0u;
+      uint32_t a[2][4];
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int rowa = row0 + rloc[2 * mt], rowb = row0 + rloc[2 * mt + 1];
+        const __nv_bfloat16* ba = Blr + static_cast<int64_t>(rowa < M ? rowa : 0) * r;
+        const __nv_bfloat16* bb = Blr + static_cast<int64_t>(rowb < M ? rowb : 0) * r;
+        a[mt][0] = (rowa < M && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(ba + kc)) : 0u;
+        a[mt][1] = (rowb < M && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bb + kc)) : 0u;
+        a[mt][2] = (rowa < M && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(ba + kc + 8)) : 0u;
+        a[mt][3] = (rowb < M && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(bb + kc + 8)) : 0u;
+      }
 #pragma unroll
       for (int tt = 0; tt < NTT; ++tt) {
-        const int64_t n = 8 * tt + g;
+        const int n = 8 * tt + g;
         const bool n_ok = n < T;
-        const __nv_bfloat16* axn = AX + (n_ok ? n : 0) * ax_ld;
+        const __nv_bfloat16* axn = AX + static_cast<int64_t>(n_ok ? n : 0) * ax_ld;
         const uint32_t b0 = (n_ok && lo_ok) ? __ldg(reinterpret_cast<const uint32_t*>(axn + kc)) : 0u;
         const uint32_t b1 = (n_ok && hi_ok) ? __ldg(reinterpret_cast<const uint32_t*>(axn + kc + 8)) : 0u;
-        mma_m16n8k16_bf16(acc[tt], a, b0, b1);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) mma_m16n8k16_bf16(acc[0][mt][tt], a[mt], b0, b1);
       }
     }
   }
 
-  // the odd-stage warps hand their sums to the even-stage warps of the same
-  // rows, which add them (a fixed order) and store Y: C rows g, g + 8 are
-  // rows ra, rb; columns 2c, 2c + 1 of token tile tt are tokens 8 tt + 2c,
-  // 8 tt + 2c + 1
-  if (kpar == 1) {
+  // quarters 1..3 hand their sums to quarter 0 of the same rows, which adds
+  // them in quarter order and stores Y: C rows g, g + 8 of tile mt are rows
+  // rloc[2 mt], rloc[2 mt + 1]; columns 2c, 2c + 1 of token tile tt are
+  // tokens 8 tt + 2c, 8 tt + 2c + 1
+  if (!PS && kUA > 1) {
 #pragma unroll
-    for (int tt = 0; tt < NTT; ++tt)
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) red[rg][tt][e][lane] = acc[tt][e];
+      for (int tt = 0; tt < NTT; ++tt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[0][mt][tt][e] += acc[kUA - 1][mt][tt][e];
+  }
+  if (kq > 0) {
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int tt = 0; tt < NTT; ++tt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) red[kq - 1][rg][mt][tt][e][lane] = acc[0][mt][tt][e];
   }
   asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumers) : "memory");
-  if (kpar == 1 || *abort_flag) return;
+  if (kq > 0 || *abort_flag) return;
 #pragma unroll
-  for (int tt = 0; tt < NTT; ++tt) {
+  for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float v = acc[tt][e] + red[rg][tt][e][lane];
-      const int64_t row = (e < 2) ? ra : rb;
-      const int64_t t = 8 * tt + 2 * c + (e & 1);
-      if (row < M && t < T) {
-        if (y_f32) static_cast<float*>(Y)[t * ldy + row] = v;
-        else static_cast<__nv_bfloat16*>(Y)[t * ldy + row] = __float2bfloat16_rn(v);
+    for (int tt = 0; tt < NTT; ++tt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float x = acc[0][mt][tt][e];
+#pragma unroll
+        for (int q = 0; q < kQuarters - 1; ++q) x += red[q][rg][mt][tt][e][lane];
+        const int row = row0 + rloc[2 * mt + (e >> 1)];
+        const int t = 8 * tt + 2 * c + (e & 1);
+        if (row < M && t < T) {
+          const int64_t at = static_cast<int64_t>(t) * ldy + row;
+          if (y_f32) static_cast<float*>(Y)[at] = x;
+          else static_cast<__nv_bfloat16*>(Y)[at] = __float2bfloat16_rn(x);
+        }
       }
     }
   }
@@ -500,32 +529,46 @@ cudaError_t launch_decode_typed(const CUtensorMap& tmC, const CUtensorMap& tmX,
   if (attr_err != cudaSuccess) return attr_err;
   const dim3 grid(static_cast<unsigned>((a.M + kRowsPerCta - 1) / kRowsPerCta));
   return launch_kernel(ttq_decode_kernel<BITS, NTT, PS>, grid, dim3(32 * (1 + kConsumers)), smem,
-                       stream, pdl, tmC, tmX, a.scales, a.zeros, a.K, a.M, a.T, group_shift,
+                       stream, pdl, tmC, tmX, a.scales, a.zeros, static_cast<int>(a.K),
+                       static_cast<int>(a.M), static_cast<int>(a.T), group_shift,
                        static_cast<const __nv_bfloat16*>(a.Blr),
-                       static_cast<const __nv_bfloat16*>(a.AX), a.r, a.ax_ld, a.Y, a.ldy,
-                       a.y_f32 ? 1 : 0, a.status);
+                       static_cast<const __nv_bfloat16*>(a.AX), static_cast<int>(a.r),
+                       static_cast<int>(a.ax_ld), a.Y, static_cast<int>(a.ldy), a.y_f32 ? 1 : 0,
+                       a.status);
 }
 
 template <int BITS>
 cudaError_t launch_decode_bits(const CUtensorMap& tmC, const CUtensorMap& tmX,
                                const DecodeArgs& a, int gs, cudaStream_t stream, bool pdl) {
-  const bool ps = a.group >= kStageK;
-  if (a.T > 8)
-    return ps ? launch_decode_typed<BITS, 2, true>(tmC, tmX, a, gs, stream, pdl)
-              : launch_decode_typed<BITS, 2, false>(tmC, tmX, a, gs, stream, pdl);
-  return ps ? launch_decode_typed<BITS, 1, true>(tmC, tmX, a, gs, stream, pdl)
-            : launch_decode_typed<BITS, 1, false>(tmC, tmX, a, gs, stream, pdl);
+  // two token tiles share each dequantised operand, and their block sums
+  // would not fit in registers besides: s goes into the operand there
+  if (a.T > 8) return launch_decode_typed<BITS, 2, false>(tmC, tmX, a, gs, stream, pdl);
+  return a.group >= 2 * kUnitK
+             ? launch_decode_typed<BITS, 1, true>(tmC, tmX, a, gs, stream, pdl)
+             : launch_decode_typed<BITS, 1, false>(tmC, tmX, a, gs, stream, pdl);
 }
 
 }  // namespace
 
-int decode_code_box_words(int bits) { return kStageK * bits / 32; }
-int decode_code_box_rows() { return kRowsPerCta; }
+DecodeMapShape decode_map_shape(int bits, int T) {
+  DecodeMapShape m;
+  m.piece_words = kUnitK * bits / 32 * (bits == 3 ? 2 : 1);
+  m.code_rows = kRowsPerCta;
+  m.code_pieces = kUnits / (bits == 3 ? 2 : 1);
+  m.unit_k = kUnitK;
+  m.x_tokens = T <= 8 ? 8 : 16;
+  m.x_units = kUnits;
+  return m;
+}
 
 cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
                                const CUtensorMap& tmX, cudaStream_t stream, bool pdl) {
   if (a.M == 0 || a.T == 0) return cudaSuccess;
-  if (a.T > 16 || a.K % 32 != 0 || a.group < 32 || (a.group & (a.group - 1)) != 0)
+  // 32-bit indexing inside the kernel
+  if (a.T > 16 || a.K % (kUnitK * (a.bits == 3 ? 2 : 1)) != 0 || a.group < 32 ||
+      (a.group & (a.group - 1)) != 0 ||
+      a.K > (int64_t{1} << 30) || a.M > (int64_t{1} << 30) || a.r > (int64_t{1} << 20) ||
+      a.ax_ld > (int64_t{1} << 20) || a.ldy > (int64_t{1} << 30))
     return cudaErrorInvalidValue;
   int gs = 0;
   while ((1 << (gs + 1)) <= a.group) ++gs;

@@ -151,6 +151,28 @@ bool encode_codes(CUtensorMap* m, const uint32_t* base, int64_t wpr, int64_t row
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A 3-D view of a dense buffer: dims[0] innermost (element stride 1),
+// strides (bytes) of dims 1 and 2 in any order, reads outside the view
+// return zeros.
+bool encode_3d(CUtensorMap* m, const void* base, CUtensorMapDataType type, const int64_t (&dims)[3],
+               const int64_t (&strides)[2], const int (&box)[3], CUtensorMapSwizzle swizzle) {
+  EncodeFn enc = get_encode();
+  if (enc == nullptr) return false;
+  for (int i = 0; i < 3; ++i)
+    if (dims[i] < 1 || box[i] < 1 || box[i] > 256) return false;
+  for (int i = 0; i < 2; ++i)
+    if (strides[i] % 16 != 0) return false;
+  const cuuint64_t gd[3] = {static_cast<cuuint64_t>(dims[0]), static_cast<cuuint64_t>(dims[1]),
+                            static_cast<cuuint64_t>(dims[2])};
+  const cuuint64_t gs[2] = {static_cast<cuuint64_t>(strides[0]), static_cast<cuuint64_t>(strides[1])};
+  const cuuint32_t bx[3] = {static_cast<cuuint32_t>(box[0]), static_cast<cuuint32_t>(box[1]),
+                            static_cast<cuuint32_t>(box[2])};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, type, 3, const_cast<void*>(base), gd, gs, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // bf16 Y [rows][cols] (row stride cols), stored as box_rows x box_cols tiles
 // without swizzle.
 bool encode_y_bf16(CUtensorMap* m, void* base, int64_t cols, int64_t rows, int box_cols,
@@ -205,13 +227,20 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     pdl = true;
   }
   if (!wq && T <= 16) {
-    // a few tokens: the product is bound by the code bytes; they stream
-    // through shared memory and are dequantised in registers for
-    // warp-level MMAs (when the code rows are 16-byte strided)
+    // a few tokens: the product is bound by turning code bytes into
+    // operands; they stream through shared memory in large stages and are
+    // dequantised in registers for warp-level MMAs (when the shape allows
+    // the unit-major views below)
+    const DecodeMapShape sh = decode_map_shape(bits, static_cast<int>(T));
+    const int64_t wpr = d * bits / 32;
     CUtensorMap tmC, tmX;
-    if (encode_codes(&tmC, codes, d * bits / 32, dp, decode_code_box_words(bits),
-                     decode_code_box_rows()) &&
-        encode_16bit(&tmX, Xh, true, d, T, d, T <= 8 ? 8 : 16)) {
+    if (d % (sh.unit_k * (bits == 3 ? 2 : 1)) == 0 && wpr % sh.piece_words == 0 &&
+        encode_3d(&tmC, codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, {sh.piece_words, dp, wpr / sh.piece_words},
+                  {wpr * 4, int64_t{sh.piece_words} * 4}, {sh.piece_words, sh.code_rows, sh.code_pieces},
+                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        encode_3d(&tmX, Xh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, {sh.unit_k, T, d / sh.unit_k},
+                  {d * 2, int64_t{sh.unit_k} * 2}, {sh.unit_k, sh.x_tokens, sh.x_units},
+                  CU_TENSOR_MAP_SWIZZLE_128B)) {
       DecodeArgs a;
       a.scales = scales;
       a.zeros = zeros;

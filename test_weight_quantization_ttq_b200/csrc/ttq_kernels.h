@@ -118,8 +118,9 @@ struct GemmMaps {
 
 // Steps (2)-(3) for T <= 16 tokens: Y[t][j] = sum_i s (q - z) Xh[t][i]
 // (+ sum_k Blr[j][k] AX[t][k] when r > 0, both bf16) with the codes
-// dequantised in registers for warp-level tensor-core MMAs.  K % 32 == 0,
-// group a power of two >= 32; Y [T][ldy] float32 or bf16.
+// dequantised in registers for warp-level tensor-core MMAs.  K a multiple
+// of 64 (128 for INT3), group a power of two >= 32; Y [T][ldy] float32 or
+// bf16.
 struct DecodeArgs {
   const uint16_t* scales = nullptr;  // [M][K / group] binary16
   const uint16_t* zeros = nullptr;
@@ -133,12 +134,16 @@ struct DecodeArgs {
   bool y_f32 = false;
   uint32_t* status = nullptr;
 };
-// The tensor maps it reads: tmC the codes [M][K bits / 32] as uint32 in
-// boxes of decode_code_box_words(bits) x decode_code_box_rows() without
-// swizzle; tmX binary16 Xh [T][K] in boxes of 64 channels x (T <= 8 ? 8 : 16)
-// tokens, 128-byte swizzled.
-int decode_code_box_words(int bits);
-int decode_code_box_rows();
+// The 3-D tensor maps it reads.  tmC: the codes as uint32 seen as
+// [K bits / 32 / piece_words][M][piece_words] (piece stride piece_words
+// words, row stride K bits / 32 words), box piece_words x code_rows x
+// code_pieces, no swizzle.  tmX: binary16 Xh seen as [K / unit_k][T][unit_k]
+// (unit stride unit_k, token stride K), box unit_k x x_tokens x x_units,
+// 128-byte swizzle.
+struct DecodeMapShape {
+  int piece_words, code_rows, code_pieces, unit_k, x_tokens, x_units;
+};
+DecodeMapShape decode_map_shape(int bits, int T);
 cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
                                const CUtensorMap& tmX, cudaStream_t stream, bool pdl = false);
 
