@@ -52,7 +52,7 @@ NCU_TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch (ncu flushes
     # L2 before it, so the W_hat and X D^-1/2 the previous kernels left in L2
     # are read from DRAM here)
-    "85c1fd19c22fa1ef": 53151488,
+    "6d92159a384ee5ea": 53043712,
 }
 
 
@@ -407,6 +407,90 @@ def run_ours(args):
     print(json.dumps(line), flush=True)
 
 
+def run_decode(args):
+    """The decode workload (d = 4096, d' = 14336, INT4 g128, T = args.decode
+    tokens): the forward timed over K steps, then its three kernels one entry
+    point each (statistic + binary16 X D^{-1/2}, quantiser, product from the
+    packed codes).  One GPU; one JSON line.  W rotates over enough copies
+    that every step reads it from HBM."""
+    import torch
+
+    from test_weight_quantization_ttq_b200 import synth, ttq
+
+    T = int(args.decode)
+    if not 1 <= T <= 16:
+        raise SystemExit("--decode takes 1..16 tokens")
+    spec = synth.C4.with_(T=T)
+    d, dp, bits, group = spec.d, spec.dp, spec.bits, spec.group
+    data = synth.generate(spec)
+    X = torch.from_numpy(data["X"]).to(torch.bfloat16).cuda()
+    W0 = torch.from_numpy(data["W"]).to(torch.bfloat16)
+    nsets = max(2, -(-2 * L2_BYTES // (2 * d * dp)))
+    Ws = [W0.cuda() for _ in range(nsets)]
+    Y = torch.empty((T, dp), dtype=torch.bfloat16, device="cuda")
+    ws = ttq.new_workspace(d, dp, T, 0, bits, group)
+    stream = torch.cuda.current_stream()
+
+    def fwd(i):
+        ttq.ttq_linear_forward(X, Ws[i % nsets], None, None, spec.p, spec.lam, spec.alpha, bits,
+                               group, ws=ws, Y=Y)
+
+    sampler = ClockSampler(0)
+    sampler.start()
+    for i in range(args.warmup):
+        fwd(i)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        fwd(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    st, flags = ttq.ttq_get_status(ws)
+    if st != ttq.TTQ_OK:
+        raise RuntimeError(f"device status {ttq.status_string(st)} (flags {flags:#x})")
+
+    views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
+    Dbuf = views["D"]
+    Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
+    codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda")
+    sc = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
+    ze = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        ttq.ttq_act_norm_scale(X, spec.p, spec.lam, spec.alpha, ws=ws, Xs=Xsbuf, copy_out=False)
+        ev[i][1].record(stream)
+        ttq.ttq_quantize_weight(Ws[i % nsets], Dbuf, bits, group, codes=codes, scales=sc, zeros=ze)
+        ev[i][2].record(stream)
+        ttq.ttq_dequant_gemm(codes, sc, ze, None, Xsbuf, None, None, bits, group, Y=Y)
+        ev[i][3].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    t = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev) / 1e3 for j in range(3)]
+    peaks = _measured_peaks()
+    code_bytes = dp * d * bits / 8 + 4.0 * dp * d / group
+    qdq_bytes = 2.0 * dp * d + code_bytes + 4.0 * d
+    prod_bytes = code_bytes + 2.0 * T * d + 2.0 * T * dp
+    hbm = peaks["hbm_gbs"]
+    kernels = [
+        {"kernel": "act_norm_scale_kernel", "us": t[0] * 1e6},
+        {"kernel": "qdq_pack_kernel", "us": t[1] * 1e6, "bytes": qdq_bytes,
+         "achieved_gbs": qdq_bytes / t[1] / 1e9, "frac": qdq_bytes / t[1] / 1e9 / hbm},
+        {"kernel": "ttq_decode_kernel", "us": t[2] * 1e6, "bytes": prod_bytes,
+         "achieved_gbs": prod_bytes / t[2] / 1e9, "frac": prod_bytes / t[2] / 1e9 / hbm},
+    ]
+    print(json.dumps({"metric": "TTQ linear decode tokens/s", "value": T * args.steps / (ms / 1e3),
+                      "unit": "tokens/s", "ms_per_step": ms / args.steps, "steps": args.steps,
+                      "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": f"decode_4096x14336_T{T}", "d": d, "dp": dp, "T": T,
+                                 "bits": bits, "group": group,
+                                 "l2": f"W rotates over {nsets} copies (> L2)"},
+                      "kernels": kernels, "hbm_peak_gbs": hbm, "clocks": clocks}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -416,10 +500,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="short run for a profiler: no clock warm-up loop, no CPU baseline, no e2e leg")
+    ap.add_argument("--decode", type=int, default=0, metavar="T",
+                    help="time the decode workload (d = 4096, d' = 14336, INT4 g128) at T <= 16 tokens instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.decode:
+        run_decode(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
