@@ -409,10 +409,12 @@ def run_ours(args):
 
 def run_decode(args):
     """The decode workload (d = 4096, d' = 14336, INT4 g128, T = args.decode
-    tokens): the forward timed over K steps, then its three kernels one entry
-    point each (statistic + binary16 X D^{-1/2}, quantiser, product from the
-    packed codes).  One GPU; one JSON line.  W rotates over enough copies
-    that every step reads it from HBM."""
+    tokens): K forwards, then K launches of each of its three kernels (one
+    entry point each: statistic + binary16 X D^{-1/2}, quantiser, product
+    from the packed codes).  A few-token step is shorter than its host-side
+    launch cost, so each batch of K calls is captured once in a CUDA graph and
+    the graph replay is timed.  One GPU; one JSON line.  W rotates over
+    enough copies that every step reads it from HBM."""
     import torch
 
     from test_weight_quantization_ttq_b200 import synth, ttq
@@ -429,47 +431,70 @@ def run_decode(args):
     Ws = [W0.cuda() for _ in range(nsets)]
     Y = torch.empty((T, dp), dtype=torch.bfloat16, device="cuda")
     ws = ttq.new_workspace(d, dp, T, 0, bits, group)
+    views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
+    Dbuf = views["D"]
+    Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
+    # the quantiser writes, and the product reads, one of ncs code sets in
+    # turn (more than L2 together)
+    ncs = max(2, -(-2 * L2_BYTES // (dp * d * bits // 8)))
+    codes = [torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda") for _ in range(ncs)]
+    sc = [torch.empty((dp, d // group), dtype=torch.int16, device="cuda") for _ in range(ncs)]
+    ze = [torch.empty((dp, d // group), dtype=torch.int16, device="cuda") for _ in range(ncs)]
     stream = torch.cuda.current_stream()
 
     def fwd(i):
         ttq.ttq_linear_forward(X, Ws[i % nsets], None, None, spec.p, spec.lam, spec.alpha, bits,
                                group, ws=ws, Y=Y)
 
+    def stat(i):
+        ttq.ttq_act_norm_scale(X, spec.p, spec.lam, spec.alpha, ws=ws, Xs=Xsbuf, copy_out=False)
+
+    def qdq(i):
+        k = i % ncs
+        ttq.ttq_quantize_weight(Ws[i % nsets], Dbuf, bits, group, codes=codes[k], scales=sc[k],
+                                zeros=ze[k])
+
+    def prod(i):
+        k = i % ncs
+        ttq.ttq_dequant_gemm(codes[k], sc[k], ze[k], None, Xsbuf, None, None, bits, group, Y=Y)
+
+    def graph_of(fn):
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(args.steps):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        return g
+
+    def time_graph(g):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / 1e3   # seconds for K calls
+
+    stat(0)
+    for k in range(ncs):   # every code set holds real codes before the product is timed
+        qdq(k)
+    g_fwd = graph_of(fwd)
     sampler = ClockSampler(0)
     sampler.start()
-    for i in range(args.warmup):
-        fwd(i)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        fwd(i)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    t_end = time.time() + (0.0 if args.profile else 1.0)
+    while time.time() < t_end:
+        g_fwd.replay()
+        torch.cuda.synchronize()
+    t_fwd = time_graph(g_fwd)
+    clocks = sampler.stop()
     st, flags = ttq.ttq_get_status(ws)
     if st != ttq.TTQ_OK:
         raise RuntimeError(f"device status {ttq.status_string(st)} (flags {flags:#x})")
-
-    views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
-    Dbuf = views["D"]
-    Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
-    codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda")
-    sc = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
-    ze = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    torch.cuda.synchronize()
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        ttq.ttq_act_norm_scale(X, spec.p, spec.lam, spec.alpha, ws=ws, Xs=Xsbuf, copy_out=False)
-        ev[i][1].record(stream)
-        ttq.ttq_quantize_weight(Ws[i % nsets], Dbuf, bits, group, codes=codes, scales=sc, zeros=ze)
-        ev[i][2].record(stream)
-        ttq.ttq_dequant_gemm(codes, sc, ze, None, Xsbuf, None, None, bits, group, Y=Y)
-        ev[i][3].record(stream)
-    torch.cuda.synchronize()
-    clocks = sampler.stop()
-    t = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev) / 1e3 for j in range(3)]
+    t = [time_graph(graph_of(fn)) / args.steps for fn in (stat, qdq, prod)]
     peaks = _measured_peaks()
     code_bytes = dp * d * bits / 8 + 4.0 * dp * d / group
     qdq_bytes = 2.0 * dp * d + code_bytes + 4.0 * d
@@ -482,12 +507,14 @@ def run_decode(args):
         {"kernel": "ttq_decode_kernel", "us": t[2] * 1e6, "bytes": prod_bytes,
          "achieved_gbs": prod_bytes / t[2] / 1e9, "frac": prod_bytes / t[2] / 1e9 / hbm},
     ]
-    print(json.dumps({"metric": "TTQ linear decode tokens/s", "value": T * args.steps / (ms / 1e3),
-                      "unit": "tokens/s", "ms_per_step": ms / args.steps, "steps": args.steps,
+    print(json.dumps({"metric": "TTQ linear decode tokens/s", "value": T * args.steps / t_fwd,
+                      "unit": "tokens/s", "ms_per_step": t_fwd * 1e3 / args.steps, "steps": args.steps,
                       "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
                       "config": {"workload": f"decode_4096x14336_T{T}", "d": d, "dp": dp, "T": T,
                                  "bits": bits, "group": group,
-                                 "l2": f"W rotates over {nsets} copies (> L2)"},
+                                 "l2": f"W rotates over {nsets} copies and the codes over {ncs} "
+                                       "sets (each more than L2)",
+                                 "timing": "CUDA graph of K calls, CUDA events around its replay"},
                       "kernels": kernels, "hbm_peak_gbs": hbm, "clocks": clocks}), flush=True)
 
 
