@@ -146,3 +146,44 @@ def sample_rows(dp: int, n: int, seed: int = 12345) -> np.ndarray:
     n = min(n, dp)
     picked = set(g.choice(dp, size=max(0, n - 2), replace=False).tolist()) | {0, dp - 1}
     return np.array(sorted(picked), dtype=np.int64)
+
+
+# ------------------------------------------------------- low-rank structure
+# Inputs for the static low-rank initialisation (B, A from W): a weight with
+# a known spectrum, and the Gaussian test matrix a randomised range finder
+# draws.  Both are drawn here so that the CUDA path and the oracle see the
+# same values; nothing below computes any part of the method.
+
+def orthonormal_columns(n: int, m: int, seed: int) -> np.ndarray:
+    """n x m float64 with orthonormal columns (Q of a seeded Gaussian, its
+    column signs fixed so that diag(R) > 0)."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    q, rr = np.linalg.qr(g.standard_normal((n, m)))
+    return q * np.where(np.diag(rr) < 0, -1.0, 1.0)
+
+
+def spectral_weight(dp: int, d: int, sigma: np.ndarray, seed: int = 0) -> dict:
+    """W = U diag(sigma) V^T (float64, d' x d) from seeded orthonormal U
+    (d' x m) and V (d x m), m = len(sigma); returns W, U, V and sigma so that
+    a test knows W's singular triplets without computing them."""
+    sigma = np.asarray(sigma, dtype=np.float64)
+    m = sigma.size
+    U = orthonormal_columns(dp, m, seed * 2 + 1)
+    V = orthonormal_columns(d, m, seed * 2 + 2)
+    return {"W": (U * sigma) @ V.T, "U": U, "V": V, "sigma": sigma}
+
+
+def geometric_spectrum(m: int, top: float = 1.0, ratio: float = 0.9, gap_at: int = 0,
+                       gap: float = 1.0) -> np.ndarray:
+    """sigma_i = top * ratio^i, i < m, divided by `gap` from index gap_at on
+    (a spectral gap after the first gap_at values when gap > 1)."""
+    s = top * ratio ** np.arange(m, dtype=np.float64)
+    if gap_at > 0:
+        s[gap_at:] /= gap
+    return s
+
+
+def gaussian_test_matrix(d: int, l: int, seed: int = 7) -> np.ndarray:
+    """d x l float32 standard normal draws (the range finder's test matrix)."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    return g.standard_normal((d, l), dtype=np.float32)
