@@ -518,6 +518,62 @@ def run_decode(args):
                       "kernels": kernels, "hbm_peak_gbs": hbm, "clocks": clocks}), flush=True)
 
 
+def run_lowrank(args):
+    """The static low-rank initialisation at the 70B-like MLP shape
+    (d' = 28672, d = 8192, bf16 W, r = 64, 8 extra sampled directions, 2
+    subspace iterations): K calls timed with CUDA events.  Reported against
+    the fp32 CUDA-core peak (148 SMs x 128 lanes x 2 flops x the max SM
+    clock), since its products run on CUDA cores.  One GPU; one JSON line."""
+    import torch
+
+    from test_weight_quantization_ttq_b200 import synth, ttq
+
+    dp, d, r, over, q = 28672, 8192, 64, 8, 2
+    l = r + over
+    g = torch.Generator(device="cuda").manual_seed(1)
+    W = (torch.randn((dp, d), generator=g, device="cuda") * 0.015).to(torch.bfloat16)
+    Om = torch.from_numpy(synth.gaussian_test_matrix(d, l, seed=7)).cuda()
+    n = ttq.ttq_lowrank_workspace_size(dp, d, r, over)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    ttq.ttq_workspace_init(ws)
+    B = torch.empty((dp, r), dtype=torch.bfloat16, device="cuda")
+    A = torch.empty((r, d), dtype=torch.bfloat16, device="cuda")
+    R = torch.empty_like(W)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        ttq.ttq_lowrank_init(W, r, Om, power_iters=q, ws=ws, B=B, A=A, W_res=R)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        ttq.ttq_lowrank_init(W, r, Om, power_iters=q, ws=ws, B=B, A=A, W_res=R)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    t = e0.elapsed_time(e1) / 1e3 / args.steps
+    st, flags = ttq.ttq_get_status(ws)
+    # multiply-adds: W passes (W Omega, q x (W^T Q, W Z), W^T Q) of 2 d' d l
+    # each, the residual 2 d' d r, the Gram matrices and l-column products
+    passes = 2 + 2 * q
+    flops = passes * 2.0 * dp * d * l + 2.0 * dp * d * r
+    flops += (3 * (1 + 2 * q)) * (2.0 * dp * l * l * 2) + 2.0 * d * l * l + 2.0 * (dp + d) * l * r
+    sm_max = clocks.get("sm_max_mhz") or 1965.0
+    peak = 148 * 128 * 2 * sm_max * 1e6 / 1e12
+    achieved = flops / t / 1e12
+    print(json.dumps({"metric": "TTQ low-rank init ms", "value": t * 1e3, "unit": "ms", "higher_is_better": False,
+                      "steps": args.steps, "warmup": args.warmup, "dtype": "bf16 W, fp32 products",
+                      "data": "synthetic", "status": ttq.status_string(st), "flags": flags,
+                      "config": {"workload": "lowrank_init_28672x8192_r64", "dp": dp, "d": d, "r": r,
+                                 "oversample": over, "power_iters": q},
+                      "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                                   "frac": achieved / peak,
+                                   "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x max SM clock"},
+                      "hbm_bytes_of_W_passes": (passes + 2) * 2.0 * dp * d,
+                      "clocks": clocks}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,10 +585,14 @@ def main():
                     help="short run for a profiler: no clock warm-up loop, no CPU baseline, no e2e leg")
     ap.add_argument("--decode", type=int, default=0, metavar="T",
                     help="time the decode workload (d = 4096, d' = 14336, INT4 g128) at T <= 16 tokens instead")
+    ap.add_argument("--lowrank", action="store_true",
+                    help="time the static low-rank initialisation (d' = 28672, d = 8192, r = 64) instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.decode:
+    if args.lowrank:
+        run_lowrank(args)
+    elif args.decode:
         run_decode(args)
     elif args.impl == "reference":
         run_reference(args)

@@ -99,6 +99,9 @@ typedef enum ttq_qscheme {
 #define TTQ_FLAG_SCALE_OVERFLOW 0x2u
 #define TTQ_FLAG_TIMEOUT 0x4u
 #define TTQ_FLAG_X_RANGE 0x8u /* an activation beyond the binary16 range (|x| > 65504) */
+#define TTQ_FLAG_RANK_DEFICIENT 0x10u /* ttq_lowrank_init: W's sampled range had fewer than
+                                         r + oversample independent directions (a Cholesky
+                                         pivot was not positive and was floored) */
 
 /* Byte offsets of the workspace regions for one problem shape (all 256-byte
  * aligned); `total` equals ttq_workspace_size(...).  After
@@ -324,6 +327,34 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
  * (may be NULL).  Returns TTQ_OK if no flag is set, TTQ_ERR_TIMEOUT if the
  * timeout flag is set, else TTQ_ERR_NONFINITE. */
 ttq_status ttq_get_status(const void* ws, uint32_t* flags);
+
+/* ---------------------------------------------------------------------
+ * Static low-rank initialisation (the step before the path).
+ *
+ * gist.science/zh/paper/2603.19296, section 2.2 (and gist.science/nl/paper/
+ * 2603.19296, section 2 "Kerncomponenten", item 3): W ~ W_q + B A, with the
+ * static factors B, A initialised by PCA and W_q the quantised residual.
+ * PCA of W is read as W's uncentred truncated SVD: B = U_r S_r [dp][r] and
+ * A = V_r^T [r][d] (A's rows orthonormal, B = W A^T), computed by a
+ * randomised range finder with `power_iters` subspace iterations (Halko,
+ * Martinsson, Tropp 2011) on the caller's Gaussian test matrix Omega
+ * [d][r + oversample] (float32, row-major; the random draws are an input).
+ * The closer the spectrum of W is to having a gap after r, and the more
+ * iterations, the closer B A is to the exact truncated SVD.
+ *
+ * W, B, A and W_res share `dtype` (TTQ_F32 or TTQ_BF16), row-major.
+ * W_res = W - B A (with B, A as stored, i.e. rounded to dtype) [dp][d] is
+ * written when non-NULL; it is the weight to pass to ttq_linear_forward
+ * together with A and B.  Requirements: 1 <= r, oversample >= 0,
+ * r + oversample <= min(96, dp, d), 0 <= power_iters <= 16, ws of at least
+ * ttq_lowrank_workspace_size(dp, d, r, oversample) bytes, initialised with
+ * ttq_workspace_init.  Device-side conditions set TTQ_FLAG_RANK_DEFICIENT
+ * or TTQ_FLAG_NONFINITE in the workspace status word.  Asynchronous on
+ * `stream`; deterministic for given inputs. */
+size_t ttq_lowrank_workspace_size(int64_t dp, int64_t d, int64_t r, int64_t oversample);
+ttq_status ttq_lowrank_init(const void* W, ttq_dtype dtype, int64_t dp, int64_t d, int64_t r,
+                            int64_t oversample, int power_iters, const float* Omega, void* B,
+                            void* A, void* W_res, void* ws, size_t ws_bytes, void* stream);
 
 /* Static description of a status code. */
 const char* ttq_status_string(ttq_status s);

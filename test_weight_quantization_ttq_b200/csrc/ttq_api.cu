@@ -630,6 +630,31 @@ ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const
                                TTQ_QSCHEME_ASYMMETRIC, Y, y_dtype, ws, ws_bytes, stream);
 }
 
+size_t ttq_lowrank_workspace_size(int64_t dp, int64_t d, int64_t r, int64_t oversample) {
+  if (dp < 1 || d < 1 || r < 1 || oversample < 0 || r + oversample > 96) return 0;
+  return ttq::lowrank_layout(dp, d, r + oversample).total;
+}
+
+ttq_status ttq_lowrank_init(const void* W, ttq_dtype dtype, int64_t dp, int64_t d, int64_t r,
+                            int64_t oversample, int power_iters, const float* Omega, void* B,
+                            void* A, void* W_res, void* ws, size_t ws_bytes, void* stream) {
+  if (dtype != TTQ_F32 && dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
+  if (dp < 1 || d < 1 || r < 1 || oversample < 0 || power_iters < 0 || power_iters > 16)
+    return TTQ_ERR_INVALID_ARG;
+  const int64_t l = r + oversample;
+  if (l > 96 || l > dp || l > d) return TTQ_ERR_UNSUPPORTED;
+  if (dp > (int64_t{1} << 31) || d > (int64_t{1} << 31)) return TTQ_ERR_UNSUPPORTED;
+  if (W == nullptr || Omega == nullptr || B == nullptr || A == nullptr) return TTQ_ERR_INVALID_ARG;
+  const void* ptrs[] = {W, Omega, B, A, W_res};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < ttq::lowrank_layout(dp, d, l).total) return TTQ_ERR_WORKSPACE;
+  return cuda_status(ttq::launch_lowrank_init(W, dtype == TTQ_BF16, dp, d, r, l, power_iters, Omega,
+                                              B, A, W_res, ws, device_sms(),
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 ttq_status ttq_get_status(const void* ws, uint32_t* flags) {
   if (ws == nullptr) return TTQ_ERR_INVALID_ARG;
   uint32_t f = 0;

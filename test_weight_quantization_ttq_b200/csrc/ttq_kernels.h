@@ -147,6 +147,19 @@ DecodeMapShape decode_map_shape(int bits, int T);
 cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
                                const CUtensorMap& tmX, cudaStream_t stream, bool pdl = false);
 
+// Static low-rank initialisation (B, A from a randomised truncated SVD of
+// W; residual W - B A).  Workspace offsets (bytes) past the 4 KiB status
+// header; l = r + oversample.
+struct LowrankLayout {
+  size_t Y, Q, Bt, partial, G, Rinv, U, sigma, inv_sigma, total;
+  int64_t partial_floats;
+};
+LowrankLayout lowrank_layout(int64_t dp, int64_t d, int64_t l);
+size_t lowrank_small_smem(int l, bool eig);
+cudaError_t launch_lowrank_init(const void* W, bool w_bf16, int64_t dp, int64_t d, int64_t r, int64_t l,
+                                int power_iters, const float* Omega, void* Bout, void* Aout, void* Wres,
+                                void* ws, int num_sms, cudaStream_t stream);
+
 // Words per row of the code tile one K block of 64 channels needs.
 int gemm_code_tile_words(int bits);
 

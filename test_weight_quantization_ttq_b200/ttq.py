@@ -33,6 +33,7 @@ TTQ_FLAG_NONFINITE = 0x1
 TTQ_FLAG_SCALE_OVERFLOW = 0x2
 TTQ_FLAG_TIMEOUT = 0x4
 TTQ_FLAG_X_RANGE = 0x8
+TTQ_FLAG_RANK_DEFICIENT = 0x10
 
 # C signatures, in the order of include/ttq.h
 _P = ctypes.c_void_p
@@ -71,6 +72,8 @@ SIGNATURES = {
                                   _P, _INT, _P, _SZ, _P]),
     "ttq_linear_forward_kernels": (_INT, [_INT, _I64, _I64, _I64, _I64, _F, ctypes.POINTER(ctypes.c_int)]),
     "ttq_get_status": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "ttq_lowrank_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
+    "ttq_lowrank_init": (_INT, [_P, _INT, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P, _P, _SZ, _P]),
     "ttq_status_string": (ctypes.c_char_p, [_INT]),
     "ttq_version": (ctypes.c_char_p, []),
 }
@@ -372,6 +375,39 @@ def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, 
     else:
         _check(lib().ttq_linear_forward_ex(*args, scheme, *tail), "ttq_linear_forward_ex")
     return Y
+
+
+def ttq_lowrank_workspace_size(dp, d, r, oversample) -> int:
+    return int(lib().ttq_lowrank_workspace_size(dp, d, r, oversample))
+
+
+def ttq_lowrank_init(W, r, Omega, power_iters=2, ws=None, B=None, A=None, W_res=None,
+                     residual=True, stream=None):
+    """Static low-rank factors of W [d'][d] (float32 or bf16): B [d'][r],
+    A [r][d] from a randomised truncated SVD with the Gaussian test matrix
+    Omega [d][r + oversample] (float32), and W_res = W - B A (when
+    `residual`).  Returns (B, A, W_res or None)."""
+    dp, d = W.shape
+    l = Omega.shape[1]
+    oversample = l - r
+    dt = _dtype_code(W)
+    if ws is None:
+        n = ttq_lowrank_workspace_size(dp, d, r, oversample)
+        if n == 0:
+            raise TTQError(TTQ_ERR_INVALID_ARG, "ttq_lowrank_workspace_size")
+        ws = torch.empty(n, dtype=torch.uint8, device=W.device)
+        ttq_workspace_init(ws, stream)
+    if B is None:
+        B = torch.empty((dp, r), dtype=W.dtype, device=W.device)
+    if A is None:
+        A = torch.empty((r, d), dtype=W.dtype, device=W.device)
+    if W_res is None and residual:
+        W_res = torch.empty_like(W)
+    _check(lib().ttq_lowrank_init(_dev(W, "W"), dt, dp, d, r, oversample, power_iters, _dev(Omega, "Omega"),
+                                  _dev(B, "B"), _dev(A, "A"), _dev(W_res, "W_res"), _dev(ws, "ws"),
+                                  ws.numel(), _stream(stream)),
+           "ttq_lowrank_init")
+    return B, A, W_res
 
 
 def workspace_views(ws: torch.Tensor, d, dp, T, r, bits, group, dtype=TTQ_BF16) -> dict:

@@ -115,3 +115,29 @@ def test_rejections_before_device_work(L):
     assert st == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_workspace_init(None, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_get_status(None, None) == ttq.TTQ_ERR_INVALID_ARG
+
+
+def test_lowrank_init_rejections_before_device_work(L):
+    size = L.ttq_lowrank_workspace_size
+    assert size(0, 64, 8, 8) == 0 and size(64, 64, 0, 8) == 0 and size(64, 64, 90, 8) == 0
+    n = size(300, 200, 16, 8)
+    assert n >= 4096 + 4 * 300 * 24 * 2 + 4 * 200 * 24
+    init = L.ttq_lowrank_init
+    ok = dict(W=16, dt=1, dp=300, d=200, r=16, ov=8, q=2, Om=32, B=48, A=64, R=80, ws=256, nb=n)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return init(a["W"], a["dt"], a["dp"], a["d"], a["r"], a["ov"], a["q"], a["Om"], a["B"], a["A"],
+                    a["R"], a["ws"], a["nb"], None)
+
+    assert call(dt=2) == ttq.TTQ_ERR_INVALID_ARG            # binary16 W
+    assert call(r=0) == ttq.TTQ_ERR_INVALID_ARG
+    assert call(ov=-1) == ttq.TTQ_ERR_INVALID_ARG
+    assert call(q=17) == ttq.TTQ_ERR_INVALID_ARG
+    assert call(r=90) == ttq.TTQ_ERR_UNSUPPORTED            # r + oversample > 96
+    assert call(dp=20) == ttq.TTQ_ERR_UNSUPPORTED           # r + oversample > d'
+    assert call(W=None) == ttq.TTQ_ERR_INVALID_ARG
+    assert call(Om=None) == ttq.TTQ_ERR_INVALID_ARG
+    assert call(A=72) == ttq.TTQ_ERR_INVALID_ARG            # not 16-byte aligned
+    assert call(ws=128) == ttq.TTQ_ERR_INVALID_ARG          # not 256-byte aligned
+    assert call(nb=n - 1) == ttq.TTQ_ERR_WORKSPACE
