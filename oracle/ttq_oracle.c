@@ -299,6 +299,124 @@ int ttqo_quantize_sym(const float* W, int64_t dp, int64_t d, const float* D,
   return flags;
 }
 
+/* ------------------------------------------------------------- FP8 codes
+ * blog.lo0.es (English post), the comparison with FP8 end to end: TTQ
+ * decides how s is obtained, not the format of the code, so "TTQ over FP8"
+ * is the same activation-aware scale feeding an FP8 quantiser.  Readings:
+ *   - the format is E4M3 as the OCP 8-bit floating point specification
+ *     defines it: 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits;
+ *     exponent 0 is subnormal (m/8 * 2^-6); no infinities; S.1111.111 is NaN;
+ *     the largest finite magnitude is 448 (S.1111.110);
+ *   - the scale is symmetric per group: s = binary16 round-up of
+ *     max|x| / 448 (floored at 2^-14), so |x| / s <= 448;
+ *   - the code is the E4M3 value nearest to the binary32 product x * (1/s),
+ *     ties to the even code, saturating at +-448 (the sign of a product that
+ *     rounds to zero is kept);
+ *   - the zero point is 0 (stored as binary16 +0) and the reconstruction is
+ *     s * e4m3(code); the 8-bit codes are packed like any 8-bit code (4 per
+ *     word, code i in bits 8 (i mod 4) .. of word i / 4).                  */
+double ttqo_e4m3_value(uint32_t code) {
+  const int sign = (code >> 7) & 1;
+  const int e = (code >> 3) & 15;
+  const int m = code & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) v = ldexp((double)m, -9);             /* m/8 * 2^-6 */
+  else v = ldexp(8.0 + (double)m, e - 10);           /* (1 + m/8) 2^(e-7) */
+  return sign ? -v : v;
+}
+
+/* Nearest finite E4M3 magnitude by search over the 127 non-negative finite
+ * codes, ties to the code whose last fraction bit is 0; beyond 448 the
+ * result is 448; the sign of v is kept.  NaN maps to the NaN code 0x7F.  */
+uint32_t ttqo_e4m3_from(double v) {
+  if (isnan(v)) return 0x7Fu;
+  const uint32_t sign = signbit(v) ? 0x80u : 0u;
+  const double a = fabs(v);
+  uint32_t best = 0;
+  double bestd = INFINITY;
+  for (uint32_t c = 0; c <= 0x7Eu; ++c) {
+    const double dd = fabs(ttqo_e4m3_value(c) - a);
+    if (dd < bestd || (dd == bestd && (c & 1u) == 0u)) {
+      bestd = dd;
+      best = c;
+    }
+  }
+  return best | sign;
+}
+
+/* The FP8 (E4M3) quantiser with the activation-aware scale; codes are 8 bits
+ * per weight, zeros are binary16 +0.                                      */
+int ttqo_quantize_fp8(const float* W, int64_t dp, int64_t d, const float* D, int group,
+                      uint32_t* codes, uint16_t* scales, uint16_t* zeros) {
+  if (!W || !codes || !scales || !zeros || dp < 0 || d < 1 || group < 1 || d % group != 0)
+    return TTQO_BAD_ARG;
+  int flags = TTQO_OK;
+  const int64_t wpr = ttqo_words_per_row(d, 8);
+  const int64_t ngroups = d / group;
+  float* sd = (float*)malloc(sizeof(float) * (size_t)d);
+  float* xg = (float*)malloc(sizeof(float) * (size_t)group);
+  if (!sd || !xg) {
+    free(sd);
+    free(xg);
+    return TTQO_BAD_ARG;
+  }
+  for (int64_t i = 0; i < d; ++i) {
+    sd[i] = D ? sqrtf(D[i]) : 1.0f;
+    if (!isfinite(sd[i])) flags |= TTQO_NONFINITE;
+  }
+  memset(codes, 0, sizeof(uint32_t) * (size_t)(dp * wpr));
+  for (int64_t j = 0; j < dp; ++j) {
+    uint32_t* crow = codes + j * wpr;
+    for (int64_t k = 0; k < ngroups; ++k) {
+      float amax = 0.0f;
+      for (int c = 0; c < group; ++c) {
+        const int64_t i = k * group + c;
+        const float w = W[j * d + i];
+        if (!isfinite(w)) flags |= TTQO_NONFINITE;
+        xg[c] = w * sd[i];
+        if (fabsf(xg[c]) > amax) amax = fabsf(xg[c]);
+      }
+      float s32 = amax / 448.0f;
+      if (!(s32 >= 0x1p-14f)) s32 = 0x1p-14f;
+      const uint16_t s16 = ttqo_f32_to_f16_ru(s32);
+      if ((s16 & 0x7c00) == 0x7c00) flags |= TTQO_NONFINITE;
+      const float s = ttqo_f16_to_f32(s16);
+      const float inv = 1.0f / s;
+      scales[j * ngroups + k] = s16;
+      zeros[j * ngroups + k] = 0;
+      for (int c = 0; c < group; ++c) {
+        const float prod = xg[c] * inv;               /* binary32 product */
+        put_code(crow, k * group + c, 8, ttqo_e4m3_from((double)prod));
+      }
+    }
+  }
+  free(sd);
+  free(xg);
+  return flags;
+}
+
+/* FP8 reconstruction: w_hat[j][i] = s_jk e4m3(q_ji) Dr_i in fp64, for the
+ * listed rows (rows == NULL: rows 0..nrows-1); Dr == NULL means D = I.     */
+int ttqo_dequant_rows_fp8(const uint32_t* codes, const uint16_t* scales, const double* Dr,
+                          int64_t dp, int64_t d, int group, const int64_t* rows, int64_t nrows,
+                          double* What) {
+  if (!codes || !scales || !What || d < 1 || group < 1 || d % group != 0 || nrows < 0)
+    return TTQO_BAD_ARG;
+  const int64_t wpr = ttqo_words_per_row(d, 8);
+  const int64_t ngroups = d / group;
+  for (int64_t rr = 0; rr < nrows; ++rr) {
+    const int64_t j = rows ? rows[rr] : rr;
+    if (j < 0 || j >= dp) return TTQO_BAD_ARG;
+    for (int64_t i = 0; i < d; ++i) {
+      const double sc = (double)ttqo_f16_to_f32(scales[j * ngroups + i / group]);
+      const double val = ttqo_e4m3_value((uint32_t)ttqo_code_at(codes + j * wpr, i, 8));
+      What[rr * d + i] = sc * val * (Dr ? Dr[i] : 1.0);
+    }
+  }
+  return TTQO_OK;
+}
+
 /* Step 3: W_hat = Q[.] D^{-1/2}: w_hat[j][i] = s_jk (q_ji - z_jk) Dr_i, in
  * fp64, for the listed rows only (rows == NULL means rows 0..nrows-1).
  * Dr == NULL means D = I.                                                  */

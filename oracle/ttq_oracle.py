@@ -75,6 +75,14 @@ class Oracle:
         lib.ttqo_quantize.restype = ctypes.c_int
         lib.ttqo_quantize_sym.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, ctypes.c_int, _P, _P, _P]
         lib.ttqo_quantize_sym.restype = ctypes.c_int
+        lib.ttqo_e4m3_value.argtypes = [ctypes.c_uint32]
+        lib.ttqo_e4m3_value.restype = ctypes.c_double
+        lib.ttqo_e4m3_from.argtypes = [ctypes.c_double]
+        lib.ttqo_e4m3_from.restype = ctypes.c_uint32
+        lib.ttqo_quantize_fp8.argtypes = [_P, _I64, _I64, _P, ctypes.c_int, _P, _P, _P]
+        lib.ttqo_quantize_fp8.restype = ctypes.c_int
+        lib.ttqo_dequant_rows_fp8.argtypes = [_P, _P, _P, _I64, _I64, ctypes.c_int, _P, _I64, _P]
+        lib.ttqo_dequant_rows_fp8.restype = ctypes.c_int
         lib.ttqo_dequant_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, ctypes.c_int, ctypes.c_int, _P, _I64, _P]
         lib.ttqo_dequant_rows.restype = ctypes.c_int
         lib.ttqo_project.argtypes = [_P, _I64, _P, _I64, _I64, _P]
@@ -128,6 +136,48 @@ class Oracle:
         st = fn(W.ctypes.data, dp, d, Dp, bits, group,
                 codes.ctypes.data, scales.ctypes.data, zeros.ctypes.data)
         return codes, scales, zeros, st
+
+    # -- FP8 (E4M3) codes --------------------------------------------------
+    def e4m3_value(self, code: int) -> float:
+        return float(self.lib.ttqo_e4m3_value(int(code)))
+
+    def e4m3_from(self, v: float) -> int:
+        return int(self.lib.ttqo_e4m3_from(float(v)))
+
+    def quantize_fp8(self, W: np.ndarray, D: np.ndarray | None, group: int):
+        """The E4M3 quantiser with the activation-aware scale; 8-bit codes
+        packed 4 per word, zeros all binary16 +0."""
+        W = np.ascontiguousarray(W, dtype=np.float32)
+        dp, d = W.shape
+        codes = np.zeros((dp, self.words_per_row(d, 8)), np.uint32)
+        ng = d // group if group > 0 and d % group == 0 else 1
+        scales = np.zeros((dp, ng), np.uint16)
+        zeros = np.zeros((dp, ng), np.uint16)
+        Dp = None
+        if D is not None:
+            D32 = np.ascontiguousarray(D, dtype=np.float32)
+            Dp = D32.ctypes.data
+        st = self.lib.ttqo_quantize_fp8(W.ctypes.data, dp, d, Dp, group, codes.ctypes.data,
+                                        scales.ctypes.data, zeros.ctypes.data)
+        return codes, scales, zeros, st
+
+    def dequant_rows_fp8(self, codes, scales, Dr, d: int, group: int, rows=None):
+        codes = np.ascontiguousarray(codes, dtype=np.uint32)
+        scales = np.ascontiguousarray(scales, dtype=np.uint16)
+        dp = codes.shape[0]
+        rows_arr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+        nrows = dp if rows is None else rows_arr.size
+        What = np.empty((nrows, d), np.float64)
+        Drp = None
+        if Dr is not None:
+            Dr64 = np.ascontiguousarray(Dr, dtype=np.float64)
+            Drp = Dr64.ctypes.data
+        st = self.lib.ttqo_dequant_rows_fp8(codes.ctypes.data, scales.ctypes.data, Drp, dp, d, group,
+                                            None if rows_arr is None else rows_arr.ctypes.data, nrows,
+                                            What.ctypes.data)
+        if st != OK:
+            raise ValueError(f"dequant_rows_fp8 failed ({st})")
+        return What
 
     def code_at(self, codes_row: np.ndarray, i: int, bits: int) -> int:
         r = np.ascontiguousarray(codes_row, dtype=np.uint32)

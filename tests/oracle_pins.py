@@ -445,6 +445,100 @@ def check_method_effect(O):
     assert e_ttq < 0.8 * e_rtn, (e_ttq, e_rtn)
 
 
+# ---------------------------------------------------------------- FP8 codes
+# E4M3 as the OCP 8-bit floating point specification defines it: sign,
+# 4 exponent bits with bias 7, 3 fraction bits, subnormals at exponent 0,
+# no infinities, S.1111.111 NaN, largest finite 448.  The values below are
+# written out from that definition (not produced by the oracle).
+_E4M3_KNOWN = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x30: 0.5,
+               0x38: 1.0, 0x39: 1.125, 0x3C: 1.5, 0x40: 2.0, 0x44: 3.0, 0x6C: 96.0, 0x6D: 104.0,
+               0x77: 240.0, 0x78: 256.0, 0x7E: 448.0, 0x80: -0.0, 0xB8: -1.0, 0xFE: -448.0}
+
+
+def _e4m3_by_definition(code: int) -> float:
+    e, m = (code >> 3) & 15, code & 7
+    if e == 15 and m == 7:
+        return float("nan")
+    v = m / 8 * 2.0 ** -6 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7)
+    return -v if code & 0x80 else v
+
+
+def check_e4m3_table(O):
+    for c, v in _E4M3_KNOWN.items():
+        got = O.e4m3_value(c)
+        assert got == v and np.signbit(got) == np.signbit(v), (hex(c), got, v)
+    for c in range(256):
+        want = _e4m3_by_definition(c)
+        got = O.e4m3_value(c)
+        assert (np.isnan(want) and np.isnan(got)) or got == want, (hex(c), got, want)
+    finite = [O.e4m3_value(c) for c in range(0x7F)]
+    assert all(b > a for a, b in zip(finite, finite[1:]))          # monotone in the code
+    assert sum(np.isnan(O.e4m3_value(c)) for c in range(256)) == 2  # 0x7F and 0xFF
+
+
+def check_e4m3_rounding(O):
+    vals = [_e4m3_by_definition(c) for c in range(0x7F)]
+    for c in range(0x7E):
+        a, b = vals[c], vals[c + 1]
+        mid = (a + b) / 2
+        even = c if c % 2 == 0 else c + 1
+        assert O.e4m3_from(mid) == even, (hex(c), mid)              # ties to the even code
+        assert O.e4m3_from(mid * (1 - 2.0 ** -30)) == c
+        assert O.e4m3_from(mid * (1 + 2.0 ** -30)) == c + 1
+        assert O.e4m3_from(-b) == (c + 1) | 0x80
+    for big in (448.0, 460.0, 464.0, 500.0, 1e30):
+        assert O.e4m3_from(big) == 0x7E and O.e4m3_from(-big) == 0xFE
+    assert O.e4m3_from(-0.0) == 0x80 and O.e4m3_from(2.0 ** -11) == 0x00
+    assert O.e4m3_from(-(2.0 ** -10) * 1.5) == 0x81                 # nearer 2^-9 than 0
+
+
+def check_fp8_worked_example(O):
+    # one group of 8, D = I: the group's largest magnitude is 448, so s = 1
+    # and each code is the E4M3 rounding of the weight itself (100 lies
+    # half-way between 96 and 104 and goes to the even code, 96)
+    row = np.array([[0.0, 1.0, 2.0, 3.0, 448.0, -448.0, 0.5, 100.0]], np.float32)
+    codes, sc, ze, st = O.quantize_fp8(row, None, 8)
+    assert st == 0
+    assert sc.tolist() == [[0x3C00]] and ze.tolist() == [[0]]
+    assert codes.tolist() == [[0x44403800, 0x6C30FE7E]], [hex(x) for x in codes.ravel()]
+    What = O.dequant_rows_fp8(codes, sc, None, 8, 8)
+    assert What.tolist() == [[0.0, 1.0, 2.0, 3.0, 448.0, -448.0, 0.5, 96.0]]
+
+
+def check_fp8_properties(O):
+    g = np.random.Generator(np.random.PCG64(77))
+    d, group = 256, 64
+    W = (g.standard_normal((6, d)) * 0.05).astype(np.float32)
+    W[:, 17] *= 60.0
+    D = np.exp(g.uniform(-3, 3, d)).astype(np.float32)
+    codes, sc, ze, st = O.quantize_fp8(W, D, group)
+    assert st == 0 and not ze.any()
+    q = codes.view(np.uint8).reshape(6, d)                       # bytes in code order
+    s = _f16_bits_to_f64(sc)
+    x = W.astype(np.float64) * np.sqrt(D.astype(np.float64))
+    vals = np.vectorize(_e4m3_by_definition)(q.astype(np.int64))
+    rec = np.repeat(s, group, axis=1) * vals
+    sg = np.repeat(s, group, axis=1)
+    # 3 fraction bits: half an ulp is 2^-4 relative in the normal range,
+    # 2^-10 s absolute among the subnormals (plus binary32 slack)
+    assert np.all(np.abs(rec - x) <= 2.0 ** -4 * np.abs(x) * (1 + 1e-5) + 2.0 ** -10 * sg * (1 + 1e-5))
+    # the oracle's reconstruction s e4m3(q) D^-1/2 against the same
+    # statement in numpy (scales far from 1, D^-1/2 far from 1)
+    Dr = 1.0 / np.sqrt(D.astype(np.float64))
+    What = O.dequant_rows_fp8(codes, sc, Dr, d, group)
+    assert np.max(np.abs(What - rec * Dr)) <= 1e-12 * np.max(np.abs(rec * Dr))
+    # every group's largest magnitude is coded as +-448
+    for j in range(6):
+        for k in range(d // group):
+            blk = x[j, k * group:(k + 1) * group]
+            i = int(np.argmax(np.abs(blk)))
+            assert q[j, k * group + i] & 0x7F == 0x7E
+    # odd symmetry: -W flips exactly the sign bit of every code
+    codes_n, sc_n, _, _ = O.quantize_fp8(-W, D, group)
+    assert np.array_equal(sc_n, sc)
+    assert np.array_equal(codes_n.view(np.uint8), codes.view(np.uint8) ^ 0x80)
+
+
 ALL_CHECKS = [
     check_hand_example,
     check_f16_round_up,
@@ -458,6 +552,10 @@ ALL_CHECKS = [
     check_quantizer_properties,
     check_scaling_and_rows,
     check_dequant_layout,
+    check_e4m3_table,
+    check_e4m3_rounding,
+    check_fp8_worked_example,
+    check_fp8_properties,
     check_projection,
     check_x_rescale,
     check_nonfinite,

@@ -58,6 +58,15 @@ MUTANTS = [
     ("project_channel_reversed", "acc += What[r * d + i] * X[t * d + i];",
      "acc += What[r * d + i] * X[t * d + (d - 1 - i)];"),
     ("lowrank_dropped", "Y[t * nrows + r] += acc;", "Y[t * nrows + r] += 0.0 * acc;"),
+    ("e4m3_exponent_bias", "else v = ldexp(8.0 + (double)m, e - 10);", "else v = ldexp(8.0 + (double)m, e - 11);"),
+    ("e4m3_subnormal_scale", "if (e == 0) v = ldexp((double)m, -9);", "if (e == 0) v = ldexp((double)m, -10);"),
+    ("e4m3_nan_code", "if (e == 15 && m == 7) return NAN;", "if (e == 15 && m == 6) return NAN;"),
+    ("e4m3_ties_odd", "if (dd < bestd || (dd == bestd && (c & 1u) == 0u)) {",
+     "if (dd < bestd || (dd == bestd && (c & 1u) == 1u)) {"),
+    ("e4m3_sign_dropped", "return best | sign;", "return best;"),
+    ("fp8_wrong_max", "float s32 = amax / 448.0f;", "float s32 = amax / 240.0f;"),
+    ("fp8_dequant_drops_scale", "What[rr * d + i] = sc * val * (Dr ? Dr[i] : 1.0);",
+     "What[rr * d + i] = val * (Dr ? Dr[i] : 1.0);"),
     ("lowrank_A_transposed", "for (int64_t i = 0; i < d; ++i) acc += A[k * d + i] * X[t * d + i];",
      "for (int64_t i = 0; i < d; ++i) acc += A[(i % rank) * d + (k * d + i) / rank % d] * X[t * d + i];"),
 ]
