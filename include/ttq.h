@@ -88,10 +88,20 @@ typedef enum ttq_dtype {
  * point (the default everywhere).  TTQ_QSCHEME_SYMMETRIC: levels
  * +-(2^(bits-1) - 1) with scale max|x| / (2^(bits-1) - 1); the codes are
  * stored as level + 2^(bits-1), and the zero point 2^(bits-1) is stored in
- * `zeros`, so both schemes dequantise as scales * (code - zeros). */
+ * `zeros`, so both schemes dequantise as scales * (code - zeros).
+ * TTQ_QSCHEME_FP8_E4M3 (blog.lo0.es, the comparison with FP8 end to end:
+ * TTQ derives s, the code format is free): bits must be 8; the code is the
+ * E4M3 value (OCP 8-bit floating point: bias 7, 3 fraction bits, largest
+ * 448) nearest to the binary32 product x * (1/s), ties to even, saturating,
+ * with s = binary16 round-up of max|x| / 448 per group; one byte per weight
+ * (four per word, weight i in bits 8 (i mod 4) of word i / 4), zeros +0,
+ * reconstruction scales * e4m3(code).  The forward always materialises the
+ * binary16 s * e4m3(q) for this scheme; ttq_dequant_gemm does not take
+ * 8-bit codes.  INT schemes take bits 2..4. */
 typedef enum ttq_qscheme {
   TTQ_QSCHEME_ASYMMETRIC = 0,
-  TTQ_QSCHEME_SYMMETRIC = 1
+  TTQ_QSCHEME_SYMMETRIC = 1,
+  TTQ_QSCHEME_FP8_E4M3 = 2
 } ttq_qscheme;
 
 /* Device status word bits (ttq_get_status). */
@@ -121,8 +131,9 @@ typedef struct ttq_workspace_layout {
   size_t xh;      /* binary16 [T][d] X D^{-1/2} for the product   */
   size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32, r > 0) */
   size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32, r > 0) */
-  size_t wq;      /* binary16 [d'][d] s (q - z) that ttq_linear_forward's
-                     product reads when T > 256 (0: not in this layout) */
+  size_t wq;      /* binary16 [d'][d] s (q - z) (s e4m3(q) for 8-bit codes)
+                     that ttq_linear_forward's product reads when T > 256 or
+                     bits == 8 (0: not in this layout) */
   size_t total;
   int64_t splits; /* number of token splits of the statistic pass */
   int64_t ax_ld;  /* row stride (elements) of A X                 */

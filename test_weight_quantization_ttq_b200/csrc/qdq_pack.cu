@@ -22,6 +22,8 @@
 // scalar one (checked on B200 against __fmul_rn).
 // The kernel is HBM-bound: it reads W once and writes d*b/8 + 4d/g bytes per
 // row.
+#include <cuda_fp8.h>
+
 #include <type_traits>
 
 #include "ttq_device.cuh"
@@ -310,6 +312,137 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_flag(status, TTQ_FLAG_NONFINITE);
 }
 
+// FP8 (E4M3) codes with the activation-aware scale (blog.lo0.es, the
+// comparison with FP8 end to end: TTQ derives s, the code format is free):
+//   x = W_ji sqrt(D_i); s32 = max|x| / 448, floored at 2^-14;
+//   s = binary16 round-up(s32); inv = 1 / s;
+//   code = E4M3 round-to-nearest-even, saturating at +-448, of the binary32
+//          product x * inv (the sign of a product that rounds to 0 is kept);
+//   zero = +0;  reconstruction s * e4m3(code).
+// Layout as in qdq_pack_kernel (16 consecutive channels per thread, the
+// group's threads reduce the range with shuffles); the 16 one-byte codes
+// of a thread are one 16-byte store.  With WQ the kernel also writes the
+// binary16 s * e4m3(code) (the E4M3 value converts to binary16 exactly; the
+// product with s rounds once).
+template <typename WT, bool WQ>
+__global__ void __launch_bounds__(kThreads, 2) qdq_fp8_kernel(
+    const WT* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D, int group,
+    int cw, uint32_t* __restrict__ codes, __half* __restrict__ scales,
+    __half* __restrict__ zeros, __half* __restrict__ wq, uint32_t* __restrict__ status) {
+  const int tpr = cw >> 4;
+  const int rpi = kThreads / tpr;
+  const int tx = threadIdx.x % tpr;
+  const int ty = threadIdx.x / tpr;
+  const int lane = threadIdx.x & 31;
+  const int gthreads = group >> 4;
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * cw + tx * 16;
+  const int64_t ngroups = d / group;
+  const int64_t kgroup = col / group;
+  const int64_t wpr = d / 4;            // four one-byte codes per word
+  allow_dependents_launch();
+  constexpr int kRows = 4;
+  const int64_t step = static_cast<int64_t>(gridDim.y) * rpi;
+  const int64_t stride = kRows * step;
+  Raw16<WT> cur[kRows], nxt[kRows];
+  auto load_rows = [&](int64_t b, Raw16<WT>(&dst)[kRows]) {
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      const int64_t row = b + u * step + ty;
+      if (row < dp) load16(W + row * d + col, dst[u]);
+      else zero16(dst[u]);
+    }
+  };
+  if (static_cast<int64_t>(blockIdx.y) * rpi < dp) load_rows(static_cast<int64_t>(blockIdx.y) * rpi, cur);
+  grid_dependency_wait();
+
+  float2 h[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    h[i] = D != nullptr ? make_float2(__fsqrt_rn(__ldg(D + col + 2 * i)), __fsqrt_rn(__ldg(D + col + 2 * i + 1)))
+                        : make_float2(1.f, 1.f);
+  float hchk = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hchk += h[i].x + h[i].y;
+  bool bad = !(hchk <= 3.402823466e38f);
+  bool ovf = false;
+  // binary32(1 / m) for the binary16 significands m = 1 + k/1024 (see
+  // qdq_pack_kernel)
+  __shared__ float rcp_sig[1024];
+  for (int k = threadIdx.x; k < 1024; k += kThreads)
+    rcp_sig[k] = __fdiv_rn(1.0f, 1.0f + static_cast<float>(k) * 0.0009765625f);
+  __syncthreads();
+
+  auto process = [&](int64_t b, const Raw16<WT>(&buf)[kRows]) {
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+      const int64_t row = b + u * step + ty;
+      const bool active = row < dp;
+      float2 x[8];
+      unpack16(buf[u], x);
+      float mn = 0.f, mx = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        x[i] = __fmul2_rn(x[i], h[i]);
+        mn = min3_nan(mn, x[i].x, x[i].y);
+        mx = max3_nan(mx, x[i].x, x[i].y);
+      }
+      for (int o = gthreads >> 1; o > 0; o >>= 1) {
+        mn = min_nan(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max_nan(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      bad |= !(__fsub_rn(mx, mn) <= 3.402823466e38f);
+      const float amax = max_nan(mx, -mn);                 // max |x| of the group
+      float s32 = __fdiv_rn(amax, 448.0f);
+      if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
+      const __half s16 = __float2half_ru(s32);
+      const float s = __half2float(s16);
+      const uint32_t sbits = __half_as_ushort(s16);
+      const int sexp = static_cast<int>((sbits >> 10) & 31u) - 15;
+      const float inv = __int_as_float(__float_as_int(rcp_sig[sbits & 1023u]) - sexp * (1 << 23));
+      const float2 inv2 = make_float2(inv, inv);
+      // eight E4M3 pairs (channel 2i in the low byte), two per word
+      uint32_t pr[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        pr[i] = static_cast<uint32_t>(
+            __nv_cvt_float2_to_fp8x2(__fmul2_rn(x[i], inv2), __NV_SATFINITE, __NV_E4M3));
+      if (active) {
+        *reinterpret_cast<uint4*>(codes + row * wpr + (col >> 2)) =
+            make_uint4(pr[0] | (pr[1] << 16), pr[2] | (pr[3] << 16), pr[4] | (pr[5] << 16),
+                       pr[6] | (pr[7] << 16));
+      }
+      if (WQ && active) {
+        const __half2 s2 = __half2half2(s16);
+        uint32_t wh[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const __half2_raw r2 = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(pr[i]), __NV_E4M3);
+          wh[i] = half2_as_u32(__hmul2(u32_as_half2(static_cast<uint32_t>(r2.x) | (static_cast<uint32_t>(r2.y) << 16)), s2));
+        }
+        uint4* dst = reinterpret_cast<uint4*>(wq + row * d + col);
+        dst[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        dst[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+      }
+      if (active && (tx & (gthreads - 1)) == 0) {
+        scales[row * ngroups + kgroup] = s16;
+        zeros[row * ngroups + kgroup] = __ushort_as_half(0);
+        ovf |= static_cast<bool>(__hisinf(s16)) || s * 448.0f > 65504.f;
+      }
+    }
+  };
+  int64_t base = static_cast<int64_t>(blockIdx.y) * rpi;
+  for (; base < dp; base += 2 * stride) {
+    if (base + stride < dp) load_rows(base + stride, nxt);
+    process(base, cur);
+    if (base + stride >= dp) break;
+    if (base + 2 * stride < dp) load_rows(base + 2 * stride, cur);
+    process(base + stride, nxt);
+  }
+  if (__any_sync(0xffffffffu, ovf) && lane == 0)
+    set_flag(status, TTQ_FLAG_NONFINITE | TTQ_FLAG_SCALE_OVERFLOW);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_flag(status, TTQ_FLAG_NONFINITE);
+}
+
 // Largest tile width (a power of two in [32, 4096]) that divides d and is a
 // multiple of the group.
 int tile_width(int64_t d, int group) {
@@ -491,6 +624,37 @@ cudaError_t launch_qdq_pack(const void* W, bool w_f32, int64_t dp, int64_t d, co
                          scales, zeros, wq, status, num_sms, stream, pdl);
   return launch_scheme(static_cast<const __nv_bfloat16*>(W), dp, d, D, bits, group, symmetric,
                        codes, scales, zeros, wq, status, num_sms, stream, pdl);
+}
+
+cudaError_t launch_qdq_fp8(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
+                           int group, uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                           uint32_t* status, int num_sms, cudaStream_t stream, bool pdl, void* wq) {
+  if (dp == 0) return cudaSuccess;
+  const int cw = tile_width(d, group);
+  const int rpi = kThreads / (cw >> 4);
+  const int64_t gx = d / cw;
+  const int64_t want = static_cast<int64_t>(num_sms) * 2;
+  int64_t gy = (want + gx - 1) / gx;
+  const int64_t max_gy = (dp + rpi - 1) / rpi;
+  if (gy > max_gy) gy = max_gy;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  __half* s = reinterpret_cast<__half*>(scales);
+  __half* z = reinterpret_cast<__half*>(zeros);
+  __half* w = static_cast<__half*>(wq);
+  if (w_f32) {
+    const float* Wf = static_cast<const float*>(W);
+    return wq ? launch_kernel(qdq_fp8_kernel<float, true>, grid, dim3(kThreads), 0, stream, pdl, Wf, dp,
+                              d, D, group, cw, codes, s, z, w, status)
+              : launch_kernel(qdq_fp8_kernel<float, false>, grid, dim3(kThreads), 0, stream, pdl, Wf,
+                              dp, d, D, group, cw, codes, s, z, w, status);
+  }
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
+  return wq ? launch_kernel(qdq_fp8_kernel<__nv_bfloat16, true>, grid, dim3(kThreads), 0, stream, pdl,
+                            Wb, dp, d, D, group, cw, codes, s, z, w, status)
+            : launch_kernel(qdq_fp8_kernel<__nv_bfloat16, false>, grid, dim3(kThreads), 0, stream, pdl,
+                            Wb, dp, d, D, group, cw, codes, s, z, w, status);
 }
 
 cudaError_t launch_to_bf16(const float* src, void* dst, int64_t n, cudaStream_t stream) {

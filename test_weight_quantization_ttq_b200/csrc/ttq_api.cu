@@ -36,14 +36,22 @@ int device_sms() {
 }
 
 bool valid_qparams(int bits, int group) {
-  return (bits >= 2 && bits <= 4) && (group == 32 || group == 64 || group == 128 || group == 256);
+  return ((bits >= 2 && bits <= 4) || bits == 8) &&
+         (group == 32 || group == 64 || group == 128 || group == 256);
+}
+
+// Whether a code scheme takes this bit width: the INT schemes 2..4 bits,
+// FP8 (E4M3) exactly 8.
+bool scheme_bits_ok(ttq_qscheme scheme, int bits) {
+  return scheme == TTQ_QSCHEME_FP8_E4M3 ? bits == 8 : (bits >= 2 && bits <= 4);
 }
 
 // Whether ttq_linear_forward materialises the dequantised weight s (q - z)
 // in binary16 and runs the product on it (more than one 256-token tile:
 // dequantising inside the product would repeat the work once per tile)
 // instead of dequantising the codes inside the product.
-bool materialize_w(int64_t dp, int64_t T) { return dp > 0 && T > 256; }
+// 8-bit (FP8) codes are always materialised: no product reads them.
+bool materialize_w(int64_t dp, int64_t T, int bits) { return dp > 0 && (T > 256 || bits == 8); }
 
 // Computes the workspace layout; false for an unsupported shape.
 bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
@@ -89,7 +97,7 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
     l.ab = off;
     off = align_up(off + (static_cast<size_t>(r) * d + static_cast<size_t>(dp) * r) * 2);
   }
-  if (has_q && materialize_w(dp, T)) {
+  if (has_q && materialize_w(dp, T, bits)) {
     l.wq = off;
     off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d) * 2);
   }
@@ -436,12 +444,13 @@ ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, in
                                   const float* D, int bits, int group, ttq_qscheme scheme,
                                   uint32_t* codes, uint16_t* scales, uint16_t* zeros,
                                   uint16_t* W_hat, void* ws, size_t ws_bytes, void* stream) {
-  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC)
+  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC &&
+      scheme != TTQ_QSCHEME_FP8_E4M3)
     return TTQ_ERR_INVALID_ARG;
   if (W_hat && !aligned16(W_hat)) return TTQ_ERR_INVALID_ARG;
   if (dtype != TTQ_F32 && dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
   if (bits < 1 || bits > 8 || group < 1) return TTQ_ERR_INVALID_ARG;
-  if (!valid_qparams(bits, group)) return TTQ_ERR_UNSUPPORTED;
+  if (!valid_qparams(bits, group) || !scheme_bits_ok(scheme, bits)) return TTQ_ERR_UNSUPPORTED;
   if (d < group || d % group != 0 || dp < 0) return TTQ_ERR_INVALID_ARG;
   if (dp > 0 && (W == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr))
     return TTQ_ERR_INVALID_ARG;
@@ -449,6 +458,10 @@ ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, in
   if ((W && !aligned16(W)) || (D && !aligned16(D)) || (codes && !aligned16(codes)))
     return TTQ_ERR_INVALID_ARG;
   if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
+  if (scheme == TTQ_QSCHEME_FP8_E4M3)
+    return cuda_status(launch_qdq_fp8(W, dtype == TTQ_F32, dp, d, D, group, codes, scales, zeros,
+                                      static_cast<uint32_t*>(ws), device_sms(),
+                                      static_cast<cudaStream_t>(stream), false, W_hat));
   return cuda_status(launch_qdq_pack(W, dtype == TTQ_F32, dp, d, D, bits, group, codes, scales,
                                      zeros, static_cast<uint32_t*>(ws), device_sms(),
                                      static_cast<cudaStream_t>(stream), false, W_hat,
@@ -510,8 +523,8 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
                             int bits, int group, void* Y, ttq_dtype y_dtype, void* ws,
                             size_t ws_bytes, void* stream) {
   if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
-  if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
-    return TTQ_ERR_UNSUPPORTED;
+  if (bits >= 1 && bits <= 8 && group >= 1 && (!valid_qparams(bits, group) || bits == 8))
+    return TTQ_ERR_UNSUPPORTED;   // no product reads 8-bit (FP8) codes
   ttq_workspace_layout L;
   if (!make_layout(d, dp, T, r, bits, group, dtype, &L)) return TTQ_ERR_INVALID_ARG;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
@@ -564,9 +577,11 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, co
                                  ttq_qscheme scheme, void* Y, ttq_dtype y_dtype, void* ws,
                                  size_t ws_bytes, void* stream) {
   if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
-  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC)
+  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC &&
+      scheme != TTQ_QSCHEME_FP8_E4M3)
     return TTQ_ERR_INVALID_ARG;
-  if (bits >= 1 && bits <= 8 && group >= 1 && !valid_qparams(bits, group))
+  if (bits >= 1 && bits <= 8 && group >= 1 &&
+      (!valid_qparams(bits, group) || !scheme_bits_ok(scheme, bits)))
     return TTQ_ERR_UNSUPPORTED;
   if (dtype == TTQ_F16) return TTQ_ERR_INVALID_ARG;
   ttq_workspace_layout L;
@@ -601,9 +616,13 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, co
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));
   uint16_t* scales = reinterpret_cast<uint16_t*>(ws_at(ws, L.scales));
   uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
-  void* wq = materialize_w(dp, T) ? ws_at(ws, L.wq) : nullptr;
-  st = cuda_status(launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros, status,
-                                   device_sms(), s, true, wq, scheme == TTQ_QSCHEME_SYMMETRIC));
+  void* wq = materialize_w(dp, T, bits) ? ws_at(ws, L.wq) : nullptr;
+  st = cuda_status(scheme == TTQ_QSCHEME_FP8_E4M3
+                       ? launch_qdq_fp8(W, f32, dp, d, D, group, codes, scales, zeros, status,
+                                        device_sms(), s, true, wq)
+                       : launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros,
+                                         status, device_sms(), s, true, wq,
+                                         scheme == TTQ_QSCHEME_SYMMETRIC));
   if (st != TTQ_OK || T == 0) return st;
 
   // (3) Y = W_hat X (+ B (A X))

@@ -147,6 +147,13 @@ DecodeMapShape decode_map_shape(int bits, int T);
 cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
                                const CUtensorMap& tmX, cudaStream_t stream, bool pdl = false);
 
+// Step (2) with FP8 (E4M3) codes: one byte per weight (4 per word), the
+// symmetric per-group scale binary16 round-up(max|x| / 448), zeros +0;
+// with wq also the binary16 s * e4m3(code).
+cudaError_t launch_qdq_fp8(const void* W, bool w_f32, int64_t dp, int64_t d, const float* D,
+                           int group, uint32_t* codes, uint16_t* scales, uint16_t* zeros,
+                           uint32_t* status, int num_sms, cudaStream_t stream, bool pdl, void* wq);
+
 // Static low-rank initialisation (B, A from a randomised truncated SVD of
 // W; residual W - B A).  Workspace offsets (bytes) past the 4 KiB status
 // header; l = r + oversample.

@@ -28,6 +28,7 @@ TTQ_F16 = 2
 
 TTQ_QSCHEME_ASYMMETRIC = 0
 TTQ_QSCHEME_SYMMETRIC = 1
+TTQ_QSCHEME_FP8_E4M3 = 2
 
 TTQ_FLAG_NONFINITE = 0x1
 TTQ_FLAG_SCALE_OVERFLOW = 0x2

@@ -141,3 +141,28 @@ def test_lowrank_init_rejections_before_device_work(L):
     assert call(A=72) == ttq.TTQ_ERR_INVALID_ARG            # not 16-byte aligned
     assert call(ws=128) == ttq.TTQ_ERR_INVALID_ARG          # not 256-byte aligned
     assert call(nb=n - 1) == ttq.TTQ_ERR_WORKSPACE
+
+
+def test_fp8_scheme_rules_before_device_work(L):
+    qw = L.ttq_quantize_weight_ex
+    ASYM, SYM, FP8 = ttq.TTQ_QSCHEME_ASYMMETRIC, ttq.TTQ_QSCHEME_SYMMETRIC, ttq.TTQ_QSCHEME_FP8_E4M3
+    # 8-bit codes only with the FP8 scheme, and FP8 only with 8 bits
+    assert qw(16, 1, 4, 64, None, 8, 64, ASYM, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert qw(16, 1, 4, 64, None, 8, 64, SYM, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert qw(16, 1, 4, 64, None, 4, 64, FP8, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert qw(16, 1, 4, 64, None, 8, 48, FP8, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
+    assert qw(16, 1, 4, 64, None, 8, 64, 3, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    # no product reads 8-bit codes
+    st = L.ttq_dequant_gemm(16, 16, 16, None, 16, None, None, 1, 64, 64, 4, 0, 8, 64, 16, 1, 256, 1 << 30, None)
+    assert st == ttq.TTQ_ERR_UNSUPPORTED
+    # the default (asymmetric) forward refuses 8 bits; the FP8 forward checks its workspace
+    st = L.ttq_linear_forward(16, 16, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 8, 64, 16, 1, 256, 1 << 30, None)
+    assert st == ttq.TTQ_ERR_UNSUPPORTED
+    st = L.ttq_linear_forward_ex(16, 16, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 8, 64, FP8, 16, 1, 256, 64,
+                                 None)
+    assert st == ttq.TTQ_ERR_WORKSPACE
+    # FP8 layouts always hold the binary16 W_hat; INT layouts only for T > 256
+    for T, bits, present in [(4, 8, True), (1, 8, True), (4, 4, False), (300, 4, True)]:
+        lay = ttq.WorkspaceLayout()
+        assert L.ttq_workspace_get_layout(256, 64, T, 0, bits, 64, 1, lay) == ttq.TTQ_OK
+        assert (lay.wq != 0) == present, (T, bits)
