@@ -42,7 +42,6 @@
 // Every barrier wait is bounded (1 s); a wait that gives up sets
 // TTQ_FLAG_TIMEOUT, stops the CTA's other warps, lets the copies in flight
 // land, and the CTA returns without storing Y.
-#include <mutex>
 
 #include "ttq_device.cuh"
 #include "ttq_kernels.h"
@@ -518,15 +517,19 @@ template <int BITS, int NTT, bool PS>
 cudaError_t launch_decode_typed(const CUtensorMap& tmC, const CUtensorMap& tmX,
                                 const DecodeArgs& a, int group_shift, cudaStream_t stream,
                                 bool pdl) {
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
   constexpr size_t smem = decode_smem_bytes<BITS, NTT>();
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(ttq_decode_kernel<BITS, NTT, PS>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(smem));
-  });
-  if (attr_err != cudaSuccess) return attr_err;
+  // the attribute belongs to a device: set once per device (the first
+  // launch on it, normally outside any graph capture)
+  static bool attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    const cudaError_t attr_err = cudaFuncSetAttribute(ttq_decode_kernel<BITS, NTT, PS>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(smem));
+    if (attr_err != cudaSuccess) return attr_err;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   const dim3 grid(static_cast<unsigned>((a.M + kRowsPerCta - 1) / kRowsPerCta));
   return launch_kernel(ttq_decode_kernel<BITS, NTT, PS>, grid, dim3(32 * (1 + kConsumers)), smem,
                        stream, pdl, tmC, tmX, a.scales, a.zeros, static_cast<int>(a.K),
