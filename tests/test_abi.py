@@ -166,3 +166,20 @@ def test_fp8_scheme_rules_before_device_work(L):
         lay = ttq.WorkspaceLayout()
         assert L.ttq_workspace_get_layout(256, 64, T, 0, bits, 64, 1, lay) == ttq.TTQ_OK
         assert (lay.wq != 0) == present, (T, bits)
+
+
+def declared_arity():
+    """Parameter count of every ttq_* function declared in the header."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(ttq_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header():
+    arity = declared_arity()
+    assert set(arity) == set(ttq.SIGNATURES)
+    for name, (_, argtypes) in ttq.SIGNATURES.items():
+        assert len(argtypes) == arity[name], (name, len(argtypes), arity[name])
