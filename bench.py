@@ -200,12 +200,26 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-def _config():
+SCHEMES = {"asym": None, "sym": "symmetric INT", "fp8": "FP8 E4M3"}
+
+
+def _config(scheme: str = "asym"):
     w = WORKLOAD
-    return {"workload": f"{w['name']}: TTQ linear, d=d'={w['d']}, T={w['T']}, INT{w['bits']} g{w['group']}, "
-                        f"p={w['p']}, lambda={w['lam']}, alpha={w['alpha']}, bf16 X/W/Y",
-            "d": w["d"], "d_out": w["dp"], "tokens": w["T"], "bits": w["bits"], "group": w["group"],
-            "l2": "inputs rotate over sets whose size exceeds L2 (no warm-L2 reads of X or W)"}
+    code = f"INT{w['bits']}" if scheme == "asym" else (f"symmetric INT{w['bits']}" if scheme == "sym" else "FP8 E4M3")
+    cfg = {"workload": f"{w['name']}: TTQ linear, d=d'={w['d']}, T={w['T']}, {code} g{w['group']}, "
+                       f"p={w['p']}, lambda={w['lam']}, alpha={w['alpha']}, bf16 X/W/Y",
+           "d": w["d"], "d_out": w["dp"], "tokens": w["T"], "bits": w["bits"] if scheme != "fp8" else 8,
+           "group": w["group"],
+           "l2": "inputs rotate over sets whose size exceeds L2 (no warm-L2 reads of X or W)"}
+    if scheme != "asym":
+        cfg["scheme"] = SCHEMES[scheme]
+    return cfg
+
+
+def _metric(scheme: str = "asym") -> str:
+    if scheme == "asym":
+        return METRIC
+    return METRIC.replace("(INT4", "(symmetric INT4" if scheme == "sym" else "(FP8 E4M3")
 
 
 # ------------------------------------------------------- multi-rank helpers
@@ -251,6 +265,9 @@ def run_ours(args):
     w = WORKLOAD
     spec = synth.C2
     d, dp, T, bits, group = w["d"], w["dp"], w["T"], w["bits"], w["group"]
+    scheme = {"asym": None, "sym": ttq.TTQ_QSCHEME_SYMMETRIC, "fp8": ttq.TTQ_QSCHEME_FP8_E4M3}[args.scheme]
+    if args.scheme == "fp8":
+        bits = 8
     data = synth.generate(spec.with_(seed=rank))
     set_bytes = 2 * (d * dp + T * d + T * dp)
     nsets = max(2, -(-2 * L2_BYTES // set_bytes))
@@ -268,7 +285,7 @@ def run_ours(args):
     def step(i):
         k = i % nsets
         ttq.ttq_linear_forward(Xs[k], Ws[k], None, None, w["p"], w["lam"], w["alpha"], bits, group,
-                               ws=ws, Y=Ys[k])
+                               ws=ws, Y=Ys[k], scheme=scheme)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -320,8 +337,12 @@ def run_ours(args):
         ev[i][0].record(stream)
         ttq.ttq_act_norm_scale(Xs[k], w["p"], w["lam"], w["alpha"], ws=ws, Xs=Xsbuf, copy_out=False)
         ev[i][1].record(stream)
-        ttq.ttq_quantize_dequant_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc,
-                                        zeros=ze, W_hat=W_hat)
+        if scheme is None:
+            ttq.ttq_quantize_dequant_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc,
+                                            zeros=ze, W_hat=W_hat)
+        else:
+            ttq.ttq_quantize_weight_ex(Ws[k], Dbuf, bits, group, scheme, ws=ws, codes=codes, scales=sc,
+                                       zeros=ze, W_hat=W_hat)
         ev[i][2].record(stream)
         ttq.ttq_dequantized_gemm(W_hat, Xsbuf, ws=ws, Y=Ys[k])
         ev[i][3].record(stream)
@@ -356,7 +377,7 @@ def run_ours(args):
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "profile_run": True,
+            print(json.dumps({"metric": _metric(args.scheme), "value": value, "unit": "tokens/s", "profile_run": True,
                               "roofline": roofline, "kernels": kernels}), flush=True)
         return
 
@@ -398,9 +419,9 @@ def run_ours(args):
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": _metric(args.scheme), "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(),
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": _config(args.scheme),
         "roofline": roofline, "kernels": kernels, "rho": rho, "cpu_baseline": cpu, "e2e": e2e,
         "clocks": clocks, "gpu_launches": n_kernels * args.steps,
     }
@@ -583,6 +604,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", action="store_true",
                     help="short run for a profiler: no clock warm-up loop, no CPU baseline, no e2e leg")
+    ap.add_argument("--scheme", choices=sorted(SCHEMES), default="asym",
+                    help="code scheme of the q_proj prefill workload (asym: the default INT4; fp8 uses 8-bit E4M3 codes)")
     ap.add_argument("--decode", type=int, default=0, metavar="T",
                     help="time the decode workload (d = 4096, d' = 14336, INT4 g128) at T <= 16 tokens instead")
     ap.add_argument("--lowrank", action="store_true",
