@@ -335,9 +335,17 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
 
 /* Reads the workspace status word (a blocking device-to-host copy; the caller
  * synchronises its stream first).  *flags receives the raw TTQ_FLAG_* bits
- * (may be NULL).  Returns TTQ_OK if no flag is set, TTQ_ERR_TIMEOUT if the
- * timeout flag is set, else TTQ_ERR_NONFINITE. */
+ * (may be NULL).  Returns ttq_status_from_flags of those bits. */
 ttq_status ttq_get_status(const void* ws, uint32_t* flags);
+
+/* The status that a set of TTQ_FLAG_* bits stands for (host only, no device
+ * work): TTQ_ERR_TIMEOUT if the timeout flag is set; else TTQ_ERR_NONFINITE
+ * if any other bit except TTQ_FLAG_RANK_DEFICIENT is set (a non-finite
+ * value, a binary16 scale overflow, an activation beyond binary16, or a bit
+ * this version does not define); else TTQ_OK.  TTQ_FLAG_RANK_DEFICIENT is a
+ * warning: a weight of rank below r + oversample is a valid input to
+ * ttq_lowrank_init, whose outputs stay finite. */
+ttq_status ttq_status_from_flags(uint32_t flags);
 
 /* ---------------------------------------------------------------------
  * Static low-rank initialisation (the step before the path).

@@ -679,8 +679,12 @@ ttq_status ttq_get_status(const void* ws, uint32_t* flags) {
   uint32_t f = 0;
   if (cudaMemcpy(&f, ws, sizeof(f), cudaMemcpyDeviceToHost) != cudaSuccess) return TTQ_ERR_CUDA;
   if (flags) *flags = f;
-  if (f & TTQ_FLAG_TIMEOUT) return TTQ_ERR_TIMEOUT;
-  if (f) return TTQ_ERR_NONFINITE;
+  return ttq_status_from_flags(f);
+}
+
+ttq_status ttq_status_from_flags(uint32_t flags) {
+  if (flags & TTQ_FLAG_TIMEOUT) return TTQ_ERR_TIMEOUT;
+  if (flags & ~TTQ_FLAG_RANK_DEFICIENT) return TTQ_ERR_NONFINITE;
   return TTQ_OK;
 }
 

@@ -73,6 +73,7 @@ SIGNATURES = {
                                   _P, _INT, _P, _SZ, _P]),
     "ttq_linear_forward_kernels": (_INT, [_INT, _I64, _I64, _I64, _I64, _F, ctypes.POINTER(ctypes.c_int)]),
     "ttq_get_status": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "ttq_status_from_flags": (_INT, [ctypes.c_uint32]),
     "ttq_lowrank_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
     "ttq_lowrank_init": (_INT, [_P, _INT, _I64, _I64, _I64, _I64, _INT, _P, _P, _P, _P, _P, _SZ, _P]),
     "ttq_status_string": (ctypes.c_char_p, [_INT]),
@@ -169,6 +170,11 @@ def ttq_get_status(ws: torch.Tensor) -> tuple[int, int]:
     flags = ctypes.c_uint32(0)
     st = lib().ttq_get_status(_dev(ws, "ws"), ctypes.byref(flags))
     return int(st), int(flags.value)
+
+
+def ttq_status_from_flags(flags: int) -> int:
+    """The status a set of TTQ_FLAG_* bits stands for (host only)."""
+    return int(lib().ttq_status_from_flags(int(flags) & 0xFFFFFFFF))
 
 
 # ---------------------------------------------------------- entry points

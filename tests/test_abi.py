@@ -40,6 +40,18 @@ def test_version_and_status_strings(L):
     assert ttq.status_string(99) == "unknown status"
 
 
+def test_status_from_flags(L):
+    f = ttq.ttq_status_from_flags
+    assert f(0) == ttq.TTQ_OK
+    # a weight of low rank is a warning, not an error
+    assert f(ttq.TTQ_FLAG_RANK_DEFICIENT) == ttq.TTQ_OK
+    for bit in (ttq.TTQ_FLAG_NONFINITE, ttq.TTQ_FLAG_SCALE_OVERFLOW, ttq.TTQ_FLAG_X_RANGE, 0x80000000):
+        assert f(bit) == ttq.TTQ_ERR_NONFINITE, bit
+        assert f(bit | ttq.TTQ_FLAG_RANK_DEFICIENT) == ttq.TTQ_ERR_NONFINITE, bit
+    # a timed-out wait outranks every other condition
+    assert f(ttq.TTQ_FLAG_TIMEOUT | ttq.TTQ_FLAG_NONFINITE | ttq.TTQ_FLAG_RANK_DEFICIENT) == ttq.TTQ_ERR_TIMEOUT
+
+
 def test_workspace_layout_is_consistent(L):
     for (d, dp, T, r, bits, g, dt) in [(4096, 4096, 2048, 0, 4, 128, ttq.TTQ_BF16),
                                        (8192, 28672, 4096, 64, 2, 64, ttq.TTQ_BF16),

@@ -112,6 +112,7 @@ def test_lowrank_zero_weight_is_flagged_and_finite():
     W = np.zeros((128, 96), dtype=np.float32)
     Wd, B, A, R, st, flags, _, _ = _run(W, 8, 8, 1, torch.float32)
     assert flags & ttq.TTQ_FLAG_RANK_DEFICIENT
+    assert st == ttq.TTQ_OK, flags          # rank deficiency is a warning
     assert not flags & ttq.TTQ_FLAG_NONFINITE
     assert torch.count_nonzero(B) == 0 and torch.count_nonzero(A) == 0 and torch.count_nonzero(R) == 0
 
