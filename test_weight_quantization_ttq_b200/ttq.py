@@ -131,7 +131,66 @@ def _dev(t: torch.Tensor | None, name: str) -> int | None:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    cur = torch.cuda.current_device()
+    if t.device.index is not None and t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device}; the library runs on the current device cuda:{cur}")
     return t.data_ptr()
+
+
+# The C ABI takes bare pointers and sizes, so the sizes it is given must
+# describe the tensors behind the pointers: the checks below run before any
+# device work and raise instead of letting a kernel read or write past a
+# buffer.
+_F32 = (torch.float32,)
+_F16 = (torch.float16,)
+_FLOAT_IN = (torch.float32, torch.bfloat16)
+
+
+def _matrix(t: torch.Tensor | None, name: str, rows=None, cols=None, dtypes=None) -> None:
+    """t (when given) is 2-D, rows x cols where those are given, of one of `dtypes`."""
+    if t is None:
+        return
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    if (rows is not None and t.shape[0] != rows) or (cols is not None and t.shape[1] != cols):
+        want = (rows if rows is not None else "*", cols if cols is not None else "*")
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {want}")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {list(dtypes)}")
+
+
+def _vector(t: torch.Tensor | None, name: str, n: int) -> None:
+    """t (when given) holds exactly n float32 values (D, D^{-1/2})."""
+    if t is None:
+        return
+    if t.dtype != torch.float32 or t.numel() != n:
+        raise ValueError(f"{name} must hold {n} float32 values, got {t.numel()} {t.dtype}")
+
+
+def _room(t: torch.Tensor | None, name: str, nbytes: int) -> None:
+    """t (when given) spans at least nbytes (packed codes, binary16 scales)."""
+    if t is None:
+        return
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name} spans {t.numel() * t.element_size()} bytes, needs {nbytes}")
+
+
+def _qsizes(d: int, bits: int, group: int, where: str) -> tuple[int, int]:
+    """(code bytes, scale bytes) of one row of W."""
+    if bits < 1 or group < 1:
+        raise TTQError(TTQ_ERR_INVALID_ARG, where)
+    return d * bits // 32 * 4, d // group * 2
+
+
+def _lowrank_pair(A: torch.Tensor | None, B: torch.Tensor | None) -> int:
+    """r of the low-rank term: A [r][d] and B [d'][r] are given together."""
+    if (A is None) != (B is None):
+        raise ValueError("A and B of the low-rank term are given together or not at all")
+    return 0 if A is None else A.shape[0]
+
+
+def _nbytes(ws: torch.Tensor) -> int:
+    return ws.numel() * ws.element_size()
 
 
 def _stream(stream) -> int | None:
@@ -152,7 +211,7 @@ def ttq_workspace_get_layout(d, dp, T, r, bits, group, dtype=TTQ_BF16) -> Worksp
 
 
 def ttq_workspace_init(ws: torch.Tensor, stream=None) -> None:
-    _check(lib().ttq_workspace_init(_dev(ws, "ws"), ws.numel(), _stream(stream)), "ttq_workspace_init")
+    _check(lib().ttq_workspace_init(_dev(ws, "ws"), _nbytes(ws), _stream(stream)), "ttq_workspace_init")
 
 
 def new_workspace(d, dp, T, r, bits, group, dtype=TTQ_BF16, device="cuda", stream=None) -> torch.Tensor:
@@ -178,16 +237,28 @@ def ttq_status_from_flags(flags: int) -> int:
 
 
 # ---------------------------------------------------------- entry points
+def _quant_outputs(dp, d, D, bits, group, codes, scales, zeros, W_hat, where) -> None:
+    cb, sb = _qsizes(d, bits, group, where)
+    _vector(D, "D", d)
+    _room(codes, "codes", dp * cb)
+    _room(scales, "scales", dp * sb)
+    _room(zeros, "zeros", dp * sb)
+    _matrix(W_hat, "W_hat", dp, d, _F16)
+
+
 def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None, copy_out=True):
     """D[i] = (||X[:, i]||_p + lambda)^alpha and D^{-1/2}; X is [T][d].
     With copy_out=False nothing is copied out: D and D^{-1/2} are returned
     as views of the workspace, where the entry point writes them."""
+    _matrix(X, "X", dtypes=_FLOAT_IN)
     T, d = X.shape
+    _vector(D, "D", d)
+    _vector(D_rsqrt, "D_rsqrt", d)
     if ws is None:
         ws = new_workspace(d, 0, T, 0, 4, 32, _dtype_code(X), X.device, stream)
     if not copy_out:
         _check(lib().ttq_act_norm(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, None, None,
-                                  _dev(ws, "ws"), ws.numel(), _stream(stream)), "ttq_act_norm")
+                                  _dev(ws, "ws"), _nbytes(ws), _stream(stream)), "ttq_act_norm")
         L = ttq_workspace_get_layout(d, 0, T, 0, 4, 32, _dtype_code(X))
         return (ws[L.D: L.D + 4 * d].view(torch.float32), ws[L.D_rsqrt: L.D_rsqrt + 4 * d].view(torch.float32))
     if D is None:
@@ -195,7 +266,7 @@ def ttq_act_norm(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, stream=None, c
     if D_rsqrt is None:
         D_rsqrt = torch.empty(d, dtype=torch.float32, device=X.device)
     _check(lib().ttq_act_norm(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, _dev(D, "D"),
-                              _dev(D_rsqrt, "D_rsqrt"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+                              _dev(D_rsqrt, "D_rsqrt"), _dev(ws, "ws"), _nbytes(ws), _stream(stream)),
            "ttq_act_norm")
     return D, D_rsqrt
 
@@ -205,7 +276,11 @@ def ttq_act_norm_scale(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, Xs=None,
     """D, D^{-1/2} and Xs [T][d] binary16 = X * D^{-1/2} in one pass over X.
     With copy_out=False, D and D^{-1/2} are not given to the entry point and
     are returned as views of the workspace, where it writes them."""
+    _matrix(X, "X", dtypes=_FLOAT_IN)
     T, d = X.shape
+    _vector(D, "D", d)
+    _vector(D_rsqrt, "D_rsqrt", d)
+    _matrix(Xs, "Xs", T, d, _F16)
     if ws is None:
         ws = new_workspace(d, 0, T, 0, 4, 32, _dtype_code(X), X.device, stream)
     if Xs is None:
@@ -219,7 +294,7 @@ def ttq_act_norm_scale(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, Xs=None,
     else:
         dptr = drptr = None
     _check(lib().ttq_act_norm_scale(_dev(X, "X"), _dtype_code(X), d, T, p, lam, alpha, dptr, drptr,
-                                    _dev(Xs, "Xs"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+                                    _dev(Xs, "Xs"), _dev(ws, "ws"), _nbytes(ws), _stream(stream)),
            "ttq_act_norm_scale")
     if not copy_out:
         L = ttq_workspace_get_layout(d, 0, T, 0, 4, 32, _dtype_code(X))
@@ -240,7 +315,10 @@ def ttq_linear_forward_kernels(d, dp, T, r=0, p=2.0, dtype=TTQ_BF16) -> int:
 def ttq_act_norm_noalloc(X, p, lam, alpha, D=None, D_rsqrt=None, stream=None):
     """ttq_act_norm without a workspace: the library's own fixed scratch array
     is used (d <= 16384; calls overlapping on the GPU race)."""
+    _matrix(X, "X", dtypes=_FLOAT_IN)
     T, d = X.shape
+    _vector(D, "D", d)
+    _vector(D_rsqrt, "D_rsqrt", d)
     if D is None:
         D = torch.empty(d, dtype=torch.float32, device=X.device)
     if D_rsqrt is None:
@@ -253,7 +331,9 @@ def ttq_act_norm_noalloc(X, p, lam, alpha, D=None, D_rsqrt=None, stream=None):
 
 def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zeros=None, stream=None):
     """codes [d'][d*bits/32] uint32, scales/zeros [d'][d/group] binary16 bits (int16 storage)."""
+    _matrix(W, "W", dtypes=_FLOAT_IN)
     dp, d = W.shape
+    _quant_outputs(dp, d, D, bits, group, codes, scales, zeros, None, "ttq_quantize_weight")
     dev = W.device
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
@@ -265,7 +345,7 @@ def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zer
         zeros = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
     _check(lib().ttq_quantize_weight(_dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group,
                                      _dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
-                                     _dev(ws, "ws"), ws.numel(), _stream(stream)),
+                                     _dev(ws, "ws"), _nbytes(ws), _stream(stream)),
            "ttq_quantize_weight")
     return codes, scales, zeros
 
@@ -274,7 +354,9 @@ def ttq_quantize_weight_ex(W, D, bits, group, scheme, ws=None, codes=None, scale
                            W_hat=None, stream=None):
     """Codes, scales and zeros under the given TTQ_QSCHEME_*; W_hat (binary16
     s (q - z), optional) is written when given."""
+    _matrix(W, "W", dtypes=_FLOAT_IN)
     dp, d = W.shape
+    _quant_outputs(dp, d, D, bits, group, codes, scales, zeros, W_hat, "ttq_quantize_weight_ex")
     dev = W.device
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
@@ -286,7 +368,7 @@ def ttq_quantize_weight_ex(W, D, bits, group, scheme, ws=None, codes=None, scale
         zeros = torch.empty((dp, d // group), dtype=torch.int16, device=dev)
     _check(lib().ttq_quantize_weight_ex(
         _dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group, scheme, _dev(codes, "codes"),
-        _dev(scales, "scales"), _dev(zeros, "zeros"), _dev(W_hat, "W_hat"), _dev(ws, "ws"), ws.numel(),
+        _dev(scales, "scales"), _dev(zeros, "zeros"), _dev(W_hat, "W_hat"), _dev(ws, "ws"), _nbytes(ws),
         _stream(stream)), "ttq_quantize_weight_ex")
     return codes, scales, zeros
 
@@ -294,7 +376,9 @@ def ttq_quantize_weight_ex(W, D, bits, group, scheme, ws=None, codes=None, scale
 def ttq_quantize_dequant_weight(W, D, bits, group, ws=None, codes=None, scales=None, zeros=None,
                                 W_hat=None, stream=None):
     """ttq_quantize_weight plus W_hat [d'][d] binary16 (torch.float16) = s (q - z)."""
+    _matrix(W, "W", dtypes=_FLOAT_IN)
     dp, d = W.shape
+    _quant_outputs(dp, d, D, bits, group, codes, scales, zeros, W_hat, "ttq_quantize_dequant_weight")
     dev = W.device
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
@@ -309,33 +393,39 @@ def ttq_quantize_dequant_weight(W, D, bits, group, ws=None, codes=None, scales=N
     _check(lib().ttq_quantize_dequant_weight(
         _dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group, _dev(codes, "codes"),
         _dev(scales, "scales"), _dev(zeros, "zeros"), _dev(W_hat, "W_hat"), _dev(ws, "ws"),
-        ws.numel(), _stream(stream)), "ttq_quantize_dequant_weight")
+        _nbytes(ws), _stream(stream)), "ttq_quantize_dequant_weight")
     return codes, scales, zeros, W_hat
 
 
 def ttq_dequantized_gemm(W_hat, Xs, ws=None, Y=None, y_dtype=torch.bfloat16, stream=None):
     """Y [T][d'] = W_hat Xs^T from a binary16 dequantised weight and binary16 X D^{-1/2}."""
+    _matrix(W_hat, "W_hat", dtypes=_F16)
     dp, d = W_hat.shape
+    _matrix(Xs, "Xs", cols=d, dtypes=_F16)
     T = Xs.shape[0]
+    _matrix(Y, "Y", T, dp, _FLOAT_IN)
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, 4, 32, TTQ_BF16, W_hat.device, stream)
     if Y is None:
         Y = torch.empty((T, dp), dtype=y_dtype, device=W_hat.device)
     _check(lib().ttq_dequantized_gemm(_dev(W_hat, "W_hat"), _dev(Xs, "Xs"), d, dp, T, _dev(Y, "Y"),
-                                      _dtype_code(Y), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+                                      _dtype_code(Y), _dev(ws, "ws"), _nbytes(ws), _stream(stream)),
            "ttq_dequantized_gemm")
     return Y
 
 
 def ttq_scale_activations(X, D_rsqrt, ws=None, Xs=None, stream=None):
     """Xs [T][d] binary16 (torch.float16) = X * D^{-1/2}, the product's B operand."""
+    _matrix(X, "X", dtypes=_FLOAT_IN + _F16)
     T, d = X.shape
+    _vector(D_rsqrt, "D_rsqrt", d)
+    _matrix(Xs, "Xs", T, d, _F16)
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, 4, 32, TTQ_BF16, X.device, stream)
     if Xs is None:
         Xs = torch.empty((T, d), dtype=torch.float16, device=X.device)
     _check(lib().ttq_scale_activations(_dev(X, "X"), _dtype_code(X), d, T, _dev(D_rsqrt, "D_rsqrt"),
-                                       _dev(Xs, "Xs"), _dev(ws, "ws"), ws.numel(), _stream(stream)),
+                                       _dev(Xs, "Xs"), _dev(ws, "ws"), _nbytes(ws), _stream(stream)),
            "ttq_scale_activations")
     return Xs
 
@@ -344,9 +434,18 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
                      y_dtype=None, stream=None):
     """Y [T][d'] = W_hat X (+ B (A X)) from quantised weights; Y in y_dtype
     (default: the dtype of X, or of a given Y)."""
+    _matrix(X, "X", dtypes=_FLOAT_IN + _F16)
     T, d = X.shape
     dp = codes.shape[0]
-    r = 0 if A is None else A.shape[0]
+    r = _lowrank_pair(A, B)
+    cb, sb = _qsizes(d, bits, group, "ttq_dequant_gemm")
+    _room(codes, "codes", dp * cb)
+    _room(scales, "scales", dp * sb)
+    _room(zeros, "zeros", dp * sb)
+    _vector(D_rsqrt, "D_rsqrt", d)
+    _matrix(A, "A", r, d, (X.dtype,))
+    _matrix(B, "B", dp, r, (X.dtype,))
+    _matrix(Y, "Y", T, dp, _FLOAT_IN)
     dt = _dtype_code(X)
     if ws is None:
         ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
@@ -356,7 +455,7 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
     _check(lib().ttq_dequant_gemm(_dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
                                   _dev(D_rsqrt, "D_rsqrt"), _dev(X, "X"), _dev(A, "A"), _dev(B, "B"), dt,
                                   d, dp, T, r, bits, group, _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"),
-                                  ws.numel(), _stream(stream)),
+                                  _nbytes(ws), _stream(stream)),
            "ttq_dequant_gemm")
     return Y
 
@@ -366,9 +465,14 @@ def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, 
     """The TTQ linear layer: Y [T][d'] = Q[W D^{1/2}] D^{-1/2} X + B (A X);
     Y in y_dtype (default: the dtype of X, or of a given Y).  scheme: None
     (ttq_linear_forward) or a TTQ_QSCHEME_* code (ttq_linear_forward_ex)."""
+    _matrix(X, "X", dtypes=_FLOAT_IN)
     T, d = X.shape
+    _matrix(W, "W", cols=d, dtypes=(X.dtype,))
     dp = W.shape[0]
-    r = 0 if A is None else A.shape[0]
+    r = _lowrank_pair(A, B)
+    _matrix(A, "A", r, d, (X.dtype,))
+    _matrix(B, "B", dp, r, (X.dtype,))
+    _matrix(Y, "Y", T, dp, _FLOAT_IN)
     dt = _dtype_code(X)
     if ws is None:
         ws = new_workspace(d, dp, T, r, bits, group, dt, X.device, stream)
@@ -376,7 +480,7 @@ def ttq_linear_forward(X, W, A, B, p, lam, alpha, bits, group, ws=None, Y=None, 
         Y = torch.empty((T, dp), dtype=y_dtype or X.dtype, device=X.device)
     args = (_dev(X, "X"), _dev(W, "W"), _dev(A, "A"), _dev(B, "B"), dt, d, dp, T, r, p, lam, alpha, bits,
             group)
-    tail = (_dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"), ws.numel(), _stream(stream))
+    tail = (_dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"), _nbytes(ws), _stream(stream))
     if scheme is None:
         _check(lib().ttq_linear_forward(*args, *tail), "ttq_linear_forward")
     else:
@@ -394,7 +498,12 @@ def ttq_lowrank_init(W, r, Omega, power_iters=2, ws=None, B=None, A=None, W_res=
     A [r][d] from a randomised truncated SVD with the Gaussian test matrix
     Omega [d][r + oversample] (float32), and W_res = W - B A (when
     `residual`).  Returns (B, A, W_res or None)."""
+    _matrix(W, "W", dtypes=_FLOAT_IN)
     dp, d = W.shape
+    _matrix(Omega, "Omega", d, None, _F32)
+    _matrix(B, "B", dp, r, (W.dtype,))
+    _matrix(A, "A", r, d, (W.dtype,))
+    _matrix(W_res, "W_res", dp, d, (W.dtype,))
     l = Omega.shape[1]
     oversample = l - r
     dt = _dtype_code(W)
@@ -412,7 +521,7 @@ def ttq_lowrank_init(W, r, Omega, power_iters=2, ws=None, B=None, A=None, W_res=
         W_res = torch.empty_like(W)
     _check(lib().ttq_lowrank_init(_dev(W, "W"), dt, dp, d, r, oversample, power_iters, _dev(Omega, "Omega"),
                                   _dev(B, "B"), _dev(A, "A"), _dev(W_res, "W_res"), _dev(ws, "ws"),
-                                  ws.numel(), _stream(stream)),
+                                  _nbytes(ws), _stream(stream)),
            "ttq_lowrank_init")
     return B, A, W_res
 
