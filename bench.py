@@ -366,7 +366,7 @@ def run_ours(args):
     kernels = [
         {"kernel": "act_norm_scale_kernel", "ms": t_stat * 1e3, "bound": "hbm", "bytes": stat_bytes,
          "achieved_gbs": stat_bytes / t_stat / 1e9, "frac": stat_bytes / t_stat / 1e9 / peaks["hbm_gbs"]},
-        {"kernel": "qdq_pack_kernel", "ms": t_qdq * 1e3, "bound": "hbm", "bytes": qdq_bytes,
+        {"kernel": "qdq_fp8_kernel" if args.scheme == "fp8" else "qdq_pack_kernel", "ms": t_qdq * 1e3, "bound": "hbm", "bytes": qdq_bytes,
          "achieved_gbs": qdq_bytes / t_qdq / 1e9, "frac": qdq_bytes / t_qdq / 1e9 / peaks["hbm_gbs"]},
         {"kernel": "ttq_gemm_kernel", "ms": t_gemm * 1e3, "bound": "tensor", "flops": flops,
          "achieved_tflops": gemm_tflops, "frac": gemm_tflops / peaks["bf16_tflops"]},
@@ -389,7 +389,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     for _ in range(2):
         Xd.copy_(Xh, non_blocking=True)
-        ttq.ttq_linear_forward(Xd, Ws[0], None, None, w["p"], w["lam"], w["alpha"], bits, group, ws=ws, Y=Ys[0])
+        ttq.ttq_linear_forward(Xd, Ws[0], None, None, w["p"], w["lam"], w["alpha"], bits, group, ws=ws, Y=Ys[0],
+                               scheme=scheme)
         Yh.copy_(Ys[0], non_blocking=True)
     torch.cuda.synchronize()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -397,7 +398,7 @@ def run_ours(args):
     for i in range(args.steps):
         Xd.copy_(Xh, non_blocking=True)
         ttq.ttq_linear_forward(Xd, Ws[i % nsets], None, None, w["p"], w["lam"], w["alpha"], bits, group,
-                               ws=ws, Y=Ys[0])
+                               ws=ws, Y=Ys[0], scheme=scheme)
         Yh.copy_(Ys[0], non_blocking=True)
     f1.record(stream)
     torch.cuda.synchronize()
