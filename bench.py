@@ -540,6 +540,108 @@ def run_decode(args):
                       "kernels": kernels, "hbm_peak_gbs": hbm, "clocks": clocks}), flush=True)
 
 
+def _floor_us(spec, hbm, tc):
+    """Lower bound on one forward (microseconds) from the method's
+    algorithmic bytes and flops at the measured peaks: the statistic and
+    quantiser at HBM bandwidth, the product at the slower of its bytes and
+    its flops.  The bytes are what the method must move (X in, the scaled X,
+    W in, codes and scales out and back in, Y out); the binary16 W_hat this
+    implementation adds for long inputs is not part of the floor."""
+    d, dp, T, b, g, r = spec.d, spec.dp, spec.T, spec.bits, spec.group, spec.r
+    e = 4 if spec.dtype == "f32" else 2
+    stat = e * d * T + 2 * d * T + 8 * d                       # X in, X D^-1/2 out, D and D^-1/2
+    codes = dp * d * b / 8 + 4 * dp * d / g
+    qdq = e * dp * d + codes + 4 * d
+    prod = codes + 2 * d * T + e * T * dp + (2 * r * (d + dp) + 2 * r * T if r else 0)
+    flops = 2.0 * dp * d * T + 2.0 * r * (d + dp) * T
+    return 1e6 * ((stat + qdq) / hbm + max(prod / hbm, flops / tc)), stat + qdq + prod, flops
+
+
+def run_table(args):
+    """Forward time of ttq_linear_forward at every configured workload point
+    (the fp32 d = 256 case, the q_proj prefill, the three MLP projections at
+    T = 512 and their block, decode at T = 1, 4, 16, and the 70B-like MLP
+    shape at T = 1 .. 4096 with p = 2, alpha = 0.5), each next to the floor
+    its algorithmic bytes and flops give at the measured peaks.  K calls are
+    captured in a CUDA graph and its replay is timed with CUDA events; W
+    rotates over enough copies to exceed L2.  One GPU; one JSON line per
+    point and a closing line with the clocks."""
+    import numpy as np
+    import torch
+
+    from test_weight_quantization_ttq_b200 import synth, ttq
+
+    peaks = _measured_peaks()
+    hbm, tc = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
+    stream = torch.cuda.current_stream()
+    points = [synth.C1, synth.C2, synth.C3_GATE, synth.C3_UP, synth.C3_DOWN]
+    points += [synth.C4.with_(T=t) for t in synth.C4_TOKENS]
+    points += [synth.C5.with_(T=t, p=2.0, alpha=0.5) for t in synth.C5_TOKENS]
+    sampler = ClockSampler(0)
+    sampler.start()
+    cached = (None, None)      # (spec name and seed, W copies): one weight on the device at a time
+    block_us = 0.0
+    for spec in points:
+        key = (spec.name, spec.seed)
+        f32 = spec.dtype == "f32"
+        tdt = torch.float32 if f32 else torch.bfloat16
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).cuda()
+        data = synth.generate(spec, need_w=cached[0] != key)
+        if cached[0] != key:
+            cached = (None, None)
+            torch.cuda.empty_cache()
+            W0 = dev(data["W"])
+            n = max(1, min(8, -(-2 * L2_BYTES // (W0.numel() * W0.element_size()))))
+            cached = (key, [W0] + [W0.clone() for _ in range(n - 1)])
+        Ws = cached[1]
+        X = dev(data["X"])
+        A = dev(data["A"]) if spec.r else None
+        B = dev(data["B"]) if spec.r else None
+        Y = torch.empty((spec.T, spec.dp), dtype=tdt, device="cuda")
+        ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group,
+                               ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)
+        floor_us, nbytes, flops = _floor_us(spec, hbm, tc)
+        k = args.steps if floor_us < 200 else max(5, args.steps // 10)
+
+        def fwd(i):
+            ttq.ttq_linear_forward(X, Ws[i % len(Ws)], A, B, spec.p, spec.lam, spec.alpha, spec.bits,
+                                   spec.group, ws=ws, Y=Y)
+
+        for i in range(args.warmup):
+            fwd(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(k):
+                fwd(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / k
+        st, flags = ttq.ttq_get_status(ws)
+        if st != ttq.TTQ_OK:
+            raise RuntimeError(f"{spec.name} T={spec.T}: device status {ttq.status_string(st)} (flags {flags:#x})")
+        if spec.name.startswith("mlp_") and spec.T == 512:
+            block_us += us
+        print(json.dumps({"table": "forward", "workload": f"{spec.name}_T{spec.T}", "d": spec.d, "dp": spec.dp,
+                          "T": spec.T, "bits": spec.bits, "group": spec.group, "r": spec.r, "p": spec.p,
+                          "alpha": spec.alpha, "dtype": spec.dtype, "us": us, "tokens_per_s": spec.T / us * 1e6,
+                          "floor_us": floor_us, "frac_of_floor": floor_us / us,
+                          "algorithmic_bytes": nbytes, "flops": flops, "calls_timed": k,
+                          "kernels_per_call": ttq.ttq_linear_forward_kernels(
+                              spec.d, spec.dp, spec.T, spec.r, spec.p, ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)}),
+              flush=True)
+        del g, ws, Y, X, A, B
+    print(json.dumps({"table": "mlp_block_4096x11008_T512", "us": block_us, "tokens_per_s": 512 / block_us * 1e6,
+                      "note": "gate + up + down projections; the SiLU gating between them is not timed",
+                      "hbm_peak_gbs": peaks["hbm_gbs"], "bf16_peak_tflops": peaks["bf16_tflops"],
+                      "peak_source": peaks["source"], "clocks": sampler.stop()}), flush=True)
+
+
 def run_lowrank(args):
     """The static low-rank initialisation at the 70B-like MLP shape
     (d' = 28672, d = 8192, bf16 W, r = 64, 8 extra sampled directions, 2
@@ -611,10 +713,14 @@ def main():
                     help="time the decode workload (d = 4096, d' = 14336, INT4 g128) at T <= 16 tokens instead")
     ap.add_argument("--lowrank", action="store_true",
                     help="time the static low-rank initialisation (d' = 28672, d = 8192, r = 64) instead")
+    ap.add_argument("--table", action="store_true",
+                    help="time the forward at every configured workload point, one JSON line each, instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.lowrank:
+    if args.table:
+        run_table(args)
+    elif args.lowrank:
         run_lowrank(args)
     elif args.decode:
         run_decode(args)
