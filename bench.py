@@ -385,28 +385,88 @@ def run_ours(args):
     # ---- end to end: pinned host X in, host Y out, inside the timed region
     Xh = X0.pin_memory()
     Yh = torch.empty((T, dp), dtype=torch.bfloat16).pin_memory()
-    Xd = torch.empty_like(Xs[0])
+
+    def fwd_on(Xd, k, Yd, s=None):
+        ttq.ttq_linear_forward(Xd, Ws[k % nsets], None, None, w["p"], w["lam"], w["alpha"], bits, group, ws=ws,
+                               Y=Yd, scheme=scheme, stream=s)
+
+    def e2e_serial():
+        """One stream: copy in, forward, copy out, step after step."""
+        Xd = torch.empty_like(Xs[0])
+        for i in range(2):
+            Xd.copy_(Xh, non_blocking=True)
+            fwd_on(Xd, i, Ys[0])
+            Yh.copy_(Ys[0], non_blocking=True)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(args.steps):
+            Xd.copy_(Xh, non_blocking=True)
+            fwd_on(Xd, i, Ys[0])
+            Yh.copy_(Ys[0], non_blocking=True)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        return f0.elapsed_time(f1)
+
+    def e2e_pipelined():
+        """Three streams (copy in, forward, copy out) over two device buffers
+        of X and Y: step i's copies overlap the forwards of steps i - 1 and
+        i + 1.  Each step still copies its own X in and its own Y out inside
+        the timed region."""
+        s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        Xd = [torch.empty_like(Xs[0]) for _ in range(2)]
+        Yd = [torch.empty((T, dp), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+        in_done = [torch.cuda.Event() for _ in range(2)]
+        cmp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
+
+        def step(i):
+            b = i % 2
+            if i >= 2:
+                s_in.wait_event(cmp_done[b])      # the forward of step i - 2 has read Xd[b]
+            with torch.cuda.stream(s_in):
+                Xd[b].copy_(Xh, non_blocking=True)
+                in_done[b].record(s_in)
+            s_cmp.wait_event(in_done[b])
+            if i >= 2:
+                s_cmp.wait_event(out_done[b])     # step i - 2's Y has left Yd[b]
+            fwd_on(Xd[b], i, Yd[b], s_cmp)
+            cmp_done[b].record(s_cmp)
+            s_out.wait_event(cmp_done[b])
+            with torch.cuda.stream(s_out):
+                Yh.copy_(Yd[b], non_blocking=True)
+                out_done[b].record(s_out)
+
+        torch.cuda.synchronize()
+        for i in range(4):
+            step(i)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(s_in)
+        s_cmp.wait_stream(s_in)
+        s_out.wait_stream(s_in)
+        for i in range(args.steps):
+            step(i)
+        f1.record(s_out)
+        torch.cuda.synchronize()
+        return f0.elapsed_time(f1)
+
     barrier()
     torch.cuda.synchronize()
-    for _ in range(2):
-        Xd.copy_(Xh, non_blocking=True)
-        ttq.ttq_linear_forward(Xd, Ws[0], None, None, w["p"], w["lam"], w["alpha"], bits, group, ws=ws, Y=Ys[0],
-                               scheme=scheme)
-        Yh.copy_(Ys[0], non_blocking=True)
-    torch.cuda.synchronize()
-    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
-    for i in range(args.steps):
-        Xd.copy_(Xh, non_blocking=True)
-        ttq.ttq_linear_forward(Xd, Ws[i % nsets], None, None, w["p"], w["lam"], w["alpha"], bits, group,
-                               ws=ws, Y=Ys[0], scheme=scheme)
-        Yh.copy_(Ys[0], non_blocking=True)
-    f1.record(stream)
-    torch.cuda.synchronize()
+    e2e_mode = "pipelined: copy-in, forward and copy-out streams over two device buffers of X and Y"
+    try:
+        e2e_local = e2e_pipelined()
+    except Exception as exc:  # keep the bench line: time the one-stream form instead
+        torch.cuda.synchronize()
+        e2e_mode = f"serial, one stream (pipelined form failed: {type(exc).__name__}: {exc})"[:300]
+        e2e_local = e2e_serial()
+    # the last step's Y, read back, equals the device result of the same inputs
+    e2e_check = bool(torch.equal(Yh, Ys[0].cpu()))
     barrier()
-    e2e_ms = max_over_ranks(f0.elapsed_time(f1))
+    e2e_ms = max_over_ranks(e2e_local)
     e2e = {"value": _job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2)}
+           "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
+           "mode": e2e_mode, "result_check": e2e_check}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
