@@ -43,6 +43,8 @@
 // TTQ_FLAG_TIMEOUT, stops the CTA's other warps, lets the copies in flight
 // land, and the CTA returns without storing Y.
 
+#include <atomic>
+
 #include "ttq_device.cuh"
 #include "ttq_kernels.h"
 
@@ -519,16 +521,17 @@ cudaError_t launch_decode_typed(const CUtensorMap& tmC, const CUtensorMap& tmX,
                                 bool pdl) {
   constexpr size_t smem = decode_smem_bytes<BITS, NTT>();
   // the attribute belongs to a device: set once per device (the first
-  // launch on it, normally outside any graph capture)
-  static bool attr_set[64] = {};
+  // launch on it, normally outside any graph capture); host threads that
+  // race here both set the same value
+  static std::atomic<bool> attr_set[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_relaxed)) {
     const cudaError_t attr_err = cudaFuncSetAttribute(ttq_decode_kernel<BITS, NTT, PS>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                       static_cast<int>(smem));
     if (attr_err != cudaSuccess) return attr_err;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_relaxed);
   }
   const dim3 grid(static_cast<unsigned>((a.M + kRowsPerCta - 1) / kRowsPerCta));
   return launch_kernel(ttq_decode_kernel<BITS, NTT, PS>, grid, dim3(32 * (1 + kConsumers)), smem,

@@ -2,6 +2,7 @@
 // workspace layout, TMA descriptor set-up and the order of the kernels of
 // one TTQ linear call.  Nothing here allocates device memory or
 // synchronises; every call only enqueues work on the caller's stream.
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -24,14 +25,17 @@ size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int device_sms() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[64] = {};   // host threads that race here store the same value
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return kPlanSMs;
-  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  if (dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
     n = kPlanSMs;
-  if (dev < 64) cache[dev] = n;
+  if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
