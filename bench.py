@@ -56,6 +56,20 @@ NCU_TRAFFIC = {
 }
 
 
+def _host_cpu() -> dict:
+    """The host the CPU oracle ran on: its logical core count and CPU model."""
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
+
+
 def _rank_env():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
         int(os.environ.get("LOCAL_RANK", "0"))
@@ -194,6 +208,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "host": _host_cpu(),
                          "cpu_seconds": spent},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -348,9 +363,9 @@ def run_ours(args):
         ttq.ttq_dequantized_gemm(W_hat, Xsbuf, ws=ws, Y=Ys[k])
         ev[i][3].record(stream)
     torch.cuda.synchronize()
-    t_stat = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_qdq = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t_gemm = statistics.mean(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    t_stat = statistics.median(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_qdq = statistics.median(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_gemm = statistics.median(e[2].elapsed_time(e[3]) for e in ev) / 1e3
 
     peaks = _measured_peaks()
     flops = 2.0 * dp * d * T
@@ -472,7 +487,7 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rows_sample = 512
         est, spent = _oracle_sample(data, rows_sample)
-        cpu = {"value": T / est, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+        cpu = {"value": T / est, "unit": "tokens/s", "cores": 1, "kind": "oracle", "host": _host_cpu(),
                "sample": f"statistic and quantiser over the full layer, projection for {rows_sample} of {dp} "
                          f"output rows, extrapolated linearly in d' ({spent:.1f} s of CPU work)"}
 
