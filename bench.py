@@ -363,9 +363,9 @@ def run_ours(args):
         ttq.ttq_dequantized_gemm(W_hat, Xsbuf, ws=ws, Y=Ys[k])
         ev[i][3].record(stream)
     torch.cuda.synchronize()
-    t_stat = statistics.median(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_qdq = statistics.median(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    t_gemm = statistics.median(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    t_stat = statistics.mean(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_qdq = statistics.mean(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    t_gemm = statistics.mean(e[2].elapsed_time(e[3]) for e in ev) / 1e3
 
     peaks = _measured_peaks()
     flops = 2.0 * dp * d * T
