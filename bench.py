@@ -673,61 +673,66 @@ def run_table(args):
     cached = (None, None)      # (spec name and seed, W copies): one weight on the device at a time
     block_us = 0.0
     for spec in points:
-        key = (spec.name, spec.seed)
-        f32 = spec.dtype == "f32"
-        tdt = torch.float32 if f32 else torch.bfloat16
-        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).cuda()
-        data = synth.generate(spec, need_w=cached[0] != key)
-        if cached[0] != key:
-            cached = (None, None)
-            torch.cuda.empty_cache()
-            W0 = dev(data["W"])
-            n = max(1, min(8, -(-2 * L2_BYTES // (W0.numel() * W0.element_size()))))
-            cached = (key, [W0] + [W0.clone() for _ in range(n - 1)])
-        Ws = cached[1]
-        X = dev(data["X"])
-        A = dev(data["A"]) if spec.r else None
-        B = dev(data["B"]) if spec.r else None
-        Y = torch.empty((spec.T, spec.dp), dtype=tdt, device="cuda")
-        ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group,
-                               ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)
-        floor_us, nbytes, flops = _floor_us(spec, hbm, tc)
-        k = args.steps if floor_us < 200 else max(5, args.steps // 10)
+        try:
+            key = (spec.name, spec.seed)
+            f32 = spec.dtype == "f32"
+            tdt = torch.float32 if f32 else torch.bfloat16
+            dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).cuda()
+            data = synth.generate(spec, need_w=cached[0] != key)
+            if cached[0] != key:
+                cached = (None, None)
+                torch.cuda.empty_cache()
+                W0 = dev(data["W"])
+                n = max(1, min(8, -(-2 * L2_BYTES // (W0.numel() * W0.element_size()))))
+                cached = (key, [W0] + [W0.clone() for _ in range(n - 1)])
+            Ws = cached[1]
+            X = dev(data["X"])
+            A = dev(data["A"]) if spec.r else None
+            B = dev(data["B"]) if spec.r else None
+            Y = torch.empty((spec.T, spec.dp), dtype=tdt, device="cuda")
+            ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group,
+                                   ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)
+            floor_us, nbytes, flops = _floor_us(spec, hbm, tc)
+            k = args.steps if floor_us < 200 else max(5, args.steps // 10)
 
-        def fwd(i):
-            ttq.ttq_linear_forward(X, Ws[i % len(Ws)], A, B, spec.p, spec.lam, spec.alpha, spec.bits,
-                                   spec.group, ws=ws, Y=Y)
+            def fwd(i):
+                ttq.ttq_linear_forward(X, Ws[i % len(Ws)], A, B, spec.p, spec.lam, spec.alpha, spec.bits,
+                                       spec.group, ws=ws, Y=Y)
 
-        for i in range(args.warmup):
-            fwd(i)
-        torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for i in range(k):
+            for i in range(args.warmup):
                 fwd(i)
-        g.replay()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        us = e0.elapsed_time(e1) * 1e3 / k
-        st, flags = ttq.ttq_get_status(ws)
-        if st != ttq.TTQ_OK:
-            raise RuntimeError(f"{spec.name} T={spec.T}: device status {ttq.status_string(st)} (flags {flags:#x})")
-        if spec.name.startswith("mlp_") and spec.T == 512:
-            block_us += us
-        print(json.dumps({"table": "forward", "workload": f"{spec.name}_T{spec.T}", "d": spec.d, "dp": spec.dp,
-                          "T": spec.T, "bits": spec.bits, "group": spec.group, "r": spec.r, "p": spec.p,
-                          "alpha": spec.alpha, "dtype": spec.dtype, "us": us, "tokens_per_s": spec.T / us * 1e6,
-                          "floor_us": floor_us, "frac_of_floor": floor_us / us,
-                          "algorithmic_bytes": nbytes, "flops": flops, "calls_timed": k,
-                          "kernels_per_call": ttq.ttq_linear_forward_kernels(
-                              spec.d, spec.dp, spec.T, spec.r, spec.p, ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)}),
-              flush=True)
-        del g, ws, Y, X, A, B
-    print(json.dumps({"table": "mlp_block_4096x11008_T512", "us": block_us, "tokens_per_s": 512 / block_us * 1e6,
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(k):
+                    fwd(i)
+            g.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us = e0.elapsed_time(e1) * 1e3 / k
+            st, flags = ttq.ttq_get_status(ws)
+            if st != ttq.TTQ_OK:
+                raise RuntimeError(f"{spec.name} T={spec.T}: device status {ttq.status_string(st)} (flags {flags:#x})")
+            if spec.name.startswith("mlp_") and spec.T == 512:
+                block_us += us
+            print(json.dumps({"table": "forward", "workload": f"{spec.name}_T{spec.T}", "d": spec.d, "dp": spec.dp,
+                              "T": spec.T, "bits": spec.bits, "group": spec.group, "r": spec.r, "p": spec.p,
+                              "alpha": spec.alpha, "dtype": spec.dtype, "us": us, "tokens_per_s": spec.T / us * 1e6,
+                              "floor_us": floor_us, "frac_of_floor": floor_us / us,
+                              "algorithmic_bytes": nbytes, "flops": flops, "calls_timed": k,
+                              "kernels_per_call": ttq.ttq_linear_forward_kernels(
+                                  spec.d, spec.dp, spec.T, spec.r, spec.p, ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)}),
+                  flush=True)
+            del g, ws, Y, X, A, B
+        except Exception as exc:  # one point failing does not lose the others
+            torch.cuda.synchronize()
+            print(json.dumps({"table": "forward", "workload": f"{spec.name}_T{spec.T}",
+                              "error": f"{type(exc).__name__}: {exc}"[:300]}), flush=True)
+    print(json.dumps({"table": "mlp_block_4096x11008_T512", "us": block_us, "tokens_per_s": 512 / block_us * 1e6 if block_us > 0 else None,
                       "note": "gate + up + down projections; the SiLU gating between them is not timed",
                       "hbm_peak_gbs": peaks["hbm_gbs"], "bf16_peak_tflops": peaks["bf16_tflops"],
                       "peak_source": peaks["source"], "clocks": sampler.stop()}), flush=True)
