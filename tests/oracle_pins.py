@@ -226,6 +226,7 @@ def check_symmetric_worked_example(O):
     just above it) and errors up to s/2 ~ 2.14 on the unit values; without
     the 30 the scale is 1/7 and the errors at most ~0.071, thirty times
     less.  Levels are +-7 around the stored zero point 8."""
+    g = json.load(open(os.path.join(GOLDEN, "blog_int4_outlier.json")))["printed"]
     bits, group = 4, 32
     row = np.ones(32, np.float32)
     row[1::2] = -1.0
@@ -240,6 +241,9 @@ def check_symmetric_worked_example(O):
     rec = s * (q.astype(np.float64) - 8.0)
     unit_err = np.abs(rec - row)[np.arange(32) != 5]
     assert unit_err.max() <= s / 2 and abs(s / 2 - 2.1428571) < 2e-3, (unit_err.max(), s)
+    # the values the page prints, to their printed digits
+    assert abs(s - g["shared_scale"]) <= 0.005 and abs(s / 2 - g["shared_max_error_typical"]) <= 0.005
+    assert abs(s / 2 / 1.0 - g["shared_relative_error_typical"]) <= 0.005
     # segregated: the same unit values without the outlier
     row2 = row.copy()
     row2[5] = 1.0
@@ -248,7 +252,9 @@ def check_symmetric_worked_example(O):
     assert 1.0 / 7.0 <= s2 <= 1.0 / 7.0 * (1 + 2.0 ** -10), s2
     err2 = np.abs(s2 * (_unpack_np(codes2, 32, bits)[0] - 8.0) - row2)
     assert err2.max() <= s2 / 2 and abs(s2 / 2 - 0.0714286) < 1e-4
-    assert 29.0 < s / s2 < 31.0
+    assert abs(s2 - g["segregated_scale"]) <= 0.0005 and abs(s2 / 2 - g["segregated_max_error_typical"]) <= 0.0005
+    assert abs(s2 / 2 - g["segregated_relative_error_typical"]) <= 0.005
+    assert abs(s / s2 - g["error_ratio"]) <= 0.5
     # the asymmetric quantiser on the outlier group: s = (30 - m) / 15, m = -1
     codes3, sc3, ze3, _ = O.quantize(row[None, :], None, bits, group)
     s3 = float(_f16_bits_to_f64(sc3)[0, 0])
