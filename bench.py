@@ -388,7 +388,13 @@ def run_ours(args):
         {"kernel": "ttq_gemm_kernel", "ms": t_gemm * 1e3, "bound": "tensor", "flops": flops,
          "achieved_tflops": gemm_tflops, "frac": gemm_tflops / peaks["bf16_tflops"]},
     ]
-    rho = {"measured": (t_stat + t_qdq) / t_gemm, "closed_form": 1.0 / dp + 3.0 / T}
+    # the paper's relative cost of the test-time steps against the product
+    # (gist.science/zh/paper/2603.19296, section 2.3) and the blog's per-step
+    # overhead Delta / T (blog.lo0.es, "Test-time quantization", section "The
+    # overhead: the cost of measuring at every step"): Delta = statistic +
+    # quantiser, T = the whole forward
+    rho = {"measured": (t_stat + t_qdq) / t_gemm, "closed_form": 1.0 / dp + 3.0 / T,
+           "delta_over_forward": (t_stat + t_qdq) / (ms / args.steps / 1e3)}
 
     if args.profile:
         if world > 1:
