@@ -23,17 +23,33 @@ constexpr int kPlanSMs = 148;  // the same split plan as ttq_act_norm
 // host it is only a stand-in, so its device address is looked up below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of the scratch array on the current device, looked up once
-// per device (with that device current) and cached; null on failure.
+// Device address of the scratch array on the current device, looked up with
+// that device current and cached per device; null on failure.  A device
+// reset (cudaDeviceReset, or the primary context released and created
+// again) loads the library's module anew, possibly elsewhere, so a cached
+// address that no longer names device memory of this device is looked up
+// again.
+bool still_valid(const void* p, int dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();  // clear the non-sticky error of the query
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
 void* noalloc_scratch() {
   static void* addr[64] = {};
   static std::mutex mu;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
-  if (addr[dev] == nullptr) {
+  if (addr[dev] == nullptr || !still_valid(addr[dev], dev)) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      addr[dev] = nullptr;
+      return nullptr;
+    }
     addr[dev] = p;
   }
   return addr[dev];

@@ -151,17 +151,10 @@ def test_dequant_gemm_matches_oracle(O, case):
     assert torch.equal(Yb, Y.to(torch.bfloat16))
 
 
-FORWARD_CASES = [
-    synth.C1,
-    synth.C2,
-    synth.C3_GATE,
-    synth.C3_DOWN,
-    synth.C4.with_(T=1),
-    synth.C4.with_(T=4),
-    synth.C4.with_(T=16),
-    synth.C5.with_(T=1, p=2.0, alpha=0.5),
-    synth.C5.with_(T=128, p=1.0, alpha=0.25),
-    synth.C5.with_(T=4096, p=2.0, alpha=0.25),
+# every configured workload point: the fp32 d = 256 layer, the q_proj
+# prefill, the three MLP projections, decode at T = 1, 4, 16 and all twenty
+# points of the 70B-like MLP shape (T x p x alpha)
+FORWARD_CASES = [spec for name in ("C1", "C2", "C3", "C4", "C5") for spec in synth.CONFIGS[name]] + [
     _small("ragged_all", d=96, dp=200, T=19, bits=3, group=32),
     # 256-row tiles with ragged row and token tails
     _small("ragged_256row_tiles", d=4096, dp=4296, T=2000, bits=4, group=128, n_out=40),
@@ -175,7 +168,7 @@ FORWARD_CASES = [
 
 @pytest.mark.parametrize("spec", FORWARD_CASES, ids=lambda s: f"{s.name}-T{s.T}-p{s.p}-a{s.alpha}")
 def test_forward_matches_oracle(O, spec):
-    data = P.inputs(spec)
+    data = P.inputs_shared_w(spec)
     rows = synth.sample_rows(spec.dp, 96)
     ref = O.forward(data["X"].astype(np.float64), data["W"], *P.params(spec), spec.bits,
                     spec.group, A=data.get("A"), B=data.get("B"), rows=rows)
@@ -197,17 +190,30 @@ def test_forward_matches_oracle(O, spec):
     views = ttq.workspace_views(ws, spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
     D = views["D"].cpu().numpy().astype(np.float64)
     assert np.max(np.abs(D - ref["D"]) / ref["D"]) <= P.D_RTOL
+    codes_dev = views["codes"]
+    sc_dev, ze_dev = views["scales"], views["zeros"]
+    if ttq.ttq_workspace_get_layout(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt).tickets:
+        # the forward took the single-pass product, which writes no codes: the
+        # same kernel, given the forward's own D and X D^(-1/2), stores them on
+        # request, and its Y is the forward's to the bit
+        codes_dev = torch.empty_like(views["codes"])
+        sc_dev, ze_dev = torch.empty_like(views["scales"]), torch.empty_like(views["zeros"])
+        Y1 = ttq.ttq_quantize_gemm(W, views["D"], views["xh"], A, B, X if spec.r else None, spec.bits,
+                                   spec.group, y_dtype=torch.float32, codes=codes_dev, scales=sc_dev,
+                                   zeros=ze_dev)
+        torch.cuda.synchronize()
+        assert torch.equal(Y1, Y)
     # The quantiser is bit-exact for a shared D (test_quantize_bit_exact); here
     # each side uses its own D, so codes, scales and zeros must agree in every
     # group whose channels got the same binary32 D on both sides.
     same_d = views["D"].cpu().numpy() == ref["D"].astype(np.float32)
     group_ok = same_d.reshape(-1, spec.group).all(axis=1)          # [d/group]
     wpg = spec.group * spec.bits // 32                               # words per group
-    codes = P.u32(views["codes"]).reshape(spec.dp, -1, wpg)
+    codes = P.u32(codes_dev).reshape(spec.dp, -1, wpg)
     ref_codes = ref["codes"].reshape(spec.dp, -1, wpg)
     assert np.array_equal(codes[:, group_ok], ref_codes[:, group_ok])
-    assert np.array_equal(P.u16(views["scales"])[:, group_ok], ref["scales"][:, group_ok])
-    assert np.array_equal(P.u16(views["zeros"])[:, group_ok], ref["zeros"][:, group_ok])
+    assert np.array_equal(P.u16(sc_dev)[:, group_ok], ref["scales"][:, group_ok])
+    assert np.array_equal(P.u16(ze_dev)[:, group_ok], ref["zeros"][:, group_ok])
     assert group_ok.mean() >= 0.99, f"D differs in {np.count_nonzero(~same_d)} channels"
     err = P.y_error(Y.cpu().numpy()[:, rows], ref["Y"])
     assert err <= P.Y_TOL, err

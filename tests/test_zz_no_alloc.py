@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import ttq_oracle
 from test_weight_quantization_ttq_b200 import synth, ttq
 
 pytestmark = pytest.mark.gpu
@@ -19,14 +20,14 @@ pytestmark = pytest.mark.gpu
 D_RTOL = 1e-5  # the statistic's tolerance throughout the parity tests
 
 
-def _check_close(a, b):
-    a = a.cpu().numpy().astype(np.float64)
-    b = b.cpu().numpy().astype(np.float64)
-    assert np.all(np.isfinite(a)) and np.max(np.abs(a - b) / np.abs(b)) <= D_RTOL
+def _check_oracle(got, ref):
+    got = got.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got)) and np.max(np.abs(got - ref) / np.abs(ref)) <= D_RTOL
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_noalloc_matches_workspace_entry_point(dtype):
+    O = ttq_oracle.get()
     specs = [synth.LinearSpec("noalloc_a", d=4096, dp=0, T=2048, bits=4, group=128, dtype=dtype,
                               n_outliers=40, outlier_lo=20.0, outlier_hi=100.0, seed=3),
              synth.LinearSpec("noalloc_b", d=264, dp=0, T=45, bits=4, group=8, dtype=dtype, p=3.0,
@@ -38,8 +39,15 @@ def test_noalloc_matches_workspace_entry_point(dtype):
         D0, Dr0 = ttq.ttq_act_norm(X, spec.p, spec.lam, spec.alpha)
         D1, Dr1 = ttq.ttq_act_norm_noalloc(X, spec.p, spec.lam, spec.alpha)
         torch.cuda.synchronize()
-        _check_close(D1, D0)
-        _check_close(Dr1, Dr0)
+        # the same split plan, kernel and merge order as the workspace entry
+        # point: the same bits
+        assert torch.equal(D1, D0) and torch.equal(Dr1, Dr0)
+        # and the oracle's D, D^(-1/2) within the statistic's tolerance
+        pf, lf, af = (float(np.float32(v)) for v in (spec.p, spec.lam, spec.alpha))
+        D_ref, Dr_ref, st = O.act_norm(x.astype(np.float64), pf, lf, af)
+        assert st == 0
+        _check_oracle(D1, D_ref)
+        _check_oracle(Dr1, Dr_ref)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
