@@ -11,9 +11,9 @@ tokens, INT4 with groups of 128, p = 2, lambda = 1e-3, alpha = 0.5.
 
 Metric: tokens/s of the layer (whole job over all ranks; each rank runs its
 own independent problem, so scaling is weak and there is no collective on the
-data path).  Timing: CUDA events on the launching stream around exactly K
-steps after W warm-up steps, barrier + synchronize on both sides, max over
-ranks.  The inputs rotate over enough (X, W) sets that each step's operands
+data path).  Timing: exactly K steps after W warm-up steps, captured once
+as a CUDA graph whose replay is bracketed by CUDA events on the launching
+stream, barrier + synchronize on both sides, max over ranks.  The inputs rotate over enough (X, W) sets that each step's operands
 exceed the 126 MB L2, so no step reads its inputs from a warm L2.
 
 Extra keys: roofline of the dominant kernel (live CUDA-event timing of each
@@ -225,7 +225,8 @@ def _config(scheme: str = "asym"):
                        f"p={w['p']}, lambda={w['lam']}, alpha={w['alpha']}, bf16 X/W/Y",
            "d": w["d"], "d_out": w["dp"], "tokens": w["T"], "bits": w["bits"] if scheme != "fp8" else 8,
            "group": w["group"],
-           "l2": "inputs rotate over sets whose size exceeds L2 (no warm-L2 reads of X or W)"}
+           "l2": "inputs rotate over sets whose size exceeds L2 (no warm-L2 reads of X or W)",
+           "timing": "the K steps captured in one CUDA graph; CUDA events around its replay"}
     if scheme != "asym":
         cfg["scheme"] = SCHEMES[scheme]
     return cfg
@@ -283,17 +284,19 @@ def run_ours(args):
     scheme = {"asym": None, "sym": ttq.TTQ_QSCHEME_SYMMETRIC, "fp8": ttq.TTQ_QSCHEME_FP8_E4M3}[args.scheme]
     if args.scheme == "fp8":
         bits = 8
-    data = synth.generate(spec.with_(seed=rank))
     set_bytes = 2 * (d * dp + T * d + T * dp)
     nsets = max(2, -(-2 * L2_BYTES // set_bytes))
+    # each rotating set is its own seeded draw of the workload: each step
+    # reads cold memory, and a step that read another set's buffers would
+    # give another result
+    sets = [synth.generate(spec.with_(seed=rank * nsets + k)) for k in range(nsets)]
+    data = sets[0]
     Xs, Ws, Ys = [], [], []
-    X0 = torch.from_numpy(data["X"]).to(torch.bfloat16)
-    W0 = torch.from_numpy(data["W"]).to(torch.bfloat16)
-    for i in range(nsets):
-        # distinct buffers with the same values: each step reads cold memory
-        Xs.append(X0.cuda())
-        Ws.append(W0.cuda())
+    for k in range(nsets):
+        Xs.append(torch.from_numpy(sets[k]["X"]).to(torch.bfloat16).cuda())
+        Ws.append(torch.from_numpy(sets[k]["W"]).to(torch.bfloat16).cuda())
         Ys.append(torch.empty((T, dp), dtype=torch.bfloat16, device="cuda"))
+    del sets
     ws = ttq.new_workspace(d, dp, T, 0, bits, group)
     stream = torch.cuda.current_stream()
 
@@ -307,26 +310,33 @@ def run_ours(args):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+    # the K timed steps are captured once in a CUDA graph and the graph is
+    # replayed: a forward is a few tens of microseconds, about what the host
+    # takes to launch its kernels, so launching them one by one would time
+    # the host
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(args.steps):
+            step(i)
+    graph.replay()
+    torch.cuda.synchronize()
     # keep the GPU busy for ~1.5 s so the clock samples describe a loaded GPU
     t_end = time.time() + (0.0 if args.profile else 1.5)
-    i = 0
     while time.time() < t_end:
-        for _ in range(50):
-            step(i)
-            i += 1
+        graph.replay()
         torch.cuda.synchronize()
 
-    # ---- value: exactly K forward steps
+    # ---- value: exactly K forward steps (one replay of the K-step graph)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(args.steps):
-        step(i)
+    graph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms = max_over_ranks(e0.elapsed_time(e1))
+    del graph
     clocks = sampler.stop()
     st, flags = ttq.ttq_get_status(ws)
     if st != ttq.TTQ_OK:
@@ -336,7 +346,8 @@ def run_ours(args):
     # ---- per-kernel durations over K steps: the forward's kernels, one entry
     # point each (statistic fused with X D^{-1/2} in binary16, quantiser with
     # the dequantised binary16 weight, product on it)
-    n_kernels = ttq.ttq_linear_forward_kernels(d, dp, T, 0, w["p"])
+    n_kernels = ttq.ttq_linear_forward_kernels(d, dp, T, 0, w["p"], ttq.TTQ_BF16, bits, group,
+                                               scheme if scheme is not None else ttq.TTQ_QSCHEME_ASYMMETRIC)
     views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
     Dbuf = views["D"]  # written in place by ttq_act_norm_scale (copy_out=False)
     Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
@@ -370,9 +381,17 @@ def run_ours(args):
 
     peaks = _measured_peaks()
     flops = 2.0 * dp * d * T
-    stat_bytes = 4.0 * d * T + 8.0 * d  # X read once, X D^{-1/2} written, D and D^{-1/2}
-    # W read, codes, scales and zeros and the binary16 W_hat written, D read
-    qdq_bytes = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d + 2.0 * dp * d
+    hbm = peaks["hbm_gbs"]
+    # algorithmic bytes of each step (what the method must move): the
+    # statistic reads X and writes D, D^{-1/2}; the quantiser reads W and D
+    # and writes codes, scales and zeros
+    stat_alg = 2.0 * d * T + 8.0 * d
+    qdq_alg = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d
+    # bytes this implementation moves besides: the statistic also writes the
+    # product's binary16 X D^{-1/2}; the quantiser also writes the binary16
+    # dequantised weight that the prefill product reads
+    stat_moved = stat_alg + 2.0 * d * T
+    qdq_moved = qdq_alg + 2.0 * dp * d
     gemm_tflops = flops / t_gemm / 1e12
     traffic = NCU_TRAFFIC.get(_kernel_hash())
     roofline = {"kernel": "ttq_gemm_kernel<0, 256> (tcgen05 GEMM on the binary16 dequantised weight)", "bound": "tensor",
@@ -380,11 +399,15 @@ def run_ours(args):
                 "frac": gemm_tflops / peaks["bf16_tflops"], "traffic": traffic,
                 "peak_source": f"{peaks['source']} bf16 burst (cuBLAS 8192^3)",
                 "algorithmic_flops_per_launch": flops}
+
+    def hbm_entry(name, t, alg, moved):
+        return {"kernel": name, "ms": t * 1e3, "bound": "hbm", "bytes": alg,
+                "achieved_gbs": alg / t / 1e9, "frac": alg / t / 1e9 / hbm,
+                "bytes_moved": moved, "moved_gbs": moved / t / 1e9, "frac_of_moved": moved / t / 1e9 / hbm}
+
     kernels = [
-        {"kernel": "act_norm_scale_kernel", "ms": t_stat * 1e3, "bound": "hbm", "bytes": stat_bytes,
-         "achieved_gbs": stat_bytes / t_stat / 1e9, "frac": stat_bytes / t_stat / 1e9 / peaks["hbm_gbs"]},
-        {"kernel": "qdq_fp8_kernel" if args.scheme == "fp8" else "qdq_pack_kernel", "ms": t_qdq * 1e3, "bound": "hbm", "bytes": qdq_bytes,
-         "achieved_gbs": qdq_bytes / t_qdq / 1e9, "frac": qdq_bytes / t_qdq / 1e9 / peaks["hbm_gbs"]},
+        hbm_entry("act_norm_scale_kernel", t_stat, stat_alg, stat_moved),
+        hbm_entry("qdq_fp8_kernel" if args.scheme == "fp8" else "qdq_pack_kernel", t_qdq, qdq_alg, qdq_moved),
         {"kernel": "ttq_gemm_kernel", "ms": t_gemm * 1e3, "bound": "tensor", "flops": flops,
          "achieved_tflops": gemm_tflops, "frac": gemm_tflops / peaks["bf16_tflops"]},
     ]
@@ -404,8 +427,9 @@ def run_ours(args):
                               "roofline": roofline, "kernels": kernels}), flush=True)
         return
 
-    # ---- end to end: pinned host X in, host Y out, inside the timed region
-    Xh = X0.pin_memory()
+    # ---- end to end: pinned host X in, host Y out, inside the timed region;
+    # step i copies in set i's X and multiplies by set i's W
+    Xh = [Xs[k].cpu().pin_memory() for k in range(nsets)]
     Yh = torch.empty((T, dp), dtype=torch.bfloat16).pin_memory()
 
     def fwd_on(Xd, k, Yd, s=None):
@@ -416,14 +440,14 @@ def run_ours(args):
         """One stream: copy in, forward, copy out, step after step."""
         Xd = torch.empty_like(Xs[0])
         for i in range(2):
-            Xd.copy_(Xh, non_blocking=True)
+            Xd.copy_(Xh[i % nsets], non_blocking=True)
             fwd_on(Xd, i, Ys[0])
             Yh.copy_(Ys[0], non_blocking=True)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for i in range(args.steps):
-            Xd.copy_(Xh, non_blocking=True)
+            Xd.copy_(Xh[i % nsets], non_blocking=True)
             fwd_on(Xd, i, Ys[0])
             Yh.copy_(Ys[0], non_blocking=True)
         f1.record(stream)
@@ -447,7 +471,7 @@ def run_ours(args):
             if i >= 2:
                 s_in.wait_event(cmp_done[b])      # the forward of step i - 2 has read Xd[b]
             with torch.cuda.stream(s_in):
-                Xd[b].copy_(Xh, non_blocking=True)
+                Xd[b].copy_(Xh[i % nsets], non_blocking=True)
                 in_done[b].record(s_in)
             s_cmp.wait_event(in_done[b])
             if i >= 2:
@@ -482,13 +506,36 @@ def run_ours(args):
         torch.cuda.synchronize()
         e2e_mode = f"serial, one stream (pipelined form failed: {type(exc).__name__}: {exc})"[:300]
         e2e_local = e2e_serial()
-    # the last step's Y, read back, equals the device result of the same inputs
-    e2e_check = bool(torch.equal(Yh, Ys[0].cpu()))
+    # the last step's Y, read back, equals a forward of that step's own set
+    last = (args.steps - 1) % nsets
+    Yref = torch.empty((T, dp), dtype=torch.bfloat16, device="cuda")
+    fwd_on(Xs[last], last, Yref)
+    e2e_check = bool(torch.equal(Yh, Yref.cpu()))
     barrier()
     e2e_ms = max_over_ranks(e2e_local)
     e2e = {"value": _job_throughput(world, args.steps, T, e2e_ms), "unit": "tokens/s",
-           "h2d_bytes_per_step": int(Xh.numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
+           "h2d_bytes_per_step": int(Xh[0].numel() * 2), "d2h_bytes_per_step": int(Yh.numel() * 2),
            "mode": e2e_mode, "result_check": e2e_check}
+
+    # ---- the other regimes the layer serves, measured in the same run (one
+    # GPU): decode at 1 and 16 tokens (HBM-bound, the test-time steps
+    # dominate) and the 70B-like MLP shape at 1 and 4096 tokens
+    extra = {}
+    if world == 1 and not args.no_extra:
+        for t in (1, 16):
+            try:
+                extra[f"decode_T{t}"] = _decode_point(t, 50, 5, peaks)
+            except Exception as exc:
+                torch.cuda.synchronize()
+                extra[f"decode_T{t}"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        cache = _WeightCache()
+        for t in (1, 4096):
+            try:
+                extra[f"mlp70b_T{t}"] = _time_forward(synth.C5.with_(T=t, p=2.0, alpha=0.5), 50, 5, cache, peaks)
+            except Exception as exc:
+                torch.cuda.synchronize()
+                extra[f"mlp70b_T{t}"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        cache.drop(torch)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -509,24 +556,23 @@ def run_ours(args):
         "roofline": roofline, "kernels": kernels, "rho": rho, "cpu_baseline": cpu, "e2e": e2e,
         "clocks": clocks, "gpu_launches": n_kernels * args.steps,
     }
+    line.update(extra)
     print(json.dumps(line), flush=True)
 
 
-def run_decode(args):
-    """The decode workload (d = 4096, d' = 14336, INT4 g128, T = args.decode
-    tokens): K forwards, then K launches of each of its three kernels (one
-    entry point each: statistic + binary16 X D^{-1/2}, quantiser, product
-    from the packed codes).  A few-token step is shorter than its host-side
-    launch cost, so each batch of K calls is captured once in a CUDA graph and
-    the graph replay is timed.  One GPU; one JSON line.  W rotates over
-    enough copies that every step reads it from HBM."""
+def _decode_point(T, steps, warmup, peaks):
+    """The decode workload (d = 4096, d' = 14336, INT4 g128) at T <= 16
+    tokens: K forwards (statistic, then the single-pass product that reads
+    W once), then K calls of each of its two entry points, and for
+    comparison the two-pass form (quantiser writing codes, then the product
+    reading them).  A few-token step is shorter than its host-side launch
+    cost, so each batch of K calls is captured once in a CUDA graph and the
+    graph replay is timed.  W rotates over enough copies that every step
+    reads it from HBM.  Returns one dict."""
     import torch
 
     from test_weight_quantization_ttq_b200 import synth, ttq
 
-    T = int(args.decode)
-    if not 1 <= T <= 16:
-        raise SystemExit("--decode takes 1..16 tokens")
     spec = synth.C4.with_(T=T)
     d, dp, bits, group = spec.d, spec.dp, spec.bits, spec.group
     data = synth.generate(spec)
@@ -539,8 +585,8 @@ def run_decode(args):
     views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
     Dbuf = views["D"]
     Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
-    # the quantiser writes, and the product reads, one of ncs code sets in
-    # turn (more than L2 together)
+    # the two-pass form's quantiser writes, and its product reads, one of ncs
+    # code sets in turn (more than L2 together)
     ncs = max(2, -(-2 * L2_BYTES // (dp * d * bits // 8)))
     codes = [torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda") for _ in range(ncs)]
     sc = [torch.empty((dp, d // group), dtype=torch.int16, device="cuda") for _ in range(ncs)]
@@ -554,6 +600,9 @@ def run_decode(args):
     def stat(i):
         ttq.ttq_act_norm_scale(X, spec.p, spec.lam, spec.alpha, ws=ws, Xs=Xsbuf, copy_out=False)
 
+    def one_pass(i):
+        ttq.ttq_quantize_gemm(Ws[i % nsets], Dbuf, Xsbuf, None, None, None, bits, group, ws=ws, Y=Y)
+
     def qdq(i):
         k = i % ncs
         ttq.ttq_quantize_weight(Ws[i % nsets], Dbuf, bits, group, codes=codes[k], scales=sc[k],
@@ -564,12 +613,12 @@ def run_decode(args):
         ttq.ttq_dequant_gemm(codes[k], sc[k], ze[k], None, Xsbuf, None, None, bits, group, Y=Y)
 
     def graph_of(fn):
-        for i in range(args.warmup):
+        for i in range(warmup):
             fn(i)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            for i in range(args.steps):
+            for i in range(steps):
                 fn(i)
         g.replay()
         torch.cuda.synchronize()
@@ -588,39 +637,61 @@ def run_decode(args):
     for k in range(ncs):   # every code set holds real codes before the product is timed
         qdq(k)
     g_fwd = graph_of(fwd)
-    sampler = ClockSampler(0)
-    sampler.start()
-    t_end = time.time() + (0.0 if args.profile else 1.0)
-    while time.time() < t_end:
-        g_fwd.replay()
-        torch.cuda.synchronize()
     t_fwd = time_graph(g_fwd)
-    clocks = sampler.stop()
     st, flags = ttq.ttq_get_status(ws)
     if st != ttq.TTQ_OK:
         raise RuntimeError(f"device status {ttq.status_string(st)} (flags {flags:#x})")
-    t = [time_graph(graph_of(fn)) / args.steps for fn in (stat, qdq, prod)]
-    peaks = _measured_peaks()
+    t = [time_graph(graph_of(fn)) / steps for fn in (stat, one_pass, qdq, prod)]
+    hbm = peaks["hbm_gbs"]
     code_bytes = dp * d * bits / 8 + 4.0 * dp * d / group
+    stat_bytes = 2.0 * T * d + 8.0 * d
+    # the single pass reads W, X D^(-1/2) and sqrt(D) and writes Y
+    one_bytes = 2.0 * dp * d + 2.0 * T * d + 4.0 * d + 2.0 * T * dp
     qdq_bytes = 2.0 * dp * d + code_bytes + 4.0 * d
     prod_bytes = code_bytes + 2.0 * T * d + 2.0 * T * dp
-    hbm = peaks["hbm_gbs"]
+    t_fwd_step = t_fwd / steps
+    # the forward's floor: W read once at HBM bandwidth (a layer that looks at
+    # every weight at every step can do no better)
+    read_once = 2.0 * dp * d + 2.0 * T * d + 2.0 * T * dp
+
+    def entry(name, tt, nbytes):
+        return {"kernel": name, "us": tt * 1e6, "bytes": nbytes, "achieved_gbs": nbytes / tt / 1e9,
+                "frac": nbytes / tt / 1e9 / hbm}
+
     kernels = [
-        {"kernel": "act_norm_scale_kernel", "us": t[0] * 1e6},
-        {"kernel": "qdq_pack_kernel", "us": t[1] * 1e6, "bytes": qdq_bytes,
-         "achieved_gbs": qdq_bytes / t[1] / 1e9, "frac": qdq_bytes / t[1] / 1e9 / hbm},
-        {"kernel": "ttq_decode_kernel", "us": t[2] * 1e6, "bytes": prod_bytes,
-         "achieved_gbs": prod_bytes / t[2] / 1e9, "frac": prod_bytes / t[2] / 1e9 / hbm},
+        entry("act_norm_scale_kernel", t[0], stat_bytes),
+        entry("ttq_fused_decode_kernel (ttq_quantize_gemm: + a sqrt(D) pass of 8d bytes)", t[1], one_bytes),
     ]
-    print(json.dumps({"metric": "TTQ linear decode tokens/s", "value": T * args.steps / t_fwd,
-                      "unit": "tokens/s", "ms_per_step": t_fwd * 1e3 / args.steps, "steps": args.steps,
-                      "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
-                      "config": {"workload": f"decode_4096x14336_T{T}", "d": d, "dp": dp, "T": T,
-                                 "bits": bits, "group": group,
-                                 "l2": f"W rotates over {nsets} copies and the codes over {ncs} "
-                                       "sets (each more than L2)",
-                                 "timing": "CUDA graph of K calls, CUDA events around its replay"},
-                      "kernels": kernels, "hbm_peak_gbs": hbm, "clocks": clocks}), flush=True)
+    two_pass = [entry("qdq_pack_kernel", t[2], qdq_bytes), entry("ttq_decode_kernel", t[3], prod_bytes)]
+    return {"workload": f"decode_4096x14336_T{T}", "d": d, "dp": dp, "T": T, "bits": bits, "group": group,
+            "us": t_fwd_step * 1e6, "tokens_per_s": T / t_fwd_step,
+            "read_once_floor_us": read_once / (hbm * 1e9) * 1e6,
+            "frac_of_read_once_floor": read_once / (hbm * 1e9) / t_fwd_step,
+            "kernels_per_call": ttq.ttq_linear_forward_kernels(d, dp, T, 0, spec.p, ttq.TTQ_BF16, bits, group),
+            "l2": f"W rotates over {nsets} copies and the codes over {ncs} sets (each more than L2)",
+            "timing": "CUDA graph of K calls, CUDA events around its replay",
+            "kernels": kernels, "two_pass_for_comparison": two_pass}
+
+
+def run_decode(args):
+    """--decode T: the decode workload alone, one JSON line (see
+    _decode_point), with the clocks sampled while it runs."""
+    T = int(args.decode)
+    if not 1 <= T <= 16:
+        raise SystemExit("--decode takes 1..16 tokens")
+    peaks = _measured_peaks()
+    sampler = ClockSampler(0)
+    sampler.start()
+    row = _decode_point(T, args.steps, args.warmup, peaks)
+    clocks = sampler.stop()
+    print(json.dumps({"metric": "TTQ linear decode tokens/s", "value": row["tokens_per_s"], "unit": "tokens/s",
+                      "ms_per_step": row["us"] / 1e3, "steps": args.steps, "warmup": args.warmup,
+                      "dtype": "bf16", "data": "synthetic", "config": {k: row[k] for k in
+                      ("workload", "d", "dp", "T", "bits", "group", "l2", "timing")},
+                      "read_once_floor_us": row["read_once_floor_us"],
+                      "frac_of_read_once_floor": row["frac_of_read_once_floor"],
+                      "kernels": row["kernels"], "hbm_peak_gbs": peaks["hbm_gbs"], "clocks": clocks}),
+          flush=True)
 
 
 def _gpu_backlog(seconds: float) -> None:
@@ -655,6 +726,89 @@ def _floor_us(spec, hbm, tc):
     return 1e6 * ((stat + qdq) / hbm + max(prod / hbm, flops / tc)), stat + qdq + prod, flops
 
 
+class _WeightCache:
+    """The weight copies of one workload recipe on the device (enough
+    copies that together they exceed L2, at most 8); one recipe is held at a
+    time."""
+
+    def __init__(self):
+        self.key, self.Ws = None, None
+
+    def get(self, spec, data_w, torch):
+        key = (spec.name, spec.seed, spec.dtype)
+        if self.key != key:
+            self.key, self.Ws = None, None
+            torch.cuda.empty_cache()
+            tdt = torch.float32 if spec.dtype == "f32" else torch.bfloat16
+            W0 = torch.from_numpy(data_w).to(tdt).cuda()
+            n = max(1, min(8, -(-2 * L2_BYTES // (W0.numel() * W0.element_size()))))
+            self.key, self.Ws = key, [W0] + [W0.clone() for _ in range(n - 1)]
+        return self.Ws
+
+    def drop(self, torch):
+        self.key, self.Ws = None, None
+        torch.cuda.empty_cache()
+
+
+def _time_forward(spec, steps, warmup, cache, peaks):
+    """Device time of one ttq_linear_forward at one workload point: K calls
+    captured in a CUDA graph, CUDA events around its replay, W rotating over
+    copies that exceed L2.  Returns a dict with the time next to the floor
+    of the point's algorithmic bytes and flops at the measured peaks."""
+    import numpy as np
+    import torch
+
+    from test_weight_quantization_ttq_b200 import synth, ttq
+
+    hbm, tc = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
+    stream = torch.cuda.current_stream()
+    f32 = spec.dtype == "f32"
+    tdt = torch.float32 if f32 else torch.bfloat16
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).cuda()
+    need_w = cache.key != (spec.name, spec.seed, spec.dtype)
+    data = synth.generate(spec, need_w=need_w)
+    Ws = cache.get(spec, data.get("W"), torch)
+    X = dev(data["X"])
+    A = dev(data["A"]) if spec.r else None
+    B = dev(data["B"]) if spec.r else None
+    Y = torch.empty((spec.T, spec.dp), dtype=tdt, device="cuda")
+    dt = ttq.TTQ_F32 if f32 else ttq.TTQ_BF16
+    ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
+    floor_us, nbytes, flops = _floor_us(spec, hbm, tc)
+    k = steps if floor_us < 200 else max(5, steps // 10)
+
+    def fwd(i):
+        ttq.ttq_linear_forward(X, Ws[i % len(Ws)], A, B, spec.p, spec.lam, spec.alpha, spec.bits,
+                               spec.group, ws=ws, Y=Y)
+
+    for i in range(warmup):
+        fwd(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(k):
+            fwd(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / k
+    st, flags = ttq.ttq_get_status(ws)
+    if st != ttq.TTQ_OK:
+        raise RuntimeError(f"{spec.name} T={spec.T}: device status {ttq.status_string(st)} (flags {flags:#x})")
+    out = {"workload": f"{spec.name}_T{spec.T}", "d": spec.d, "dp": spec.dp, "T": spec.T, "bits": spec.bits,
+           "group": spec.group, "r": spec.r, "p": spec.p, "alpha": spec.alpha, "dtype": spec.dtype,
+           "us": us, "tokens_per_s": spec.T / us * 1e6, "floor_us": floor_us, "frac_of_floor": floor_us / us,
+           "algorithmic_bytes": nbytes, "flops": flops, "calls_timed": k,
+           "kernels_per_call": ttq.ttq_linear_forward_kernels(spec.d, spec.dp, spec.T, spec.r, spec.p, dt,
+                                                               spec.bits, spec.group)}
+    del g
+    return out
+
+
 def run_table(args):
     """Forward time of ttq_linear_forward at every configured workload point
     (the fp32 d = 256 case, the q_proj prefill, the three MLP projections at
@@ -664,77 +818,24 @@ def run_table(args):
     captured in a CUDA graph and its replay is timed with CUDA events; W
     rotates over enough copies to exceed L2.  One GPU; one JSON line per
     point and a closing line with the clocks."""
-    import numpy as np
     import torch
 
-    from test_weight_quantization_ttq_b200 import synth, ttq
+    from test_weight_quantization_ttq_b200 import synth
 
     peaks = _measured_peaks()
-    hbm, tc = peaks["hbm_gbs"] * 1e9, peaks["bf16_tflops"] * 1e12
-    stream = torch.cuda.current_stream()
     points = [synth.C1, synth.C2, synth.C3_GATE, synth.C3_UP, synth.C3_DOWN]
     points += [synth.C4.with_(T=t) for t in synth.C4_TOKENS]
     points += [synth.C5.with_(T=t, p=2.0, alpha=0.5) for t in synth.C5_TOKENS]
     sampler = ClockSampler(0)
     sampler.start()
-    cached = (None, None)      # (spec name and seed, W copies): one weight on the device at a time
+    cache = _WeightCache()
     block_us = 0.0
     for spec in points:
         try:
-            key = (spec.name, spec.seed)
-            f32 = spec.dtype == "f32"
-            tdt = torch.float32 if f32 else torch.bfloat16
-            dev = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(tdt).cuda()
-            data = synth.generate(spec, need_w=cached[0] != key)
-            if cached[0] != key:
-                cached = (None, None)
-                torch.cuda.empty_cache()
-                W0 = dev(data["W"])
-                n = max(1, min(8, -(-2 * L2_BYTES // (W0.numel() * W0.element_size()))))
-                cached = (key, [W0] + [W0.clone() for _ in range(n - 1)])
-            Ws = cached[1]
-            X = dev(data["X"])
-            A = dev(data["A"]) if spec.r else None
-            B = dev(data["B"]) if spec.r else None
-            Y = torch.empty((spec.T, spec.dp), dtype=tdt, device="cuda")
-            ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group,
-                                   ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)
-            floor_us, nbytes, flops = _floor_us(spec, hbm, tc)
-            k = args.steps if floor_us < 200 else max(5, args.steps // 10)
-
-            def fwd(i):
-                ttq.ttq_linear_forward(X, Ws[i % len(Ws)], A, B, spec.p, spec.lam, spec.alpha, spec.bits,
-                                       spec.group, ws=ws, Y=Y)
-
-            for i in range(args.warmup):
-                fwd(i)
-            torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                for i in range(k):
-                    fwd(i)
-            g.replay()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
-            us = e0.elapsed_time(e1) * 1e3 / k
-            st, flags = ttq.ttq_get_status(ws)
-            if st != ttq.TTQ_OK:
-                raise RuntimeError(f"{spec.name} T={spec.T}: device status {ttq.status_string(st)} (flags {flags:#x})")
+            row = _time_forward(spec, args.steps, args.warmup, cache, peaks)
             if spec.name.startswith("mlp_") and spec.T == 512:
-                block_us += us
-            print(json.dumps({"table": "forward", "workload": f"{spec.name}_T{spec.T}", "d": spec.d, "dp": spec.dp,
-                              "T": spec.T, "bits": spec.bits, "group": spec.group, "r": spec.r, "p": spec.p,
-                              "alpha": spec.alpha, "dtype": spec.dtype, "us": us, "tokens_per_s": spec.T / us * 1e6,
-                              "floor_us": floor_us, "frac_of_floor": floor_us / us,
-                              "algorithmic_bytes": nbytes, "flops": flops, "calls_timed": k,
-                              "kernels_per_call": ttq.ttq_linear_forward_kernels(
-                                  spec.d, spec.dp, spec.T, spec.r, spec.p, ttq.TTQ_F32 if f32 else ttq.TTQ_BF16)}),
-                  flush=True)
-            del g, ws, Y, X, A, B
+                block_us += row["us"]
+            print(json.dumps({"table": "forward", **row}), flush=True)
         except Exception as exc:  # one point failing does not lose the others
             torch.cuda.synchronize()
             print(json.dumps({"table": "forward", "workload": f"{spec.name}_T{spec.T}",
@@ -808,6 +909,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the decode and 70B-like MLP points added to the default line")
     ap.add_argument("--profile", action="store_true",
                     help="short run for a profiler: no clock warm-up loop, no CPU baseline, no e2e leg")
     ap.add_argument("--scheme", choices=sorted(SCHEMES), default="asym",

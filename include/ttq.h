@@ -41,7 +41,8 @@
  *    caller, and must be 16-byte aligned.  The library never allocates
  *    device memory and keeps no per-call state.  Temporary storage is the
  *    caller's workspace `ws` of `ws_bytes` >= ttq_workspace_size(...) bytes
- *    (256-byte aligned); its first bytes hold a device status word.
+ *    (256-byte aligned); its header (the first 20480 bytes, or all of a
+ *    smaller workspace) holds a device status word and internal counters.
  *    Initialise a fresh workspace once with ttq_workspace_init.
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
  *    only enqueues work on that stream and returns; the library never
@@ -137,6 +138,13 @@ typedef struct ttq_workspace_layout {
   size_t total;
   int64_t splits; /* number of token splits of the statistic pass */
   int64_t ax_ld;  /* row stride (elements) of A X                 */
+  size_t axp;     /* float32 [ax_splits][T][r] partial sums of A X split along d
+                     (0 when A X is not split) */
+  size_t D_sqrt;  /* float32 [d] sqrtf(D_ii) for the single-pass decode product */
+  size_t ypart;   /* float32 partial output tiles of the single-pass decode product */
+  size_t tickets; /* uint32 arrival tickets of its 128-row tiles (inside the
+                     zeroed header; 0: not in this layout) */
+  int64_t ax_splits; /* K splits of the A X product (1: none; 0 when r == 0) */
 } ttq_workspace_layout;
 
 /* Workspace bytes needed by every entry point below for this shape
@@ -149,8 +157,10 @@ ttq_status ttq_workspace_get_layout(int64_t d, int64_t dp, int64_t T, int64_t r,
                                     int bits, int group, ttq_dtype dtype,
                                     ttq_workspace_layout* out);
 
-/* Clears the status word and internal counters of a workspace (enqueued on
- * `stream`).  Call once after allocating a workspace, and to reset flags. */
+/* Clears the header of a workspace: the status word and internal counters,
+ * the first min(ws_bytes, 20480) bytes (enqueued on `stream`; ws_bytes must
+ * be at least 4096).  Call once after allocating a workspace, to reset flags,
+ * and after TTQ_ERR_TIMEOUT. */
 ttq_status ttq_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Step (1), the per-channel activation statistic
@@ -202,7 +212,11 @@ ttq_status ttq_act_norm_scale(const void* X, ttq_dtype dtype, int64_t d, int64_t
  * that loads the library holds 2 MiB + 4 KiB for it until the process exits,
  * and d may be at most 16384 (larger d returns TTQ_ERR_UNSUPPORTED).
  *   The first call on a device looks up the array's device address on the
- * current device; make that first call before any stream capture.  All calls
+ * current device; make that first call before any stream capture.  Every
+ * later call checks that the cached address still names device memory of
+ * that device and looks it up again if not (after cudaDeviceReset, or once
+ * the primary context was released and created anew, the array may sit
+ * elsewhere; make the first call after such a reset outside a capture too).  All calls
  * share the one array, so calls whose work overlaps on the GPU (other
  * streams, other threads) race: order them on one stream.  Each call clears
  * the array's status word and tickets first; device flags are not reported
@@ -324,18 +338,51 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A,
                                  int bits, int group, ttq_qscheme scheme, void* Y,
                                  ttq_dtype y_dtype, void* ws, size_t ws_bytes, void* stream);
 
-/* Number of kernels one ttq_linear_forward call with these sizes enqueues
- * on the current device (host query; no device work), in *kernels:
- * the statistic pass (fused with the scaling of X when it fits, see
- * ttq_act_norm_scale), the quantiser, the product, and for r > 0 the A X
- * product (plus two bf16 conversions of a float32 A and B).  An interface
- * query of this library; the method has no counterpart. */
+/* Number of kernels one ttq_linear_forward_ex call with these sizes and
+ * this code scheme enqueues on the current device (host query; no device
+ * work), in *kernels: the statistic pass (fused with the scaling of X when
+ * it fits, see ttq_act_norm_scale), the quantiser and the product (one
+ * kernel together where the forward takes the single-pass decode product,
+ * see ttq_quantize_gemm), and for r > 0 the A X product (plus the
+ * reduction of its K splits, and two bf16 conversions of a float32 A and
+ * B).  An interface query of this library; the method has no counterpart. */
 ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,
-                                      int64_t r, float p, int* kernels);
+                                      int64_t r, float p, int bits, int group,
+                                      ttq_qscheme scheme, int* kernels);
+
+/* Steps (2)-(3) in one pass over the weight, for a few tokens: reads bf16 W
+ * once, forms Q[W D^{1/2}] group by group in the binary32 order stated at
+ * the top of this file, and multiplies it with the binary16 X D^{-1/2} on
+ * the tensor cores, so that the codes never travel through memory
+ * (gist.science/zh/paper/2603.19296, section 2.1 for W_hat, section 2.3 for
+ * the cost it attacks: at decode the 3d'd test-time term outweighs the
+ * d'dT product, and reading W once is its floor).
+ *   Y [T][d'] (y_dtype) = sum_i s (q - z) Xs[t][i]  (+ B (A X) when r > 0),
+ * accumulated in fp32 (each group's sum of (q - z) Xs is scaled by s once).
+ * W bf16 [dp][d]; D float32 [d]; Xs binary16 [T][d] = X D^{-1/2} as
+ * ttq_act_norm_scale writes it; A [r][d], B [dp][r] and X [T][d] bf16 (only
+ * for r > 0).  codes, scales, zeros: NULL, or all three given and filled
+ * exactly as ttq_quantize_weight fills them (same bits).
+ *   Limits: 1 <= T <= 16, d a multiple of 128, bits 2..4, group 32, 64 or
+ * 128, dp <= 524288 (else TTQ_ERR_UNSUPPORTED).  Workspace as for
+ * ttq_linear_forward (TTQ_BF16) of the same sizes; its tile tickets start at
+ * zero (ttq_workspace_init) and every call leaves them at zero.  Flags as
+ * ttq_quantize_weight, and TIMEOUT (then re-initialise the workspace).
+ * ttq_linear_forward takes this product itself for bf16 layers with the
+ * asymmetric codes and at most 16 tokens (without storing codes). */
+ttq_status ttq_quantize_gemm(const void* W, const float* D, const uint16_t* Xs, const void* A,
+                             const void* B, const void* X, int64_t d, int64_t dp, int64_t T,
+                             int64_t r, int bits, int group, uint32_t* codes, uint16_t* scales,
+                             uint16_t* zeros, void* Y, ttq_dtype y_dtype, void* ws,
+                             size_t ws_bytes, void* stream);
 
 /* Reads the workspace status word (a blocking device-to-host copy; the caller
  * synchronises its stream first).  *flags receives the raw TTQ_FLAG_* bits
- * (may be NULL).  Returns ttq_status_from_flags of those bits. */
+ * (may be NULL).  Returns ttq_status_from_flags of those bits.
+ *   After TTQ_ERR_TIMEOUT the workspace must be reset with
+ * ttq_workspace_init before its next use: a statistic pass whose barrier
+ * among its blocks gave up leaves that barrier's counter off zero, and the
+ * next call would otherwise start from it. */
 ttq_status ttq_get_status(const void* ws, uint32_t* flags);
 
 /* The status that a set of TTQ_FLAG_* bits stands for (host only, no device

@@ -105,7 +105,8 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
     const XT* __restrict__ X, int64_t d, int64_t T, double p, double lambda, double alpha,
     int64_t splits, int64_t rows_per_split, double* __restrict__ partial,
     uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
-    __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
+    float* __restrict__ Dh, __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb,
+    uint32_t* __restrict__ status) {
   __shared__ double red[8][kChannelsPerBlock + 2];
   __shared__ int is_last;
   allow_dependents_launch();
@@ -205,6 +206,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
     const bool ok = finish_channel<PK>(tot, p, lambda, alpha, &df, &drf);
     D[c] = df;
     Dr[c] = drf;
+    if (Dh != nullptr) Dh[c] = __fsqrt_rn(df);   // the quantiser's h = sqrtf(D)
     if (!ok) set_flag(status, TTQ_FLAG_NONFINITE);
   }
   if (threadIdx.x == 0) counters[cb] = 0u;  // ready for the next call
@@ -262,12 +264,14 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
     const XT* __restrict__ X, int64_t d, int64_t T, double p, double lambda, double alpha,
     int64_t splits, int64_t rows_per_split, double* __restrict__ partial,
     uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
-    __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb, uint32_t* __restrict__ status) {
+    float* __restrict__ Dh, __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb,
+    uint32_t* __restrict__ status) {
   constexpr int R = reg_rows<XT>();
   __shared__ double red[8][kChannelsPerBlock + 2];
   __shared__ float dr_s[kChannelsPerBlock];
   __shared__ int barrier_ok;
   allow_dependents_launch();
+  grid_dependency_wait();   // (a no-op for the cooperative launch)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -331,6 +335,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
     if (sp == 0) {
       D[c] = df;
       Dr[c] = drf;
+      if (Dh != nullptr) Dh[c] = __fsqrt_rn(df);   // the quantiser's h = sqrtf(D)
       if (!ok) set_flag(status, TTQ_FLAG_NONFINITE);
     }
   }
@@ -368,29 +373,29 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
 template <typename XT, int PK>
 cudaError_t launch_typed(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
                          int64_t splits, int64_t rows_per_split, double* partial,
-                         uint32_t* counters, float* D, float* Dr, void* xh, void* xb,
+                         uint32_t* counters, float* D, float* Dr, float* Dh, void* xh, void* xb,
                          uint32_t* status, cudaStream_t stream, bool pdl) {
   const dim3 grid(static_cast<unsigned>((d + kChannelsPerBlock - 1) / kChannelsPerBlock),
                   static_cast<unsigned>(splits));
   return launch_kernel(act_norm_kernel<XT, PK>, grid, dim3(kThreads), 0, stream, pdl, X, d, T,
                        static_cast<double>(p), static_cast<double>(lambda),
                        static_cast<double>(alpha), splits, rows_per_split, partial, counters, D,
-                       Dr, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
+                       Dr, Dh, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
 }
 
 template <typename XT>
 cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
                      int64_t splits, int64_t rows_per_split, double* partial, uint32_t* counters,
-                     float* D, float* Dr, void* xh, void* xb, uint32_t* status,
+                     float* D, float* Dr, float* Dh, void* xh, void* xb, uint32_t* status,
                      cudaStream_t stream, bool pdl) {
   if (p == 1.0f)
     return launch_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                               counters, D, Dr, xh, xb, status, stream, pdl);
+                               counters, D, Dr, Dh, xh, xb, status, stream, pdl);
   if (p == 2.0f)
     return launch_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                               counters, D, Dr, xh, xb, status, stream, pdl);
+                               counters, D, Dr, Dh, xh, xb, status, stream, pdl);
   return launch_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                             counters, D, Dr, xh, xb, status, stream, pdl);
+                             counters, D, Dr, Dh, xh, xb, status, stream, pdl);
 }
 
 // How many blocks of the fused kernel fit on one SM (0 when the query
@@ -433,7 +438,7 @@ template <typename XT, int PK>
 cudaError_t launch_fused_typed(const XT* X, int64_t d, int64_t T, float p, float lambda,
                                float alpha, int64_t splits, int64_t rows_per_split,
                                double* partial, uint32_t* counters, float* D, float* Dr,
-                               void* xh, void* xb, uint32_t* status, int num_sms,
+                               float* Dh, void* xh, void* xb, uint32_t* status, int num_sms,
                                cudaStream_t stream, bool* launched) {
   *launched = false;
   if (!fused_fits<XT, PK>(d, splits, rows_per_split, num_sms)) return cudaSuccess;
@@ -444,14 +449,22 @@ cudaError_t launch_fused_typed(const XT* X, int64_t d, int64_t T, float p, float
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  if (splits > 1) {
+    // the blocks of a column block wait for one another: all must be resident
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    // one split: each block's barrier has itself alone to wait for, so a
+    // plain launch does, and it may overlap the previous kernel's tail
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+  }
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, act_norm_scale_kernel<XT, PK>, X, d, T, static_cast<double>(p),
       static_cast<double>(lambda), static_cast<double>(alpha), splits, rows_per_split, partial,
-      counters, D, Dr, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
+      counters, D, Dr, Dh, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
   *launched = e == cudaSuccess;
   return e;
 }
@@ -459,21 +472,37 @@ cudaError_t launch_fused_typed(const XT* X, int64_t d, int64_t T, float p, float
 template <typename XT>
 cudaError_t launch_fused_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
                            int64_t splits, int64_t rows_per_split, double* partial,
-                           uint32_t* counters, float* D, float* Dr, void* xh, void* xb,
+                           uint32_t* counters, float* D, float* Dr, float* Dh, void* xh, void* xb,
                            uint32_t* status, int num_sms, cudaStream_t stream, bool* launched) {
   if (p == 1.0f)
     return launch_fused_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                                     counters, D, Dr, xh, xb, status, num_sms, stream,
+                                     counters, D, Dr, Dh, xh, xb, status, num_sms, stream,
                                      launched);
   if (p == 2.0f)
     return launch_fused_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                                     counters, D, Dr, xh, xb, status, num_sms, stream,
+                                     counters, D, Dr, Dh, xh, xb, status, num_sms, stream,
                                      launched);
   return launch_fused_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                                   counters, D, Dr, xh, xb, status, num_sms, stream, launched);
+                                   counters, D, Dr, Dh, xh, xb, status, num_sms, stream, launched);
+}
+
+__global__ void sqrt_f32_kernel(const float* __restrict__ D, float* __restrict__ h, int64_t d) {
+  allow_dependents_launch();
+  grid_dependency_wait();
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < d;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    h[i] = __fsqrt_rn(D[i]);
 }
 
 }  // namespace
+
+cudaError_t launch_sqrt_f32(const float* D, float* h, int64_t d, cudaStream_t stream) {
+  if (d == 0) return cudaSuccess;
+  int64_t blocks = (d + 255) / 256;
+  if (blocks > 1024) blocks = 1024;
+  return launch_kernel(sqrt_f32_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                       false, D, h, d);
+}
 
 void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split) {
   // about two resident blocks per SM, and at most 16 splits so that the
@@ -496,12 +525,12 @@ void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* 
 cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                             float lambda, float alpha, int64_t splits, int64_t rows_per_split,
                             double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
-                            void* xb, uint32_t* status, cudaStream_t stream, bool pdl) {
+                            void* xb, uint32_t* status, cudaStream_t stream, bool pdl, float* Dh) {
   if (x_f32)
     return launch_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits, rows_per_split,
-                    partial, counters, D, Dr, xh, xb, status, stream, pdl);
+                    partial, counters, D, Dr, Dh, xh, xb, status, stream, pdl);
   return launch_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
-                  rows_per_split, partial, counters, D, Dr, xh, nullptr, status, stream, pdl);
+                  rows_per_split, partial, counters, D, Dr, Dh, xh, nullptr, status, stream, pdl);
 }
 
 bool act_norm_scale_fused(bool x_f32, int64_t d, int64_t splits, int64_t rows_per_split, float p,
@@ -515,13 +544,13 @@ cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t 
                                   int64_t rows_per_split, double* partial,
                                   uint32_t* counters, float* D, float* Dr, void* xh,
                                   void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
-                                  bool* launched) {
+                                  bool* launched, float* Dh) {
   if (x_f32)
     return launch_fused_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits,
-                          rows_per_split, partial, counters, D, Dr, xh, xb, status, num_sms,
+                          rows_per_split, partial, counters, D, Dr, Dh, xh, xb, status, num_sms,
                           stream, launched);
   return launch_fused_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
-                        rows_per_split, partial, counters, D, Dr, xh, nullptr, status,
+                        rows_per_split, partial, counters, D, Dr, Dh, xh, nullptr, status,
                         num_sms, stream, launched);
 }
 

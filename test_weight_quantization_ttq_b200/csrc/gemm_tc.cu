@@ -60,6 +60,8 @@ struct GemmDev {
   int a_f16;            // plain mode: binary16 A operand (else bf16)
   int BN;
   int stages;
+  int kb_per_split;     // split-K: K blocks per split (0: no split)
+  int64_t split_stride; // split-K: elements between the splits' partial outputs
   uint32_t* status;
 };
 
@@ -279,7 +281,10 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
   const int64_t n0 = static_cast<int64_t>(blockIdx.y) * BN;
   const int kb_main = static_cast<int>((g.K + kBK - 1) / kBK);
   const int kb_tail = static_cast<int>((g.K_tail + kBK - 1) / kBK);
-  const int kb_total = kb_main + kb_tail;
+  // this CTA's K blocks [kb_lo, kb_total): all of them, or one split of the
+  // main blocks (split-K runs only in the plain mode without a tail)
+  const int kb_lo = g.kb_per_split > 0 ? static_cast<int>(blockIdx.z) * g.kb_per_split : 0;
+  const int kb_total = g.kb_per_split > 0 ? min(kb_main, kb_lo + g.kb_per_split) : kb_main + kb_tail;
   // accumulator h of a 256-row tile starts at column 256 * h
   const uint32_t tmem_cols =
       kSub == 2 ? 512u : (BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u);
@@ -323,7 +328,7 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
     if (lane == 0) {
       int s = 0;
       uint32_t ph = 0;
-      for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
+      for (int kb = kb_lo; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag)) {
           *abort_flag = 1;
           set_flag(g.status, TTQ_FLAG_TIMEOUT);
@@ -361,7 +366,7 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
       const uint32_t idesc_tail = idesc_f16kind(kFmtBF16, 128, static_cast<uint32_t>(BN));
       int s = 0;
       uint32_t ph = 0;
-      for (int kb = 0; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
+      for (int kb = kb_lo; kb < kb_total; ++kb, s = (s + 1 == stages) ? 0 : s + 1, ph ^= (s == 0)) {
         if (!mbar_wait(&full[s], ph, abort_flag)) {
           *abort_flag = 1;
           set_flag(g.status, TTQ_FLAG_TIMEOUT);
@@ -377,7 +382,7 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
           for (int h = 0; h < kSub; ++h) {
             const uint64_t adesc = smem_desc_sw128(a_addr + h * kSubTileBytes);
             mma_f16kind_ss(tmem_base + 256u * h, adesc + 2u * k, bdesc + 2u * k, idesc,
-                           (kb | k) != 0 ? 1u : 0u);
+                           (kb != kb_lo || k != 0) ? 1u : 0u);
           }
         }
         mma_commit(&empty[s]);
@@ -495,12 +500,19 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
     }
 
     int ok = 1;
-    if (lane == 0) ok = mbar_wait(accum, 0, abort_flag) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      set_flag(g.status, TTQ_FLAG_TIMEOUT);
+    if (lane == 0) {
+      ok = mbar_wait(accum, 0, abort_flag) ? 1 : 0;
+      if (!ok) {
+        *abort_flag = 1;
+        set_flag(g.status, TTQ_FLAG_TIMEOUT);
+        // the MMA issuer commits `accum` after its loop even when it stops
+        // early: wait for that (with a fresh limit, not cut short by the
+        // abort) so that no MMA still writes the tensor memory freed below
+        int never = 0;
+        mbar_wait(accum, 0, &never);
+      }
     }
+    ok = __shfl_sync(0xffffffffu, ok, 0);
     tc_fence_after_sync();
     // warp w may read tensor-memory lanes 32 (w % 4) .. +31.  BM = 128: the
     // two warps of a lane quadrant split the columns; BM = 256: warps 2-5
@@ -557,6 +569,7 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
       if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
     } else {
       const bool store = good && j < g.M;
+      const int64_t yoff = g.kb_per_split > 0 ? static_cast<int64_t>(blockIdx.z) * g.split_stride : 0;
       for (int ch = ch0; ch < nchunks; ch += chs) {
         uint32_t rr[16];
         tmem_load_16(tmem_base + 256u * acc + (static_cast<uint32_t>(q * 32) << 16) + ch * 16, rr);
@@ -564,7 +577,7 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
         if (store) {
           const int64_t t0 = n0 + ch * 16;
           if (g.y_f32) {
-            float* Y = static_cast<float*>(g.Y);
+            float* Y = static_cast<float*>(g.Y) + yoff;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               if (t0 + i < g.T) Y[(t0 + i) * g.ldy + j] = __uint_as_float(rr[i]);
@@ -623,8 +636,16 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.BN = BN;
   g.stages = stages;
   g.status = a.status;
+  const bool split = a.k_splits > 1;
+  if (split && (BITS != 0 || a.K_tail != 0 || !a.y_f32 || a.kb_per_split < 1 ||
+                static_cast<int64_t>(a.k_splits - 1) * a.kb_per_split >= (a.K + kBK - 1) / kBK))
+    return cudaErrorInvalidValue;   // every split must own at least one K block
+  g.kb_per_split = split ? a.kb_per_split : 0;
+  g.split_stride = split ? a.split_stride : 0;
+  if (split) g.y_tma = 0;
   const dim3 grid(static_cast<unsigned>((a.M + BM - 1) / BM),
-                  static_cast<unsigned>((a.T + BN - 1) / BN));
+                  static_cast<unsigned>((a.T + BN - 1) / BN),
+                  static_cast<unsigned>(split ? a.k_splits : 1));
   return launch_kernel(ttq_gemm_kernel<BITS, BM, TC>, grid, dim3(cta_threads<BM>()), smem, stream,
                        pdl, maps.a0, maps.b0, maps.a1, maps.b1, maps.c0, maps.y, g);
 }
@@ -644,7 +665,42 @@ cudaError_t launch_bits(const GemmArgs& a, const GemmMaps& maps, int BN, int BM,
   return launch_tile<BITS, 128, false>(a, maps, BN, stream, pdl);
 }
 
+// AX[t][k] = bf16(sum over s of P[s][t][k]), the splits added in order.
+__global__ void ax_reduce_kernel(const float* __restrict__ P, int splits, int64_t T, int64_t r,
+                                 __nv_bfloat16* __restrict__ AX, int64_t ax_ld) {
+  allow_dependents_launch();
+  grid_dependency_wait();
+  const int64_t n = T * r;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < splits; ++s) acc += __ldcg(P + s * n + i);
+    const int64_t t = i / r;
+    AX[t * ax_ld + (i - t * r)] = __float2bfloat16_rn(acc);
+  }
+}
+
 }  // namespace
+
+AxSplit ax_split_plan(int64_t r, int64_t T, int64_t d, int num_sms) {
+  const int64_t kb = (d + kBK - 1) / kBK;
+  const int64_t tiles = ((r + 127) / 128) * ((T + gemm_block_n(T) - 1) / gemm_block_n(T));
+  int64_t s = tiles > 0 ? num_sms / tiles : 1;
+  if (s > kb / 4) s = kb / 4;
+  if (s < 2) return {1, static_cast<int>(kb)};
+  const int64_t per = (kb + s - 1) / s;
+  return {static_cast<int>((kb + per - 1) / per), static_cast<int>(per)};
+}
+
+cudaError_t launch_ax_reduce(const float* P, int splits, int64_t T, int64_t r, void* AX,
+                             int64_t ax_ld, cudaStream_t stream, bool pdl) {
+  const int64_t n = T * r;
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  return launch_kernel(ax_reduce_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                       pdl, P, splits, T, r, static_cast<__nv_bfloat16*>(AX), ax_ld);
+}
 
 int gemm_code_tile_words(int bits) { return bits == 2 ? 4 : 8; }
 

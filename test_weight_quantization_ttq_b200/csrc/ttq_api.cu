@@ -14,9 +14,13 @@ namespace ttq {
 namespace {
 
 constexpr size_t kAlign = 256;
-// status header: word 0 the flags, words 64.. one counter per column block
-// of the statistic pass (merge tickets / barrier counts, left at zero)
-constexpr size_t kStatusBytes = 4096;
+// Workspace header, zeroed by ttq_workspace_init and left at zero by every
+// call: word 0 the flags; words 64..1023 one counter per column block of the
+// statistic pass (merge tickets / barrier counts); bytes 4096..20479 one
+// arrival ticket per 128-row tile of the single-pass decode product.
+constexpr size_t kStatusBytes = 4096;           // the least workspace an entry point takes
+constexpr size_t kTicketsOffset = 4096;
+constexpr size_t kHeaderBytes = kTicketsOffset + 4 * static_cast<size_t>(kFusedDecodeMaxTiles);
 constexpr int64_t kMaxColumnBlocks = 960;       // tickets after the first 256 bytes
 constexpr int kPlanSMs = 148;                   // fixed so the layout is device-independent
 
@@ -57,6 +61,15 @@ bool scheme_bits_ok(ttq_qscheme scheme, int bits) {
 // 8-bit (FP8) codes are always materialised: no product reads them.
 bool materialize_w(int64_t dp, int64_t T, int bits) { return dp > 0 && (T > 256 || bits == 8); }
 
+// Whether ttq_linear_forward takes the single-pass decode product (W read
+// once, quantised and multiplied in one kernel, no codes written) for this
+// shape: bf16 layers with the asymmetric INT codes and at most 16 tokens.
+bool single_pass_decode(ttq_dtype dtype, ttq_qscheme scheme, int64_t d, int64_t dp, int64_t T,
+                        int bits, int group) {
+  return dtype == TTQ_BF16 && scheme == TTQ_QSCHEME_ASYMMETRIC &&
+         fused_decode_supported(dp, d, T, bits, group);
+}
+
 // Computes the workspace layout; false for an unsupported shape.
 bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
                  ttq_dtype dtype, ttq_workspace_layout* L) {
@@ -70,7 +83,7 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
   act_norm_plan(d, T, kPlanSMs, &splits, &rps);
   size_t off = 0;
   l.status = off;
-  off += kStatusBytes;
+  off += kHeaderBytes;
   l.D = off;
   off = align_up(off + 4 * static_cast<size_t>(d));
   l.D_rsqrt = off;
@@ -86,10 +99,26 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
     off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d / group) * 2);
   }
   l.ax_ld = 0;
+  l.ax_splits = 0;
   if (r > 0) {
     l.ax_ld = r;
     l.ax = off;
     off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(r) * 2);
+    const AxSplit sp = ax_split_plan(r, T, d, kPlanSMs);
+    l.ax_splits = sp.splits;
+    if (sp.splits > 1) {
+      l.axp = off;
+      off = align_up(off + static_cast<size_t>(sp.splits) * static_cast<size_t>(T) *
+                               static_cast<size_t>(r) * 4);
+    }
+  }
+  if (has_q && dtype == TTQ_BF16 && fused_decode_supported(dp, d, T, bits, group)) {
+    // the single-pass decode product: sqrt(D), its partial tiles and tickets
+    l.D_sqrt = off;
+    off = align_up(off + 4 * static_cast<size_t>(d));
+    l.ypart = off;
+    off = align_up(off + 4 * static_cast<size_t>(fused_decode_plan(dp, d, T).part_floats));
+    l.tickets = kTicketsOffset;
   }
   if (has_q) {
     l.xh = off;
@@ -204,6 +233,47 @@ ttq_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TTQ_OK : TTQ_E
 
 uint8_t* ws_at(void* ws, size_t off) { return static_cast<uint8_t*>(ws) + off; }
 
+// A X [T][r] bf16 into the workspace: the plain-operand mode of the GEMM
+// (M = r rows of A), split along K when its few output tiles would leave
+// most SMs idle (float32 partials, then a reduction in split order).
+ttq_status run_ax(const void* Ab, const void* Xb, int64_t d, int64_t T, int64_t r, void* ws,
+                  const ttq_workspace_layout& L, cudaStream_t stream, bool pdl) {
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  void* ax = ws_at(ws, L.ax);
+  const int bn = gemm_block_n(T);
+  GemmMaps m;
+  if (!encode_16bit(&m.a0, Ab, false, d, r, d, 128) || !encode_16bit(&m.b0, Xb, false, d, T, d, bn))
+    return TTQ_ERR_CUDA;
+  m.a1 = m.a0;
+  m.b1 = m.b0;
+  m.c0 = m.b0;
+  m.y = m.b0;
+  GemmArgs a;
+  a.bits = 0;
+  a.K = d;
+  a.M = r;
+  a.T = T;
+  a.K_tail = 0;
+  a.status = status;
+  const AxSplit sp = ax_split_plan(r, T, d, kPlanSMs);
+  if (sp.splits > 1 && L.axp != 0 && L.ax_splits == sp.splits) {
+    float* P = reinterpret_cast<float*>(ws_at(ws, L.axp));
+    a.Y = P;
+    a.ldy = r;
+    a.y_f32 = true;
+    a.k_splits = sp.splits;
+    a.kb_per_split = sp.kb_per_split;
+    a.split_stride = T * r;
+    ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, 128, stream, pdl));
+    if (st != TTQ_OK) return st;
+    return cuda_status(launch_ax_reduce(P, sp.splits, T, r, ax, L.ax_ld, stream, true));
+  }
+  a.Y = ax;
+  a.ldy = L.ax_ld;
+  a.y_f32 = false;
+  return cuda_status(launch_dequant_gemm(a, m, bn, 128, stream, pdl));
+}
+
 // Y = W_hat X (+ B (A X)) from quantised weights.  Xh is binary16
 // X D^(-1/2); Xb, Ab, Bb are bf16 X, A, B (used only when r > 0).
 ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_t* zeros,
@@ -214,27 +284,8 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   if (T == 0 || dp == 0) return TTQ_OK;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   void* ax = r > 0 ? ws_at(ws, L.ax) : nullptr;
-  const int bn = gemm_block_n(T);
   if (r > 0) {
-    // A X: the plain-operand mode of the same kernel, M = r rows of A.
-    GemmMaps m;
-    if (!encode_16bit(&m.a0, Ab, false, d, r, d, 128) || !encode_16bit(&m.b0, Xb, false, d, T, d, bn))
-      return TTQ_ERR_CUDA;
-    m.a1 = m.a0;
-    m.b1 = m.b0;
-    m.c0 = m.b0;
-    m.y = m.b0;
-    GemmArgs a;
-    a.bits = 0;
-    a.K = d;
-    a.M = r;
-    a.T = T;
-    a.K_tail = 0;
-    a.Y = ax;
-    a.ldy = L.ax_ld;
-    a.y_f32 = false;
-    a.status = status;
-    const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bn, 128, stream, pdl));
+    const ttq_status st = run_ax(Ab, Xb, d, T, r, ws, L, stream, pdl);
     if (st != TTQ_OK) return st;
     pdl = true;
   }
@@ -316,6 +367,46 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   return cuda_status(launch_dequant_gemm(a, m, bnm, bm, stream, pdl));
 }
 
+// Steps (2)-(3) in one pass over bf16 W (T <= 16): sqrt(D) in Dh, binary16
+// X D^(-1/2) in Xh; codes/scales/zeros stored when codes is non-null.
+ttq_status run_single_pass(const void* W, const float* Dh, const void* Xh, const void* Xb,
+                           const void* Ab, const void* Bb, int64_t d, int64_t dp, int64_t T,
+                           int64_t r, int bits, int group, uint32_t* codes, uint16_t* scales,
+                           uint16_t* zeros, void* Y, bool y_f32, void* ws,
+                           const ttq_workspace_layout& L, cudaStream_t stream, bool pdl) {
+  if (T == 0 || dp == 0) return TTQ_OK;
+  if (r > 0) {
+    const ttq_status st = run_ax(Ab, Xb, d, T, r, ws, L, stream, pdl);
+    if (st != TTQ_OK) return st;
+    pdl = true;
+  }
+  CUtensorMap tmW, tmX;
+  if (!encode_16bit(&tmW, W, false, d, dp, d, 128) ||
+      !encode_16bit(&tmX, Xh, true, d, T, d, T <= 8 ? 8 : 16))
+    return TTQ_ERR_CUDA;
+  FusedDecodeArgs a;
+  a.Dh = Dh;
+  a.K = d;
+  a.M = dp;
+  a.T = T;
+  a.bits = bits;
+  a.group = group;
+  a.Blr = Bb;
+  a.AX = r > 0 ? ws_at(ws, L.ax) : nullptr;
+  a.r = r;
+  a.ax_ld = L.ax_ld;
+  a.Y = Y;
+  a.ldy = dp;
+  a.y_f32 = y_f32;
+  a.codes = codes;
+  a.scales = scales;
+  a.zeros = zeros;
+  a.part = reinterpret_cast<float*>(ws_at(ws, L.ypart));
+  a.tickets = reinterpret_cast<uint32_t*>(ws_at(ws, L.tickets));
+  a.status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
+  return cuda_status(launch_fused_decode(a, tmW, tmX, stream, pdl));
+}
+
 // Step (1) and, when xh is non-null, the product's binary16 operand
 // X D^(-1/2) in xh: one fused cooperative kernel when every block's tile of
 // X fits in shared memory and the grid is resident at once, else the
@@ -324,7 +415,8 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
 // float32 X (or null).
 ttq_status run_statistic(const void* X, ttq_dtype dtype, int64_t d, int64_t T, float p,
                          float lambda, float alpha, const ttq_workspace_layout& L, void* ws,
-                         float* D, float* Dr, void* xh, void* xb, cudaStream_t s) {
+                         float* D, float* Dr, void* xh, void* xb, cudaStream_t s,
+                         float* Dh = nullptr) {
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   double* partial = reinterpret_cast<double*>(ws_at(ws, L.partial));
   const bool f32 = dtype == TTQ_F32;
@@ -335,12 +427,12 @@ ttq_status run_statistic(const void* X, ttq_dtype dtype, int64_t d, int64_t T, f
     const ttq_status st = cuda_status(launch_act_norm_scale(X, f32, d, T, p, lambda, alpha,
                                                             splits, rps, partial, status + 64, D,
                                                             Dr, xh, xb, status, device_sms(), s,
-                                                            &fused));
+                                                            &fused, Dh));
     if (st != TTQ_OK || fused) return st;
   }
   ttq_status st = cuda_status(launch_act_norm(X, f32, d, T, p, lambda, alpha, splits, rps,
                                               partial, status + 64, D, Dr, nullptr, xb, status,
-                                              s));
+                                              s, false, Dh));
   if (st != TTQ_OK || xh == nullptr) return st;
   return cuda_status(launch_scale_to_f16(X, dtype, Dr, xh, T, d, status, device_sms(), s, true));
 }
@@ -369,7 +461,8 @@ ttq_status ttq_workspace_get_layout(int64_t d, int64_t dp, int64_t T, int64_t r,
 ttq_status ttq_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (ws == nullptr || ws_bytes < kStatusBytes || (reinterpret_cast<uintptr_t>(ws) & 255u))
     return TTQ_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)));
+  const size_t n = ws_bytes < kHeaderBytes ? ws_bytes : kHeaderBytes;
+  return cuda_status(cudaMemsetAsync(ws, 0, n, static_cast<cudaStream_t>(stream)));
 }
 
 ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T, float p,
@@ -426,9 +519,13 @@ ttq_status ttq_act_norm_scale(const void* X, ttq_dtype dtype, int64_t d, int64_t
 }
 
 ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,
-                                      int64_t r, float p, int* kernels) {
+                                      int64_t r, float p, int bits, int group, ttq_qscheme scheme,
+                                      int* kernels) {
   if (kernels == nullptr || (dtype != TTQ_F32 && dtype != TTQ_BF16)) return TTQ_ERR_INVALID_ARG;
   if (d < 8 || d % 8 != 0 || dp < 0 || T < 0 || r < 0 || !(p >= 1.0f) || !std::isfinite(p))
+    return TTQ_ERR_INVALID_ARG;
+  if (scheme != TTQ_QSCHEME_ASYMMETRIC && scheme != TTQ_QSCHEME_SYMMETRIC &&
+      scheme != TTQ_QSCHEME_FP8_E4M3)
     return TTQ_ERR_INVALID_ARG;
   int64_t splits, rps;
   act_norm_plan(d, T, kPlanSMs, &splits, &rps);
@@ -436,13 +533,50 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
   int n = 1;  // statistic
   if (dp > 0) {
     if (!act_norm_scale_fused(f32, d, splits, rps, p, device_sms())) ++n;  // separate scaling
-    ++n;                                                                   // quantiser
-    if (T > 0) n += 1 + (r > 0 ? 1 + (f32 ? 2 : 0) : 0);  // product (+ A X, + bf16 A, B)
+    const bool one_pass = T > 0 && single_pass_decode(dtype, scheme, d, dp, T, bits, group);
+    if (!one_pass) ++n;                                                    // quantiser
+    if (T > 0) {
+      ++n;                                                                 // product
+      if (r > 0) {
+        n += 1 + (f32 ? 2 : 0);                                            // A X (+ bf16 A, B)
+        if (ax_split_plan(r, T, d, kPlanSMs).splits > 1) ++n;              // its split reduction
+      }
+    }
   }
   *kernels = n;
   return TTQ_OK;
 }
 
+ttq_status ttq_quantize_gemm(const void* W, const float* D, const uint16_t* Xs, const void* A,
+                             const void* B, const void* X, int64_t d, int64_t dp, int64_t T,
+                             int64_t r, int bits, int group, uint32_t* codes, uint16_t* scales,
+                             uint16_t* zeros, void* Y, ttq_dtype y_dtype, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
+  if (d < 8 || d % 8 != 0 || dp < 0 || T < 0 || r < 0) return TTQ_ERR_INVALID_ARG;
+  if (!valid_qparams(bits, group) || bits == 8 || d % group != 0) return TTQ_ERR_UNSUPPORTED;
+  const bool work = dp > 0 && T > 0;
+  if (work && !fused_decode_supported(dp, d, T, bits, group)) return TTQ_ERR_UNSUPPORTED;
+  ttq_workspace_layout L;
+  if (!make_layout(d, dp, T, r, bits, group, TTQ_BF16, &L)) return TTQ_ERR_INVALID_ARG;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
+  if (ws_bytes < L.total) return TTQ_ERR_WORKSPACE;
+  if (work && (W == nullptr || D == nullptr || Xs == nullptr || Y == nullptr))
+    return TTQ_ERR_INVALID_ARG;
+  if (r > 0 && (A == nullptr || B == nullptr || X == nullptr)) return TTQ_ERR_INVALID_ARG;
+  if ((codes == nullptr) != (scales == nullptr) || (codes == nullptr) != (zeros == nullptr))
+    return TTQ_ERR_INVALID_ARG;
+  const void* ptrs[] = {W, D, Xs, A, B, X, codes, scales, zeros, Y};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return TTQ_ERR_INVALID_ARG;
+  if (!work) return TTQ_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* Dh = reinterpret_cast<float*>(ws_at(ws, L.D_sqrt));
+  const ttq_status st = cuda_status(launch_sqrt_f32(D, Dh, d, s));
+  if (st != TTQ_OK) return st;
+  return run_single_pass(W, Dh, Xs, X, A, B, d, dp, T, r, bits, group, codes, scales, zeros, Y,
+                         y_dtype == TTQ_F32, ws, L, s, true);
+}
 
 ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
                                   const float* D, int bits, int group, ttq_qscheme scheme,
@@ -613,8 +747,16 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, co
 
   // (1) D and D^{-1/2} (a float32 X is also written as bf16 for the
   // low-rank product), then the product's B operand X D^{-1/2} in binary16
-  ttq_status st = run_statistic(X, dtype, d, T, p, lambda, alpha, L, ws, D, Dr, xh, xb, s);
+  const bool one_pass = T > 0 && single_pass_decode(dtype, scheme, d, dp, T, bits, group);
+  float* Dh = one_pass ? reinterpret_cast<float*>(ws_at(ws, L.D_sqrt)) : nullptr;
+  ttq_status st = run_statistic(X, dtype, d, T, p, lambda, alpha, L, ws, D, Dr, xh, xb, s, Dh);
   if (st != TTQ_OK || dp == 0) return st;
+  if (one_pass) {
+    // (2)-(3) at a few tokens: W read once, quantised and multiplied in one
+    // kernel; no codes are written
+    return run_single_pass(W, Dh, xh, X, A, B, d, dp, T, r, bits, group, nullptr, nullptr,
+                           nullptr, Y, y_dtype == TTQ_F32, ws, L, s, true);
+  }
 
   // (2) codes, scales, zeros of Q[W D^{1/2}]
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));

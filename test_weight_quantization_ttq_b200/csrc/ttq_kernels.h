@@ -37,11 +37,16 @@ void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* 
 // `counters` ceil(d/256) uint32 that start (and are left) at zero.  When
 // xh is non-null X is also written out as binary16 [T][d] (flag X_RANGE if
 // some |x| > 65504); when xb is non-null a float32 X is also written out as
-// bf16 [T][d].
+// bf16 [T][d].  When Dh is non-null it also receives sqrtf(D) (binary32,
+// correctly rounded: the quantiser's h).
 cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                             float lambda, float alpha, int64_t splits, int64_t rows_per_split,
                             double* partial, uint32_t* counters, float* D, float* Dr, void* xh,
-                            void* xb, uint32_t* status, cudaStream_t stream, bool pdl = false);
+                            void* xb, uint32_t* status, cudaStream_t stream, bool pdl = false,
+                            float* Dh = nullptr);
+
+// h = sqrtf(D) (binary32, correctly rounded) for d channels.
+cudaError_t launch_sqrt_f32(const float* D, float* h, int64_t d, cudaStream_t stream);
 
 // Whether launch_act_norm_scale would run (on the current device).
 bool act_norm_scale_fused(bool x_f32, int64_t d, int64_t splits, int64_t rows_per_split, float p,
@@ -60,7 +65,7 @@ cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t 
                                   int64_t rows_per_split, double* partial,
                                   uint32_t* counters, float* D, float* Dr, void* xh,
                                   void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
-                                  bool* launched);
+                                  bool* launched, float* Dh = nullptr);
 
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null); with wq
 // non-null also the dequantised weight s (q - z) as binary16 [dp][d].
@@ -105,6 +110,12 @@ struct GemmArgs {
   bool a_f16 = false;      // plain mode: the A operand (maps.a0) is binary16, not bf16
   bool codes_tma = false;  // codes tile loaded by TMA (maps.c0); else per-thread loads
   bool y_tma = false;      // bf16 Y stored by TMA (maps.y, box block_m x block_n)
+  // split-K (plain mode without a low-rank tail only): split z of k_splits
+  // covers K blocks [z * kb_per_split, (z + 1) * kb_per_split) and writes
+  // its float32 partial product to Y + z * split_stride (y_f32 must be set)
+  int k_splits = 1;
+  int kb_per_split = 0;
+  int64_t split_stride = 0;
 };
 
 struct GemmMaps {
@@ -147,6 +158,44 @@ DecodeMapShape decode_map_shape(int bits, int T);
 cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
                                const CUtensorMap& tmX, cudaStream_t stream, bool pdl = false);
 
+// Steps (2)-(3) in one pass over W for T <= 16 tokens: quantise bf16 W
+// [M][K] with sqrt(D) (Dh), multiply by binary16 X' [T][K] (tmX) on
+// warp-level MMAs, add B (A X) (bf16, when r > 0) and store Y [T][ldy];
+// codes, scales and zeros (all three or none) are stored as the quantiser
+// stores them.  K a multiple of 128, group 32, 64 or 128, bits 2..4.
+// Persistent grid of fused_decode_plan().grid CTAs over row tiles of 128;
+// `part` holds plan.part_floats floats, `tickets` plan.row_tiles uint32
+// that are zero before and after the call.  tmW: bf16 W [M][K], box 64 x
+// 128, 128-byte swizzle; tmX: binary16 X' [T][K], box 64 x (T <= 8 ? 8 :
+// 16), 128-byte swizzle.
+constexpr int kFusedDecodePlanSMs = 148;     // fixed so the layout is device-independent
+constexpr int64_t kFusedDecodeMaxTiles = 4096;
+struct FusedDecodePlan {
+  int grid;
+  int64_t row_tiles, units, part_floats;
+};
+FusedDecodePlan fused_decode_plan(int64_t dp, int64_t d, int64_t T);
+bool fused_decode_supported(int64_t dp, int64_t d, int64_t T, int bits, int group);
+struct FusedDecodeArgs {
+  const float* Dh = nullptr;
+  int64_t K = 0, M = 0, T = 0;
+  int bits = 4, group = 128;
+  const void* Blr = nullptr;   // bf16 [M][r]
+  const void* AX = nullptr;    // bf16 [T][ax_ld]
+  int64_t r = 0, ax_ld = 0;
+  void* Y = nullptr;
+  int64_t ldy = 0;
+  bool y_f32 = false;
+  uint32_t* codes = nullptr;
+  uint16_t* scales = nullptr;
+  uint16_t* zeros = nullptr;
+  float* part = nullptr;
+  uint32_t* tickets = nullptr;
+  uint32_t* status = nullptr;
+};
+cudaError_t launch_fused_decode(const FusedDecodeArgs& a, const CUtensorMap& tmW,
+                                const CUtensorMap& tmX, cudaStream_t stream, bool pdl = false);
+
 // Step (2) with FP8 (E4M3) codes: one byte per weight (4 per word), the
 // symmetric per-group scale binary16 round-up(max|x| / 448), zeros +0;
 // with wq also the binary16 s * e4m3(code).
@@ -166,6 +215,20 @@ size_t lowrank_small_smem(int l, bool eig);
 cudaError_t launch_lowrank_init(const void* W, bool w_bf16, int64_t dp, int64_t d, int64_t r, int64_t l,
                                 int power_iters, const float* Omega, void* Bout, void* Aout, void* Wres,
                                 void* ws, int num_sms, cudaStream_t stream);
+
+// Split-K plan of the low-rank product A X (M = r rows of A, T tokens, K =
+// d): the number of K splits that brings its few output tiles up to about
+// one wave on num_sms SMs with at least 4 K blocks of 64 per split (1: no
+// split), and the K blocks each split covers.
+struct AxSplit {
+  int splits, kb_per_split;
+};
+AxSplit ax_split_plan(int64_t r, int64_t T, int64_t d, int num_sms);
+
+// AX [T][ax_ld] bf16 = the sum over the splits, in split order, of the
+// float32 partials P [splits][T][r] (one rounding at the end).
+cudaError_t launch_ax_reduce(const float* P, int splits, int64_t T, int64_t r, void* AX,
+                             int64_t ax_ld, cudaStream_t stream, bool pdl);
 
 // Words per row of the code tile one K block of 64 channels needs.
 int gemm_code_tile_words(int bits);

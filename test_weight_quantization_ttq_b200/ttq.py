@@ -47,7 +47,8 @@ _SZ = ctypes.c_size_t
 class WorkspaceLayout(ctypes.Structure):
     _fields_ = [("status", _SZ), ("D", _SZ), ("D_rsqrt", _SZ), ("partial", _SZ), ("codes", _SZ),
                 ("scales", _SZ), ("zeros", _SZ), ("ax", _SZ), ("xh", _SZ), ("xb", _SZ), ("ab", _SZ),
-                ("wq", _SZ), ("total", _SZ), ("splits", _I64), ("ax_ld", _I64)]
+                ("wq", _SZ), ("total", _SZ), ("splits", _I64), ("ax_ld", _I64), ("axp", _SZ),
+                ("D_sqrt", _SZ), ("ypart", _SZ), ("tickets", _SZ), ("ax_splits", _I64)]
 
 
 SIGNATURES = {
@@ -71,7 +72,11 @@ SIGNATURES = {
                                 _P, _INT, _P, _SZ, _P]),
     "ttq_linear_forward": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT, _INT,
                                   _P, _INT, _P, _SZ, _P]),
-    "ttq_linear_forward_kernels": (_INT, [_INT, _I64, _I64, _I64, _I64, _F, ctypes.POINTER(ctypes.c_int)]),
+    "ttq_linear_forward_kernels": (_INT, [_INT, _I64, _I64, _I64, _I64, _F, _INT, _INT, _INT,
+                                          ctypes.POINTER(ctypes.c_int)]),
+    "ttq_testing_wait_timeout": (_INT, [_INT, ctypes.c_uint64, _INT, _P, _SZ, _P]),
+    "ttq_quantize_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _INT, _INT, _P, _P, _P,
+                                 _P, _INT, _P, _SZ, _P]),
     "ttq_get_status": (_INT, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "ttq_status_from_flags": (_INT, [ctypes.c_uint32]),
     "ttq_lowrank_workspace_size": (_SZ, [_I64, _I64, _I64, _I64]),
@@ -303,11 +308,12 @@ def ttq_act_norm_scale(X, p, lam, alpha, ws=None, D=None, D_rsqrt=None, Xs=None,
     return D, D_rsqrt, Xs
 
 
-def ttq_linear_forward_kernels(d, dp, T, r=0, p=2.0, dtype=TTQ_BF16) -> int:
-    """Kernels one ttq_linear_forward call of these sizes enqueues on the
-    current device."""
+def ttq_linear_forward_kernels(d, dp, T, r=0, p=2.0, dtype=TTQ_BF16, bits=4, group=128,
+                               scheme=TTQ_QSCHEME_ASYMMETRIC) -> int:
+    """Kernels one ttq_linear_forward(_ex) call of these sizes and this code
+    scheme enqueues on the current device."""
     n = ctypes.c_int(0)
-    _check(lib().ttq_linear_forward_kernels(dtype, d, dp, T, r, p, ctypes.byref(n)),
+    _check(lib().ttq_linear_forward_kernels(dtype, d, dp, T, r, p, bits, group, scheme, ctypes.byref(n)),
            "ttq_linear_forward_kernels")
     return n.value
 
@@ -457,6 +463,55 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
                                   d, dp, T, r, bits, group, _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"),
                                   _nbytes(ws), _stream(stream)),
            "ttq_dequant_gemm")
+    return Y
+
+
+TTQ_TESTING_WAIT_MBARRIER = 0
+TTQ_TESTING_WAIT_GRID_BARRIER = 1
+
+
+def ttq_testing_wait_timeout(kind, limit_ns, blocks, ws, stream=None) -> None:
+    """Test hook: `blocks` blocks each make one wait of `kind` that cannot
+    complete, with a limit of limit_ns; they set TTQ_FLAG_TIMEOUT in ws."""
+    _check(lib().ttq_testing_wait_timeout(kind, limit_ns, blocks, _dev(ws, "ws"), _nbytes(ws),
+                                          _stream(stream)), "ttq_testing_wait_timeout")
+
+
+def ttq_quantize_gemm(W, D, Xs, A, B, X, bits, group, ws=None, Y=None, y_dtype=torch.bfloat16,
+                      codes=None, scales=None, zeros=None, stream=None):
+    """Steps (2)-(3) in one pass over bf16 W [d'][d] for T <= 16 tokens:
+    Y [T][d'] = Q[W D^{1/2}] Xs (+ B (A X)), Xs the binary16 X D^{-1/2}
+    [T][d]; A [r][d], B [d'][r], X [T][d] bf16 for the low-rank term.
+    codes/scales/zeros: None, or all three buffers to receive the codes."""
+    _matrix(Xs, "Xs", dtypes=_F16)
+    T, d = Xs.shape
+    _matrix(W, "W", cols=d, dtypes=(torch.bfloat16,))
+    dp = W.shape[0]
+    _vector(D, "D", d)
+    r = _lowrank_pair(A, B)
+    _matrix(A, "A", r, d, (torch.bfloat16,))
+    _matrix(B, "B", dp, r, (torch.bfloat16,))
+    if r > 0:
+        _matrix(X, "X", T, d, (torch.bfloat16,))
+    given = [t is not None for t in (codes, scales, zeros)]
+    if any(given) and not all(given):
+        raise TTQError(TTQ_ERR_INVALID_ARG, "ttq_quantize_gemm: codes, scales and zeros go together")
+    if all(given):
+        cb, sb = _qsizes(d, bits, group, "ttq_quantize_gemm")
+        _room(codes, "codes", dp * cb)
+        _room(scales, "scales", dp * sb)
+        _room(zeros, "zeros", dp * sb)
+    _matrix(Y, "Y", T, dp, _FLOAT_IN)
+    if ws is None:
+        ws = new_workspace(d, dp, T, r, bits, group, TTQ_BF16, W.device, stream)
+    if Y is None:
+        Y = torch.empty((T, dp), dtype=y_dtype, device=W.device)
+    _check(lib().ttq_quantize_gemm(_dev(W, "W"), _dev(D, "D"), _dev(Xs, "Xs"), _dev(A, "A"), _dev(B, "B"),
+                                   _dev(X if r > 0 else None, "X"), d, dp, T, r, bits, group,
+                                   _dev(codes, "codes"), _dev(scales, "scales"), _dev(zeros, "zeros"),
+                                   _dev(Y, "Y"), _dtype_code(Y), _dev(ws, "ws"), _nbytes(ws),
+                                   _stream(stream)),
+           "ttq_quantize_gemm")
     return Y
 
 

@@ -118,14 +118,20 @@ def test_forward_kernel_count_matches_launches():
     cases = [(synth.C2.with_(dp=512), 3, True),
              (_spec("wide_two_kernel", d=8192, dp=64, T=2048), 4, False),
              (_spec("f32_lowrank", d=448, dp=96, T=77, dtype="f32", r=16), 6, True),
-             (_spec("no_tokens", d=512, dp=64, T=0), 2, True)]
+             (_spec("no_tokens", d=512, dp=64, T=0), 2, True),
+             # a few tokens: statistic, then the single-pass product
+             (_spec("decode", d=1024, dp=640, T=1, bits=4, group=128), 2, True),
+             # with a low-rank pair whose A X is split along d: A X, its
+             # reduction, then the single-pass product
+             (_spec("decode_lowrank", d=8192, dp=256, T=3, bits=2, group=64, r=64), 4, True)]
     for spec, expected, fused in cases:
         data = P.inputs(spec)
         X, W = P.to_dev(data["X"], spec.dtype), P.to_dev(data["W"], spec.dtype)
         A = P.to_dev(data["A"], spec.dtype) if spec.r else None
         B = P.to_dev(data["B"], spec.dtype) if spec.r else None
         ws = ttq.new_workspace(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, _dt(spec))
-        n = ttq.ttq_linear_forward_kernels(spec.d, spec.dp, spec.T, spec.r, spec.p, _dt(spec))
+        n = ttq.ttq_linear_forward_kernels(spec.d, spec.dp, spec.T, spec.r, spec.p, _dt(spec),
+                                           spec.bits, spec.group)
         assert n == expected, spec.name
         torch.cuda.synchronize()
         with profile(activities=[ProfilerActivity.CUDA]) as prof:
