@@ -87,14 +87,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // false) after kWaitLimitNs or as soon as *abort becomes non-zero.
 // The clock is read only every 64th failed try (try_wait itself suspends
 // the thread for a while between polls).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// limit_ns: the time limit (kWaitLimitNs unless a test asks for less).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t n = 1;; ++n) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((n & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
 }
@@ -106,11 +108,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // that publishes the block's earlier global writes), waits with acquire
 // loads until all n have arrived, and adds 1 when it leaves; the block that
 // brings it to 2n sets it back to zero.  A wait
-// longer than kWaitLimitNs sets TTQ_FLAG_TIMEOUT and lets the block go on
-// (its later results are then not valid); the result is false in that case.
+// longer than limit_ns sets TTQ_FLAG_TIMEOUT and lets the block go on (its
+// later results are then not valid, and the count is left off zero until
+// the workspace is re-initialised); the result is false in that case.
 // `ok_smem` is a shared int used to broadcast the outcome to the block.
 __device__ __forceinline__ bool group_barrier(uint32_t* count, uint32_t n, uint32_t* status,
-                                              int* ok_smem) {
+                                              int* ok_smem, uint64_t limit_ns = kWaitLimitNs) {
   __syncthreads();
   if (threadIdx.x == 0) {
     int ok = 1;
@@ -122,7 +125,7 @@ __device__ __forceinline__ bool group_barrier(uint32_t* count, uint32_t n, uint3
       uint32_t cur;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(count) : "memory");
       if (cur >= n) break;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         set_flag(status, TTQ_FLAG_TIMEOUT);
         ok = 0;
         break;

@@ -1,5 +1,5 @@
 """The C ABI library on the CPU: it loads, exports every entry point that
-include/ttq.h declares, and its host-side logic (workspace layout, argument
+include/*.h declare, and its host-side logic (workspace layout, argument
 checks that reject before any device work) behaves as documented.  No
 compute call is made here."""
 import os
@@ -10,7 +10,12 @@ import pytest
 from test_weight_quantization_ttq_b200 import build as ttq_build
 from test_weight_quantization_ttq_b200 import ttq
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "ttq.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+HEADERS = sorted(os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h"))
+
+
+def _header_text():
+    return "".join(open(h).read() for h in HEADERS)
 
 
 @pytest.fixture(scope="module")
@@ -20,7 +25,7 @@ def L():
 
 
 def declared_functions():
-    text = open(HEADER).read()
+    text = _header_text()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(ttq_[a-z_0-9]+)\s*\(", text)))
 
@@ -164,8 +169,11 @@ def test_fp8_scheme_rules_before_device_work(L):
     assert qw(16, 1, 4, 64, None, 4, 64, FP8, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
     assert qw(16, 1, 4, 64, None, 8, 48, FP8, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
     assert qw(16, 1, 4, 64, None, 8, 64, 3, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
-    # no product reads 8-bit codes
-    st = L.ttq_dequant_gemm(16, 16, 16, None, 16, None, None, 1, 64, 64, 4, 0, 8, 64, 16, 1, 256, 1 << 30, None)
+    # 8-bit codes are read by the decode product only: at most 16 tokens,
+    # d a multiple of 64
+    st = L.ttq_dequant_gemm(16, 16, 16, None, 16, None, None, 1, 64, 64, 17, 0, 8, 64, 16, 1, 256, 1 << 30, None)
+    assert st == ttq.TTQ_ERR_UNSUPPORTED
+    st = L.ttq_dequant_gemm(16, 16, 16, None, 16, None, None, 1, 96, 64, 4, 0, 8, 32, 16, 1, 256, 1 << 30, None)
     assert st == ttq.TTQ_ERR_UNSUPPORTED
     # the default (asymmetric) forward refuses 8 bits; the FP8 forward checks its workspace
     st = L.ttq_linear_forward(16, 16, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 8, 64, 16, 1, 256, 1 << 30, None)
@@ -173,8 +181,10 @@ def test_fp8_scheme_rules_before_device_work(L):
     st = L.ttq_linear_forward_ex(16, 16, None, None, 1, 64, 64, 4, 0, 2.0, 0.0, 0.5, 8, 64, FP8, 16, 1, 256, 64,
                                  None)
     assert st == ttq.TTQ_ERR_WORKSPACE
-    # FP8 layouts always hold the binary16 W_hat; INT layouts only for T > 256
-    for T, bits, present in [(4, 8, True), (1, 8, True), (4, 4, False), (300, 4, True)]:
+    # FP8 layouts hold the binary16 W_hat beyond the decode product's reach
+    # (T > 16); INT layouts only for T > 256
+    for T, bits, present in [(4, 8, False), (1, 8, False), (16, 8, False), (17, 8, True),
+                             (4, 4, False), (300, 4, True)]:
         lay = ttq.WorkspaceLayout()
         assert L.ttq_workspace_get_layout(256, 64, T, 0, bits, 64, 1, lay) == ttq.TTQ_OK
         assert (lay.wq != 0) == present, (T, bits)
@@ -182,7 +192,7 @@ def test_fp8_scheme_rules_before_device_work(L):
 
 def declared_arity():
     """Parameter count of every ttq_* function declared in the header."""
-    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"/\*.*?\*/", "", _header_text(), flags=re.S)
     out = {}
     for m in re.finditer(r"\b(ttq_[a-z_0-9]+)\s*\(([^;{]*?)\)\s*;", text):
         params = m.group(2).strip()
