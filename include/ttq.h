@@ -96,9 +96,11 @@ typedef enum ttq_dtype {
  * 448) nearest to the binary32 product x * (1/s), ties to even, saturating,
  * with s = binary16 round-up of max|x| / 448 per group; one byte per weight
  * (four per word, weight i in bits 8 (i mod 4) of word i / 4), zeros +0,
- * reconstruction scales * e4m3(code).  The forward always materialises the
- * binary16 s * e4m3(q) for this scheme; ttq_dequant_gemm does not take
- * 8-bit codes.  INT schemes take bits 2..4. */
+ * reconstruction scales * e4m3(code).  For T <= 16 tokens and d a
+ * multiple of 64 the forward's product reads the 8-bit codes themselves
+ * (E4M3 pairs converted to binary16 in registers), and ttq_dequant_gemm
+ * takes them there; otherwise the forward materialises the binary16
+ * s * e4m3(q) and multiplies by that.  INT schemes take bits 2..4. */
 typedef enum ttq_qscheme {
   TTQ_QSCHEME_ASYMMETRIC = 0,
   TTQ_QSCHEME_SYMMETRIC = 1,
@@ -133,8 +135,9 @@ typedef struct ttq_workspace_layout {
   size_t xb;      /* bf16 [T][d] copy of float32 X (TTQ_F32, r > 0) */
   size_t ab;      /* bf16 copies of float32 A and B (TTQ_F32, r > 0) */
   size_t wq;      /* binary16 [d'][d] s (q - z) (s e4m3(q) for 8-bit codes)
-                     that ttq_linear_forward's product reads when T > 256 or
-                     bits == 8 (0: not in this layout) */
+                     that ttq_linear_forward's product reads when T > 256, or
+                     for 8-bit codes beyond the decode product's reach
+                     (T > 16 or d % 64 != 0); 0: not in this layout */
   size_t total;
   int64_t splits; /* number of token splits of the statistic pass */
   int64_t ax_ld;  /* row stride (elements) of A X                 */
@@ -290,7 +293,9 @@ ttq_status ttq_scale_activations(const void* X, ttq_dtype dtype, int64_t d, int6
  * holds X D^{-1/2} when D_rsqrt is NULL (as written by
  * ttq_scale_activations): then only the product runs; it needs r == 0.
  * Y [T][dp] is written in y_dtype (TTQ_F32 or TTQ_BF16): TTQ_F32 keeps the
- * fp32 accumulator as is, TTQ_BF16 rounds it to nearest-even once. */
+ * fp32 accumulator as is, TTQ_BF16 rounds it to nearest-even once.
+ * bits = 8 takes FP8 (E4M3) codes (TTQ_QSCHEME_FP8_E4M3, zeros ignored)
+ * for T <= 16 and d a multiple of 64 only (else TTQ_ERR_UNSUPPORTED). */
 ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
                             const uint16_t* zeros, const float* D_rsqrt,
                             const void* X, const void* A, const void* B,

@@ -263,26 +263,7 @@ __global__ void __launch_bounds__(kFdThreads, 2) ttq_fused_decode_kernel(
   const int64_t u_begin = U * blockIdx.x / NC;
   const int64_t u_end = U * (blockIdx.x + 1) / NC;
 
-  for (int k = threadIdx.x; k < 1024; k += kFdThreads)
-    rcp_sig[k] = __fdiv_rn(1.0f, 1.0f + static_cast<float>(k) * 0.0009765625f);
-  if (threadIdx.x == 0) {
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kFdWarps);
-    }
-    abort_s = 0;
-    last_s = 0;
-    fence_barrier_init();
-    prefetch_tensormap(&tmW);
-    prefetch_tensormap(&tmX);
-  }
-  __syncthreads();
-  allow_dependents_launch();
-
   const bool producer = threadIdx.x == 0;
-  // the weight does not depend on the kernels before this one: the first
-  // stages' W boxes are requested before waiting for them
   auto issue_w = [&](int64_t u, int s) {
     const int64_t tile = u / a.nsl;
     const int32_t k0 = static_cast<int32_t>((u - tile * a.nsl) * kFdK);
@@ -302,8 +283,27 @@ __global__ void __launch_bounds__(kFdThreads, 2) ttq_fused_decode_kernel(
   };
   const int64_t n_units = u_end - u_begin;
   const int first_issue = static_cast<int>(n_units < kStages ? n_units : kStages);
-  if (producer)
+  if (producer) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kFdWarps);
+    }
+    abort_s = 0;
+    last_s = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmW);
+    prefetch_tensormap(&tmX);
+    // the weight does not depend on the kernels before this one: the first
+    // stages' W boxes are requested before anything else
     for (int i = 0; i < first_issue; ++i) issue_w(u_begin + i, i);
+  }
+  // binary32 1 / (1 + k/1024) for the binary16 significands (1/s of a
+  // normal binary16 s = m 2^e is this times 2^-e, exactly)
+  for (int k = threadIdx.x; k < 1024; k += kFdThreads)
+    rcp_sig[k] = __fdiv_rn(1.0f, 1.0f + static_cast<float>(k) * 0.0009765625f);
+  __syncthreads();
+  allow_dependents_launch();
   grid_dependency_wait();
   if (producer)
     for (int i = 0; i < first_issue; ++i) issue_xh(u_begin + i, i);

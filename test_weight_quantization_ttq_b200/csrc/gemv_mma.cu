@@ -29,7 +29,10 @@
 // matching pairs of X' are put together with byte permutes.  The X' tiles
 // are 128-byte swizzled, which makes their reads free of bank conflicts.
 //
-// The operand is (m + q) - (m + z) = q - z, exact in binary16.  For up to 8
+// The operand is (m + q) - (m + z) = q - z, exact in binary16; FP8 (E4M3)
+// codes (one byte per channel) convert to their binary16 values exactly and
+// need no zero point (the blog.lo0.es comparison with FP8: the activation-
+// aware scale feeding an FP8 code).  For up to 8
 // tokens with quantisation groups that span whole stages (group >= 128) s
 // multiplies the fp32 sum of a stage once per row; otherwise the operand is
 // the binary16 s (q - z) (one rounding), as in the large-tile product.
@@ -42,6 +45,8 @@
 // Every barrier wait is bounded (1 s); a wait that gives up sets
 // TTQ_FLAG_TIMEOUT, stops the CTA's other warps, lets the copies in flight
 // land, and the CTA returns without storing Y.
+
+#include <cuda_fp8.h>
 
 #include <atomic>
 
@@ -72,15 +77,15 @@ constexpr uint32_t code_tile_bytes() { return kRowsPerCta * kStageK * BITS / 8; 
 // X' of a stage: [unit][8 NTT tokens][64 channels], 128-byte swizzled
 template <int NTT>
 constexpr uint32_t xh_tile_bytes() { return kUnits * 8u * NTT * 128u; }
-template <int NTT>
-constexpr int num_stages() { return NTT == 1 ? 4 : 3; }
+template <int BITS, int NTT>
+constexpr int num_stages() { return BITS == 8 ? 2 : (NTT == 1 ? 4 : 3); }
 template <int BITS, int NTT>
 constexpr uint32_t stage_bytes() {
   return (xh_tile_bytes<NTT>() + code_tile_bytes<BITS>() + 1023u) & ~1023u;
 }
 template <int BITS, int NTT>
 constexpr size_t decode_smem_bytes() {
-  return static_cast<size_t>(num_stages<NTT>()) * stage_bytes<BITS, NTT>() + 1024;
+  return static_cast<size_t>(num_stages<BITS, NTT>()) * stage_bytes<BITS, NTT>() + 1024;
 }
 
 __device__ __forceinline__ void mma_m16n8k16_f16(float (&c)[4], const uint32_t (&a)[4],
@@ -144,13 +149,33 @@ __device__ __forceinline__ constexpr uint32_t kind_magic(int k) {
                    : (k == 0 ? 0x6400u : 0x5400u);
 }
 
+// Two E4M3 codes (low 16 bits of v) as a binary16 pair: exact, every E4M3
+// value is a binary16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_h2(uint32_t v) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
 // (m + q) pairs P[0..7] of the lane's 16 channels of unit u of its piece,
 // for one row (row_addr: the row's first byte in the piece).  INT4: P[i] =
 // channels (i, i + 4), P[4 + i] = (8 + i, 12 + i); INT2: P[i] = (i, i + 8);
-// INT3: P[i] = (2i, 2i + 1).
+// INT3: P[i] = (2i, 2i + 1); 8-bit E4M3 codes: the binary16 values of
+// channels (2i, 2i + 1) themselves (zero point 0).
+
 template <int BITS>
 __device__ __forceinline__ void code_pairs(uint32_t row_addr, int u, int c, uint32_t (&P)[8]) {
-  if (BITS == 4) {
+  if (BITS == 8) {
+    // E4M3 codes, one byte per channel in channel order: the lane's 16
+    // channels are 16 bytes, and each byte pair converts to the binary16
+    // pair (2i, 2i + 1) exactly (every E4M3 value is a binary16 value)
+    const uint4 w = lds128(row_addr + 64 * u + 16 * c);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      P[2 * k] = e4m3x2_to_h2(ws[k]);
+      P[2 * k + 1] = e4m3x2_to_h2(ws[k] >> 16);
+    }
+  } else if (BITS == 4) {
     const uint2 w = lds64(row_addr + 32 * u + 8 * c);
     const uint32_t lo8 = w.x >> 8, hi8 = w.y >> 8;
     P[0] = (w.x & 0x000F000Fu) | 0x64006400u;   // channels 0, 4
@@ -217,7 +242,7 @@ __global__ void __launch_bounds__(32 * (1 + kConsumers), 2) ttq_decode_kernel(
     int T, int group_shift, const __nv_bfloat16* __restrict__ Blr,
     const __nv_bfloat16* __restrict__ AX, int r, int ax_ld, void* __restrict__ Y, int ldy,
     int y_f32, uint32_t* status) {
-  constexpr int kStages = num_stages<NTT>();
+  constexpr int kStages = num_stages<BITS, NTT>();
   extern __shared__ uint8_t dsm[];
   __shared__ __align__(8) uint64_t full[kStages];
   __shared__ __align__(8) uint64_t empty[kStages];
@@ -390,7 +415,8 @@ __global__ void __launch_bounds__(32 * (1 + kConsumers), 2) ttq_decode_kernel(
           code_pairs<BITS>(prow + 8u * i * kPieceRow, h, c, P[i]);
 #pragma unroll
           for (int p = 0; p < 8; ++p) {
-            const __half2 x = __hsub2(bits_h2(P[i][p]), bits_h2(zc[i][pair_kind<BITS>(p)]));
+            const __half2 x = BITS == 8 ? bits_h2(P[i][p])
+                                        : __hsub2(bits_h2(P[i][p]), bits_h2(zc[i][pair_kind<BITS>(p)]));
             P[i][p] = PS ? h2_bits(x) : h2_bits(__hmul2(x, bits_h2(s2[i])));
           }
         }
@@ -582,6 +608,7 @@ cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
     case 2: return launch_decode_bits<2>(tmC, tmX, a, gs, stream, pdl);
     case 3: return launch_decode_bits<3>(tmC, tmX, a, gs, stream, pdl);
     case 4: return launch_decode_bits<4>(tmC, tmX, a, gs, stream, pdl);
+    case 8: return launch_decode_bits<8>(tmC, tmX, a, gs, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

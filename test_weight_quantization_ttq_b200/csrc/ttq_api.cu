@@ -59,7 +59,10 @@ bool scheme_bits_ok(ttq_qscheme scheme, int bits) {
 // dequantising inside the product would repeat the work once per tile)
 // instead of dequantising the codes inside the product.
 // 8-bit (FP8) codes are always materialised: no product reads them.
-bool materialize_w(int64_t dp, int64_t T, int bits) { return dp > 0 && (T > 256 || bits == 8); }
+bool decode_reads_fp8(int64_t d, int64_t T) { return T <= 16 && d % 64 == 0; }
+bool materialize_w(int64_t dp, int64_t T, int bits, int64_t d) {
+  return dp > 0 && (T > 256 || (bits == 8 && !decode_reads_fp8(d, T)));
+}
 
 // Whether ttq_linear_forward takes the single-pass decode product (W read
 // once, quantised and multiplied in one kernel, no codes written) for this
@@ -130,7 +133,7 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
     l.ab = off;
     off = align_up(off + (static_cast<size_t>(r) * d + static_cast<size_t>(dp) * r) * 2);
   }
-  if (has_q && materialize_w(dp, T, bits)) {
+  if (has_q && materialize_w(dp, T, bits, d)) {
     l.wq = off;
     off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d) * 2);
   }
@@ -323,6 +326,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
       return cuda_status(launch_decode_gemm(a, tmC, tmX, stream, pdl));
     }
   }
+  if (!wq && bits == 8) return TTQ_ERR_UNSUPPORTED;  // no other product reads 8-bit codes
   // wq: the product reads the materialised binary16 s (q - z) by TMA
   int bm = 128, bnm = 16;
   gemm_tile_shape(wq ? 0 : bits, dp, T, device_sms(), &bm, &bnm);
@@ -661,8 +665,9 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales, const
                             int bits, int group, void* Y, ttq_dtype y_dtype, void* ws,
                             size_t ws_bytes, void* stream) {
   if (y_dtype != TTQ_F32 && y_dtype != TTQ_BF16) return TTQ_ERR_INVALID_ARG;
-  if (bits >= 1 && bits <= 8 && group >= 1 && (!valid_qparams(bits, group) || bits == 8))
-    return TTQ_ERR_UNSUPPORTED;   // no product reads 8-bit (FP8) codes
+  if (bits >= 1 && bits <= 8 && group >= 1 &&
+      (!valid_qparams(bits, group) || (bits == 8 && !decode_reads_fp8(d, T))))
+    return TTQ_ERR_UNSUPPORTED;   // 8-bit (FP8) codes: only the decode product reads them
   ttq_workspace_layout L;
   if (!make_layout(d, dp, T, r, bits, group, dtype, &L)) return TTQ_ERR_INVALID_ARG;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
@@ -762,7 +767,7 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, co
   uint32_t* codes = reinterpret_cast<uint32_t*>(ws_at(ws, L.codes));
   uint16_t* scales = reinterpret_cast<uint16_t*>(ws_at(ws, L.scales));
   uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
-  void* wq = materialize_w(dp, T, bits) ? ws_at(ws, L.wq) : nullptr;
+  void* wq = materialize_w(dp, T, bits, d) ? ws_at(ws, L.wq) : nullptr;
   st = cuda_status(scheme == TTQ_QSCHEME_FP8_E4M3
                        ? launch_qdq_fp8(W, f32, dp, d, D, group, codes, scales, zeros, status,
                                         device_sms(), s, true, wq)
