@@ -826,6 +826,8 @@ def run_table(args):
     points = [synth.C1, synth.C2, synth.C3_GATE, synth.C3_UP, synth.C3_DOWN]
     points += [synth.C4.with_(T=t) for t in synth.C4_TOKENS]
     points += [synth.C5.with_(T=t, p=2.0, alpha=0.5) for t in synth.C5_TOKENS]
+    if args.only:
+        points = [sp for sp in points if args.only in f"{sp.name}_T{sp.T}"]
     sampler = ClockSampler(0)
     sampler.start()
     cache = _WeightCache()
@@ -921,6 +923,9 @@ def main():
                     help="time the static low-rank initialisation (d' = 28672, d = 8192, r = 64) instead")
     ap.add_argument("--table", action="store_true",
                     help="time the forward at every configured workload point, one JSON line each, instead")
+    ap.add_argument("--only", default="", metavar="NAME",
+                    help="with --table: only the points whose workload name (e.g. mlp70b_8192x28672_T128) "
+                         "contains NAME")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

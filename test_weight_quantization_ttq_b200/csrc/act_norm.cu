@@ -50,7 +50,15 @@ __device__ __forceinline__ bool finish_channel(double tot, double p, double lamb
   } else {
     n = pow(tot, 1.0 / p);
   }
-  const double dv = pow(n + lambda, alpha);
+  // (n + lambda)^alpha: the exponents the workloads use through correctly
+  // rounded square roots (alpha = 1/2 is then the correctly rounded power
+  // itself), any other through pow
+  const double y = n + lambda;
+  const double dv = alpha == 0.5   ? sqrt(y)
+                    : alpha == 1.0  ? y
+                    : alpha == 0.25 ? sqrt(sqrt(y))
+                    : alpha == 0.0  ? 1.0
+                                    : pow(y, alpha);
   const double drv = 1.0 / sqrt(dv);
   *df = static_cast<float>(dv);
   *drf = static_cast<float>(drv);
@@ -313,23 +321,28 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
   __syncthreads();
   const int ci = threadIdx.x;
   const int64_t c = cb * kChannelsPerBlock + ci;
-  {
-    double sum = 0.0;
+  double own = 0.0;   // this split's sum of |x|^p for channel c
 #pragma unroll
-    for (int w = 0; w < 8; ++w) sum += red[w][ci];
-    if (c < d) partial[sp * d + c] = sum;
-  }
+  for (int w = 0; w < 8; ++w) own += red[w][ci];
 
-  // (2) every split of this column block has published; merge in split order
-  group_barrier(counters + cb, static_cast<uint32_t>(splits), status, &barrier_ok);
+  // (2) every split of this column block has published; merge in split order.
+  // With one split the merge is that split's own sum (0 + v is v), so the
+  // block needs neither the round trip through global memory nor the barrier.
+  if (splits > 1) {
+    if (c < d) partial[sp * d + c] = own;
+    group_barrier(counters + cb, static_cast<uint32_t>(splits), status, &barrier_ok);
+  }
   float drf = 0.f;
   if (c < d) {
-    double v[16];
+    double tot = own;
+    if (splits > 1) {
+      double v[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
-    double tot = 0.0;
+      for (int k = 0; k < 16; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
+      tot = 0.0;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) tot += v[k];
+      for (int k = 0; k < 16; ++k) tot += v[k];
+    }
     float df;
     const bool ok = finish_channel<PK>(tot, p, lambda, alpha, &df, &drf);
     if (sp == 0) {
