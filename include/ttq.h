@@ -145,7 +145,7 @@ typedef struct ttq_workspace_layout {
                      (0 when A X is not split) */
   size_t D_sqrt;  /* float32 [d] sqrtf(D_ii) for the single-pass decode product */
   size_t ypart;   /* float32 partial output tiles of the single-pass decode product */
-  size_t tickets; /* uint32 arrival tickets of its 128-row tiles (inside the
+  size_t tickets; /* uint32 arrival tickets of its 256-row tiles (inside the
                      zeroed header; 0: not in this layout) */
   int64_t ax_splits; /* K splits of the A X product (1: none; 0 when r == 0) */
 } ttq_workspace_layout;
@@ -369,7 +369,7 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
  * for r > 0).  codes, scales, zeros: NULL, or all three given and filled
  * exactly as ttq_quantize_weight fills them (same bits).
  *   Limits: 1 <= T <= 16, d a multiple of 128, bits 2..4, group 32, 64 or
- * 128, dp <= 524288 (else TTQ_ERR_UNSUPPORTED).  Workspace as for
+ * 128, dp <= 1048576 (else TTQ_ERR_UNSUPPORTED).  Workspace as for
  * ttq_linear_forward (TTQ_BF16) of the same sizes; its tile tickets start at
  * zero (ttq_workspace_init) and every call leaves them at zero.  Flags as
  * ttq_quantize_weight, and TIMEOUT (then re-initialise the workspace).

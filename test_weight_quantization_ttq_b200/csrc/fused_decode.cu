@@ -9,18 +9,19 @@
 // quantiser forms them (same binary32 operations in the same order), and are
 // stored only when the caller asks for them.
 //
-// Work: the weight is cut into units of 128 rows x 128 input channels; the
+// Work: the weight is cut into units of 256 rows x 128 input channels; the
 // units are numbered row-tile-major and every CTA takes one contiguous range
-// of them (a persistent grid of two CTAs per SM, equal shares), so no SM
+// of them (a persistent grid of one CTA per SM, equal shares), so no SM
 // idles at the end.  A row tile whose units fall to two or more CTAs is
 // finished by the last of them to arrive: each writes its partial sums to
 // the workspace and takes a ticket, and the last adds the partials in CTA
 // order (a fixed order: the result does not depend on timing).
 //
 // Per unit, lane 0 of warp 0 loads by TMA into one stage of a ring: the
-// 128 x 128 tile of W (two 64-channel boxes, 128-byte swizzle), the unit's
+// 256 x 128 tile of W (two 64-channel boxes, 128-byte swizzle), the unit's
 // 128 channels of X' (two boxes, 8 or 16 tokens) and of sqrt(D).  Each of
-// the 8 warps owns 16 rows of the tile.  Lane (g, c) (g = lane / 4, c =
+// the 16 warps owns 16 rows of the tile; a stage is refilled once all of
+// them have released it, which keeps them in step.  Lane (g, c) (g = lane / 4, c =
 // lane % 4) holds rows pi(g) and pi(g) + 8 of the warp's 16 (pi(g) =
 // g / 2 + 4 (g % 2), which keeps its shared-memory reads free of bank
 // conflicts) and channels 8 (4m + c) .. + 7 for m = 0..3: a row's group
@@ -43,14 +44,14 @@
 namespace ttq {
 namespace {
 
-constexpr int kFdWarps = 8;
+constexpr int kFdWarps = 16;
 constexpr int kFdThreads = 32 * kFdWarps;
 constexpr int kFdRows = 16 * kFdWarps;               // rows of W per unit
 constexpr int kFdK = 128;                            // channels per unit
-constexpr uint32_t kFdWBox = kFdRows * 64 * 2;       // one 64-channel box of W: 16 KiB
+constexpr uint32_t kFdWBox = kFdRows * 64 * 2;       // one 64-channel box of W: 32 KiB
 
 template <int NTT>
-constexpr int fd_stages() { return NTT == 1 ? 3 : 2; }
+constexpr int fd_stages() { return 3; }
 // X' box: 8 NTT tokens x 64 channels of binary16
 template <int NTT>
 constexpr uint32_t fd_x_box() { return 8u * NTT * 128u; }
@@ -236,7 +237,7 @@ __device__ __forceinline__ void store_chunk_codes(uint32_t* codes, int64_t wpr, 
 }
 
 template <int BITS, int NTT, int GROUP, bool CODES>
-__global__ void __launch_bounds__(kFdThreads, 2) ttq_fused_decode_kernel(
+__global__ void __launch_bounds__(kFdThreads, 1) ttq_fused_decode_kernel(
     const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
     const FdDev a) {
   constexpr int kStages = fd_stages<NTT>();
@@ -282,7 +283,11 @@ __global__ void __launch_bounds__(kFdThreads, 2) ttq_fused_decode_kernel(
     bulk_load(base + 2u * kXBox, a.Dh + k0, kFdK * 4u, &full[s]);
   };
   const int64_t n_units = u_end - u_begin;
-  const int first_issue = static_cast<int>(n_units < kStages ? n_units : kStages);
+  // only the first stage is requested at launch: every CTA asks at once, and
+  // a CTA's first stage lands sooner when it does not compete with the
+  // others' second and third; those follow once it has landed
+  const int first_issue = n_units > 0 ? 1 : 0;
+  const int ring_fill = static_cast<int>(n_units < kStages ? n_units : kStages);
   if (producer) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) {
@@ -349,6 +354,13 @@ __global__ void __launch_bounds__(kFdThreads, 2) ttq_fused_decode_kernel(
       }
     }
     ok = __all_sync(0xffffffffu, ok);
+    if (producer && i == 0 && ok) {
+      for (int k = 1; k < ring_fill; ++k) {
+        issue_w(u_begin + k, k);
+        issue_xh(u_begin + k, k);
+      }
+      issued = ring_fill;
+    }
     if (ok) {
       const uint32_t base = smem + static_cast<uint32_t>(s) * kStage;
       const uint32_t xbase = base + 2u * kFdWBox;
@@ -391,17 +403,32 @@ __global__ void __launch_bounds__(kFdThreads, 2) ttq_fused_decode_kernel(
             mxb = max3_nan(mxb, xb[m][p].x, xb[m][p].y);
           }
         }
-#pragma unroll
-        for (int o = 1; o <= 2; o <<= 1) {
-          mna = min_nan(mna, __shfl_xor_sync(0xffffffffu, mna, o));
-          mxa = max_nan(mxa, __shfl_xor_sync(0xffffffffu, mxa, o));
-          mnb = min_nan(mnb, __shfl_xor_sync(0xffffffffu, mnb, o));
-          mxb = max_nan(mxb, __shfl_xor_sync(0xffffffffu, mxb, o));
+        // The lanes of a pair (c, c ^ 1) split the two rows: even c takes
+        // row A, odd c row B.  Each hands the other the range of the row it
+        // does not take, the pair (c, c ^ 2) completes the range, each lane
+        // computes its row's s, 1/s and z, and the pair swaps them.
+        const bool keep_a = (c & 1) == 0;
+        float kmn = min_nan(keep_a ? mna : mnb,
+                            __shfl_xor_sync(0xffffffffu, keep_a ? mnb : mna, 1));
+        float kmx = max_nan(keep_a ? mxa : mxb,
+                            __shfl_xor_sync(0xffffffffu, keep_a ? mxb : mxa, 1));
+        kmn = min_nan(kmn, __shfl_xor_sync(0xffffffffu, kmn, 2));
+        kmx = max_nan(kmx, __shfl_xor_sync(0xffffffffu, kmx, 2));
+        const GroupQ<BITS> qk = group_params<BITS>(kmn, kmx, rcp_sig);
+        bad |= qk.bad;
+        ovf |= qk.ovf;
+        GroupQ<BITS> qo;   // the partner's row
+        qo.sf = __shfl_xor_sync(0xffffffffu, qk.sf, 1);
+        qo.inv = __shfl_xor_sync(0xffffffffu, qk.inv, 1);
+        qo.zz = __shfl_xor_sync(0xffffffffu, qk.zz, 1);
+        {
+          const uint32_t sz = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(qk.s16) |
+                                                               (static_cast<uint32_t>(qk.z) << 16), 1);
+          qo.s16 = static_cast<uint16_t>(sz & 0xFFFFu);
+          qo.z = static_cast<uint16_t>(sz >> 16);
         }
-        const GroupQ<BITS> qa = group_params<BITS>(mna, mxa, rcp_sig);
-        const GroupQ<BITS> qb = group_params<BITS>(mnb, mxb, rcp_sig);
-        bad |= qa.bad | qb.bad;
-        ovf |= qa.ovf | qb.ovf;
+        const GroupQ<BITS>& qa = keep_a ? qk : qo;
+        const GroupQ<BITS>& qb = keep_a ? qo : qk;
         const uint32_t za = (0x6400u + qa.z) * 0x00010001u;
         const uint32_t zb = (0x6400u + qb.z) * 0x00010001u;
         float part[NTT][4];
@@ -622,13 +649,17 @@ FusedDecodePlan fused_decode_plan(int64_t dp, int64_t d, int64_t T) {
   FusedDecodePlan p;
   p.row_tiles = (dp + kFdRows - 1) / kFdRows;
   p.units = p.row_tiles * (d / kFdK);
-  // never more CTAs than units: every CTA then owns at least one unit, so
-  // the CTAs that share a row tile are consecutive and all take its ticket
-  p.grid = static_cast<int>(p.units < 2 * kFusedDecodePlanSMs ? p.units : 2 * kFusedDecodePlanSMs);
+  // one CTA per SM (its 16 warps share one ring, so none races ahead of the
+  // others as a second CTA on the SM would), and never more CTAs than
+  // units: every CTA then owns at least one unit, so the CTAs that share a
+  // row tile are consecutive and all take its ticket
+  p.grid = static_cast<int>(p.units < kFusedDecodePlanSMs ? p.units : kFusedDecodePlanSMs);
   if (p.grid < 1) p.grid = 1;
   p.part_floats = static_cast<int64_t>(p.grid) * 2 * kFdWarps * 32 * 4 * (T > 8 ? 2 : 1);
   return p;
 }
+
+int fused_decode_rows() { return kFdRows; }
 
 bool fused_decode_supported(int64_t dp, int64_t d, int64_t T, int bits, int group) {
   return T >= 1 && T <= 16 && dp >= 1 && d >= kFdK && d % kFdK == 0 && bits >= 2 && bits <= 4 &&

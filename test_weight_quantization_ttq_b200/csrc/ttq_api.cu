@@ -385,7 +385,7 @@ ttq_status run_single_pass(const void* W, const float* Dh, const void* Xh, const
     pdl = true;
   }
   CUtensorMap tmW, tmX;
-  if (!encode_16bit(&tmW, W, false, d, dp, d, 128) ||
+  if (!encode_16bit(&tmW, W, false, d, dp, d, fused_decode_rows()) ||
       !encode_16bit(&tmX, Xh, true, d, T, d, T <= 8 ? 8 : 16))
     return TTQ_ERR_CUDA;
   FusedDecodeArgs a;

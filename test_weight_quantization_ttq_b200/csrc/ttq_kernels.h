@@ -163,10 +163,10 @@ cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
 // warp-level MMAs, add B (A X) (bf16, when r > 0) and store Y [T][ldy];
 // codes, scales and zeros (all three or none) are stored as the quantiser
 // stores them.  K a multiple of 128, group 32, 64 or 128, bits 2..4.
-// Persistent grid of fused_decode_plan().grid CTAs over row tiles of 128;
+// Persistent grid of fused_decode_plan().grid CTAs over row tiles of 256;
 // `part` holds plan.part_floats floats, `tickets` plan.row_tiles uint32
 // that are zero before and after the call.  tmW: bf16 W [M][K], box 64 x
-// 128, 128-byte swizzle; tmX: binary16 X' [T][K], box 64 x (T <= 8 ? 8 :
+// 256, 128-byte swizzle; tmX: binary16 X' [T][K], box 64 x (T <= 8 ? 8 :
 // 16), 128-byte swizzle.
 constexpr int kFusedDecodePlanSMs = 148;     // fixed so the layout is device-independent
 constexpr int64_t kFusedDecodeMaxTiles = 4096;
@@ -175,6 +175,7 @@ struct FusedDecodePlan {
   int64_t row_tiles, units, part_floats;
 };
 FusedDecodePlan fused_decode_plan(int64_t dp, int64_t d, int64_t T);
+int fused_decode_rows();   // rows of W per unit (the W box height)
 bool fused_decode_supported(int64_t dp, int64_t d, int64_t T, int bits, int group);
 struct FusedDecodeArgs {
   const float* Dh = nullptr;
