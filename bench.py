@@ -351,9 +351,6 @@ def run_ours(args):
     views = ttq.workspace_views(ws, d, dp, T, 0, bits, group)
     Dbuf = views["D"]  # written in place by ttq_act_norm_scale (copy_out=False)
     Xsbuf = torch.empty((T, d), dtype=torch.float16, device="cuda")
-    codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device="cuda")
-    sc = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
-    ze = torch.empty((dp, d // group), dtype=torch.int16, device="cuda")
     W_hat = torch.empty((dp, d), dtype=torch.float16, device="cuda")
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     barrier()
@@ -365,12 +362,13 @@ def run_ours(args):
         ev[i][0].record(stream)
         ttq.ttq_act_norm_scale(Xs[k], w["p"], w["lam"], w["alpha"], ws=ws, Xs=Xsbuf, copy_out=False)
         ev[i][1].record(stream)
+        # as in the forward, the materialised weight alone (no codes)
         if scheme is None:
-            ttq.ttq_quantize_dequant_weight(Ws[k], Dbuf, bits, group, ws=ws, codes=codes, scales=sc,
-                                            zeros=ze, W_hat=W_hat)
+            ttq.ttq_quantize_dequant_weight(Ws[k], Dbuf, bits, group, ws=ws, W_hat=W_hat,
+                                            with_codes=False)
         else:
-            ttq.ttq_quantize_weight_ex(Ws[k], Dbuf, bits, group, scheme, ws=ws, codes=codes, scales=sc,
-                                       zeros=ze, W_hat=W_hat)
+            ttq.ttq_quantize_weight_ex(Ws[k], Dbuf, bits, group, scheme, ws=ws, W_hat=W_hat,
+                                       with_codes=False)
         ev[i][2].record(stream)
         ttq.ttq_dequantized_gemm(W_hat, Xsbuf, ws=ws, Y=Ys[k])
         ev[i][3].record(stream)
@@ -387,11 +385,12 @@ def run_ours(args):
     # and writes codes, scales and zeros
     stat_alg = 2.0 * d * T + 8.0 * d
     qdq_alg = 2.0 * dp * d + dp * d * bits / 8 + 4.0 * dp * d / group + 4.0 * d
-    # bytes this implementation moves besides: the statistic also writes the
-    # product's binary16 X D^{-1/2}; the quantiser also writes the binary16
-    # dequantised weight that the prefill product reads
+    # bytes this implementation moves: the statistic also writes the
+    # product's binary16 X D^{-1/2}; the quantiser reads W and D and writes
+    # the binary16 dequantised weight that the prefill product reads, in
+    # place of the codes, scales and zeros
     stat_moved = stat_alg + 2.0 * d * T
-    qdq_moved = qdq_alg + 2.0 * dp * d
+    qdq_moved = 2.0 * dp * d + 2.0 * dp * d + 4.0 * d
     gemm_tflops = flops / t_gemm / 1e12
     traffic = NCU_TRAFFIC.get(_kernel_hash())
     roofline = {"kernel": "ttq_gemm_kernel<0, 256> (tcgen05 GEMM on the binary16 dequantised weight)", "bound": "tensor",
@@ -848,6 +847,86 @@ def run_table(args):
                       "peak_source": peaks["source"], "clocks": sampler.stop()}), flush=True)
 
 
+def run_ab_dequant(args):
+    """Where the prefill product gets its weight operand: the
+    materialised form (the quantiser also writes the binary16 s (q - z), the
+    plain tcgen05 GEMM reads it by TMA) against dequantisation inside the
+    product's main loop (the quantiser writes codes only; the GEMM's
+    producer warps turn each TMA-fed code tile into the binary16 operand in
+    shared memory).  At the q_proj prefill (d = d' = 4096, T = 2048, INT4
+    g128) and the 70B-like MLP shape at T = 4096 (INT2 g64, no low-rank
+    term), each pair of entry points and each kernel in a CUDA graph of K
+    calls, W rotating over copies larger than L2.  One JSON line per
+    workload."""
+    import torch
+
+    from test_weight_quantization_ttq_b200 import synth, ttq
+
+    stream = torch.cuda.current_stream()
+    peaks = _measured_peaks()
+
+    def graph_time(fn, k):
+        for i in range(args.warmup):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(k):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / k
+
+    for spec in (synth.C2, synth.C5.with_(T=4096, r=0)):
+        data = synth.generate(spec)
+        X = torch.from_numpy(data["X"]).to(torch.bfloat16).cuda()
+        W0 = torch.from_numpy(data["W"]).to(torch.bfloat16).cuda()
+        n = max(2, -(-2 * L2_BYTES // (W0.numel() * 2)))
+        Ws = [W0] + [W0.clone() for _ in range(n - 1)]
+        d, dp, T, b, g = spec.d, spec.dp, spec.T, spec.bits, spec.group
+        D, Dr, Xs = ttq.ttq_act_norm_scale(X, spec.p, spec.lam, spec.alpha)
+        ws = ttq.new_workspace(d, dp, T, 0, b, g)
+        codes = torch.empty((dp, d * b // 32), dtype=torch.int32, device="cuda")
+        sc = torch.empty((dp, d // g), dtype=torch.int16, device="cuda")
+        ze = torch.empty_like(sc)
+        Wh = torch.empty((dp, d), dtype=torch.float16, device="cuda")
+        Y = torch.empty((T, dp), dtype=torch.bfloat16, device="cuda")
+        k = max(3, min(args.steps, 20))
+
+        def quant_wq(i):
+            ttq.ttq_quantize_dequant_weight(Ws[i % n], D, b, g, ws=ws, codes=codes, scales=sc, zeros=ze, W_hat=Wh)
+
+        def gemm_wq(i):
+            ttq.ttq_dequantized_gemm(Wh, Xs, ws=ws, Y=Y)
+
+        def quant(i):
+            ttq.ttq_quantize_weight(Ws[i % n], D, b, g, ws=ws, codes=codes, scales=sc, zeros=ze)
+
+        def gemm_codes(i):
+            ttq.ttq_dequant_gemm(codes, sc, ze, None, Xs, None, None, b, g, ws=ws, Y=Y)
+
+        t = {name: graph_time(fn, k) for name, fn in (
+            ("materialised_quantiser", quant_wq), ("materialised_gemm", gemm_wq),
+            ("materialised_pair", lambda i: (quant_wq(i), gemm_wq(i))),
+            ("in_mainloop_quantiser", quant), ("in_mainloop_gemm", gemm_codes),
+            ("in_mainloop_pair", lambda i: (quant(i), gemm_codes(i))))}
+        st, flags = ttq.ttq_get_status(ws)
+        flops = 2.0 * dp * d * T
+        print(json.dumps({"ab": "prefill weight operand: materialised binary16 W_hat vs in-mainloop dequantisation",
+                          "workload": f"{spec.name}_T{T}", "d": d, "dp": dp, "T": T, "bits": b, "group": g,
+                          "us": t, "gemm_tflops": {"materialised": flops / t["materialised_gemm"] / 1e6,
+                                                   "in_mainloop": flops / t["in_mainloop_gemm"] / 1e6},
+                          "bf16_peak_tflops": peaks["bf16_tflops"], "calls_timed": k,
+                          "status": ttq.status_string(st)}), flush=True)
+        del Ws, W0
+        torch.cuda.empty_cache()
+
+
 def run_lowrank(args):
     """The static low-rank initialisation at the 70B-like MLP shape
     (d' = 28672, d = 8192, bf16 W, r = 64, 8 extra sampled directions, 2
@@ -923,6 +1002,9 @@ def main():
                     help="time the static low-rank initialisation (d' = 28672, d = 8192, r = 64) instead")
     ap.add_argument("--table", action="store_true",
                     help="time the forward at every configured workload point, one JSON line each, instead")
+    ap.add_argument("--ab-dequant", action="store_true",
+                    help="A/B of the prefill weight operand: materialised W_hat vs dequantisation in the "
+                         "product's main loop, instead")
     ap.add_argument("--only", default="", metavar="NAME",
                     help="with --table: only the points whose workload name (e.g. mlp70b_8192x28672_T128) "
                          "contains NAME")
@@ -931,6 +1013,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.table:
         run_table(args)
+    elif args.ab_dequant:
+        run_ab_dequant(args)
     elif args.lowrank:
         run_lowrank(args)
     elif args.decode:

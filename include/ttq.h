@@ -119,8 +119,13 @@ typedef enum ttq_qscheme {
 /* Byte offsets of the workspace regions for one problem shape (all 256-byte
  * aligned); `total` equals ttq_workspace_size(...).  After
  * ttq_linear_forward the regions hold that call's intermediates: D and
- * D_rsqrt as float32 [d], the codes/scales/zeros of W_hat, and A X as bf16
- * [T][ax_ld].  Offsets of regions the shape does not use are 0 with
+ * D_rsqrt as float32 [d], A X as bf16 [T][ax_ld], and the codes/scales/
+ * zeros of W_hat where the product read them (INT codes at 17 to 256
+ * tokens and with a non-bf16 or symmetric layer at up to 16; FP8 codes at
+ * up to 16 tokens).  Where the product read the materialised binary16 W_hat
+ * (wq: more than 256 tokens; FP8 above 16) that alone is kept, no codes;
+ * the single-pass product (bf16, asymmetric, up to 16 tokens) keeps
+ * neither.  Offsets of regions the shape does not use are 0 with
  * size 0.  Returns TTQ_ERR_INVALID_ARG for an unsupported shape. */
 typedef struct ttq_workspace_layout {
   size_t status;  /* uint32 status word, then internal counters */
@@ -187,17 +192,17 @@ ttq_status ttq_act_norm(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
  * W_hat = Q[W D^{1/2}] D^{-1/2}, carried by X).  X [T][d] in TTQ_F32 or
  * TTQ_BF16, d % 8 == 0; Xs binary16 [T][d] (uint16 bit patterns), required
  * when T > 0; D and D_rsqrt float32 [d] or NULL (then written to the
- * workspace only).  When each token split of the statistic pass has at
- * most 128 rows (64 for float32 X; the splits are those of ttq_act_norm:
- * about 296 blocks of 256 channels, at most 16 splits) and the whole grid
- * can be resident at once, this is one cooperative kernel that reads X
- * from HBM once and keeps it in registers; otherwise it is the two kernels
- * of ttq_act_norm and ttq_scale_activations.  The results are the same bits
- * either way.  The
+ * workspace only).  The token splits are those of ttq_act_norm (the
+ * layout's `splits`): for T <= 2048, enough for about two 128-channel
+ * blocks per SM and for at most 256 rows each, at most 8; for longer T,
+ * at most 16.  When there are at most 8 splits of at most 256 rows (128 for
+ * float32 X), this is one kernel that reads X from HBM once and keeps it in
+ * registers, the splits of a column block forming one thread-block cluster;
+ * otherwise it is the two kernels of ttq_act_norm and
+ * ttq_scale_activations.  The results are the same bits either way.  The
  * workspace is the one ttq_act_norm needs (it must have been cleared by
  * ttq_workspace_init once; the call leaves its counters at zero).  Flags as
- * ttq_act_norm and ttq_scale_activations (NONFINITE, X_RANGE; TIMEOUT if
- * the fused kernel's wait for the other splits gave up). */
+ * ttq_act_norm and ttq_scale_activations (NONFINITE, X_RANGE). */
 ttq_status ttq_act_norm_scale(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
                               float p, float lambda, float alpha, float* D,
                               float* D_rsqrt, uint16_t* Xs, void* ws, size_t ws_bytes,
@@ -244,7 +249,9 @@ ttq_status ttq_quantize_weight(const void* W, ttq_dtype dtype, int64_t dp, int64
 
 /* ttq_quantize_weight with a choice of code scheme and an optional
  * dequantised binary16 weight (as ttq_quantize_dequant_weight writes it;
- * W_hat may be NULL).  With TTQ_QSCHEME_SYMMETRIC the binary32 order is
+ * W_hat may be NULL).  With W_hat given, codes, scales and zeros may all
+ * be NULL: then W_hat alone is written (the same values; the flags as
+ * with the codes).  With TTQ_QSCHEME_SYMMETRIC the binary32 order is
  *   h = sqrtf(D_i); x = W_ji * h; M = max_group |x|;
  *   s32 = M / (2^(bits-1) - 1), floored at 2^-14; s = binary16 round-up;
  *   inv = 1 / s; level = clamp(rint(x * inv), -(2^(bits-1)-1), 2^(bits-1)-1)
@@ -264,7 +271,9 @@ ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, in
  * section 2.1) without its D^{-1/2} factor, which the product's other
  * operand X D^{-1/2} carries.  q - z is exact and the product is rounded
  * once, so these are the operand values ttq_dequant_gemm forms from the
- * codes.  Everything else as ttq_quantize_weight. */
+ * codes.  codes, scales and zeros may all be NULL (W_hat alone is written,
+ * as the forward does when it materialises the weight).  Everything else
+ * as ttq_quantize_weight. */
 ttq_status ttq_quantize_dequant_weight(const void* W, ttq_dtype dtype, int64_t dp, int64_t d,
                                        const float* D, int bits, int group, uint32_t* codes,
                                        uint16_t* scales, uint16_t* zeros, uint16_t* W_hat,
@@ -322,13 +331,15 @@ ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64
  * `y_dtype` (TTQ_F32: the fp32 accumulator; TTQ_BF16: rounded once to
  * nearest-even).  A and B may be NULL when r == 0.  W is taken to be the
  * residual that the static low-rank pair complements (gist.science/zh,
- * section 2.2).  The workspace keeps D, D_rsqrt, codes, scales and zeros of
- * this call.  For T > 256 the quantiser also writes the dequantised weight
- * s (q - z) in binary16 to the workspace (layout field wq) and the product
- * reads it as a plain tensor-core operand, so that no 256-token tile
- * dequantises the codes again; for T <= 256 the product dequantises the
- * codes itself (as ttq_dequant_gemm does).  Both give the same operand
- * values. */
+ * section 2.2).  The workspace keeps D and D_rsqrt of this call and the
+ * quantised weight in the form the product read (see ttq_workspace_layout).
+ * For T > 256 the quantiser writes the dequantised weight s (q - z) in
+ * binary16 to the workspace (layout field wq) instead of the codes, and the
+ * product reads it as a plain tensor-core operand, so that no 256-token
+ * tile dequantises the codes again; for 17 <= T <= 256 the product
+ * dequantises the codes itself (as ttq_dequant_gemm does); for T <= 16
+ * (bf16, asymmetric codes) one kernel quantises W in registers and
+ * multiplies (as ttq_quantize_gemm).  All give the same operand values. */
 ttq_status ttq_linear_forward(const void* X, const void* W, const void* A,
                               const void* B, ttq_dtype dtype, int64_t d, int64_t dp,
                               int64_t T, int64_t r, float p, float lambda, float alpha,

@@ -3,17 +3,24 @@
 // (gist.science/zh/paper/2603.19296, section 2.1).  X is [T][d] (token
 // major), so channel i is a column: the reduction runs down the columns.
 //
-// Layout of the work: a block owns 256 consecutive channels and one split of
-// the tokens.  Each lane loads 8 consecutive channels of a row (one 16-byte
-// load for bf16), each of the 8 warps walks every 8th row of the split, and
-// the warps' sums are merged in shared memory in a fixed order; sums are kept
-// in fp64 (the pass is bound by memory, not by the fp64 pipe).  The split's
-// partial sums go to global memory; the last block to finish a column block
-// (an atomic ticket) merges all splits in fp64, in split order, so the
-// result does not depend on scheduling.  On the way it writes the binary16
-// copy of X that the tensor-core product consumes (and, for float32 X with a
-// low-rank term, a bf16 copy).  The pass is HBM-bound: it reads X once (2dT
-// bytes for bf16) and writes 2dT bytes of binary16 X plus 8d bytes.
+// The order of the sums, shared by both kernels below so that D is the same
+// bits whichever runs: the tokens are cut into `splits` consecutive splits
+// (act_norm_plan); within a split, |x|^p of channel i is accumulated in fp64
+// over 16 row phases (phase j holds rows j, j + 16, j + 32, ... of the split,
+// in increasing order), the 16 phase sums are added in phase order, and the
+// split sums in split order.  fp64 is cheap here: the pass is bound by
+// memory, not by the fp64 pipe.
+//
+// act_norm_kernel (any T): a block owns 256 consecutive channels and one
+// split; lane l loads channels 8l..8l+7 of a row (one 16-byte load for
+// bf16), warp w walks rows w, w + 8, ... of the split and so holds phases w
+// and w + 8.  The split's sums go to global memory; the last block of a
+// column block to finish (an atomic ticket) merges the splits.
+//
+// act_norm_scale_kernel (each split's rows fit in registers): the fused
+// statistic and product operand X D^(-1/2), reading X from HBM once; the
+// splits of a column block form one thread-block cluster and merge through
+// distributed shared memory.
 #include <map>
 #include <mutex>
 #include <utility>
@@ -24,8 +31,12 @@
 namespace ttq {
 namespace {
 
-constexpr int kChannelsPerBlock = 256;
+constexpr int kChannelsPerBlock = 256;  // act_norm_kernel's column block
+constexpr int kClusterChannels = 128;   // act_norm_scale_kernel's column block
 constexpr int kThreads = 256;
+constexpr int kPhases = 16;             // row phases of a split
+constexpr int kMaxSplits = 16;          // token splits (act_norm_plan)
+constexpr int kMaxClusterSplits = 8;    // portable cluster size
 
 // |x|^p in fp64: exact for p = 1 and for p = 2 with 16-bit inputs, so the
 // merged sums (and hence D rounded to binary32) match an fp64 reference.
@@ -115,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
     uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
     float* __restrict__ Dh, __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb,
     uint32_t* __restrict__ status) {
-  __shared__ double red[8][kChannelsPerBlock + 2];
+  __shared__ double red[kPhases][kChannelsPerBlock + 2];
   __shared__ int is_last;
   allow_dependents_launch();
   grid_dependency_wait();
@@ -126,16 +137,19 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
   const int64_t sp = blockIdx.y;
   const int64_t c0 = cb * kChannelsPerBlock + lane * 8;
 
-  double acc[8];
+  // acc[h]: phase warp + 8h (rows warp + 8m of the split with m % 2 == h)
+  double acc[2][8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+  for (int e = 0; e < 8; ++e) acc[0][e] = acc[1][e] = 0.0;
 
   const int64_t t_begin = sp * rows_per_split;
   const int64_t t_end = min(T, t_begin + rows_per_split);
   float amax = 0.f;
   if (c0 < d) {
-    // each warp takes rows t_begin + warp + 8k, kBatch at a time; the next
-    // batch is loaded while the current one is summed
+    // rows t_begin + warp + 8m, kBatch at a time (batches start at even m);
+    // the next batch is loaded while the current one is summed.  A row past
+    // the split is loaded as zeros and adds +0 to its phase, which leaves
+    // the (non-negative or NaN) sum unchanged.
     constexpr int kBatch = 4;
     float v[kBatch][8], vn[kBatch][8];
     auto load_batch = [&](int64_t t0, float (&dst)[kBatch][8]) {
@@ -160,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          acc[e] += abs_pow<PK>(buf[k][e], p);
+          acc[k & 1][e] += abs_pow<PK>(buf[k][e], p);
           amax = fmaxf(amax, fabsf(buf[k][e]));
         }
       }
@@ -181,14 +195,17 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
   if (xh != nullptr && __any_sync(0xffffffffu, amax > 65504.f) && lane == 0)
     set_flag(status, TTQ_FLAG_X_RANGE);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
+  for (int e = 0; e < 8; ++e) {
+    red[warp][lane * 8 + e] = acc[0][e];
+    red[warp + 8][lane * 8 + e] = acc[1][e];
+  }
   __syncthreads();
 
   const int ci = threadIdx.x;
   const int64_t c = cb * kChannelsPerBlock + ci;
   double sum = 0.0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) sum += red[w][ci];
+  for (int j = 0; j < kPhases; ++j) sum += red[j][ci];
   if (c < d) partial[sp * d + c] = sum;
 
   // Ticket: the last split block of this column block merges all splits.
@@ -203,13 +220,14 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
   __threadfence();
 
   if (c < d) {
-    // fixed order; up to 16 partials loaded at once (one L2 round trip)
-    double v[16];
+    // split order; all partials loaded at once (one L2 round trip); the
+    // +0 of an absent split leaves the sum unchanged
+    double v[kMaxSplits];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
+    for (int k = 0; k < kMaxSplits; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
     double tot = 0.0;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) tot += v[k];
+    for (int k = 0; k < kMaxSplits; ++k) tot += v[k];
     float df, drf;
     const bool ok = finish_channel<PK>(tot, p, lambda, alpha, &df, &drf);
     D[c] = df;
@@ -222,18 +240,21 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_kernel(
 
 // ---------------------------------------------------------------------------
 // Fused form of the statistic pass and of the binary16 operand X D^(-1/2).
-// Block (cb, sp) is the block of act_norm_kernel with the same index: warp w
-// takes rows w, w + 8, ... of the split, lane l channels 8l..8l+7 of the
-// column block.  Each thread loads all of its rows (at most kRegRows<XT>)
-// into registers at once, sums |x|^p over them in the same order as
-// act_norm_kernel, publishes the split's partial sums, and waits until every
-// split of its column block has done so (a barrier among the blocks of the
-// column block; the grid is launched cooperatively so that all of them are
-// resident).  Each block then merges its column block's splits in split
-// order (the same merge as act_norm_kernel, so D is identical), and writes
-// binary16(x * D^(-1/2)) from the registers.  X is read from HBM once.
+// Block (cb, sp) owns channels 128 cb .. 128 cb + 127 and split sp of the
+// tokens.  Lane l of warp w takes channels 8 (l % 16) .. + 7 of the rows of
+// phase j = 2w + l / 16 (rows j, j + 16, ... of the split), so a warp reads
+// two whole 256-byte row segments per load.  Each thread loads all of its
+// rows (at most reg_rows<XT>()) into registers at once, sums |x|^p over them
+// in increasing row order, and the block adds its 16 phase sums in phase
+// order.  The splits of a column block are the blocks of one thread-block
+// cluster: each publishes its split sums in shared memory, and after the
+// cluster barrier every block reads all of them through distributed shared
+// memory and adds them in split order (the merge of act_norm_kernel, so D is
+// identical).  It then writes binary16(x * D^(-1/2)) from the registers.  X
+// is read from HBM once, and no block waits on another beyond its cluster,
+// so no grid-wide residency is needed.
 
-// Rows per warp held in registers: 16 uint4 of X per thread.
+// Rows per thread held in registers: 16 uint4 of X.
 template <typename XT>
 __host__ __device__ constexpr int reg_rows() { return sizeof(XT) == 2 ? 16 : 8; }
 
@@ -270,45 +291,46 @@ struct Raw8<float> {
 template <typename XT, int PK>
 __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
     const XT* __restrict__ X, int64_t d, int64_t T, double p, double lambda, double alpha,
-    int64_t splits, int64_t rows_per_split, double* __restrict__ partial,
-    uint32_t* __restrict__ counters, float* __restrict__ D, float* __restrict__ Dr,
+    int64_t splits, int64_t rows_per_split, float* __restrict__ D, float* __restrict__ Dr,
     float* __restrict__ Dh, __half* __restrict__ xh, __nv_bfloat16* __restrict__ xb,
     uint32_t* __restrict__ status) {
   constexpr int R = reg_rows<XT>();
-  __shared__ double red[8][kChannelsPerBlock + 2];
-  __shared__ float dr_s[kChannelsPerBlock];
-  __shared__ int barrier_ok;
+  __shared__ double red[kPhases][kClusterChannels + 2];
+  __shared__ double own_s[kClusterChannels];   // this split's sums, read by the cluster
+  __shared__ float dr_s[kClusterChannels];
   allow_dependents_launch();
-  grid_dependency_wait();   // (a no-op for the cooperative launch)
+  grid_dependency_wait();
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int phase = 2 * warp + (lane >> 4);
+  const int cl = (lane & 15) * 8;
   const int64_t cb = blockIdx.x;
-  const int64_t sp = blockIdx.y;
-  const int cl = lane * 8;
-  const int64_t c0 = cb * kChannelsPerBlock + cl;
+  const int64_t sp = blockIdx.y;   // also this block's rank in its cluster
+  const int64_t c0 = cb * kClusterChannels + cl;
   const bool active = c0 < d;
   const int64_t t_begin = sp * rows_per_split;
   const int64_t t_end = min(T, t_begin + rows_per_split);
+  const bool clustered = splits > 1;
 
   // all rows of this thread in flight at once
   Raw8<XT> raw[R];
   if (active) {
 #pragma unroll
     for (int k = 0; k < R; ++k) {
-      const int64_t t = t_begin + warp + 8 * k;
+      const int64_t t = t_begin + phase + kPhases * k;
       if (t < t_end) raw[k].load(X + t * d + c0);
     }
   }
 
-  // (1) this split's sums of |x|^p, rows in increasing order
+  // (1) this phase's sums of |x|^p, rows in increasing order
   double acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
   if (active) {
 #pragma unroll
     for (int k = 0; k < R; ++k) {
-      if (t_begin + warp + 8 * k < t_end) {
+      if (t_begin + phase + kPhases * k < t_end) {
         float v[8];
         raw[k].unpack(v);
 #pragma unroll
@@ -317,31 +339,36 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[warp][cl + e] = acc[e];
+  for (int e = 0; e < 8; ++e) red[phase][cl + e] = acc[e];
   __syncthreads();
-  const int ci = threadIdx.x;
-  const int64_t c = cb * kChannelsPerBlock + ci;
-  double own = 0.0;   // this split's sum of |x|^p for channel c
+  const int ci = threadIdx.x;   // channel of the merge, threads < 128
+  const int64_t c = cb * kClusterChannels + ci;
+  if (ci < kClusterChannels) {
+    double own = 0.0;
 #pragma unroll
-  for (int w = 0; w < 8; ++w) own += red[w][ci];
+    for (int j = 0; j < kPhases; ++j) own += red[j][ci];
+    own_s[ci] = own;
+  }
 
-  // (2) every split of this column block has published; merge in split order.
-  // With one split the merge is that split's own sum (0 + v is v), so the
-  // block needs neither the round trip through global memory nor the barrier.
-  if (splits > 1) {
-    if (c < d) partial[sp * d + c] = own;
-    group_barrier(counters + cb, static_cast<uint32_t>(splits), status, &barrier_ok);
+  // (2) every split of this column block has published; merge in split
+  // order.  With one split the merge is that split's own sum (0 + v is v).
+  if (clustered) {
+    cluster_arrive_release();
+    cluster_wait_acquire();
+  } else {
+    __syncthreads();
   }
   float drf = 0.f;
-  if (c < d) {
-    double tot = own;
-    if (splits > 1) {
-      double v[16];
+  if (ci < kClusterChannels && c < d) {
+    double tot = own_s[ci];
+    if (clustered) {
+      double v[kMaxClusterSplits];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) v[k] = k < splits ? __ldcg(partial + k * d + c) : 0.0;
+      for (int k = 0; k < kMaxClusterSplits; ++k)
+        v[k] = k < splits ? ld_cluster_f64(&own_s[ci], static_cast<uint32_t>(k)) : 0.0;
       tot = 0.0;
 #pragma unroll
-      for (int k = 0; k < 16; ++k) tot += v[k];
+      for (int k = 0; k < kMaxClusterSplits; ++k) tot += v[k];
     }
     float df;
     const bool ok = finish_channel<PK>(tot, p, lambda, alpha, &df, &drf);
@@ -352,7 +379,10 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
       if (!ok) set_flag(status, TTQ_FLAG_NONFINITE);
     }
   }
-  dr_s[ci] = drf;
+  if (ci < kClusterChannels) dr_s[ci] = drf;
+  // this block has read the other blocks' sums (their shared memory must
+  // stay until every block of the cluster is past this point)
+  if (clustered) cluster_arrive_relaxed();
   __syncthreads();
 
   // (3) binary16(x * D^(-1/2)) (and the bf16 copy of a float32 X)
@@ -363,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
     for (int e = 0; e < 8; ++e) f[e] = dr_s[cl + e];
 #pragma unroll
     for (int k = 0; k < R; ++k) {
-      const int64_t t = t_begin + warp + 8 * k;
+      const int64_t t = t_begin + phase + kPhases * k;
       if (t < t_end) {
         float v[8];
         raw[k].unpack(v);
@@ -381,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
     }
   }
   if (__any_sync(0xffffffffu, out_of_range) && lane == 0) set_flag(status, TTQ_FLAG_X_RANGE);
+  if (clustered) cluster_wait_acquire();
 }
 
 template <typename XT, int PK>
@@ -411,92 +442,100 @@ cudaError_t launch_p(const XT* X, int64_t d, int64_t T, float p, float lambda, f
                              counters, D, Dr, Dh, xh, xb, status, stream, pdl);
 }
 
-// How many blocks of the fused kernel fit on one SM (0 when the query
-// fails), cached per device.
+// Whether a cluster of `splits` blocks of the fused kernel can be resident
+// on this device (false when the query fails), cached per device and size.
 template <typename XT, int PK>
-int fused_blocks_per_sm() {
+bool cluster_resident(int64_t splits) {
   static std::mutex mu;
-  static int cache[64] = {};
+  static int8_t cache[64][kMaxClusterSplits + 1] = {};
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev] == 0) {
+  int8_t& known = cache[dev][splits];
+  if (known == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, static_cast<unsigned>(splits));
+    cfg.blockDim = dim3(kThreads);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(splits);
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, act_norm_scale_kernel<XT, PK>, kThreads,
-                                                      0) != cudaSuccess)
-      return 0;
-    cache[dev] = n > 0 ? n : -1;
+    const cudaError_t e =
+        cudaOccupancyMaxActiveClusters(&n, act_norm_scale_kernel<XT, PK>, &cfg);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    known = n > 0 ? 1 : -1;
   }
-  return cache[dev] > 0 ? cache[dev] : 0;
+  return known > 0;
 }
 
 // Whether the fused kernel applies: every thread's rows fit in its
-// registers and the grid (ceil(d/256) x splits blocks) is resident at once.
+// registers and the splits of a column block form one cluster.
 template <typename XT, int PK>
-bool fused_fits(int64_t d, int64_t splits, int64_t rows_per_split, int num_sms) {
-  if (rows_per_split > 8 * reg_rows<XT>()) return false;
-  const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
-  const int per_sm = fused_blocks_per_sm<XT, PK>();
-  return per_sm > 0 && ncb * splits <= static_cast<int64_t>(per_sm) * num_sms;
+bool fused_fits(int64_t splits, int64_t rows_per_split) {
+  if (rows_per_split > kPhases * reg_rows<XT>()) return false;
+  if (splits < 1 || splits > kMaxClusterSplits) return false;
+  return splits == 1 || cluster_resident<XT, PK>(splits);
 }
 
 template <typename XT>
-bool fused_fits_p(float p, int64_t d, int64_t splits, int64_t rows_per_split, int num_sms) {
-  if (p == 1.0f) return fused_fits<XT, 1>(d, splits, rows_per_split, num_sms);
-  if (p == 2.0f) return fused_fits<XT, 2>(d, splits, rows_per_split, num_sms);
-  return fused_fits<XT, 0>(d, splits, rows_per_split, num_sms);
+bool fused_fits_p(float p, int64_t splits, int64_t rows_per_split) {
+  if (p == 1.0f) return fused_fits<XT, 1>(splits, rows_per_split);
+  if (p == 2.0f) return fused_fits<XT, 2>(splits, rows_per_split);
+  return fused_fits<XT, 0>(splits, rows_per_split);
 }
 
 template <typename XT, int PK>
 cudaError_t launch_fused_typed(const XT* X, int64_t d, int64_t T, float p, float lambda,
-                               float alpha, int64_t splits, int64_t rows_per_split,
-                               double* partial, uint32_t* counters, float* D, float* Dr,
-                               float* Dh, void* xh, void* xb, uint32_t* status, int num_sms,
+                               float alpha, int64_t splits, int64_t rows_per_split, float* D,
+                               float* Dr, float* Dh, void* xh, void* xb, uint32_t* status,
                                cudaStream_t stream, bool* launched) {
   *launched = false;
-  if (!fused_fits<XT, PK>(d, splits, rows_per_split, num_sms)) return cudaSuccess;
-  const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
+  if (!fused_fits<XT, PK>(splits, rows_per_split)) return cudaSuccess;
+  const int64_t ncb = (d + kClusterChannels - 1) / kClusterChannels;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(ncb), static_cast<unsigned>(splits));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  if (splits > 1) {
-    // the blocks of a column block wait for one another: all must be resident
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-  } else {
-    // one split: each block's barrier has itself alone to wait for, so a
-    // plain launch does, and it may overlap the previous kernel's tail
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-  }
+  // may overlap the previous kernel's tail (the kernel waits for it before
+  // touching memory); the splits of a column block are one cluster
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = static_cast<unsigned>(splits);
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = splits > 1 ? 2 : 1;
   const cudaError_t e = cudaLaunchKernelEx(
       &cfg, act_norm_scale_kernel<XT, PK>, X, d, T, static_cast<double>(p),
-      static_cast<double>(lambda), static_cast<double>(alpha), splits, rows_per_split, partial,
-      counters, D, Dr, Dh, static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
+      static_cast<double>(lambda), static_cast<double>(alpha), splits, rows_per_split, D, Dr, Dh,
+      static_cast<__half*>(xh), static_cast<__nv_bfloat16*>(xb), status);
   *launched = e == cudaSuccess;
   return e;
 }
 
 template <typename XT>
 cudaError_t launch_fused_p(const XT* X, int64_t d, int64_t T, float p, float lambda, float alpha,
-                           int64_t splits, int64_t rows_per_split, double* partial,
-                           uint32_t* counters, float* D, float* Dr, float* Dh, void* xh, void* xb,
-                           uint32_t* status, int num_sms, cudaStream_t stream, bool* launched) {
+                           int64_t splits, int64_t rows_per_split, float* D, float* Dr, float* Dh,
+                           void* xh, void* xb, uint32_t* status, cudaStream_t stream,
+                           bool* launched) {
   if (p == 1.0f)
-    return launch_fused_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                                     counters, D, Dr, Dh, xh, xb, status, num_sms, stream,
-                                     launched);
+    return launch_fused_typed<XT, 1>(X, d, T, p, lambda, alpha, splits, rows_per_split, D, Dr,
+                                     Dh, xh, xb, status, stream, launched);
   if (p == 2.0f)
-    return launch_fused_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                                     counters, D, Dr, Dh, xh, xb, status, num_sms, stream,
-                                     launched);
-  return launch_fused_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, partial,
-                                   counters, D, Dr, Dh, xh, xb, status, num_sms, stream, launched);
+    return launch_fused_typed<XT, 2>(X, d, T, p, lambda, alpha, splits, rows_per_split, D, Dr,
+                                     Dh, xh, xb, status, stream, launched);
+  return launch_fused_typed<XT, 0>(X, d, T, p, lambda, alpha, splits, rows_per_split, D, Dr, Dh,
+                                   xh, xb, status, stream, launched);
 }
 
 __global__ void sqrt_f32_kernel(const float* __restrict__ D, float* __restrict__ h, int64_t d) {
@@ -518,14 +557,26 @@ cudaError_t launch_sqrt_f32(const float* D, float* h, int64_t d, cudaStream_t st
 }
 
 void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split) {
-  // about two resident blocks per SM, and at most 16 splits so that the
-  // final merge is one batch of loads
-  const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
+  // When 8 splits of at most 256 rows cover T (the fused kernel's register
+  // capacity for bf16 X), enough splits for about two 128-channel blocks
+  // per SM and enough for the rows to fit, at most 8 (one cluster).
+  // Otherwise about two 256-channel blocks per SM, at most 16 splits.
+  // Always at least 32 rows per split.
+  const int64_t fit = (T + kPhases * 16 - 1) / (kPhases * 16);
   const int64_t target = static_cast<int64_t>(num_sms) * 2;
-  int64_t s = (target + ncb - 1) / ncb;
-  const int64_t max_by_rows = (T + 31) / 32;  // at least 32 rows per split
+  int64_t s;
+  if (fit <= kMaxClusterSplits) {
+    const int64_t ncb = (d + kClusterChannels - 1) / kClusterChannels;
+    s = (target + ncb - 1) / ncb;
+    if (s < fit) s = fit;
+    if (s > kMaxClusterSplits) s = kMaxClusterSplits;
+  } else {
+    const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
+    s = (target + ncb - 1) / ncb;
+    if (s > kMaxSplits) s = kMaxSplits;
+  }
+  const int64_t max_by_rows = (T + 31) / 32;
   if (s > max_by_rows) s = max_by_rows;
-  if (s > 16) s = 16;
   if (s < 1) s = 1;
   int64_t rps = (T + s - 1) / s;
   if (rps < 1) rps = 1;
@@ -546,25 +597,21 @@ cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, flo
                   rows_per_split, partial, counters, D, Dr, Dh, xh, nullptr, status, stream, pdl);
 }
 
-bool act_norm_scale_fused(bool x_f32, int64_t d, int64_t splits, int64_t rows_per_split, float p,
-                          int num_sms) {
-  return x_f32 ? fused_fits_p<float>(p, d, splits, rows_per_split, num_sms)
-               : fused_fits_p<__nv_bfloat16>(p, d, splits, rows_per_split, num_sms);
+bool act_norm_scale_fused(bool x_f32, int64_t splits, int64_t rows_per_split, float p) {
+  return x_f32 ? fused_fits_p<float>(p, splits, rows_per_split)
+               : fused_fits_p<__nv_bfloat16>(p, splits, rows_per_split);
 }
 
 cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                                   float lambda, float alpha, int64_t splits,
-                                  int64_t rows_per_split, double* partial,
-                                  uint32_t* counters, float* D, float* Dr, void* xh,
-                                  void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
-                                  bool* launched, float* Dh) {
+                                  int64_t rows_per_split, float* D, float* Dr, void* xh, void* xb,
+                                  uint32_t* status, cudaStream_t stream, bool* launched,
+                                  float* Dh) {
   if (x_f32)
     return launch_fused_p(static_cast<const float*>(X), d, T, p, lambda, alpha, splits,
-                          rows_per_split, partial, counters, D, Dr, Dh, xh, xb, status, num_sms,
-                          stream, launched);
+                          rows_per_split, D, Dr, Dh, xh, xb, status, stream, launched);
   return launch_fused_p(static_cast<const __nv_bfloat16*>(X), d, T, p, lambda, alpha, splits,
-                        rows_per_split, partial, counters, D, Dr, Dh, xh, nullptr, status,
-                        num_sms, stream, launched);
+                        rows_per_split, D, Dr, Dh, xh, nullptr, status, stream, launched);
 }
 
 }  // namespace ttq

@@ -255,6 +255,15 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
           dst[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
           dst[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
         }
+        // s (q - z) alone is wanted when codes is null (the forward's
+        // materialised weight): the packing and the stores below are skipped
+        // (a grid-uniform branch, so the INT3 shuffles stay uniform)
+        const bool want_codes = codes != nullptr;
+        if (active && (tx & (gthreads - 1)) == 0) {
+          // s (q - z) is formed in binary16 by the product: |q - z| <= 2^b - 1
+          ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QSPAN) > 65504.f;
+        }
+        if (!want_codes) continue;
         uint32_t lo = 0, hi = 0;  // INT4: codes 0-7 and 8-15; INT3: 24 bits each
         if (BITS == 4) {
           lo = __byte_perm(nibbles4(qp[0], qp[1]), nibbles4(qp[2], qp[3]), 0x5410);
@@ -274,8 +283,6 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
           scales[row * ngroups + kgroup] = s16;
           zeros[row * ngroups + kgroup] =
               __hsub(__ushort_as_half(static_cast<uint16_t>(0x6400u | z)), __ushort_as_half(0x6400));
-          // s (q - z) is formed in binary16 by the product: |q - z| <= 2^b - 1
-          ovf |= static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QSPAN) > 65504.f;
         }
         // the lane's 16 codes are 16*BITS bits at bit 16*BITS*(col/16)
         if (BITS == 4) {
@@ -323,7 +330,8 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
 // group's threads reduce the range with shuffles); the 16 one-byte codes
 // of a thread are one 16-byte store.  With WQ the kernel also writes the
 // binary16 s * e4m3(code) (the E4M3 value converts to binary16 exactly; the
-// product with s rounds once).
+// product with s rounds once); with WQ and codes == nullptr it writes that
+// alone (no codes, scales or zeros).
 template <typename WT, bool WQ>
 __global__ void __launch_bounds__(kThreads, 2) qdq_fp8_kernel(
     const WT* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D, int group,
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_fp8_kernel(
       for (int i = 0; i < 8; ++i)
         pr[i] = static_cast<uint32_t>(
             __nv_cvt_float2_to_fp8x2(__fmul2_rn(x[i], inv2), __NV_SATFINITE, __NV_E4M3));
-      if (active) {
+      if (active && codes != nullptr) {
         *reinterpret_cast<uint4*>(codes + row * wpr + (col >> 2)) =
             make_uint4(pr[0] | (pr[1] << 16), pr[2] | (pr[3] << 16), pr[4] | (pr[5] << 16),
                        pr[6] | (pr[7] << 16));
@@ -424,8 +432,10 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_fp8_kernel(
         dst[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
       }
       if (active && (tx & (gthreads - 1)) == 0) {
-        scales[row * ngroups + kgroup] = s16;
-        zeros[row * ngroups + kgroup] = __ushort_as_half(0);
+        if (codes != nullptr) {
+          scales[row * ngroups + kgroup] = s16;
+          zeros[row * ngroups + kgroup] = __ushort_as_half(0);
+        }
         ovf |= static_cast<bool>(__hisinf(s16)) || s * 448.0f > 65504.f;
       }
     }

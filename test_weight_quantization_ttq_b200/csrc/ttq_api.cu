@@ -412,8 +412,8 @@ ttq_status run_single_pass(const void* W, const float* Dh, const void* Xh, const
 }
 
 // Step (1) and, when xh is non-null, the product's binary16 operand
-// X D^(-1/2) in xh: one fused cooperative kernel when every block's tile of
-// X fits in shared memory and the grid is resident at once, else the
+// X D^(-1/2) in xh: one fused kernel (the splits of a column block form a
+// thread-block cluster) when each split's rows fit in registers, else the
 // statistic kernel followed by the scaling kernel.  Either way D and D_rsqrt
 // are the same bits (same splits, same merge order).  xb: bf16 copy of a
 // float32 X (or null).
@@ -429,8 +429,7 @@ ttq_status run_statistic(const void* X, ttq_dtype dtype, int64_t d, int64_t T, f
   if (xh != nullptr) {
     bool fused = false;
     const ttq_status st = cuda_status(launch_act_norm_scale(X, f32, d, T, p, lambda, alpha,
-                                                            splits, rps, partial, status + 64, D,
-                                                            Dr, xh, xb, status, device_sms(), s,
+                                                            splits, rps, D, Dr, xh, xb, status, s,
                                                             &fused, Dh));
     if (st != TTQ_OK || fused) return st;
   }
@@ -536,7 +535,7 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
   const bool f32 = dtype == TTQ_F32;
   int n = 1;  // statistic
   if (dp > 0) {
-    if (!act_norm_scale_fused(f32, d, splits, rps, p, device_sms())) ++n;  // separate scaling
+    if (!act_norm_scale_fused(f32, splits, rps, p)) ++n;                  // separate scaling
     const bool one_pass = T > 0 && single_pass_decode(dtype, scheme, d, dp, T, bits, group);
     if (!one_pass) ++n;                                                    // quantiser
     if (T > 0) {
@@ -594,7 +593,11 @@ ttq_status ttq_quantize_weight_ex(const void* W, ttq_dtype dtype, int64_t dp, in
   if (bits < 1 || bits > 8 || group < 1) return TTQ_ERR_INVALID_ARG;
   if (!valid_qparams(bits, group) || !scheme_bits_ok(scheme, bits)) return TTQ_ERR_UNSUPPORTED;
   if (d < group || d % group != 0 || dp < 0) return TTQ_ERR_INVALID_ARG;
-  if (dp > 0 && (W == nullptr || codes == nullptr || scales == nullptr || zeros == nullptr))
+  // the codes, scales and zeros are written together, or (with W_hat) all left out
+  const bool no_codes = codes == nullptr && scales == nullptr && zeros == nullptr;
+  if (dp > 0 && (W == nullptr || (no_codes ? W_hat == nullptr
+                                           : (codes == nullptr || scales == nullptr ||
+                                              zeros == nullptr))))
     return TTQ_ERR_INVALID_ARG;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
   if ((W && !aligned16(W)) || (D && !aligned16(D)) || (codes && !aligned16(codes)))
@@ -768,11 +771,16 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, co
   uint16_t* scales = reinterpret_cast<uint16_t*>(ws_at(ws, L.scales));
   uint16_t* zeros = reinterpret_cast<uint16_t*>(ws_at(ws, L.zeros));
   void* wq = materialize_w(dp, T, bits, d) ? ws_at(ws, L.wq) : nullptr;
+  // with the materialised weight the product reads W_hat alone: the codes,
+  // scales and zeros are not written
+  uint32_t* codes_out = wq ? nullptr : codes;
+  uint16_t* scales_out = wq ? nullptr : scales;
+  uint16_t* zeros_out = wq ? nullptr : zeros;
   st = cuda_status(scheme == TTQ_QSCHEME_FP8_E4M3
-                       ? launch_qdq_fp8(W, f32, dp, d, D, group, codes, scales, zeros, status,
-                                        device_sms(), s, true, wq)
-                       : launch_qdq_pack(W, f32, dp, d, D, bits, group, codes, scales, zeros,
-                                         status, device_sms(), s, true, wq,
+                       ? launch_qdq_fp8(W, f32, dp, d, D, group, codes_out, scales_out, zeros_out,
+                                        status, device_sms(), s, true, wq)
+                       : launch_qdq_pack(W, f32, dp, d, D, bits, group, codes_out, scales_out,
+                                         zeros_out, status, device_sms(), s, true, wq,
                                          scheme == TTQ_QSCHEME_SYMMETRIC));
   if (st != TTQ_OK || T == 0) return st;
 

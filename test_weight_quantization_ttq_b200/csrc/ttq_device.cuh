@@ -46,6 +46,30 @@ __device__ __forceinline__ void allow_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ----------------------------------------------------- thread-block cluster
+// The hardware barrier among all threads of all blocks of a cluster, in
+// two halves: arrive (release: this thread's earlier shared-memory writes
+// become visible to the cluster) and wait (acquire).  Every thread of every
+// block executes both, unconditionally, so the wait always completes.
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// A float64 in the shared memory of block `rank` of this cluster, at the
+// offset that `local` has in this block's shared memory.
+__device__ __forceinline__ double ld_cluster_f64(const double* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  double v;
+  asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(v) : "r"(remote) : "memory");
+  return v;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
@@ -99,44 +123,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (global_timer_ns() - t0 > limit_ns) return false;
     }
   }
-}
-
-// ------------------------------------------------------ inter-block barrier
-// Barrier among the n blocks of a grid that share the global word `count`
-// (all of them resident at once: a cooperative launch).  `count` is zero
-// before and after every use: each block adds 1 when it arrives (a release
-// that publishes the block's earlier global writes), waits with acquire
-// loads until all n have arrived, and adds 1 when it leaves; the block that
-// brings it to 2n sets it back to zero.  A wait
-// longer than limit_ns sets TTQ_FLAG_TIMEOUT and lets the block go on (its
-// later results are then not valid, and the count is left off zero until
-// the workspace is re-initialised); the result is false in that case.
-// `ok_smem` is a shared int used to broadcast the outcome to the block.
-__device__ __forceinline__ bool group_barrier(uint32_t* count, uint32_t n, uint32_t* status,
-                                              int* ok_smem, uint64_t limit_ns = kWaitLimitNs) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int ok = 1;
-    // release at gpu scope: the block's writes (ordered before this thread
-    // by the block barrier) are visible to whoever observes the increment
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(count) : "memory");
-    const uint64_t t0 = global_timer_ns();
-    for (;;) {
-      uint32_t cur;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(count) : "memory");
-      if (cur >= n) break;
-      if (global_timer_ns() - t0 > limit_ns) {
-        set_flag(status, TTQ_FLAG_TIMEOUT);
-        ok = 0;
-        break;
-      }
-      __nanosleep(32);
-    }
-    if (atomicAdd(count, 1u) == 2u * n - 1u) atomicExch(count, 0u);
-    *ok_smem = ok;
-  }
-  __syncthreads();
-  return *ok_smem != 0;
 }
 
 // -------------------------------------------------------------------- TMA

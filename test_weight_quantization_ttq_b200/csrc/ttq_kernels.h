@@ -49,23 +49,22 @@ cudaError_t launch_act_norm(const void* X, bool x_f32, int64_t d, int64_t T, flo
 cudaError_t launch_sqrt_f32(const float* D, float* h, int64_t d, cudaStream_t stream);
 
 // Whether launch_act_norm_scale would run (on the current device).
-bool act_norm_scale_fused(bool x_f32, int64_t d, int64_t splits, int64_t rows_per_split, float p,
-                          int num_sms);
+bool act_norm_scale_fused(bool x_f32, int64_t splits, int64_t rows_per_split, float p);
 
 // Step (1) fused with the binary16 operand X D^(-1/2) (written to xh, which
-// must be non-null; xb as for launch_act_norm).  One cooperative launch over
-// the same splits as launch_act_norm, with D bit-identical to it; X is read
-// once and held in registers.  `counters` as for launch_act_norm.  Launches
-// only when each thread's rows of X fit in its registers (rows_per_split <=
-// 128 for bf16, 64 for float32) and the whole grid is resident at once;
-// *launched tells whether it ran (when it did not, nothing was queued and
-// the result is cudaSuccess).
+// must be non-null; xb as for launch_act_norm).  One launch over the same
+// splits as launch_act_norm, with D bit-identical to it; the splits of a
+// 128-channel column block are one thread-block cluster.  X is read once and
+// held in registers.  Launches only when each thread's rows of X fit in its
+// registers (rows_per_split <= 256 for bf16, 128 for float32), there are at
+// most 8 splits and such a cluster can be resident; *launched tells whether
+// it ran (when it did not, nothing was queued and the result is
+// cudaSuccess).
 cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t T, float p,
                                   float lambda, float alpha, int64_t splits,
-                                  int64_t rows_per_split, double* partial,
-                                  uint32_t* counters, float* D, float* Dr, void* xh,
-                                  void* xb, uint32_t* status, int num_sms, cudaStream_t stream,
-                                  bool* launched, float* Dh = nullptr);
+                                  int64_t rows_per_split, float* D, float* Dr, void* xh, void* xb,
+                                  uint32_t* status, cudaStream_t stream, bool* launched,
+                                  float* Dh = nullptr);
 
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null); with wq
 // non-null also the dequantised weight s (q - z) as binary16 [dp][d].

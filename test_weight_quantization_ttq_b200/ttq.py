@@ -357,15 +357,23 @@ def ttq_quantize_weight(W, D, bits, group, ws=None, codes=None, scales=None, zer
 
 
 def ttq_quantize_weight_ex(W, D, bits, group, scheme, ws=None, codes=None, scales=None, zeros=None,
-                           W_hat=None, stream=None):
+                           W_hat=None, stream=None, with_codes=True):
     """Codes, scales and zeros under the given TTQ_QSCHEME_*; W_hat (binary16
-    s (q - z), optional) is written when given."""
+    s (q - z), optional) is written when given.  With with_codes=False (and
+    W_hat given) only W_hat is written and (None, None, None) is returned."""
     _matrix(W, "W", dtypes=_FLOAT_IN)
     dp, d = W.shape
     _quant_outputs(dp, d, D, bits, group, codes, scales, zeros, W_hat, "ttq_quantize_weight_ex")
     dev = W.device
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
+    if not with_codes:
+        if W_hat is None:
+            raise ValueError("ttq_quantize_weight_ex: with_codes=False needs W_hat")
+        _check(lib().ttq_quantize_weight_ex(
+            _dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group, scheme, None, None, None,
+            _dev(W_hat, "W_hat"), _dev(ws, "ws"), _nbytes(ws), _stream(stream)), "ttq_quantize_weight_ex")
+        return None, None, None
     if codes is None:
         codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device=dev)
     if scales is None:
@@ -380,14 +388,23 @@ def ttq_quantize_weight_ex(W, D, bits, group, scheme, ws=None, codes=None, scale
 
 
 def ttq_quantize_dequant_weight(W, D, bits, group, ws=None, codes=None, scales=None, zeros=None,
-                                W_hat=None, stream=None):
-    """ttq_quantize_weight plus W_hat [d'][d] binary16 (torch.float16) = s (q - z)."""
+                                W_hat=None, stream=None, with_codes=True):
+    """ttq_quantize_weight plus W_hat [d'][d] binary16 (torch.float16) = s (q - z).
+    With with_codes=False only W_hat is written (codes, scales, zeros are None)."""
     _matrix(W, "W", dtypes=_FLOAT_IN)
     dp, d = W.shape
     _quant_outputs(dp, d, D, bits, group, codes, scales, zeros, W_hat, "ttq_quantize_dequant_weight")
     dev = W.device
     if ws is None:
         ws = new_workspace(d, 0, 0, 0, bits, group, _dtype_code(W), dev, stream)
+    if W_hat is None:
+        W_hat = torch.empty((dp, d), dtype=torch.float16, device=dev)
+    if not with_codes:
+        _check(lib().ttq_quantize_dequant_weight(
+            _dev(W, "W"), _dtype_code(W), dp, d, _dev(D, "D"), bits, group, None, None, None,
+            _dev(W_hat, "W_hat"), _dev(ws, "ws"), _nbytes(ws), _stream(stream)),
+            "ttq_quantize_dequant_weight")
+        return None, None, None, W_hat
     if codes is None:
         codes = torch.empty((dp, d * bits // 32), dtype=torch.int32, device=dev)
     if scales is None:
@@ -467,7 +484,6 @@ def ttq_dequant_gemm(codes, scales, zeros, D_rsqrt, X, A, B, bits, group, ws=Non
 
 
 TTQ_TESTING_WAIT_MBARRIER = 0
-TTQ_TESTING_WAIT_GRID_BARRIER = 1
 
 
 def ttq_testing_wait_timeout(kind, limit_ns, blocks, ws, stream=None) -> None:

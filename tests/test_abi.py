@@ -79,6 +79,26 @@ def test_workspace_layout_is_consistent(L):
             assert lay.xb > 0 and lay.ab > 0
 
 
+@pytest.mark.parametrize("d,T,splits", [
+    (4096, 2048, 8),     # 32 column blocks of 128 channels: 8 splits of 256 rows (one cluster)
+    (8192, 2048, 8),     # 256 rows per split still needs 8 splits
+    (4096, 1024, 8),     # two blocks per SM would take 10: capped at a cluster of 8
+    (4096, 150, 5),      # no more splits than ceil(T / 32): 5 of 30 rows
+    (4096, 16, 1),
+    (4096, 0, 1),
+    (4096, 4096, 16),    # too many rows for 8 splits of 256: 16 blocks of 256 channels x 16
+    (8192, 8192, 10),    # 32 blocks of 256 channels: 10 splits
+])
+def test_statistic_split_plan(L, d, T, splits):
+    """The token splits of the statistic pass: the fused kernel's clusters
+    hold at most 8 splits of at most 256 rows."""
+    lay = ttq.ttq_workspace_get_layout(d, 0, T, 0, 4, 32, ttq.TTQ_BF16)
+    assert lay.splits == splits
+    if T:
+        rps = -(-T // splits)
+        assert -(-T // rps) == splits and splits <= -(-T // 32)
+
+
 def test_dequantised_weight_only_for_long_inputs(L):
     """The forward materialises s (q - z) only for more than 256 tokens."""
     for T in (0, 1, 16, 256):
@@ -118,6 +138,10 @@ def test_rejections_before_device_work(L):
     assert L.ttq_act_norm_scale(16, 1, 64, 4, 2.0, 0.0, 0.5, None, None, 40, 256, 1 << 20, None) == ttq.TTQ_ERR_INVALID_ARG
     # dequantised-weight entry points: W_hat required, shapes checked before any CUDA call
     assert L.ttq_quantize_dequant_weight(16, 1, 4, 64, None, 4, 64, 16, 16, 16, None, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    # codes, scales and zeros are given together, or all left out with W_hat given
+    assert L.ttq_quantize_weight_ex(16, 1, 4, 64, None, 4, 64, 0, None, None, None, None, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_quantize_weight_ex(16, 1, 4, 64, None, 4, 64, 0, 16, None, None, 16, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
+    assert L.ttq_quantize_weight_ex(16, 1, 4, 64, None, 4, 64, 0, None, 16, 16, 16, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_quantize_dequant_weight(16, 1, 4, 64, None, 5, 64, 16, 16, 16, 16, 256, 4096, None) == ttq.TTQ_ERR_UNSUPPORTED
     assert L.ttq_dequantized_gemm(16, 16, 60, 4, 4, 16, 1, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG
     assert L.ttq_dequantized_gemm(16, None, 64, 4, 4, 16, 1, 256, 4096, None) == ttq.TTQ_ERR_INVALID_ARG

@@ -68,6 +68,11 @@ def test_fp8_quantizer_bit_exact(O, case):
     s16 = np.repeat(sc_o.view(np.float16), group, axis=1)
     want = (s16.astype(np.float32) * _e4m3_to_f16(q).astype(np.float32)).astype(np.float16)
     assert np.array_equal(W_hat.cpu().numpy().view(np.uint16), want.view(np.uint16))
+    # W_hat alone (no codes, scales or zeros), as the forward writes it above 16 tokens
+    W_hat1 = torch.empty_like(W_hat)
+    ttq.ttq_quantize_weight_ex(W, Dd, 8, group, FP8, W_hat=W_hat1, with_codes=False)
+    torch.cuda.synchronize()
+    assert torch.equal(W_hat1.view(torch.int16), W_hat.view(torch.int16))
 
 
 FORWARD_CASES = [

@@ -1,7 +1,8 @@
 """The forward computes the statistic D and the binary16 operand X D^(-1/2)
-either in one cooperative kernel (when every block's tile of X fits in
-shared memory and the grid is resident at once) or in two kernels.  Both
-must give exactly what the stand-alone entry points ttq_act_norm and
+either in one kernel (when each token split's rows fit in registers: the
+splits of a 128-channel column block then form one thread-block cluster and
+merge through distributed shared memory) or in two kernels.  Both must give
+exactly what the stand-alone entry points ttq_act_norm and
 ttq_scale_activations give (TTQ paper, section 2.1: D_ii = (||X_i,:||_p +
 lambda)^alpha; section 2.2: the product runs on X D^(-1/2))."""
 from __future__ import annotations
@@ -29,12 +30,14 @@ def _spec(name, d, dp, T, p=2.0, alpha=0.5, dtype="bf16", r=0, bits=4, group=32)
 
 
 CASES = [
-    synth.C2.with_(dp=256),                                  # fused: 16 x 16 blocks of 128 rows
+    synth.C2.with_(dp=256),                                  # fused: 32 clusters of 8 splits of 256 rows
     _spec("ragged_channels_p3", d=96, dp=64, T=19, p=3.0),   # one partial column block, any p
     _spec("ragged_block_p1", d=288, dp=64, T=1000, p=1.0, alpha=0.25),
+    _spec("cluster_of_5", d=4096, dp=64, T=150),              # 5 splits of 30 rows
     _spec("f32_lowrank", d=448, dp=96, T=77, dtype="f32", r=16),
+    _spec("f32_two_kernel", d=1024, dp=64, T=2048, dtype="f32"),  # 256 rows: too many for f32
     _spec("one_token", d=4096, dp=64, T=1),
-    _spec("wide_two_kernel", d=8192, dp=64, T=2048),          # X too large for one resident grid
+    _spec("wide", d=8192, dp=64, T=2048),                     # 64 clusters, more than one wave
     _spec("long_two_kernel", d=4096, dp=64, T=4096, alpha=0.25),
     _spec("no_tokens", d=512, dp=64, T=0),
 ]
@@ -87,8 +90,8 @@ def test_forward_lowrank_f32_matches_oracle(O):
 
 
 def test_workspace_reused_across_shapes():
-    """The grid barrier's words are left at zero, so one workspace serves
-    calls of different grid sizes in a row."""
+    """The statistic's merge tickets are left at zero, so one workspace
+    serves calls of different grid sizes in a row."""
     big = synth.C2.with_(dp=256)
     ws = ttq.new_workspace(big.d, big.dp, big.T, 0, big.bits, big.group, ttq.TTQ_BF16)
     outs = []
@@ -111,12 +114,12 @@ def test_forward_kernel_count_matches_launches():
     """ttq_linear_forward_kernels tells how many kernels a forward call
     enqueues; a CUDA activity trace of one call sees exactly that many of the
     library's kernels (the statistic fused with the scaling of X where the
-    grid fits, two kernels where it does not)."""
+    rows fit in registers, two kernels where they do not)."""
     from torch.autograd import DeviceType
     from torch.profiler import ProfilerActivity, profile
 
     cases = [(synth.C2.with_(dp=512), 3, True),
-             (_spec("wide_two_kernel", d=8192, dp=64, T=2048), 4, False),
+             (_spec("long_two_kernel", d=8192, dp=64, T=4096), 4, False),
              (_spec("f32_lowrank", d=448, dp=96, T=77, dtype="f32", r=16), 6, True),
              (_spec("no_tokens", d=512, dp=64, T=0), 2, True),
              # a few tokens: statistic, then the single-pass product

@@ -1,10 +1,10 @@
 """For more than 256 tokens the forward writes the dequantised weight
-s (q - z) in binary16 once (with the codes) and runs the product on it as a
-plain tensor-core operand.  Those operand values must be exactly the
-dequantisation of the codes, scales and zeros the call leaves in its
-workspace (TTQ paper, section 2.1: W_hat = Q[W D^(1/2)] D^(-1/2), with the
-D^(-1/2) factor carried by X), and the product must equal the one that
-dequantises inside the GEMM (ttq_dequant_gemm) on the same operands."""
+s (q - z) in binary16 once (in place of the codes) and runs the product on
+it as a plain tensor-core operand.  Those operand values must be exactly
+the dequantisation of the codes, scales and zeros that the quantiser gives
+for the call's D (TTQ paper, section 2.1: W_hat = Q[W D^(1/2)] D^(-1/2),
+with the D^(-1/2) factor carried by X), and the product must equal the one
+that dequantises inside the GEMM (ttq_dequant_gemm) on the same operands."""
 from __future__ import annotations
 
 import numpy as np
@@ -52,16 +52,20 @@ def test_materialized_weight_is_the_dequantised_codes(O, spec):
     assert st == ttq.TTQ_OK, flags
     v = ttq.workspace_views(ws, spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt)
     assert "wq" in v
-    q = O.unpack(P.u32(v["codes"]), spec.d, spec.bits).astype(np.float64)
-    s = P.u16(v["scales"]).view(np.float16).astype(np.float64)
-    z = P.u16(v["zeros"]).view(np.float16).astype(np.float64)
+    # the forward keeps W_hat and no codes; the quantiser, given the
+    # forward's D, gives the codes W_hat must be the dequantisation of
+    codes, scales, zeros = ttq.ttq_quantize_weight(W, v["D"], spec.bits, spec.group)
+    torch.cuda.synchronize()
+    q = O.unpack(P.u32(codes), spec.d, spec.bits).astype(np.float64)
+    s = P.u16(scales).view(np.float16).astype(np.float64)
+    z = P.u16(zeros).view(np.float16).astype(np.float64)
     k = np.arange(spec.d) // spec.group
     # s (q - z) is exact in float64; one rounding to binary16
     ref = (s[:, k] * (q - z[:, k])).astype(np.float16)
     assert np.array_equal(v["wq"].cpu().numpy().view(np.uint16), ref.view(np.uint16))
     # the same product from the codes, dequantised inside the GEMM
     if spec.r == 0:
-        Y2 = ttq.ttq_dequant_gemm(v["codes"], v["scales"], v["zeros"], None, v["xh"], None, None,
+        Y2 = ttq.ttq_dequant_gemm(codes, scales, zeros, None, v["xh"], None, None,
                                   spec.bits, spec.group, y_dtype=torch.float32)
         torch.cuda.synchronize()
         rms = float(Y2.double().pow(2).mean().sqrt())
@@ -86,7 +90,10 @@ def test_composed_materialized_steps_equal_forward():
     Y2 = ttq.ttq_dequantized_gemm(W_hat, Xs, y_dtype=torch.float32)
     Yb = ttq.ttq_dequantized_gemm(W_hat, Xs, y_dtype=torch.bfloat16)
     codes1, sc1, ze1 = ttq.ttq_quantize_weight(W, D, spec.bits, spec.group)
+    # W_hat alone (no codes, scales or zeros), as the forward writes it
+    _, _, _, W_hat1 = ttq.ttq_quantize_dequant_weight(W, D, spec.bits, spec.group, with_codes=False)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)
     assert torch.equal(Yb, Y2.to(torch.bfloat16))
     assert torch.equal(codes, codes1) and torch.equal(sc, sc1) and torch.equal(ze, ze1)
+    assert torch.equal(W_hat1.view(torch.int16), W_hat.view(torch.int16))

@@ -192,7 +192,19 @@ def test_forward_matches_oracle(O, spec):
     assert np.max(np.abs(D - ref["D"]) / ref["D"]) <= P.D_RTOL
     codes_dev = views["codes"]
     sc_dev, ze_dev = views["scales"], views["zeros"]
-    if ttq.ttq_workspace_get_layout(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt).tickets:
+    if "wq" in views:
+        # the forward kept the binary16 W_hat and no codes: the quantiser,
+        # given the forward's D, gives the codes, and W_hat is their
+        # dequantisation to the bit
+        codes_dev, sc_dev, ze_dev = ttq.ttq_quantize_weight(W, views["D"], spec.bits, spec.group)
+        torch.cuda.synchronize()
+        q = O.unpack(P.u32(codes_dev), spec.d, spec.bits).astype(np.float64)
+        k = np.arange(spec.d) // spec.group
+        sv = P.u16(sc_dev).view(np.float16).astype(np.float64)[:, k]
+        zv = P.u16(ze_dev).view(np.float16).astype(np.float64)[:, k]
+        assert np.array_equal(views["wq"].cpu().numpy().view(np.uint16),
+                              (sv * (q - zv)).astype(np.float16).view(np.uint16))
+    elif ttq.ttq_workspace_get_layout(spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group, dt).tickets:
         # the forward took the single-pass product, which writes no codes: the
         # same kernel, given the forward's own D and X D^(-1/2), stores them on
         # request, and its Y is the forward's to the bit

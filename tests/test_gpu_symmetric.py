@@ -98,12 +98,24 @@ def test_symmetric_forward_matches_oracle(O, spec):
     st, flags = ttq.ttq_get_status(ws)
     assert st == ttq.TTQ_OK, flags
     v = ttq.workspace_views(ws, spec.d, spec.dp, spec.T, spec.r, spec.bits, spec.group)
+    codes_d, sc_d, ze_d = v["codes"], v["scales"], v["zeros"]
+    if "wq" in v:
+        # the forward kept the binary16 W_hat only: the quantiser, given the
+        # forward's D, gives the codes, and W_hat must be their dequantisation
+        codes_d, sc_d, ze_d = ttq.ttq_quantize_weight_ex(W, v["D"], spec.bits, spec.group, SYM)
+        torch.cuda.synchronize()
+        q = O.unpack(P.u32(codes_d), spec.d, spec.bits).astype(np.float64)
+        k = np.arange(spec.d) // spec.group
+        sv = P.u16(sc_d).view(np.float16).astype(np.float64)[:, k]
+        zv = P.u16(ze_d).view(np.float16).astype(np.float64)[:, k]
+        assert np.array_equal(v["wq"].cpu().numpy().view(np.uint16),
+                              (sv * (q - zv)).astype(np.float16).view(np.uint16))
     same_d = v["D"].cpu().numpy() == ref["D"].astype(np.float32)
     group_ok = same_d.reshape(-1, spec.group).all(axis=1)
     assert group_ok.mean() >= 0.99
     wpg = spec.group * spec.bits // 32
-    codes = P.u32(v["codes"]).reshape(spec.dp, -1, wpg)
+    codes = P.u32(codes_d).reshape(spec.dp, -1, wpg)
     assert np.array_equal(codes[:, group_ok], ref["codes"].reshape(spec.dp, -1, wpg)[:, group_ok])
-    assert np.array_equal(P.u16(v["scales"])[:, group_ok], ref["scales"][:, group_ok])
-    assert np.all(P.u16(v["zeros"]).view(np.float16) == 2 ** (spec.bits - 1))
+    assert np.array_equal(P.u16(sc_d)[:, group_ok], ref["scales"][:, group_ok])
+    assert np.all(P.u16(ze_d).view(np.float16) == 2 ** (spec.bits - 1))
     assert P.y_error(Y.cpu().numpy()[:, rows], ref["Y"]) <= P.Y_TOL
