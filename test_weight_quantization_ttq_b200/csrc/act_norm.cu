@@ -313,29 +313,32 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
   const int64_t t_end = min(T, t_begin + rows_per_split);
   const bool clustered = splits > 1;
 
+  // this thread's rows: t0 + 16 k for k < nk (none when its channels are
+  // past d), at a fixed stride from one base pointer
+  const int64_t t0 = t_begin + phase;
+  const int nk = active && t0 < t_end
+                     ? static_cast<int>(min(static_cast<int64_t>(R), (t_end - t0 + kPhases - 1) / kPhases))
+                     : 0;
+  const int64_t rs = kPhases * d;
+  const XT* xp = X + (nk > 0 ? t0 * d + c0 : 0);
+
   // all rows of this thread in flight at once
   Raw8<XT> raw[R];
-  if (active) {
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
-      const int64_t t = t_begin + phase + kPhases * k;
-      if (t < t_end) raw[k].load(X + t * d + c0);
-    }
-  }
+  for (int k = 0; k < R; ++k)
+    if (k < nk) raw[k].load(xp + k * rs);
 
   // (1) this phase's sums of |x|^p, rows in increasing order
   double acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-  if (active) {
 #pragma unroll
-    for (int k = 0; k < R; ++k) {
-      if (t_begin + phase + kPhases * k < t_end) {
-        float v[8];
-        raw[k].unpack(v);
+  for (int k = 0; k < R; ++k) {
+    if (k < nk) {
+      float v[8];
+      raw[k].unpack(v);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v[e], p);
-      }
+      for (int e = 0; e < 8; ++e) acc[e] += abs_pow<PK>(v[e], p);
     }
   }
 #pragma unroll
@@ -385,32 +388,34 @@ __global__ void __launch_bounds__(kThreads, 2) act_norm_scale_kernel(
   if (clustered) cluster_arrive_relaxed();
   __syncthreads();
 
-  // (3) binary16(x * D^(-1/2)) (and the bf16 copy of a float32 X)
-  bool out_of_range = false;
-  if (active) {
-    float f[8];
+  // (3) binary16(x * D^(-1/2)) (and the bf16 copy of a float32 X); the
+  // products go through the packed f32x2 multiply (each lane rounded as
+  // the scalar one), and their largest magnitude is checked once
+  float amax = 0.f;
+  if (nk > 0) {
+    float2 f[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) f[e] = dr_s[cl + e];
+    for (int q = 0; q < 4; ++q) f[q] = make_float2(dr_s[cl + 2 * q], dr_s[cl + 2 * q + 1]);
+    __half* hp = xh + t0 * d + c0;
 #pragma unroll
     for (int k = 0; k < R; ++k) {
-      const int64_t t = t_begin + phase + kPhases * k;
-      if (t < t_end) {
+      if (k < nk) {
         float v[8];
         raw[k].unpack(v);
         __half2 h[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float a = __fmul_rn(v[2 * q], f[2 * q]);
-          const float b = __fmul_rn(v[2 * q + 1], f[2 * q + 1]);
-          h[q] = __floats2half2_rn(a, b);
-          out_of_range |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
+          const float2 a = __fmul2_rn(make_float2(v[2 * q], v[2 * q + 1]), f[q]);
+          h[q] = __floats2half2_rn(a.x, a.y);
+          amax = fmaxf(amax, fmaxf(fabsf(a.x), fabsf(a.y)));
         }
-        *reinterpret_cast<uint4*>(xh + t * d + c0) = *reinterpret_cast<const uint4*>(h);
-        if (xb != nullptr) store8_bf16(xb + t * d + c0, v);
+        *reinterpret_cast<uint4*>(hp + k * rs) = *reinterpret_cast<const uint4*>(h);
+        if (xb != nullptr) store8_bf16(xb + t0 * d + c0 + k * rs, v);
       }
     }
   }
-  if (__any_sync(0xffffffffu, out_of_range) && lane == 0) set_flag(status, TTQ_FLAG_X_RANGE);
+  // |x D^(-1/2)| beyond binary16 (a NaN x makes D NaN, flagged there)
+  if (__any_sync(0xffffffffu, amax > 65504.f) && lane == 0) set_flag(status, TTQ_FLAG_X_RANGE);
   if (clustered) cluster_wait_acquire();
 }
 

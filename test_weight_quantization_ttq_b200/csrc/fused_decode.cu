@@ -82,22 +82,7 @@ struct FdDev {
   uint32_t* status;
 };
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
 
 __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                         uint32_t b1) {
@@ -177,7 +162,7 @@ __device__ __forceinline__ GroupQ<BITS> group_params(float mn, float mx, const f
   GroupQ<BITS> p;
   const float range = __fsub_rn(mx, mn);
   p.bad = !(range <= 3.402823466e38f);
-  float s32 = __fdiv_rn(range, static_cast<float>(QMAX));
+  float s32 = div_by_const<QMAX>(range);
   if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
   const __half s16 = __float2half_ru(s32);
   p.sf = __half2float(s16);

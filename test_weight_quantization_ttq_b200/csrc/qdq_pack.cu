@@ -9,7 +9,9 @@
 //   s32 = (M - m) / (2^b - 1), floored at 2^-14; s = binary16 round-up(s32);
 //   inv = 1 / s; z = clamp(rint(-m * inv)); q = clamp(rint(x * inv) + z),
 // where the two products inside rint are exact (one fused multiply-add
-// rounds them straight to the integer).  Every other operation is an
+// rounds them straight to the integer).  The quotient s32 is the correctly
+// rounded one, formed by div_by_const (a product with the rounded
+// reciprocal and one exact correction).  Every other operation is an
 // explicitly rounded intrinsic, so no contraction can change a result.
 //
 // Layout of the work: a block owns a tile of `cw` consecutive input channels
@@ -23,6 +25,8 @@
 // The kernel is HBM-bound: it reads W once and writes d*b/8 + 4d/g bytes per
 // row.
 #include <cuda_fp8.h>
+
+#include <atomic>
 
 #include <type_traits>
 
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
         // asymmetric: the range [m, M] over 2^b - 1 steps; symmetric: max|x|
         // over 2^(b-1) - 1 steps
         const float span = SYM ? max_nan(mx, -mn) : range;
-        float s32 = __fdiv_rn(span, static_cast<float>(QSPAN));
+        float s32 = div_by_const<QSPAN>(span);
         if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
         const __half s16 = __float2half_ru(s32);
         const float s = __half2float(s16);
@@ -319,6 +323,331 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_pack_kernel(
   if (__any_sync(0xffffffffu, bad) && lane == 0) set_flag(status, TTQ_FLAG_NONFINITE);
 }
 
+// The scale, its reciprocal and the zero point of one group of one row from
+// the group's range [mn, mx], in the quantiser's binary32 order (the same
+// operations as qdq_pack_kernel), and whether the group is bad (a NaN or
+// infinite x, or a range beyond binary32) or its scale overflows what the
+// product forms in binary16.
+template <int BITS, bool SYM>
+struct GroupParams {
+  uint32_t sz;   // binary16 bits of s in the high half, z in the low half
+  float inv;     // binary32(1 / s)
+  bool bad, ovf;
+};
+template <int BITS, bool SYM>
+__device__ __forceinline__ GroupParams<BITS, SYM> group_params(float mn, float mx,
+                                                               const float* rcp_sig) {
+  constexpr int QMAX = (1 << BITS) - 1;
+  constexpr int QSPAN = SYM ? (1 << (BITS - 1)) - 1 : QMAX;  // levels the scale spans
+  GroupParams<BITS, SYM> g;
+  const float range = __fsub_rn(mx, mn);
+  g.bad = !(range <= 3.402823466e38f);
+  const float span = SYM ? max_nan(mx, -mn) : range;
+  float s32 = div_by_const<QSPAN>(span);
+  if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
+  const __half s16 = __float2half_ru(s32);
+  const float s = __half2float(s16);
+  const uint32_t sbits = __half_as_ushort(s16);
+  const int sexp = static_cast<int>((sbits >> 10) & 31u) - 15;
+  g.inv = __int_as_float(__float_as_int(rcp_sig[sbits & 1023u]) - sexp * (1 << 23));
+  const int zi = __float_as_int(__fmaf_rn(-mn, g.inv, 12582912.0f)) - 0x4B400000;
+  const int z = SYM ? (1 << (BITS - 1)) : min(max(zi, 0), QMAX);
+  g.sz = (sbits << 16) | static_cast<uint32_t>(z);
+  g.ovf = static_cast<bool>(__hisinf(s16)) || s * static_cast<float>(QSPAN) > 65504.f;
+  return g;
+}
+
+// The same quantiser for bf16 W, with W staged in shared memory.  Block
+// (bx, by) owns the tile of cw channels at bx * cw and the row batches by,
+// by + gridDim.y, ... of kStageRows * rpi consecutive rows (32 KiB of W).
+// Thread (tx, ty) quantises rows ty, ty + rpi, ... of each batch, 16
+// channels each, as in qdq_pack_kernel.  A batch lands in one stage of a
+// ring of kQStages by one bulk copy per row segment, on the stage's
+// mbarrier (bounded waits).  Each warp copies its rows of a stage into
+// registers and releases the stage at once; the last warp to release it
+// (a shared-memory count) posts the next batch's byte count and issues its
+// copies, so the ring is refilled as soon as its data sits in registers
+// and no warp waits for another.  With no rows of W held in registers
+// between batches a thread keeps the four rows' scaled weights at once, and
+// the G = group/16 lanes of a group reduce the four rows' ranges together:
+// the first shuffle round (partner li ^ G/2) leaves each lane two rows
+// (lane bit G/2 picks the pair), the second (li ^ G/4) one row, and the
+// remaining rounds reduce that row.  Each lane then computes s, 1/s and z of
+// its own row only (with G = 2, of its two rows), and the four rows' values
+// are shuffled back to every lane of the group.  min and max are exact, so
+// no result depends on the order.
+constexpr int kStageRows = 4;   // rows per thread per batch
+constexpr int kQStages = 3;
+constexpr uint32_t kQStageBytes = kStageRows * kThreads * 16 * 2;   // 32 KiB
+constexpr uint32_t kQSmemBytes = kQStages * kQStageBytes;           // 96 KiB
+
+template <int BITS, bool WQ, bool SYM, int G>
+__global__ void __launch_bounds__(kThreads, 2) qdq_stage_kernel(
+    const __nv_bfloat16* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D,
+    int cw, uint32_t* __restrict__ codes, __half* __restrict__ scales,
+    __half* __restrict__ zeros, __half* __restrict__ wq, uint32_t* __restrict__ status) {
+  static_assert(G == 2 || G == 4 || G == 8 || G == 16, "group of 32 to 256 channels");
+  constexpr int QMAX = (1 << BITS) - 1;
+  constexpr int kWarps = kThreads / 32;
+  extern __shared__ __align__(128) uint8_t stage_smem[];   // [kQStages][rows][cw] bf16
+  __shared__ __align__(8) uint64_t full[kQStages];
+  __shared__ int released[kQStages];   // warps done with the stage's current batch
+  __shared__ int issued_s;             // batches requested so far
+  __shared__ int timeout_s;
+  __shared__ float rcp_sig[1024];
+
+  const int tpr = cw >> 4;            // threads per row (16 channels each)
+  const int rpi = kThreads / tpr;     // rows per step of the block
+  const int rows_pb = kStageRows * rpi;
+  const uint32_t row_bytes = static_cast<uint32_t>(cw) * 2u;
+  const int tx = threadIdx.x % tpr;
+  const int ty = threadIdx.x / tpr;
+  const int lane = threadIdx.x & 31;
+  const int li = lane & (G - 1);      // lane within the group
+  const int gbase = lane - li;
+  const int64_t col0 = static_cast<int64_t>(blockIdx.x) * cw;
+  const int64_t col = col0 + tx * 16;
+  const int64_t ngroups = d / (16 * G);
+  const int64_t kgroup = col / (16 * G);
+  const int64_t wpr = d * BITS / 32;
+  const int64_t nb_all = (dp + rows_pb - 1) / rows_pb;
+  const int64_t nb = blockIdx.y < nb_all ? (nb_all - blockIdx.y + gridDim.y - 1) / gridDim.y : 0;
+  const uint32_t smem0 = smem_addr(stage_smem);
+  allow_dependents_launch();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&full[s], 1);
+      released[s] = 0;
+    }
+    fence_barrier_init();
+    issued_s = static_cast<int>(nb < kQStages ? nb : kQStages);
+    timeout_s = 0;
+  }
+  __syncthreads();
+  // batch i of this block into stage i % kQStages (all lanes of one warp)
+  auto issue = [&](int64_t i) {
+    const int s = static_cast<int>(i % kQStages);
+    const int64_t r0 = (blockIdx.y + i * gridDim.y) * rows_pb;
+    const int nrows = static_cast<int>(min(static_cast<int64_t>(rows_pb), dp - r0));
+    if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nrows) * row_bytes);
+    __syncwarp();
+    const uint32_t dst = smem0 + static_cast<uint32_t>(s) * kQStageBytes;
+    for (int r = lane; r < nrows; r += 32)
+      bulk_load(dst + static_cast<uint32_t>(r) * row_bytes, W + (r0 + r) * d + col0, row_bytes,
+                &full[s]);
+  };
+  // W does not depend on the previous kernel: the first batches are
+  // requested before waiting for it (D does)
+  if (threadIdx.x < 32)
+    for (int64_t i = 0; i < nb && i < kQStages; ++i) issue(i);
+  grid_dependency_wait();
+
+  float2 h[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    h[k] = D != nullptr ? make_float2(__fsqrt_rn(__ldg(D + col + 2 * k)), __fsqrt_rn(__ldg(D + col + 2 * k + 1)))
+                        : make_float2(1.f, 1.f);
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) bad |= !(h[k].x <= 3.402823466e38f) || !(h[k].y <= 3.402823466e38f);
+  bool ovf = false;
+  for (int k = threadIdx.x; k < 1024; k += kThreads)
+    rcp_sig[k] = __fdiv_rn(1.0f, 1.0f + static_cast<float>(k) * 0.0009765625f);
+  __syncthreads();
+
+  const bool want_codes = codes != nullptr;
+  const int pa = (li & (G / 2)) != 0 ? 1 : 0;              // row pair after round 1
+  const int pb = G >= 4 && (li & (G / 4)) != 0 ? 1 : 0;    // row of the pair after round 2
+  int never = 0;
+  for (int64_t i = 0; i < nb; ++i) {
+    const int s = static_cast<int>(i % kQStages);
+    const uint32_t ph = static_cast<uint32_t>(i / kQStages) & 1u;
+    // warp-uniform (the work below shuffles)
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, &never))) {
+      if (lane == 0) {
+        set_flag(status, TTQ_FLAG_TIMEOUT);
+        timeout_s = 1;
+      }
+      break;
+    }
+    const int64_t r0 = (blockIdx.y + i * gridDim.y) * rows_pb;
+    const uint32_t base = smem0 + static_cast<uint32_t>(s) * kQStageBytes +
+                          static_cast<uint32_t>(tx) * 32u;
+    // the four rows' scaled weights and ranges (rows past dp hold stale
+    // data: their results are never stored or flagged)
+    float2 x[kStageRows][8];
+    float mn[kStageRows], mx[kStageRows];
+#pragma unroll
+    for (int u = 0; u < kStageRows; ++u) {
+      const uint32_t a = base + static_cast<uint32_t>(u * rpi + ty) * row_bytes;
+      Raw16<__nv_bfloat16> raw;
+      raw.v[0] = lds128(a);
+      raw.v[1] = lds128(a + 16u);
+      unpack16(raw, x[u]);
+      mn[u] = 0.f;
+      mx[u] = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        x[u][k] = __fmul2_rn(x[u][k], h[k]);
+        mn[u] = min3_nan(mn[u], x[u][k].x, x[u][k].y);
+        mx[u] = max3_nan(mx[u], x[u][k].x, x[u][k].y);
+      }
+    }
+    // this warp is done with stage s (the fence orders its reads before the
+    // bulk copies that will overwrite it); the last warp to say so refills it
+    fence_proxy_async_smem();
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&released[s], 1) == kWarps - 1;
+    if (__shfl_sync(0xffffffffu, last, 0)) {
+      if (lane == 0) released[s] = 0;
+      if (i + kQStages < nb) {
+        if (lane == 0) issued_s = static_cast<int>(i + kQStages + 1);
+        issue(i + kQStages);
+      }
+    }
+    // round 1 (partner li ^ G/2): keep the row pair pa, send the other
+    float kmn[2], kmx[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float smn = pa ? mn[j] : mn[2 + j];
+      const float smx = pa ? mx[j] : mx[2 + j];
+      kmn[j] = min_nan(pa ? mn[2 + j] : mn[j], __shfl_xor_sync(0xffffffffu, smn, G / 2));
+      kmx[j] = max_nan(pa ? mx[2 + j] : mx[j], __shfl_xor_sync(0xffffffffu, smx, G / 2));
+    }
+    uint32_t psz[kStageRows];
+    float pinv[kStageRows];
+    if constexpr (G == 2) {
+      // each lane holds the complete ranges of rows 2 pa and 2 pa + 1
+      GroupParams<BITS, SYM> gp[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        gp[j] = group_params<BITS, SYM>(kmn[j], kmx[j], rcp_sig);
+        const int64_t row = r0 + (2 * pa + j) * rpi + ty;
+        if (row < dp) {
+          bad |= gp[j].bad;
+          ovf |= gp[j].ovf;
+          if (want_codes) {
+            scales[row * ngroups + kgroup] = __ushort_as_half(static_cast<uint16_t>(gp[j].sz >> 16));
+            zeros[row * ngroups + kgroup] =
+                __hsub(__ushort_as_half(static_cast<uint16_t>(0x6400u | (gp[j].sz & 0xFFFFu))),
+                       __ushort_as_half(0x6400));
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kStageRows; ++u) {
+        psz[u] = __shfl_sync(0xffffffffu, gp[u & 1].sz, gbase + (u >> 1));
+        pinv[u] = __shfl_sync(0xffffffffu, gp[u & 1].inv, gbase + (u >> 1));
+      }
+    } else {
+      // round 2 (partner li ^ G/4): keep row 2 pa + pb
+      const float smn = pb ? kmn[0] : kmn[1];
+      const float smx = pb ? kmx[0] : kmx[1];
+      float rmn = min_nan(pb ? kmn[1] : kmn[0], __shfl_xor_sync(0xffffffffu, smn, G / 4));
+      float rmx = max_nan(pb ? kmx[1] : kmx[0], __shfl_xor_sync(0xffffffffu, smx, G / 4));
+#pragma unroll
+      for (int o = G / 8; o > 0; o >>= 1) {
+        rmn = min_nan(rmn, __shfl_xor_sync(0xffffffffu, rmn, o));
+        rmx = max_nan(rmx, __shfl_xor_sync(0xffffffffu, rmx, o));
+      }
+      const GroupParams<BITS, SYM> gp = group_params<BITS, SYM>(rmn, rmx, rcp_sig);
+      const int64_t row = r0 + (2 * pa + pb) * rpi + ty;
+      if (row < dp) {
+        bad |= gp.bad;
+        ovf |= gp.ovf;
+        // one lane per row stores its scale and zero
+        if (want_codes && (li & (G / 4 - 1)) == 0) {
+          scales[row * ngroups + kgroup] = __ushort_as_half(static_cast<uint16_t>(gp.sz >> 16));
+          zeros[row * ngroups + kgroup] =
+              __hsub(__ushort_as_half(static_cast<uint16_t>(0x6400u | (gp.sz & 0xFFFFu))),
+                     __ushort_as_half(0x6400));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kStageRows; ++u) {
+        const int src = gbase + (u >> 1) * (G / 2) + (u & 1) * (G / 4);
+        psz[u] = __shfl_sync(0xffffffffu, gp.sz, src);
+        pinv[u] = __shfl_sync(0xffffffffu, gp.inv, src);
+      }
+    }
+
+#pragma unroll
+    for (int u = 0; u < kStageRows; ++u) {
+      const int64_t row = r0 + u * rpi + ty;
+      const bool active = row < dp;
+      const uint32_t z = psz[u] & 0xFFFFu;
+      // codes as in qdq_pack_kernel: rint(x * inv) from the fused
+      // multiply-add with 1.5 * 2^23, plus z, clamped at the top
+      const uint32_t zz = z * 0x00010001u;
+      constexpr uint32_t QQ = static_cast<uint32_t>(QMAX) * 0x00010001u;
+      const float2 inv2 = make_float2(pinv[u], pinv[u]);
+      const float2 magic2 = make_float2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+      uint32_t qp[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float2 r = __ffma2_rn(x[u][k], inv2, magic2);
+        const uint32_t n = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
+        qp[k] = __viaddmin_s16x2(n, zz, QQ);
+      }
+      if (WQ && active) {
+        const __half2 zc2 = u32_as_half2((0x6400u | z) * 0x00010001u);
+        const __half2 s2 = u32_as_half2((psz[u] >> 16) * 0x00010001u);
+        uint32_t wh[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          wh[k] = half2_as_u32(__hmul2(__hsub2(u32_as_half2(qp[k] | 0x64006400u), zc2), s2));
+        uint4* dst = reinterpret_cast<uint4*>(wq + row * d + col);
+        dst[0] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        dst[1] = make_uint4(wh[4], wh[5], wh[6], wh[7]);
+      }
+      if (!want_codes) continue;
+      uint32_t lo = 0, hi = 0;
+      if (BITS == 4) {
+        lo = __byte_perm(nibbles4(qp[0], qp[1]), nibbles4(qp[2], qp[3]), 0x5410);
+        hi = __byte_perm(nibbles4(qp[4], qp[5]), nibbles4(qp[6], qp[7]), 0x5410);
+      } else if (BITS == 2) {
+        lo = __byte_perm(__byte_perm(crumbs4(qp[0], qp[1]), crumbs4(qp[2], qp[3]), 0x0040),
+                         __byte_perm(crumbs4(qp[4], qp[5]), crumbs4(qp[6], qp[7]), 0x0040), 0x5410);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t pair = (qp[k] & 0xFFFFu) | ((qp[k] >> 16) << BITS);
+          if (k < 4) lo |= pair << (2 * BITS * k);
+          else hi |= pair << (2 * BITS * (k - 4));
+        }
+      }
+      if (BITS == 4) {
+        if (active) *reinterpret_cast<uint2*>(codes + row * wpr + (col >> 3)) = make_uint2(lo, hi);
+      } else if (BITS == 2) {
+        if (active) codes[row * wpr + (col >> 4)] = lo;
+      } else {
+        const uint32_t a = lo | (hi << 24);
+        const uint32_t bw = hi >> 8;
+        const uint32_t oa = __shfl_down_sync(0xffffffffu, a, 1);
+        const uint32_t ob = __shfl_down_sync(0xffffffffu, bw, 1);
+        if (active && (tx & 1) == 0) {
+          uint32_t* dst = codes + row * wpr + (col >> 5) * 3;
+          dst[0] = a;
+          dst[1] = bw | (oa << 16);
+          dst[2] = (oa >> 16) | (ob << 16);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (timeout_s && threadIdx.x == 0) {
+    // a wait gave up: let the copies still in flight land before the block
+    // exits (the latest batch of each stage, each with a fresh limit)
+    for (int64_t k = issued_s - kQStages; k < issued_s; ++k)
+      if (k >= 0) mbar_wait(&full[k % kQStages], static_cast<uint32_t>(k / kQStages) & 1u, &never);
+  }
+  if (__any_sync(0xffffffffu, ovf) && lane == 0)
+    set_flag(status, TTQ_FLAG_NONFINITE | TTQ_FLAG_SCALE_OVERFLOW);
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_flag(status, TTQ_FLAG_NONFINITE);
+}
+
 // FP8 (E4M3) codes with the activation-aware scale (blog.lo0.es, the
 // comparison with FP8 end to end: TTQ derives s, the code format is free):
 //   x = W_ji sqrt(D_i); s32 = max|x| / 448, floored at 2^-14;
@@ -400,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_fp8_kernel(
       }
       bad |= !(__fsub_rn(mx, mn) <= 3.402823466e38f);
       const float amax = max_nan(mx, -mn);                 // max |x| of the group
-      float s32 = __fdiv_rn(amax, 448.0f);
+      float s32 = div_by_const<448>(amax);
       if (!(s32 >= 6.103515625e-05f)) s32 = 6.103515625e-05f;  // 2^-14
       const __half s16 = __float2half_ru(s32);
       const float s = __half2float(s16);
@@ -459,6 +788,81 @@ int tile_width(int64_t d, int group) {
   for (int c = 4096; c >= 32; c >>= 1)
     if (c >= group && d % c == 0) return c;
   return group;
+}
+
+template <int BITS, bool WQ, bool SYM, int G>
+cudaError_t launch_stage_g(dim3 grid, const __nv_bfloat16* W, int64_t dp, int64_t d,
+                           const float* D, int cw, uint32_t* codes, __half* s, __half* z,
+                           __half* wq, uint32_t* status, cudaStream_t stream, bool pdl) {
+  constexpr size_t smem = kQSmemBytes;
+  static std::atomic<bool> attr_set[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || !attr_set[dev].load(std::memory_order_relaxed)) {
+    const cudaError_t e = cudaFuncSetAttribute(qdq_stage_kernel<BITS, WQ, SYM, G>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_relaxed);
+  }
+  return launch_kernel(qdq_stage_kernel<BITS, WQ, SYM, G>, grid, dim3(kThreads), smem, stream,
+                       pdl, W, dp, d, D, cw, codes, s, z, wq, status);
+}
+
+template <int BITS, bool WQ, bool SYM>
+cudaError_t launch_stage(dim3 grid, const __nv_bfloat16* W, int64_t dp, int64_t d,
+                         const float* D, int group, int cw, uint32_t* codes, __half* s,
+                         __half* z, __half* wq, uint32_t* status, cudaStream_t stream, bool pdl) {
+  switch (group) {
+    case 32:
+      return launch_stage_g<BITS, WQ, SYM, 2>(grid, W, dp, d, D, cw, codes, s, z, wq, status,
+                                              stream, pdl);
+    case 64:
+      return launch_stage_g<BITS, WQ, SYM, 4>(grid, W, dp, d, D, cw, codes, s, z, wq, status,
+                                              stream, pdl);
+    case 128:
+      return launch_stage_g<BITS, WQ, SYM, 8>(grid, W, dp, d, D, cw, codes, s, z, wq, status,
+                                              stream, pdl);
+    case 256:
+      return launch_stage_g<BITS, WQ, SYM, 16>(grid, W, dp, d, D, cw, codes, s, z, wq, status,
+                                               stream, pdl);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+// The launch of the staged kernel for bf16 W: one block per tile of cw
+// channels and per gy row-batch slot, about two resident blocks per SM.
+template <bool WQ, bool SYM>
+cudaError_t launch_staged(const __nv_bfloat16* W, int64_t dp, int64_t d, const float* D,
+                          int bits, int group, uint32_t* codes, uint16_t* scales,
+                          uint16_t* zeros, void* wq, uint32_t* status, int num_sms,
+                          cudaStream_t stream, bool pdl) {
+  const int cw = tile_width(d, group);
+  const int rows_pb = kStageRows * (kThreads / (cw >> 4));
+  const int64_t gx = d / cw;
+  const int64_t nb_all = (dp + rows_pb - 1) / rows_pb;
+  int64_t gy = (static_cast<int64_t>(num_sms) * 2 + gx - 1) / gx;
+  if (gy > nb_all) gy = nb_all;
+  if (gy > 65535) gy = 65535;
+  if (gy < 1) gy = 1;
+  const dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(gy));
+  __half* s = reinterpret_cast<__half*>(scales);
+  __half* z = reinterpret_cast<__half*>(zeros);
+  __half* w = static_cast<__half*>(wq);
+  switch (bits) {
+    case 2:
+      return launch_stage<2, WQ, SYM>(grid, W, dp, d, D, group, cw, codes, s, z, w, status,
+                                      stream, pdl);
+    case 3:
+      return launch_stage<3, WQ, SYM>(grid, W, dp, d, D, group, cw, codes, s, z, w, status,
+                                      stream, pdl);
+    case 4:
+      return launch_stage<4, WQ, SYM>(grid, W, dp, d, D, group, cw, codes, s, z, w, status,
+                                      stream, pdl);
+    default:
+      return cudaErrorInvalidValue;
+  }
 }
 
 template <typename WT, bool WQ, bool SYM>
@@ -607,10 +1011,18 @@ template <typename WT, bool SYM>
 cudaError_t launch_wq(const WT* W, int64_t dp, int64_t d, const float* D, int bits, int group,
                       uint32_t* codes, uint16_t* scales, uint16_t* zeros, void* wq,
                       uint32_t* status, int num_sms, cudaStream_t stream, bool pdl) {
-  return wq ? launch_w<WT, true, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq, status,
-                                      num_sms, stream, pdl)
-            : launch_w<WT, false, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq, status,
-                                       num_sms, stream, pdl);
+  if constexpr (std::is_same<WT, __nv_bfloat16>::value) {
+    // bf16 W: the kernel with W staged in shared memory
+    return wq ? launch_staged<true, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                         status, num_sms, stream, pdl)
+              : launch_staged<false, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                          status, num_sms, stream, pdl);
+  } else {
+    return wq ? launch_w<WT, true, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq, status,
+                                        num_sms, stream, pdl)
+              : launch_w<WT, false, SYM>(W, dp, d, D, bits, group, codes, scales, zeros, wq,
+                                         status, num_sms, stream, pdl);
+  }
 }
 
 template <typename WT>

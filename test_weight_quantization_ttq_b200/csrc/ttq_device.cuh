@@ -32,6 +32,30 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// binary32 x / B rounded to nearest even, for the quantisers' constant
+// divisors, as the product with r = RN(1 / B) and one fused multiply-add
+// correction (e = x - q0 B is exact): 5 instructions where the general
+// correctly rounded division takes about 40.  For B = 1, 3, 7, 15 the result
+// equals RN(x / B) for every non-negative binary32 x, zero, subnormals, inf
+// and NaN included; for B = 448 it does whenever RN(x / B) >= 2^-14, and
+// both sides then agree after the quantisers' floor of the scale at 2^-14
+// (both checked exhaustively over binary32).
+template <int B>
+__device__ __forceinline__ float div_by_const(float x) {
+  static_assert(B == 1 || B == 3 || B == 7 || B == 15 || B == 448, "divisor not checked");
+  if constexpr (B == 1) {
+    return x;
+  } else {
+    constexpr float r = B == 3    ? 0x1.555556p-2f
+                        : B == 7  ? 0x1.24924ap-3f
+                        : B == 15 ? 0x1.111112p-4f
+                                  : 0x1.24924ap-9f;   // RN(1 / B)
+    const float q0 = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-q0, static_cast<float>(B), x);
+    return e == e ? __fmaf_rn(e, r, q0) : q0;   // inf and NaN keep q0
+  }
+}
+
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel on the stream is still running; it must execute
@@ -126,6 +150,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // -------------------------------------------------------------------- TMA
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned; no cluster multicast), completing that many
+// bytes of transaction count on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
 // 2-D tiled bulk copy global -> shared (no cluster multicast), completing
 // `bytes` of transaction count on `bar`.  x is the innermost coordinate.
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst,
