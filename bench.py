@@ -848,7 +848,7 @@ def run_table(args):
 
 
 def run_ab_dequant(args):
-    """Where the prefill product gets its weight operand (SURVEY row a4): the
+    """Where the prefill product gets its weight operand: the
     materialised form (the quantiser also writes the binary16 s (q - z), the
     plain tcgen05 GEMM reads it by TMA) against dequantisation inside the
     product's main loop (the quantiser writes codes only; the GEMM's

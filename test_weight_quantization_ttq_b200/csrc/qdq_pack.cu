@@ -457,8 +457,8 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_stage_kernel(
   __syncthreads();
 
   const bool want_codes = codes != nullptr;
-  const int pa = (li & (G / 2)) != 0 ? 1 : 0;              // row pair after round 1
-  const int pb = G >= 4 && (li & (G / 4)) != 0 ? 1 : 0;    // row of the pair after round 2
+  const int pa = (li & (G / 2)) != 0 ? 1 : 0;              // row pair after the first shuffle round
+  const int pb = G >= 4 && (li & (G / 4)) != 0 ? 1 : 0;    // row of the pair after the second
   int never = 0;
   for (int64_t i = 0; i < nb; ++i) {
     const int s = static_cast<int>(i % kQStages);
@@ -507,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_stage_kernel(
         issue(i + kQStages);
       }
     }
-    // round 1 (partner li ^ G/2): keep the row pair pa, send the other
+    // first shuffle round (partner li ^ G/2): keep the row pair pa, send the other
     float kmn[2], kmx[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_stage_kernel(
         pinv[u] = __shfl_sync(0xffffffffu, gp[u & 1].inv, gbase + (u >> 1));
       }
     } else {
-      // round 2 (partner li ^ G/4): keep row 2 pa + pb
+      // second shuffle round (partner li ^ G/4): keep row 2 pa + pb
       const float smn = pb ? kmn[0] : kmn[1];
       const float smx = pb ? kmx[0] : kmx[1];
       float rmn = min_nan(pb ? kmn[1] : kmn[0], __shfl_xor_sync(0xffffffffu, smn, G / 4));
