@@ -563,21 +563,21 @@ cudaError_t launch_sqrt_f32(const float* D, float* h, int64_t d, cudaStream_t st
 
 void act_norm_plan(int64_t d, int64_t T, int num_sms, int64_t* splits, int64_t* rows_per_split) {
   // When 8 splits of at most 256 rows cover T (the fused kernel's register
-  // capacity for bf16 X), enough splits for about two 128-channel blocks
-  // per SM and enough for the rows to fit, at most 8 (one cluster).
-  // Otherwise about two 256-channel blocks per SM, at most 16 splits.
-  // Always at least 32 rows per split.
+  // capacity for bf16 X), as many splits as keep the 128-channel blocks
+  // within two per SM (one wave), but enough for the rows to fit, at most 8
+  // (one cluster).  Otherwise as many as keep the 256-channel blocks within
+  // two per SM, at most 16.  Always at most one split per 32 rows.
   const int64_t fit = (T + kPhases * 16 - 1) / (kPhases * 16);
   const int64_t target = static_cast<int64_t>(num_sms) * 2;
   int64_t s;
   if (fit <= kMaxClusterSplits) {
     const int64_t ncb = (d + kClusterChannels - 1) / kClusterChannels;
-    s = (target + ncb - 1) / ncb;
+    s = target / ncb;
     if (s < fit) s = fit;
     if (s > kMaxClusterSplits) s = kMaxClusterSplits;
   } else {
     const int64_t ncb = (d + kChannelsPerBlock - 1) / kChannelsPerBlock;
-    s = (target + ncb - 1) / ncb;
+    s = target / ncb;
     if (s > kMaxSplits) s = kMaxSplits;
   }
   const int64_t max_by_rows = (T + 31) / 32;

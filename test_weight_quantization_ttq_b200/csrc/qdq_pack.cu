@@ -842,7 +842,8 @@ cudaError_t launch_staged(const __nv_bfloat16* W, int64_t dp, int64_t d, const f
   const int rows_pb = kStageRows * (kThreads / (cw >> 4));
   const int64_t gx = d / cw;
   const int64_t nb_all = (dp + rows_pb - 1) / rows_pb;
-  int64_t gy = (static_cast<int64_t>(num_sms) * 2 + gx - 1) / gx;
+  // two resident blocks per SM, all in one wave
+  int64_t gy = static_cast<int64_t>(num_sms) * 2 / gx;
   if (gy > nb_all) gy = nb_all;
   if (gy > 65535) gy = 65535;
   if (gy < 1) gy = 1;
@@ -873,7 +874,7 @@ cudaError_t launch_w(const WT* W, int64_t dp, int64_t d, const float* D, int bit
   const int rpi = kThreads / (cw >> 4);
   const int64_t gx = d / cw;
   const int64_t want = static_cast<int64_t>(num_sms) * 2;  // two resident blocks per SM
-  int64_t gy = (want + gx - 1) / gx;
+  int64_t gy = want / gx;   // all blocks resident in one wave
   const int64_t max_gy = (dp + rpi - 1) / rpi;  // each block still takes >= 1 row
   if (gy > max_gy) gy = max_gy;
   if (gy > 65535) gy = 65535;
@@ -1056,7 +1057,7 @@ cudaError_t launch_qdq_fp8(const void* W, bool w_f32, int64_t dp, int64_t d, con
   const int rpi = kThreads / (cw >> 4);
   const int64_t gx = d / cw;
   const int64_t want = static_cast<int64_t>(num_sms) * 2;
-  int64_t gy = (want + gx - 1) / gx;
+  int64_t gy = want / gx;   // all blocks resident in one wave
   const int64_t max_gy = (dp + rpi - 1) / rpi;
   if (gy > max_gy) gy = max_gy;
   if (gy > 65535) gy = 65535;

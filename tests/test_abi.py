@@ -87,11 +87,13 @@ def test_workspace_layout_is_consistent(L):
     (4096, 16, 1),
     (4096, 0, 1),
     (4096, 4096, 16),    # too many rows for 8 splits of 256: 16 blocks of 256 channels x 16
-    (8192, 8192, 10),    # 32 blocks of 256 channels: 10 splits
+    (8192, 8192, 9),     # 32 blocks of 256 channels: 9 splits keep 288 blocks in one wave
+    (11008, 512, 3),     # 86 blocks of 128 channels: 3 splits keep 258 blocks in one wave
 ])
 def test_statistic_split_plan(L, d, T, splits):
     """The token splits of the statistic pass: the fused kernel's clusters
-    hold at most 8 splits of at most 256 rows."""
+    hold at most 8 splits of at most 256 rows, and the blocks fit two per SM
+    in one wave where the rows allow."""
     lay = ttq.ttq_workspace_get_layout(d, 0, T, 0, 4, 32, ttq.TTQ_BF16)
     assert lay.splits == splits
     if T:
