@@ -149,7 +149,10 @@ typedef struct ttq_workspace_layout {
   size_t axp;     /* float32 [ax_splits][T][r] partial sums of A X split along d
                      (0 when A X is not split) */
   size_t D_sqrt;  /* float32 [d] sqrtf(D_ii) for the single-pass decode product */
-  size_t ypart;   /* float32 partial output tiles of the single-pass decode product */
+  size_t ypart;   /* float32 partial output tiles of the single-pass decode product
+                     (T <= 16), or float32 [splits][T][d'] partial sums of the
+                     product on wq when it is split along K (T > 256 and few
+                     output tiles); 0: not in this layout */
   size_t tickets; /* uint32 arrival tickets of its 256-row tiles (inside the
                      zeroed header; 0: not in this layout) */
   int64_t ax_splits; /* K splits of the A X product (1: none; 0 when r == 0) */
@@ -320,10 +323,22 @@ ttq_status ttq_dequant_gemm(const uint32_t* codes, const uint16_t* scales,
  * D^{-1/2}, as written by ttq_scale_activations); d % 8 == 0; all pointers
  * 16-byte aligned.  Y [T][dp] in y_dtype (TTQ_F32 or TTQ_BF16, rounded
  * once).  No low-rank term.  Needs a workspace of at least 4096 bytes
- * (status word). */
+ * (status word).  For more than 256 tokens and a shape with few output
+ * tiles (d' small against T and d: a long K), the product is split along K
+ * exactly as ttq_linear_forward splits it: the splits' float32 partial sums
+ * go to the workspace after its 20480-byte header and are added in split
+ * order, rounded once.  It does so when the workspace spans
+ * ttq_dequantized_gemm_workspace_size(d, dp, T) bytes, and then gives the
+ * forward's bits; with a smaller workspace it runs unsplit (the same
+ * product, its fp32 sums in another order). */
 ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64_t d,
                                 int64_t dp, int64_t T, void* Y, ttq_dtype y_dtype, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/* Workspace bytes at which ttq_dequantized_gemm takes the forward's K split
+ * for this shape (4096 when it never splits); 0 for an invalid shape.  An
+ * interface query of this library; the method has no counterpart. */
+size_t ttq_dequantized_gemm_workspace_size(int64_t d, int64_t dp, int64_t T);
 
 /* The whole TTQ linear layer, (1) -> (2) -> (3), on `stream`:
  *   Y = Q[W D^{1/2}] D^{-1/2} X + B (A X).
@@ -336,7 +351,10 @@ ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64
  * For T > 256 the quantiser writes the dequantised weight s (q - z) in
  * binary16 to the workspace (layout field wq) instead of the codes, and the
  * product reads it as a plain tensor-core operand, so that no 256-token
- * tile dequantises the codes again; for 17 <= T <= 256 the product
+ * tile dequantises the codes again (where few output tiles would leave
+ * most SMs to one long K loop, that product is split along K and the
+ * float32 partial sums are added in split order, layout field ypart); for
+ * 17 <= T <= 256 the product
  * dequantises the codes itself (as ttq_dequant_gemm does); for T <= 16
  * (bf16, asymmetric codes) one kernel quantises W in registers and
  * multiplies (as ttq_quantize_gemm).  All give the same operand values. */
@@ -359,7 +377,9 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A,
  * work), in *kernels: the statistic pass (fused with the scaling of X when
  * it fits, see ttq_act_norm_scale), the quantiser and the product (one
  * kernel together where the forward takes the single-pass decode product,
- * see ttq_quantize_gemm), and for r > 0 the A X product (plus the
+ * see ttq_quantize_gemm; plus the reduction of its K splits where the
+ * product on the materialised weight is split), and for r > 0 the A X
+ * product (plus the
  * reduction of its K splits, and two bf16 conversions of a float32 A and
  * B).  An interface query of this library; the method has no counterpart. */
 ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, int64_t T,

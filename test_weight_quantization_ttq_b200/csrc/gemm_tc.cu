@@ -30,6 +30,8 @@
 // Every barrier wait is bounded (1 s); a wait that gives up sets
 // TTQ_FLAG_TIMEOUT, tells the other roles to stop, and the CTA still frees
 // its tensor memory and returns.
+#include <algorithm>
+
 #include "ttq_device.cuh"
 #include "ttq_kernels.h"
 
@@ -282,9 +284,13 @@ __global__ void __launch_bounds__(cta_threads<BM>(), 1)
   const int kb_main = static_cast<int>((g.K + kBK - 1) / kBK);
   const int kb_tail = static_cast<int>((g.K_tail + kBK - 1) / kBK);
   // this CTA's K blocks [kb_lo, kb_total): all of them, or one split of the
-  // main blocks (split-K runs only in the plain mode without a tail)
-  const int kb_lo = g.kb_per_split > 0 ? static_cast<int>(blockIdx.z) * g.kb_per_split : 0;
-  const int kb_total = g.kb_per_split > 0 ? min(kb_main, kb_lo + g.kb_per_split) : kb_main + kb_tail;
+  // main blocks (split-K runs only in the plain mode); the last split takes
+  // the rest of the main blocks and the low-rank tail
+  const bool k_split = g.kb_per_split > 0;
+  const int kb_lo = k_split ? static_cast<int>(blockIdx.z) * g.kb_per_split : 0;
+  const int kb_total = !k_split || blockIdx.z + 1 == gridDim.z
+                           ? kb_main + kb_tail
+                           : min(kb_main, kb_lo + g.kb_per_split);
   // accumulator h of a 256-row tile starts at column 256 * h
   const uint32_t tmem_cols =
       kSub == 2 ? 512u : (BN <= 32 ? 32u : BN <= 64 ? 64u : BN <= 128 ? 128u : 256u);
@@ -637,9 +643,9 @@ cudaError_t launch_tile(const GemmArgs& a, const GemmMaps& maps, int BN, cudaStr
   g.stages = stages;
   g.status = a.status;
   const bool split = a.k_splits > 1;
-  if (split && (BITS != 0 || a.K_tail != 0 || !a.y_f32 || a.kb_per_split < 1 ||
+  if (split && (BITS != 0 || !a.y_f32 || a.kb_per_split < 1 ||
                 static_cast<int64_t>(a.k_splits - 1) * a.kb_per_split >= (a.K + kBK - 1) / kBK))
-    return cudaErrorInvalidValue;   // every split must own at least one K block
+    return cudaErrorInvalidValue;   // every split must own at least one main K block
   g.kb_per_split = split ? a.kb_per_split : 0;
   g.split_stride = split ? a.split_stride : 0;
   if (split) g.y_tma = 0;
@@ -677,6 +683,46 @@ __global__ void ax_reduce_kernel(const float* __restrict__ P, int splits, int64_
     for (int s = 0; s < splits; ++s) acc += __ldcg(P + s * n + i);
     const int64_t t = i / r;
     AX[t * ax_ld + (i - t * r)] = __float2bfloat16_rn(acc);
+  }
+}
+
+// Y[i] = the sum over s of P[s][i], the splits added in order and the sum
+// rounded once (to bf16, or kept in float32); n = T * ldy elements.
+__global__ void y_reduce_kernel(const float* __restrict__ P, int splits, int64_t n,
+                                void* __restrict__ Y, int y_f32) {
+  allow_dependents_launch();
+  grid_dependency_wait();   // the partials come from the previous kernel
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t i0 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n % 4 == 0) {
+    const int64_t nv = n / 4;
+    for (int64_t i = i0; i < nv; i += stride) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < splits; ++s) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(P + s * n) + i);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      if (y_f32) {
+        reinterpret_cast<float4*>(Y)[i] = acc;
+      } else {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+        uint2 u;
+        memcpy(&u.x, &lo, 4);
+        memcpy(&u.y, &hi, 4);
+        reinterpret_cast<uint2*>(Y)[i] = u;
+      }
+    }
+  } else {
+    for (int64_t i = i0; i < n; i += stride) {
+      float acc = 0.f;
+      for (int s = 0; s < splits; ++s) acc += __ldcs(P + s * n + i);
+      if (y_f32) static_cast<float*>(Y)[i] = acc;
+      else static_cast<__nv_bfloat16*>(Y)[i] = __float2bfloat16_rn(acc);
+    }
   }
 }
 
@@ -737,6 +783,78 @@ void gemm_tile_shape(int bits, int64_t M, int64_t T, int num_sms, int* block_m, 
   }
   *block_m = best_m;
   *block_n = best_n;
+}
+
+GemmPlan gemm_plan_plain(int64_t M, int64_t T, int64_t K, int64_t K_tail, int num_sms,
+                         bool allow_split) {
+  // Unsplit, the tile shape is gemm_tile_shape's.  A K split is weighed
+  // against it with a time model: the larger of
+  //  - the tensor-core time: waves x K blocks per CTA x 4 BN (BM = 256) or
+  //    2 BN (BM = 128) cycles (4096 multiply-adds per SM and cycle), at the
+  //    power-capped clock of about 1.7 GHz;
+  //  - the time to bring the operand tiles from L2 into shared memory: each
+  //    CTA reads (BM + BN) x 128 bytes per K block, at about 12 TB/s over the
+  //    device and at most 128 bytes per cycle into one SM;
+  // plus, with K split in s parts, the float32 partial sums written and read
+  // once more and Y written (about 6 TB/s), and the reduction's launch.  The
+  // unsplit product at 4096 x 4096 x 2048 (256 x 240 tiles) and at
+  // 4096 x 512 x 11008 (256 x 64 tiles), measured on B200, is bound by the
+  // L2 term: 48.6 and 93 us against 48.8 and 75.6 us modelled.  (As a choice
+  // among unsplit shapes the model misleads: it prefers 256 x 256 tiles,
+  // which measured 2-4% slower than gemm_tile_shape's at 4096 x 4096 x 2048
+  // and 28672 x 1024 x 8192.)  A split is taken when the model puts it 10%
+  // ahead of the unsplit shape.
+  constexpr double kClock = 1.7e9, kL2 = 12e12, kSmL2 = 128.0 * kClock, kHbm = 6e12;
+  constexpr double kLaunch = 2e-6;
+  constexpr int kMaxSplits = 8, kMinBlocksPerSplit = 8;
+  const int64_t kb = (K + kBK - 1) / kBK;
+  const int64_t kbt = (K_tail + kBK - 1) / kBK;
+  auto model = [&](int bm, int bn, int64_t s, int64_t per) {
+    const int64_t tiles = (M + bm - 1) / bm * ((T + bn - 1) / bn);
+    const int64_t ctas = tiles * s;
+    const int64_t waves = (ctas + num_sms - 1) / num_sms;
+    const int64_t kcta = per + kbt;   // the last split's blocks, tail included
+    const double t_mma = static_cast<double>(waves * kcta) * (bm == 256 ? 4.0 : 2.0) * bn / kClock;
+    const double bytes = static_cast<double>(bm + bn) * 128.0 * static_cast<double>(kcta);
+    const double t_l2 = std::max(static_cast<double>(ctas) * bytes / kL2,
+                                 static_cast<double>(waves) * bytes / kSmL2);
+    const double t_red =
+        s > 1 ? static_cast<double>(2 * s + 1) * static_cast<double>(T * M) * 4.0 / kHbm + kLaunch
+              : 0.0;
+    return std::max(t_mma, t_l2) + t_red;
+  };
+  GemmPlan plan{128, 16, 1, 0};
+  gemm_tile_shape(0, M, T, num_sms, &plan.block_m, &plan.block_n);
+  if (!allow_split) return plan;
+  const double t1 = model(plan.block_m, plan.block_n, 1, kb);
+  double ts = -1.0;
+  GemmPlan split = plan;
+  const int64_t bn_max = T >= 256 ? 256 : (T + 15) / 16 * 16;
+  for (int bm = 256; bm >= 128; bm -= 128) {
+    if (bm == 256 && M <= 128) continue;
+    for (int bn = static_cast<int>(bn_max); bn >= 16; bn -= 16) {
+      for (int64_t s = 2; s <= kMaxSplits && kb / s >= kMinBlocksPerSplit; ++s) {
+        const int64_t per = (kb + s - 1) / s;
+        if ((kb + per - 1) / per != s) continue;   // another s gives these splits
+        const double t = model(bm, bn, s, per);
+        if (ts < 0.0 || t < ts) {
+          ts = t;
+          split = GemmPlan{bm, bn, static_cast<int>(s), static_cast<int>(per)};
+        }
+      }
+    }
+  }
+  return ts >= 0.0 && ts < 0.9 * t1 ? split : plan;
+}
+
+cudaError_t launch_y_reduce(const float* P, int splits, int64_t n, void* Y, bool y_f32,
+                            cudaStream_t stream, bool pdl) {
+  if (n == 0) return cudaSuccess;
+  const int64_t work = n % 4 == 0 ? n / 4 : n;
+  int64_t blocks = (work + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  return launch_kernel(y_reduce_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, stream,
+                       pdl, P, splits, n, Y, y_f32 ? 1 : 0);
 }
 
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,

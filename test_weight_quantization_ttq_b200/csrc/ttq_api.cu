@@ -74,6 +74,13 @@ bool single_pass_decode(ttq_dtype dtype, ttq_qscheme scheme, int64_t d, int64_t 
 }
 
 // Computes the workspace layout; false for an unsupported shape.
+// The plan of the product on the materialised weight: K splits only for
+// more than 256 tokens, planned for 148 SMs whatever the device so that the
+// workspace layout does not depend on it.
+GemmPlan product_plan(int64_t dp, int64_t T, int64_t d, int64_t r, bool allow_split) {
+  return gemm_plan_plain(dp, T, d, r, kPlanSMs, allow_split && T > 256);
+}
+
 bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
                  ttq_dtype dtype, ttq_workspace_layout* L) {
   if (d < 8 || d % 8 != 0 || dp < 0 || T < 0 || r < 0 || r % 8 != 0) return false;
@@ -136,6 +143,13 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
   if (has_q && materialize_w(dp, T, bits, d)) {
     l.wq = off;
     off = align_up(off + static_cast<size_t>(dp) * static_cast<size_t>(d) * 2);
+    // the product on W_hat split along K: its float32 partial sums
+    const GemmPlan plan = product_plan(dp, T, d, r, true);
+    if (plan.splits > 1) {
+      l.ypart = off;
+      off = align_up(off + static_cast<size_t>(plan.splits) * static_cast<size_t>(T) *
+                               static_cast<size_t>(dp) * 4);
+    }
   }
   l.total = off;
   l.splits = splits;
@@ -283,7 +297,8 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
                     const void* Xh, const void* Xb, const void* Ab,
                     const void* Bb, int64_t d, int64_t dp, int64_t T, int64_t r, int bits,
                     int group, void* Y, bool y_f32, void* ws, const ttq_workspace_layout& L,
-                    cudaStream_t stream, bool pdl, const void* wq = nullptr) {
+                    cudaStream_t stream, bool pdl, const void* wq = nullptr,
+                    float* ypart = nullptr) {
   if (T == 0 || dp == 0) return TTQ_OK;
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   void* ax = r > 0 ? ws_at(ws, L.ax) : nullptr;
@@ -327,9 +342,18 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
     }
   }
   if (!wq && bits == 8) return TTQ_ERR_UNSUPPORTED;  // no other product reads 8-bit codes
-  // wq: the product reads the materialised binary16 s (q - z) by TMA
+  // wq: the product reads the materialised binary16 s (q - z) by TMA, split
+  // along K where its plan says so and ypart has room for the partial sums
   int bm = 128, bnm = 16;
-  gemm_tile_shape(wq ? 0 : bits, dp, T, device_sms(), &bm, &bnm);
+  GemmPlan plan{128, 16, 1, 0};
+  if (wq) {
+    plan = product_plan(dp, T, d, r, ypart != nullptr);
+    bm = plan.block_m;
+    bnm = plan.block_n;
+  } else {
+    gemm_tile_shape(bits, dp, T, device_sms(), &bm, &bnm);
+  }
+  const bool k_split = plan.splits > 1;
   GemmMaps m;
   if (!encode_16bit(&m.b0, Xh, true, d, T, d, bnm)) return TTQ_ERR_CUDA;
   m.a0 = m.b0;
@@ -349,7 +373,7 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   if (!codes_tma) m.c0 = m.b0;
   // bf16 Y goes out through TMA stores of 32 x 16 slabs when its rows are
   // 16-byte strided
-  const bool y_tma = !y_f32 && dp % 8 == 0 && encode_y_bf16(&m.y, Y, dp, T, 32, 16);
+  const bool y_tma = !k_split && !y_f32 && dp % 8 == 0 && encode_y_bf16(&m.y, Y, dp, T, 32, 16);
   if (!y_tma) m.y = m.b0;
   GemmArgs a;
   a.codes_tma = codes_tma;
@@ -364,11 +388,18 @@ ttq_status run_gemm(const uint32_t* codes, const uint16_t* scales, const uint16_
   a.M = dp;
   a.T = T;
   a.K_tail = r;
-  a.Y = Y;
+  a.Y = k_split ? static_cast<void*>(ypart) : Y;
   a.ldy = dp;
-  a.y_f32 = y_f32;
+  a.y_f32 = y_f32 || k_split;
   a.status = status;
-  return cuda_status(launch_dequant_gemm(a, m, bnm, bm, stream, pdl));
+  if (k_split) {
+    a.k_splits = plan.splits;
+    a.kb_per_split = plan.kb_per_split;
+    a.split_stride = T * dp;
+  }
+  const ttq_status st = cuda_status(launch_dequant_gemm(a, m, bnm, bm, stream, pdl));
+  if (st != TTQ_OK || !k_split) return st;
+  return cuda_status(launch_y_reduce(ypart, plan.splits, T * dp, Y, y_f32, stream, true));
 }
 
 // Steps (2)-(3) in one pass over bf16 W (T <= 16): sqrt(D) in Dh, binary16
@@ -540,6 +571,8 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
     if (!one_pass) ++n;                                                    // quantiser
     if (T > 0) {
       ++n;                                                                 // product
+      if (materialize_w(dp, T, bits, d) && product_plan(dp, T, d, r, true).splits > 1)
+        ++n;                                                               // its split reduction
       if (r > 0) {
         n += 1 + (f32 ? 2 : 0);                                            // A X (+ bf16 A, B)
         if (ax_split_plan(r, T, d, kPlanSMs).splits > 1) ++n;              // its split reduction
@@ -643,9 +676,22 @@ ttq_status ttq_dequantized_gemm(const uint16_t* W_hat, const uint16_t* Xs, int64
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return TTQ_ERR_INVALID_ARG;
   if (ws_bytes < kStatusBytes) return TTQ_ERR_WORKSPACE;
   if (!work) return TTQ_OK;
-  ttq_workspace_layout L = {};  // only the status word (offset 0) is used
+  ttq_workspace_layout L = {};  // the status word (offset 0); the partial sums after the header
+  float* ypart = nullptr;
+  if (ws_bytes >= ttq_dequantized_gemm_workspace_size(d, dp, T) &&
+      product_plan(dp, T, d, 0, true).splits > 1)
+    ypart = reinterpret_cast<float*>(ws_at(ws, kHeaderBytes));
   return run_gemm(nullptr, nullptr, nullptr, Xs, nullptr, nullptr, nullptr, d, dp, T, 0, 4, 32,
-                  Y, y_dtype == TTQ_F32, ws, L, static_cast<cudaStream_t>(stream), false, W_hat);
+                  Y, y_dtype == TTQ_F32, ws, L, static_cast<cudaStream_t>(stream), false, W_hat,
+                  ypart);
+}
+
+size_t ttq_dequantized_gemm_workspace_size(int64_t d, int64_t dp, int64_t T) {
+  if (d < 8 || d % 8 != 0 || dp < 0 || T < 0) return 0;
+  const GemmPlan plan = product_plan(dp, T, d, 0, true);
+  if (dp == 0 || T == 0 || plan.splits < 2) return kStatusBytes;
+  return kHeaderBytes + static_cast<size_t>(plan.splits) * static_cast<size_t>(T) *
+                            static_cast<size_t>(dp) * 4;
 }
 
 ttq_status ttq_scale_activations(const void* X, ttq_dtype dtype, int64_t d, int64_t T,
@@ -796,8 +842,9 @@ ttq_status ttq_linear_forward_ex(const void* X, const void* W, const void* A, co
     Ab = ab;
     Bb = bb;
   }
+  float* ypart = wq && L.ypart != 0 ? reinterpret_cast<float*>(ws_at(ws, L.ypart)) : nullptr;
   return run_gemm(codes, scales, zeros, xh, f32 ? xb : X, Ab, Bb, d, dp, T, r, bits, group, Y,
-                  y_dtype == TTQ_F32, ws, L, s, true, wq);
+                  y_dtype == TTQ_F32, ws, L, s, true, wq, ypart);
 }
 
 ttq_status ttq_linear_forward(const void* X, const void* W, const void* A, const void* B,

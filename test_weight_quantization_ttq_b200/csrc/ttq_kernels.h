@@ -109,9 +109,10 @@ struct GemmArgs {
   bool a_f16 = false;      // plain mode: the A operand (maps.a0) is binary16, not bf16
   bool codes_tma = false;  // codes tile loaded by TMA (maps.c0); else per-thread loads
   bool y_tma = false;      // bf16 Y stored by TMA (maps.y, box block_m x block_n)
-  // split-K (plain mode without a low-rank tail only): split z of k_splits
-  // covers K blocks [z * kb_per_split, (z + 1) * kb_per_split) and writes
-  // its float32 partial product to Y + z * split_stride (y_f32 must be set)
+  // split-K (plain mode only): split z of k_splits covers K blocks
+  // [z * kb_per_split, (z + 1) * kb_per_split), the last one the rest of the
+  // main blocks and the low-rank tail, and writes its float32 partial
+  // product to Y + z * split_stride (y_f32 must be set)
   int k_splits = 1;
   int kb_per_split = 0;
   int64_t split_stride = 0;
@@ -240,6 +241,25 @@ int gemm_block_n(int64_t T);
 // (256 only with codes), block_n a multiple of 16 up to 256 tokens, chosen
 // so that the CTAs fill the SMs in as few, as full waves as possible.
 void gemm_tile_shape(int bits, int64_t M, int64_t T, int num_sms, int* block_m, int* block_n);
+
+// Tile shape and K split of the product on the materialised binary16 weight
+// (plain mode: M rows of W_hat, T tokens, K channels, K_tail low-rank
+// channels): BM x BN tiles and `splits` parts of kb_per_split K blocks of 64
+// (splits 1, kb_per_split 0: unsplit; the last part also takes the rest of
+// the blocks and the low-rank tail).  Unsplit, the shape is gemm_tile_shape's;
+// a split is taken where a time model that counts the tensor-core time, the
+// operand traffic from L2 and the float32 partial sums with their reduction
+// (launch_y_reduce) puts it well ahead.
+struct GemmPlan {
+  int block_m, block_n, splits, kb_per_split;
+};
+GemmPlan gemm_plan_plain(int64_t M, int64_t T, int64_t K, int64_t K_tail, int num_sms,
+                         bool allow_split);
+
+// Y (n elements, bf16 or float32) = the sum over the splits, in split order,
+// of the float32 partials P [splits][n], rounded once.
+cudaError_t launch_y_reduce(const float* P, int splits, int64_t n, void* Y, bool y_f32,
+                            cudaStream_t stream, bool pdl);
 
 // The operand boxes: a0/a1 are loaded as block_m x 64, b0/b1 as block_n x 64.
 cudaError_t launch_dequant_gemm(const GemmArgs& args, const GemmMaps& maps, int block_n,

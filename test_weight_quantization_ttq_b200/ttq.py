@@ -67,6 +67,7 @@ SIGNATURES = {
     "ttq_linear_forward_ex": (_INT, [_P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _F, _F, _F, _INT,
                                      _INT, _INT, _P, _INT, _P, _SZ, _P]),
     "ttq_dequantized_gemm": (_INT, [_P, _P, _I64, _I64, _I64, _P, _INT, _P, _SZ, _P]),
+    "ttq_dequantized_gemm_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "ttq_scale_activations": (_INT, [_P, _INT, _I64, _I64, _P, _P, _P, _SZ, _P]),
     "ttq_dequant_gemm": (_INT, [_P, _P, _P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _I64, _INT, _INT,
                                 _P, _INT, _P, _SZ, _P]),
@@ -428,7 +429,10 @@ def ttq_dequantized_gemm(W_hat, Xs, ws=None, Y=None, y_dtype=torch.bfloat16, str
     T = Xs.shape[0]
     _matrix(Y, "Y", T, dp, _FLOAT_IN)
     if ws is None:
-        ws = new_workspace(d, 0, 0, 0, 4, 32, TTQ_BF16, W_hat.device, stream)
+        # room for the forward's K split of this shape, so the result is its bits
+        nbytes = max(4096, int(lib().ttq_dequantized_gemm_workspace_size(d, dp, T)))
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=W_hat.device)
+        ttq_workspace_init(ws, stream)
     if Y is None:
         Y = torch.empty((T, dp), dtype=y_dtype, device=W_hat.device)
     _check(lib().ttq_dequantized_gemm(_dev(W_hat, "W_hat"), _dev(Xs, "Xs"), d, dp, T, _dev(Y, "Y"),

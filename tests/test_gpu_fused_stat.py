@@ -118,8 +118,14 @@ def test_forward_kernel_count_matches_launches():
     from torch.autograd import DeviceType
     from torch.profiler import ProfilerActivity, profile
 
-    cases = [(synth.C2.with_(dp=512), 3, True),
-             (_spec("long_two_kernel", d=8192, dp=64, T=4096), 4, False),
+    cases = [(synth.C2, 3, True),
+             # few output tiles: statistic, quantiser, the product split
+             # along K and the reduction of its splits
+             (synth.C2.with_(dp=512), 4, True),
+             (_spec("split_product", d=4096, dp=200, T=333), 4, True),
+             # two statistic kernels; 64 rows of W against 4096 tokens and
+             # 8192 channels: the product splits along K, then its reduction
+             (_spec("long_two_kernel", d=8192, dp=64, T=4096), 5, False),
              (_spec("f32_lowrank", d=448, dp=96, T=77, dtype="f32", r=16), 6, True),
              (_spec("no_tokens", d=512, dp=64, T=0), 2, True),
              # a few tokens: statistic, then the single-pass product

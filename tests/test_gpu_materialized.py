@@ -77,10 +77,13 @@ def test_materialized_weight_is_the_dequantised_codes(O, spec):
 
 
 
-def test_composed_materialized_steps_equal_forward():
+@pytest.mark.parametrize("spec", [synth.C2.with_(T=300, dp=640),
+                                  # few output tiles: the product splits along K
+                                  synth.C2.with_(T=333, dp=200)], ids=lambda s: f"dp{s.dp}-T{s.T}")
+def test_composed_materialized_steps_equal_forward(spec):
     """ttq_act_norm_scale -> ttq_quantize_dequant_weight -> ttq_dequantized_gemm
-    is the forward for more than 256 tokens, bit for bit."""
-    spec = synth.C2.with_(T=300, dp=640)
+    is the forward for more than 256 tokens, bit for bit (also where the
+    product is split along K and its partial sums are added in split order)."""
     data = P.inputs(spec)
     X, W = P.to_dev(data["X"], "bf16"), P.to_dev(data["W"], "bf16")
     Y = ttq.ttq_linear_forward(X, W, None, None, spec.p, spec.lam, spec.alpha, spec.bits, spec.group,

@@ -163,6 +163,11 @@ FORWARD_CASES = [spec for name in ("C1", "C2", "C3", "C4", "C5") for spec in syn
     _small("decode_lowrank", d=480, dp=150, T=11, bits=4, group=32, r=16),
     _small("decode_int3_lowrank", d=736, dp=77, T=1, bits=3, group=32, r=8, dtype="f32"),
     _small("decode_int3_k768", d=768, dp=129, T=8, bits=3, group=128, r=16),
+    # the product on W_hat split along K (few output tiles, long K): ragged
+    # rows, tokens and last K block, and the low-rank tail in the last split
+    _small("split_k_ragged_lowrank", d=8224, dp=300, T=333, bits=4, group=32, r=16),
+    _small("split_k_int2_lowrank", d=4128, dp=264, T=520, bits=2, group=32, r=24),
+    _small("split_k_eight", d=4096, dp=200, T=333, bits=3, group=64),
 ]
 
 
