@@ -27,6 +27,7 @@
 #include <cuda_fp8.h>
 
 #include <atomic>
+#include <cstring>
 
 #include <type_traits>
 
@@ -383,9 +384,10 @@ constexpr uint32_t kQSmemBytes = kQStages * kQStageBytes;           // 96 KiB
 
 template <int BITS, bool WQ, bool SYM, int G>
 __global__ void __launch_bounds__(kThreads, 2) qdq_stage_kernel(
-    const __nv_bfloat16* __restrict__ W, int64_t dp, int64_t d, const float* __restrict__ D,
-    int cw, uint32_t* __restrict__ codes, __half* __restrict__ scales,
-    __half* __restrict__ zeros, __half* __restrict__ wq, uint32_t* __restrict__ status) {
+    const __grid_constant__ CUtensorMap tmW, int w_box, const __nv_bfloat16* __restrict__ W,
+    int64_t dp, int64_t d, const float* __restrict__ D, int cw, uint32_t* __restrict__ codes,
+    __half* __restrict__ scales, __half* __restrict__ zeros, __half* __restrict__ wq,
+    uint32_t* __restrict__ status) {
   static_assert(G == 2 || G == 4 || G == 8 || G == 16, "group of 32 to 256 channels");
   constexpr int QMAX = (1 << BITS) - 1;
   constexpr int kWarps = kThreads / 32;
@@ -429,6 +431,16 @@ __global__ void __launch_bounds__(kThreads, 2) qdq_stage_kernel(
   auto issue = [&](int64_t i) {
     const int s = static_cast<int>(i % kQStages);
     const int64_t r0 = (blockIdx.y + i * gridDim.y) * rows_pb;
+    if (w_box) {
+      // one tensor-map box of rows_pb rows x cw channels (a whole stage;
+      // rows past dp arrive as zeros and count toward the bytes)
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], kQStageBytes);
+        tma_load_2d(&tmW, &full[s], stage_smem + static_cast<size_t>(s) * kQStageBytes,
+                    static_cast<int32_t>(col0), static_cast<int32_t>(r0));
+      }
+      return;
+    }
     const int nrows = static_cast<int>(min(static_cast<int64_t>(rows_pb), dp - r0));
     if (lane == 0) mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nrows) * row_bytes);
     __syncwarp();
@@ -805,8 +817,14 @@ cudaError_t launch_stage_g(dim3 grid, const __nv_bfloat16* W, int64_t dp, int64_
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev].store(true, std::memory_order_relaxed);
   }
+  // narrow tiles (at most 256 channels, a batch of at most 256 rows): each
+  // batch comes in as one tensor-map box instead of one bulk copy per row
+  CUtensorMap tmW;
+  memset(&tmW, 0, sizeof(tmW));
+  const int rows_pb = kStageRows * (kThreads / (cw >> 4));
+  const int w_box = cw <= 256 && rows_pb <= 256 && encode_bf16_box(&tmW, W, d, dp, cw, rows_pb);
   return launch_kernel(qdq_stage_kernel<BITS, WQ, SYM, G>, grid, dim3(kThreads), smem, stream,
-                       pdl, W, dp, d, D, cw, codes, s, z, wq, status);
+                       pdl, tmW, w_box, W, dp, d, D, cw, codes, s, z, wq, status);
 }
 
 template <int BITS, bool WQ, bool SYM>

@@ -472,6 +472,23 @@ ttq_status run_statistic(const void* X, ttq_dtype dtype, int64_t d, int64_t T, f
 }
 
 }  // namespace
+
+bool encode_bf16_box(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int box_cols,
+                     int box_rows) {
+  EncodeFn enc = get_encode();
+  if (enc == nullptr || cols < 1 || rows < 1 || (cols * 2) % 16 != 0 || box_cols < 8 ||
+      box_cols > 256 || (box_cols * 2) % 16 != 0 || box_rows < 1 || box_rows > 256 ||
+      (reinterpret_cast<uintptr_t>(base) & 15u) != 0)
+    return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace ttq
 
 using namespace ttq;

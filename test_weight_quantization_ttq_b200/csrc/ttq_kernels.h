@@ -66,6 +66,13 @@ cudaError_t launch_act_norm_scale(const void* X, bool x_f32, int64_t d, int64_t 
                                   uint32_t* status, cudaStream_t stream, bool* launched,
                                   float* Dh = nullptr);
 
+// Tensor map of a bf16 matrix [rows][cols] (row stride cols elements, a
+// multiple of 8; base 16-byte aligned), loaded as box_rows x box_cols tiles
+// (each at most 256) without swizzle: row-major in shared memory, rows past
+// the matrix zero-filled.  False when the driver or the sizes do not allow it.
+bool encode_bf16_box(CUtensorMap* m, const void* base, int64_t cols, int64_t rows, int box_cols,
+                     int box_rows);
+
 // Step (2): codes, scales, zeros of Q[W D^{1/2}] (D may be null); with wq
 // non-null also the dequantised weight s (q - z) as binary16 [dp][d].
 // symmetric: the symmetric quantiser (zero point 2^(b-1)).
