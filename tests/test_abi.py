@@ -109,6 +109,27 @@ def test_dequantised_weight_only_for_long_inputs(L):
     assert lay.wq % 256 == 0 and lay.wq > lay.zeros and lay.wq + 4096 * 4096 * 2 <= lay.total
 
 
+def test_split_product_plan(L):
+    """The product on the materialised weight splits along K where few output
+    rows meet a long K, and only there: the 11008 -> 4096 projection at 512
+    tokens in 4 splits (its float32 partial sums in the layout's ypart
+    region, 4 x 512 x 4096 floats, and the same room after the 20 KiB header
+    for ttq_dequantized_gemm), the 4096 -> 4096 and 4096 -> 11008 layers and
+    the 8192 -> 28672 ones not at all."""
+    lay = ttq.ttq_workspace_get_layout(11008, 4096, 512, 32, 3, 128, ttq.TTQ_BF16)
+    need = 4 * 512 * 4096 * 4
+    assert lay.ypart % 256 == 0 and lay.ypart > lay.wq and lay.ypart + need <= lay.total
+    assert L.ttq_dequantized_gemm_workspace_size(11008, 4096, 512) == 20480 + need
+    for d, dp, T, r in ((4096, 4096, 2048, 0), (4096, 11008, 512, 32), (8192, 28672, 1024, 64),
+                        (8192, 28672, 4096, 64)):
+        assert ttq.ttq_workspace_get_layout(d, dp, T, r, 3, 128, ttq.TTQ_BF16).ypart == 0, (d, dp, T)
+        assert L.ttq_dequantized_gemm_workspace_size(d, dp, T) == 4096, (d, dp, T)
+    # at most 256 tokens the product is never split
+    assert ttq.ttq_workspace_get_layout(11008, 4096, 256, 32, 3, 128, ttq.TTQ_BF16).ypart == 0
+    assert L.ttq_dequantized_gemm_workspace_size(11008, 4096, 256) == 4096
+    assert L.ttq_dequantized_gemm_workspace_size(12, 4096, 512) == 0   # d % 8 != 0
+
+
 @pytest.mark.parametrize("args", [
     (4096, 4096, 2048, 0, 5, 128),   # bits not built
     (4096, 4096, 2048, 0, 4, 96),    # group not built
