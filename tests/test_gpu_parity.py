@@ -168,6 +168,9 @@ FORWARD_CASES = [spec for name in ("C1", "C2", "C3", "C4", "C5") for spec in syn
     _small("split_k_ragged_lowrank", d=8224, dp=300, T=333, bits=4, group=32, r=16),
     _small("split_k_int2_lowrank", d=4128, dp=264, T=520, bits=2, group=32, r=24),
     _small("split_k_eight", d=4096, dp=200, T=333, bits=3, group=64),
+    # T x d' odd: the split reduction's element-wise path (and Y rows of an
+    # odd length)
+    _small("split_k_odd_rows_lowrank", d=4096, dp=201, T=333, bits=4, group=32, r=16),
 ]
 
 
