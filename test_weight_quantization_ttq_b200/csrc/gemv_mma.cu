@@ -573,6 +573,118 @@ cudaError_t launch_decode_bits(const CUtensorMap& tmC, const CUtensorMap& tmX,
              : launch_decode_typed<BITS, 1, false>(tmC, tmX, a, gs, stream, pdl);
 }
 
+
+// The low-rank A X product for 17 to 512 tokens, out[t][k] = sum_i
+// A[k][i] X[t][i] (bf16 operands, fp32 sums): CTA (x, y) takes tokens
+// 64 x .. 64 x + 63 and channels [y kc, (y + 1) kc) of the reduction, brings
+// both operand slices into shared memory at once with asynchronous copies
+// (zero-filled past T and d), and its four warps each multiply 16 tokens by
+// all r rows of A with warp-level MMAs (m16n8k16, k ascending).  With one
+// channel slice the CTA rounds its sums to bf16 AX [T][ax_ld]; otherwise it
+// writes its fp32 partial sums to P [slice][T][r] for ax_reduce_kernel to add
+// in slice order.  Rows of the shared tiles are padded by 16 bytes so that
+// the fragment loads of a warp fall in 32 different banks.
+constexpr int kAxTokens = 64;
+constexpr int kAxThreads = 128;
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+
+template <int NT>   // NT = r / 8 tiles of 8 rows of A
+__global__ void __launch_bounds__(kAxThreads) ax_mma_kernel(
+    const __nv_bfloat16* __restrict__ A, const __nv_bfloat16* __restrict__ X, int64_t d, int64_t T,
+    int kc, float* __restrict__ P, __nv_bfloat16* __restrict__ AX, int64_t ax_ld) {
+  extern __shared__ __align__(16) __nv_bfloat16 ax_smem[];
+  constexpr int R = 8 * NT;
+  const int ld = kc + 8;                          // padded row, in elements
+  __nv_bfloat16* sX = ax_smem;                    // [kAxTokens][ld]
+  __nv_bfloat16* sA = ax_smem + kAxTokens * ld;   // [R][ld]
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kAxTokens;
+  const int64_t k0 = static_cast<int64_t>(blockIdx.y) * kc;
+  allow_dependents_launch();
+  grid_dependency_wait();   // X may come from the previous kernel
+
+  // both slices, 16 bytes (8 channels) per copy; d % 8 == 0, so a chunk is
+  // either inside d or wholly past it
+  const int cpr = kc / 8;                         // chunks per row
+  for (int c = threadIdx.x; c < (kAxTokens + R) * cpr; c += kAxThreads) {
+    const int row = c / cpr, ch = c - row * cpr;
+    const int64_t k = k0 + ch * 8;
+    const bool in_x = row < kAxTokens;
+    const int64_t grow = in_x ? t0 + row : row - kAxTokens;
+    const bool valid = k < d && (!in_x || grow < T);
+    const __nv_bfloat16* src = (in_x ? X : A) + (valid ? grow * d + k : 0);
+    __nv_bfloat16* dst = (in_x ? sX + row * ld : sA + (row - kAxTokens) * ld) + ch * 8;
+    cp_async16(static_cast<uint32_t>(__cvta_generic_to_shared(dst)), src, valid ? 16u : 0u);
+  }
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qr = lane >> 2, qc = (lane & 3) * 2;
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  const __nv_bfloat16* xr0 = sX + (warp * 16 + qr) * ld + qc;
+  const __nv_bfloat16* xr1 = xr0 + 8 * ld;
+  const __nv_bfloat16* ar = sA + qr * ld + qc;
+  const int ksteps = static_cast<int>(min(static_cast<int64_t>(kc), d - k0) + 15) / 16;
+  for (int s = 0; s < ksteps; ++s) {
+    const int kk = s * 16;
+    uint32_t a[4];
+    a[0] = *reinterpret_cast<const uint32_t*>(xr0 + kk);
+    a[1] = *reinterpret_cast<const uint32_t*>(xr1 + kk);
+    a[2] = *reinterpret_cast<const uint32_t*>(xr0 + kk + 8);
+    a[3] = *reinterpret_cast<const uint32_t*>(xr1 + kk + 8);
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const __nv_bfloat16* b = ar + j * 8 * ld + kk;
+      mma_m16n8k16_bf16(acc[j], a, *reinterpret_cast<const uint32_t*>(b),
+                        *reinterpret_cast<const uint32_t*>(b + 8));
+    }
+  }
+
+  const bool partial = gridDim.y > 1;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int64_t t = t0 + warp * 16 + qr + 8 * h;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int k = j * 8 + qc;
+      if (partial) {
+        float2* dst = reinterpret_cast<float2*>(P + (static_cast<int64_t>(blockIdx.y) * T + t) * R + k);
+        *dst = make_float2(acc[j][2 * h], acc[j][2 * h + 1]);
+      } else {
+        *reinterpret_cast<__nv_bfloat162*>(AX + t * ax_ld + k) =
+            __floats2bfloat162_rn(acc[j][2 * h], acc[j][2 * h + 1]);
+      }
+    }
+  }
+}
+
+template <int NT>
+cudaError_t launch_ax_mma_nt(const __nv_bfloat16* A, const __nv_bfloat16* X, int64_t d, int64_t T,
+                             int kc, int splits, float* P, __nv_bfloat16* AX, int64_t ax_ld,
+                             cudaStream_t stream, bool pdl) {
+  const size_t smem = static_cast<size_t>(kAxTokens + 8 * NT) * (kc + 8) * 2;
+  static std::atomic<size_t> attr_bytes[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 64 || attr_bytes[dev].load(std::memory_order_relaxed) < smem) {
+    const cudaError_t e = cudaFuncSetAttribute(ax_mma_kernel<NT>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_bytes[dev].store(smem, std::memory_order_relaxed);
+  }
+  const dim3 grid(static_cast<unsigned>((T + kAxTokens - 1) / kAxTokens), static_cast<unsigned>(splits));
+  return launch_kernel(ax_mma_kernel<NT>, grid, dim3(kAxThreads), smem, stream, pdl, A, X, d, T, kc,
+                       P, AX, ax_ld);
+}
+
 }  // namespace
 
 DecodeMapShape decode_map_shape(int bits, int T) {
@@ -602,6 +714,41 @@ cudaError_t launch_decode_gemm(const DecodeArgs& a, const CUtensorMap& tmC,
     case 3: return launch_decode_bits<3>(tmC, tmX, a, gs, stream, pdl);
     case 4: return launch_decode_bits<4>(tmC, tmX, a, gs, stream, pdl);
     case 8: return launch_decode_bits<8>(tmC, tmX, a, gs, stream, pdl);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+
+AxMmaPlan ax_mma_plan(int64_t r, int64_t T, int64_t d) {
+  // at up to 16 tokens the tensor-core GEMM's K splits measured faster
+  // (8192 -> 28672 at one token: 118.9 against 121.2 us per forward)
+  if (T <= 16 || T > kAxMaxTokens || r < 8 || r > 96 || r % 8 != 0) return {0, 0};
+  const int kc = r <= 32 ? 512 : 256;
+  return {static_cast<int>((d + kc - 1) / kc), kc};
+}
+
+cudaError_t launch_ax_mma(const void* A, const void* X, int64_t d, int64_t T, int64_t r,
+                          const AxMmaPlan& plan, float* P, void* AX, int64_t ax_ld,
+                          cudaStream_t stream, bool pdl) {
+  if (T == 0) return cudaSuccess;
+  if (plan.splits < 1 || (plan.splits > 1 && P == nullptr)) return cudaErrorInvalidValue;
+  const auto* a = static_cast<const __nv_bfloat16*>(A);
+  const auto* x = static_cast<const __nv_bfloat16*>(X);
+  auto* ax = static_cast<__nv_bfloat16*>(AX);
+  const int kc = plan.kc;
+  switch (r / 8) {
+    case 1: return launch_ax_mma_nt<1>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 2: return launch_ax_mma_nt<2>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 3: return launch_ax_mma_nt<3>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 4: return launch_ax_mma_nt<4>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 5: return launch_ax_mma_nt<5>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 6: return launch_ax_mma_nt<6>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 7: return launch_ax_mma_nt<7>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 8: return launch_ax_mma_nt<8>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 9: return launch_ax_mma_nt<9>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 10: return launch_ax_mma_nt<10>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 11: return launch_ax_mma_nt<11>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
+    case 12: return launch_ax_mma_nt<12>(a, x, d, T, kc, plan.splits, P, ax, ax_ld, stream, pdl);
     default: return cudaErrorInvalidValue;
   }
 }

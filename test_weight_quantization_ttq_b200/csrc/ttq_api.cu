@@ -81,6 +81,14 @@ GemmPlan product_plan(int64_t dp, int64_t T, int64_t d, int64_t r, bool allow_sp
   return gemm_plan_plain(dp, T, d, r, kPlanSMs, allow_split && T > 256);
 }
 
+// The number of parts of the low-rank A X product's reduction over d
+// (1: none): the warp-level MMA kernel's channel slices for 17 to 512
+// tokens, else the tensor-core GEMM's K splits.
+int ax_parts(int64_t r, int64_t T, int64_t d) {
+  const AxMmaPlan mp = ax_mma_plan(r, T, d);
+  return mp.splits > 0 ? mp.splits : ax_split_plan(r, T, d, kPlanSMs).splits;
+}
+
 bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int group,
                  ttq_dtype dtype, ttq_workspace_layout* L) {
   if (d < 8 || d % 8 != 0 || dp < 0 || T < 0 || r < 0 || r % 8 != 0) return false;
@@ -114,11 +122,11 @@ bool make_layout(int64_t d, int64_t dp, int64_t T, int64_t r, int bits, int grou
     l.ax_ld = r;
     l.ax = off;
     off = align_up(off + static_cast<size_t>(T) * static_cast<size_t>(r) * 2);
-    const AxSplit sp = ax_split_plan(r, T, d, kPlanSMs);
-    l.ax_splits = sp.splits;
-    if (sp.splits > 1) {
+    const int parts = ax_parts(r, T, d);
+    l.ax_splits = parts;
+    if (parts > 1) {
       l.axp = off;
-      off = align_up(off + static_cast<size_t>(sp.splits) * static_cast<size_t>(T) *
+      off = align_up(off + static_cast<size_t>(parts) * static_cast<size_t>(T) *
                                static_cast<size_t>(r) * 4);
     }
   }
@@ -257,6 +265,17 @@ ttq_status run_ax(const void* Ab, const void* Xb, int64_t d, int64_t T, int64_t 
                   const ttq_workspace_layout& L, cudaStream_t stream, bool pdl) {
   uint32_t* status = reinterpret_cast<uint32_t*>(ws_at(ws, L.status));
   void* ax = ws_at(ws, L.ax);
+  const AxMmaPlan mp = ax_mma_plan(r, T, d);
+  if (mp.splits > 0) {
+    // 17 to 512 tokens: warp-level MMAs over channel slices
+    const bool split = mp.splits > 1;
+    if (split && (L.axp == 0 || L.ax_splits != mp.splits)) return TTQ_ERR_WORKSPACE;
+    float* P = split ? reinterpret_cast<float*>(ws_at(ws, L.axp)) : nullptr;
+    const ttq_status st =
+        cuda_status(launch_ax_mma(Ab, Xb, d, T, r, mp, P, ax, L.ax_ld, stream, pdl));
+    if (st != TTQ_OK || !split) return st;
+    return cuda_status(launch_ax_reduce(P, mp.splits, T, r, ax, L.ax_ld, stream, true));
+  }
   const int bn = gemm_block_n(T);
   GemmMaps m;
   if (!encode_16bit(&m.a0, Ab, false, d, r, d, 128) || !encode_16bit(&m.b0, Xb, false, d, T, d, bn))
@@ -592,7 +611,7 @@ ttq_status ttq_linear_forward_kernels(ttq_dtype dtype, int64_t d, int64_t dp, in
         ++n;                                                               // its split reduction
       if (r > 0) {
         n += 1 + (f32 ? 2 : 0);                                            // A X (+ bf16 A, B)
-        if (ax_split_plan(r, T, d, kPlanSMs).splits > 1) ++n;              // its split reduction
+        if (ax_parts(r, T, d) > 1) ++n;                                    // its split reduction
       }
     }
   }

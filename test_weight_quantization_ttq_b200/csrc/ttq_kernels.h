@@ -233,6 +233,23 @@ struct AxSplit {
 };
 AxSplit ax_split_plan(int64_t r, int64_t T, int64_t d, int num_sms);
 
+// The low-rank A X product for 17 to kAxMaxTokens tokens on warp-level
+// MMAs: plan.splits slices of plan.kb_per_split channels of the reduction
+// (512 for r <= 32, else 256), one CTA per 64 tokens and slice.  With one
+// slice it writes bf16 AX [T][ax_ld] itself; with more it writes the fp32
+// partial sums P [splits][T][r] for launch_ax_reduce.  ax_mma_plan returns
+// splits = 0 where it does not apply (other token counts, or r not a
+// multiple of 8 in 8..96).
+constexpr int64_t kAxMaxTokens = 512;
+struct AxMmaPlan {
+  int splits;   // channel slices (0: the kernel does not apply)
+  int kc;       // channels per slice
+};
+AxMmaPlan ax_mma_plan(int64_t r, int64_t T, int64_t d);
+cudaError_t launch_ax_mma(const void* A, const void* X, int64_t d, int64_t T, int64_t r,
+                          const AxMmaPlan& plan, float* P, void* AX, int64_t ax_ld,
+                          cudaStream_t stream, bool pdl);
+
 // AX [T][ax_ld] bf16 = the sum over the splits, in split order, of the
 // float32 partials P [splits][T][r] (one rounding at the end).
 cudaError_t launch_ax_reduce(const float* P, int splits, int64_t T, int64_t r, void* AX,
