@@ -130,6 +130,27 @@ def test_split_product_plan(L):
     assert L.ttq_dequantized_gemm_workspace_size(12, 4096, 512) == 0   # d % 8 != 0
 
 
+def test_low_rank_product_parts(L):
+    """A X's reduction over d: for 17 to 512 tokens the warp-level MMA
+    kernel's channel slices (512 channels for r <= 32, 256 above), whose
+    partial sums the layout holds; otherwise the tensor-core GEMM's K splits
+    (at most one wave, at least 4 blocks of 64 channels each)."""
+    def lay(d, T, r):
+        return ttq.ttq_workspace_get_layout(d, 4096, T, r, 3, 128, ttq.TTQ_BF16)
+    for d, T, r, parts in ((4096, 512, 32, 8), (11008, 512, 32, 22), (8192, 128, 64, 32),
+                           (448 + 64, 77, 16, 1), (4096, 17, 96, 16)):
+        lo = lay(d, T, r)
+        assert lo.ax_splits == parts, (d, T, r, lo.ax_splits)
+        if parts > 1:
+            assert lo.axp % 256 == 0 and lo.axp + parts * T * r * 4 <= lo.total
+        else:
+            assert lo.axp == 0
+    for d, T, r in ((8192, 1, 64), (8192, 16, 64), (4096, 513, 32), (8192, 4096, 64)):
+        lo = lay(d, T, r)
+        kb = -(-d // 64)
+        assert 1 <= lo.ax_splits <= max(1, kb // 4), (d, T, r, lo.ax_splits)
+
+
 @pytest.mark.parametrize("args", [
     (4096, 4096, 2048, 0, 5, 128),   # bits not built
     (4096, 4096, 2048, 0, 4, 96),    # group not built
